@@ -1,0 +1,140 @@
+"""CPU oracle for the Kimi Delta Attention (KDA) forward pass.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, the smoke check and the benchmark's
+CPU-baseline / reference leg may import this package.  The library's product
+path never calls it, and it shares no code with the CUDA path.
+
+Two implementations of the same definition, both fp64 on the exact input
+values, both following "Kimi Delta Attention: The Linear Attention Behind Kimi
+K2 and Qwen3", §How Kimi Delta Attention works step by step (the order:
+decay per channel, predict from the decayed state, error scaled by beta,
+delta-rule write, read with the query scaled by 1/sqrt(d_k)):
+
+* ``forward``     -- plain C (``kda_oracle.c``), threaded over heads; used for
+                     parity at realistic sizes and for the timed CPU baseline.
+* ``forward_np``  -- plain numpy, a loop over tokens vectorised over (B, H);
+                     used for small cases and to cross-check ``forward``.
+
+Both store the state as ``[B, H, dk, dv]`` (the transpose of the page's
+(d_v, d_k) matrix), so the per-channel decay scales rows and the page's
+``S @ k`` is ``S^T k`` here.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+import subprocess
+from typing import Optional
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kda_oracle.c")
+_LIB = os.path.join(_HERE, "libkda_oracle.so")
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile ``kda_oracle.c`` into ``libkda_oracle.so`` next to it."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-pthread",
+                               _SRC, "-o", tmp, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        f = lib.kda_oracle_forward
+        f.restype = ctypes.c_int
+        f.argtypes = [ctypes.c_void_p] * 8 + [ctypes.c_int] * 5 + [ctypes.c_double, ctypes.c_int]
+        lib.kda_oracle_default_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return int(_load().kda_oracle_default_threads())
+
+
+def _as_f32(x) -> np.ndarray:
+    """Exact fp32 copy of a torch tensor (bf16 or fp32) or array."""
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").float().numpy()
+    return np.ascontiguousarray(x, dtype=np.float32)
+
+
+def _as_f64(x) -> Optional[np.ndarray]:
+    if x is None:
+        return None
+    if hasattr(x, "detach"):
+        x = x.detach().to("cpu").double().numpy()
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(a: Optional[np.ndarray]):
+    return None if a is None else a.ctypes.data_as(ctypes.c_void_p)
+
+
+def forward(q, k, v, log_alpha, beta, initial_state=None, scale=None, nthreads=0):
+    """fp64 KDA forward by the token recurrence (C implementation).
+
+    Arguments are torch tensors or numpy arrays in the library layout:
+    q, k, log_alpha ``[B,T,H,dk]``; v ``[B,T,H,dv]``; beta ``[B,T,H]``;
+    initial_state ``[B,H,dk,dv]`` or None (zeros).  ``scale`` defaults to
+    ``1/sqrt(dk)``.  Returns ``(out [B,T,H,dv], final_state [B,H,dk,dv])`` as
+    fp64 numpy arrays.
+    """
+    qf, kf, vf, af, bf = (_as_f32(x) for x in (q, k, v, log_alpha, beta))
+    B, T, H, dk = qf.shape
+    dv = vf.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    s0 = _as_f64(initial_state)
+    out = np.empty((B, T, H, dv), dtype=np.float64)
+    sT = np.empty((B, H, dk, dv), dtype=np.float64)
+    rc = _load().kda_oracle_forward(_ptr(qf), _ptr(kf), _ptr(vf), _ptr(af), _ptr(bf),
+                                    _ptr(s0), _ptr(out), _ptr(sT),
+                                    B, T, H, dk, dv, float(scale), int(nthreads))
+    if rc != 0:
+        raise RuntimeError("kda_oracle_forward failed with code %d" % rc)
+    return out, sT
+
+
+def forward_np(q, k, v, log_alpha, beta, initial_state=None, scale=None):
+    """fp64 KDA forward by the token recurrence (numpy implementation).
+
+    Same arguments and results as :func:`forward`.  Meant for small inputs.
+    """
+    qf, kf, vf, af, bf = (_as_f32(x).astype(np.float64) for x in (q, k, v, log_alpha, beta))
+    B, T, H, dk = qf.shape
+    dv = vf.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    S = np.zeros((B, H, dk, dv)) if initial_state is None else _as_f64(initial_state).copy()
+    out = np.empty((B, T, H, dv))
+    for t in range(T):
+        alpha = np.exp(af[:, t])                           # [B,H,dk]
+        S = S * alpha[..., :, None]                        # decay rows (key channels)
+        p = np.einsum("bhcx,bhc->bhx", S, kf[:, t])        # S~^T k
+        e = bf[:, t, :, None] * (vf[:, t] - p)             # beta (v - p)
+        S = S + kf[:, t][..., :, None] * e[..., None, :]   # S~ + k e^T
+        out[:, t] = scale * np.einsum("bhcx,bhc->bhx", S, qf[:, t])
+    return out, S
+
+
+def parity_error(x_gpu, x_ref) -> float:
+    """max |x_gpu - x_ref| / rms(x_ref), the parity metric for outputs and states."""
+    g = np.asarray(x_gpu, dtype=np.float64)
+    r = np.asarray(x_ref, dtype=np.float64)
+    if r.size == 0:
+        return 0.0
+    rms = math.sqrt(float(np.mean(r * r)))
+    err = float(np.max(np.abs(g - r)))
+    if rms == 0.0:
+        return err
+    return err / rms

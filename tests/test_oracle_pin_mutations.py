@@ -1,0 +1,77 @@
+"""The oracle pins catch plausible mistakes.
+
+Each case below is the numpy oracle with one deliberate slip planted in a local
+copy (on the CPU; the real oracle is untouched).  Every slip must make at least
+one pin in test_oracle_pins fail.
+"""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from tests import test_oracle_pins as pins
+
+
+def _make(mutation):
+    def fwd(q, k, v, log_alpha, beta, initial_state=None, scale=None):
+        qf, kf, vf, af, bf = (oracle._as_f32(x).astype(np.float64) for x in (q, k, v, log_alpha, beta))
+        B, T, H, dk = qf.shape
+        dv = vf.shape[-1]
+        if scale is None:
+            scale = 1.0 / math.sqrt(dk)
+        if mutation == "no_scale":
+            scale = 1.0
+        S = np.zeros((B, H, dk, dv)) if initial_state is None else oracle._as_f64(initial_state).copy()
+        out = np.empty((B, T, H, dv))
+        for t in range(T):
+            alpha = af[:, t] if mutation == "alpha_not_exp" else np.exp(af[:, t])
+            if mutation == "read_before_write":
+                pre = np.einsum("bhcx,bhc->bhx", S * alpha[..., :, None], qf[:, t])
+            S_old = S
+            if mutation == "decay_value_axis":
+                S = S * alpha[..., None, :dv] if dv <= dk else S
+            else:
+                S = S * alpha[..., :, None]
+            src = S_old if mutation == "predict_undecayed" else S
+            p = np.einsum("bhcx,bhc->bhx", src, kf[:, t])
+            e = vf[:, t] - p if mutation == "no_beta" else bf[:, t, :, None] * (vf[:, t] - p)
+            if mutation == "error_sign":
+                e = -e
+            S = S + kf[:, t][..., :, None] * e[..., None, :]
+            if mutation == "transposed_read" and dk == dv:
+                o = np.einsum("bhxc,bhc->bhx", S, qf[:, t])
+            elif mutation == "read_before_write":
+                o = pre
+            else:
+                o = np.einsum("bhcx,bhc->bhx", S, qf[:, t])
+            out[:, t] = scale * o
+        return out, S
+    return fwd
+
+
+PIN_TESTS = [pins.test_worked_example_by_hand, pins.test_beta_zero_is_pure_per_channel_decay,
+             pins.test_small_beta_no_decay_is_linear_attention,
+             pins.test_no_decay_is_deltanet_in_value_by_key_layout,
+             pins.test_scalar_decay_is_gated_deltanet, pins.test_unit_write_recalls_value_exactly,
+             pins.test_unrolled_matrix_products_tiny]
+
+
+@pytest.mark.parametrize("mutation", ["decay_value_axis", "predict_undecayed", "read_before_write",
+                                      "error_sign", "no_beta", "no_scale", "transposed_read",
+                                      "alpha_not_exp"])
+def test_some_pin_fails_on_planted_mistake(mutation):
+    fwd = _make(mutation)
+    failed = []
+    for t in PIN_TESTS:
+        try:
+            t(fwd)
+        except AssertionError:
+            failed.append(t.__name__)
+    assert failed, "no pin caught the planted mistake %r" % mutation
+
+
+def test_unmutated_copy_passes_every_pin():
+    fwd = _make("none")
+    for t in PIN_TESTS:
+        t(fwd)
