@@ -1,0 +1,501 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA forward on B200: chunked prefill and single-token decode.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl kda|reference]
+
+Prints ONE JSON line on rank 0.
+
+* ``value``: prefill tokens/s of the long-context workload (B=1, H=32,
+  T=65536, dk=dv=128, bf16 inputs, fp32 final state), whole job: the tokens
+  every rank processed divided by the slowest rank's device time for K steps.
+  One step is one ``kda_forward`` over the whole batch (chunk staging, decay
+  cumsum and scaling, intra-chunk products, UT solve, inter-chunk scan,
+  output, state I/O).  Inputs (3.77 GB per step) are far larger than the
+  126 MB L2, so no flush is needed between steps.
+* ``decode``: the decode workload (B=256, H=32, d=128, 537 MB fp32 state),
+  1024 sequential ``kda_decode_step`` calls timed as one region.
+* ``e2e``: the same metrics through the public Python API with host-resident
+  pinned inputs: every step copies that step's inputs host->device and reads
+  the outputs back device->host inside the timed region.
+* ``roofline``: the prefill kernel's algorithmic bytes per launch over its
+  CUDA-event launch time, against the measured HBM copy bandwidth.
+* ``cpu_baseline``: the fp64 CPU oracle timed on this host on a bounded slice
+  of the same workload (rank 0, N=1 only).
+
+With N > 1 (launched by torchrun) every rank runs its own independent batch
+of the same size (weak scaling); no collective touches the data path, only
+the timing (barrier, max over ranks).
+
+``--impl reference`` times the fp64 CPU oracle instead (the reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "KDA prefill tokens/s (H32,d128,T64K) & decode tok/s; % of roofline"
+HBM_FALLBACK_GBS = 6650.0
+BF16_FALLBACK_TFLOPS = 1590.0
+
+# Algorithmic cost model of the prefill per token and head (d = dk = dv):
+# bytes read/written once: q, k, v (input dtype), log_alpha (fp32), beta (fp32), out (fp32).
+# FLOPs: 5*C*d + 6*d^2 per token-head with C = 64 (triangular products counted half).
+def prefill_bytes_per_token_head(dk, dv, in_bytes):
+    return (2 * dk + dv) * in_bytes + 4 * dk + 4 + 4 * dv
+
+
+def prefill_flops_per_token_head(d, C=64):
+    return 5 * C * d + 6 * d * d
+
+
+def decode_bytes_per_head(dk, dv, in_bytes):
+    return 2 * 4 * dk * dv + (2 * dk + dv) * in_bytes + 4 * dk + 4 + 4 * dv
+
+
+# ncu DRAM traffic of the dominant kernel, per launch, keyed by the kernel
+# source it was measured on; reported only while that source is unchanged.
+MEASURED_TRAFFIC = {}
+
+
+def source_digest(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), "measured"
+    except Exception:
+        return HBM_FALLBACK_GBS, BF16_FALLBACK_TFLOPS, BF16_FALLBACK_TFLOPS, "fallback"
+
+
+# ---------------------------------------------------------------- multi-rank plumbing
+def rank_workload(w, rank):
+    """Weak scaling: rank r processes its own independent batch (seed + 1000 r)."""
+    from gated_delta_rule_109_b200 import inputs as I
+    return I.scaled(w, seed=w.seed + 1000 * rank)
+
+
+def max_over_ranks(value, device=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(value)
+    t = torch.tensor([float(value)], dtype=torch.float64, device=device or "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        if device is not None and dist.get_backend() == "nccl":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+def init_distributed(backend="nccl", timeout_s=300):
+    import torch.distributed as dist
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=timeout_s))
+    return rank, local, world
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi samples of this GPU's clocks and throttle reasons, every 200 ms."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device):
+        import torch
+        self.proc = None
+        self.path = None
+        try:
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            self.ident = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            self.ident = str(device.index or 0)
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="kda_clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.ident, "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.3)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        mx = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[4 + i] == "Active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None,
+                "samples": len(rows), "reasons": reasons}
+
+
+# ---------------------------------------------------------------- prefill
+def bench_prefill(w, K, W, device):
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    x = I.make_inputs(w, device)
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+    sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device) if w.final_state else None
+    args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+    for _ in range(W):
+        kda.forward(*args, out=out, final_state=sT, return_final_state=sT is not None)
+    torch.cuda.synchronize(device)
+    kda.check_status(device)
+    stream = torch.cuda.current_stream(device)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(K + 1)]
+    barrier(device)
+    torch.cuda.synchronize(device)
+    n0 = kda.launch_count()
+    evs[0].record(stream)
+    for i in range(K):
+        kda.forward(*args, out=out, final_state=sT, return_final_state=sT is not None)
+        evs[i + 1].record(stream)
+    torch.cuda.synchronize(device)
+    launches = kda.launch_count() - n0
+    barrier(device)
+    per = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
+    kda.check_status(device)
+    return {"ms_total": sum(per), "ms_per_launch": per, "launches": launches, "x": x}
+
+
+def bench_prefill_e2e(w, K, W, device, x):
+    """Same metric through the public API with pinned host inputs, copies inside the timed region."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    names = ("q", "k", "v", "log_alpha", "beta")
+    host = {n: x[n].cpu().pin_memory() for n in names}
+    s0h = x["initial_state"].cpu().pin_memory() if x["initial_state"] is not None else None
+    dev = {n: torch.empty_like(x[n]) for n in names}
+    s0d = torch.empty_like(x["initial_state"]) if s0h is not None else None
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+    sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device) if w.final_state else None
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    sT_h = torch.empty(sT.shape, dtype=sT.dtype).pin_memory() if sT is not None else None
+    h2d = sum(t.numel() * t.element_size() for t in host.values()) + (s0h.numel() * 4 if s0h is not None else 0)
+    d2h = out.numel() * 4 + (sT.numel() * 4 if sT is not None else 0)
+
+    def step():
+        for n in names:
+            dev[n].copy_(host[n], non_blocking=True)
+        if s0h is not None:
+            s0d.copy_(s0h, non_blocking=True)
+        kda.forward(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], s0d,
+                    out=out, final_state=sT, return_final_state=sT is not None)
+        out_h.copy_(out, non_blocking=True)
+        if sT is not None:
+            sT_h.copy_(sT, non_blocking=True)
+
+    for _ in range(W):
+        step()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    e0.record(stream)
+    for _ in range(K):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    assert torch.isfinite(out_h[0, -1]).all()
+    return {"ms_total": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------- decode
+def bench_decode(w, steps, W, device, e2e_steps):
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    x = I.make_inputs(w, device, steps=steps)
+    state = x["initial_state"].clone()
+    outs = torch.empty((steps, w.B, w.H, w.dv), dtype=torch.float32, device=device)
+
+    def run(s, st, o):
+        kda.decode_step(x["q"][s], x["k"][s], x["v"][s], x["log_alpha"][s], x["beta"][s], st, out=o)
+
+    warm_state = x["initial_state"].clone()
+    for s in range(W):
+        run(s % steps, warm_state, outs[s % steps])
+    del warm_state
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    n0 = kda.launch_count()
+    e0.record(stream)
+    for s in range(steps):
+        run(s, state, outs[s])
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    launches = kda.launch_count() - n0
+    barrier(device)
+    kda.check_status(device)
+    ms = e0.elapsed_time(e1)
+
+    # end to end: each step's inputs from pinned host memory, its output read back
+    names = ("q", "k", "v", "log_alpha", "beta")
+    n_e2e = min(e2e_steps, steps)
+    host = {n: x[n][:n_e2e].cpu().pin_memory() for n in names}
+    dbuf = {n: torch.empty_like(x[n][0]) for n in names}
+    out_h = torch.empty((n_e2e, w.B, w.H, w.dv), dtype=torch.float32).pin_memory()
+    h2d = sum(host[n][0].numel() * host[n].element_size() for n in names)
+    d2h = w.B * w.H * w.dv * 4
+    o = torch.empty((w.B, w.H, w.dv), dtype=torch.float32, device=device)
+    st2 = x["initial_state"].clone()
+    del x
+    torch.cuda.synchronize(device)
+    f0, f1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    f0.record(stream)
+    for s in range(n_e2e):
+        for n in names:
+            dbuf[n].copy_(host[n][s], non_blocking=True)
+        kda.decode_step(dbuf["q"], dbuf["k"], dbuf["v"], dbuf["log_alpha"], dbuf["beta"], st2, out=o)
+        out_h[s].copy_(o, non_blocking=True)
+    f1.record(stream)
+    torch.cuda.synchronize(device)
+    barrier(device)
+    return {"ms": ms, "launches": launches, "e2e_ms": f0.elapsed_time(f1), "e2e_steps": n_e2e,
+            "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------- CPU oracle
+def oracle_sample(w, x, budget_s, max_tokens=None, chunk_tokens=2048):
+    """Time the fp64 oracle on the first tokens of every head until ``budget_s``."""
+    import numpy as np
+    import oracle
+    T = w.T if max_tokens is None else min(w.T, max_tokens)
+    state = None if x["initial_state"] is None else x["initial_state"].cpu().double().numpy()
+    done, elapsed = 0, 0.0
+    threads = min(os.cpu_count() or 1, w.B * w.H)
+    while done < T and (elapsed < budget_s or done == 0):
+        n = min(chunk_tokens, T - done)
+        sub = {k: x[k][:, done:done + n].cpu() for k in ("q", "k", "v", "log_alpha", "beta")}
+        t0 = time.perf_counter()
+        _, state = oracle.forward(sub["q"], sub["k"], sub["v"], sub["log_alpha"], sub["beta"], state,
+                                  nthreads=threads)
+        elapsed += time.perf_counter() - t0
+        done += n
+    return {"tokens": done * w.B, "seconds": elapsed, "threads": threads,
+            "value": done * w.B / elapsed}
+
+
+def run_reference(args):
+    """The reference arm: the fp64 CPU oracle on this host, bounded per step."""
+    rank, _, world = int(os.environ.get("RANK", "0")), 0, int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return 0
+    import torch
+    from gated_delta_rule_109_b200 import inputs as I
+    w = I.PREFILL_H32_T64K
+    per_step = args.ref_tokens_per_step
+    steps_total = args.warmup + args.steps
+    T = min(w.T, per_step * steps_total)
+    ws = I.scaled(w, T=T)
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = I.make_inputs(ws, dev)
+    x = {k: (v.cpu() if v is not None else None) for k, v in x.items()}
+    import oracle
+    threads = min(os.cpu_count() or 1, w.B * w.H)
+    state = None
+    t_timed = 0.0
+    for s in range(steps_total):
+        lo, hi = (s * per_step) % T, (s * per_step) % T + per_step
+        sub = {k: x[k][:, lo:hi] for k in ("q", "k", "v", "log_alpha", "beta")}
+        t0 = time.perf_counter()
+        _, state = oracle.forward(sub["q"], sub["k"], sub["v"], sub["log_alpha"], sub["beta"], state,
+                                  nthreads=threads)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            t_timed += dt
+    tokens = per_step * w.B * args.steps
+    value = tokens / t_timed
+    sample = ("fp64 oracle, %s workload, all %d heads, %d consecutive tokens per step "
+              "(state carried), %d threads" % (w.name, w.H, per_step, threads))
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "impl": "reference",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t_timed / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                       "tokens_per_step": per_step},
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---------------------------------------------------------------- main
+def main(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
+    ap.add_argument("--workload", default="prefill_bf16_b1_h32_t65536_d128",
+                    help="prefill workload to time (name from gated_delta_rule_109_b200.inputs)")
+    ap.add_argument("--decode-steps", type=int, default=1024)
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--ref-tokens-per-step", type=int, default=1024)
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    args.warmup = max(3, args.warmup)
+
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    from gated_delta_rule_109_b200 import build as kbuild, inputs as I
+    import gated_delta_rule_109_b200 as kda
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    kda.load()          # fails loudly if libkda.so is missing
+    rank, local, world = init_distributed()
+    if world != args.gpus:
+        raise SystemExit("--gpus %d but WORLD_SIZE=%d (launch N>1 with torchrun)" % (args.gpus, world))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+
+    byname = {w.name: w for w in I.WORKLOADS}
+    w = rank_workload(byname[args.workload], rank)
+    hbm, tf_burst, tf_sust, peak_src = load_peaks()
+    in_bytes = 2 if w.dtype == "bf16" else 4
+
+    clocks = ClockSampler(device)
+    clocks.start()
+    pre = bench_prefill(w, args.steps, args.warmup, device)
+    clk = clocks.stop()
+    ms_total = max_over_ranks(pre["ms_total"], device)
+    tokens_per_step = w.B * w.T
+    value = tokens_per_step * args.steps * world / (ms_total / 1e3)
+
+    # roofline of the prefill kernel (one launch per step)
+    ms_launch = statistics.mean(pre["ms_per_launch"])
+    alg_bytes = (w.B * w.T * w.H * prefill_bytes_per_token_head(w.dk, w.dv, in_bytes)
+                 + (4 * w.B * w.H * w.dk * w.dv if w.final_state else 0)
+                 + (4 * w.B * w.H * w.dk * w.dv if w.state_sd is not None else 0))
+    achieved = alg_bytes / (ms_launch / 1e3) / 1e9
+    kfile = os.path.join(ROOT, "gated_delta_rule_109_b200", "csrc", "kda_prefill_simt.cu")
+    traffic = MEASURED_TRAFFIC.get(("kda_prefill_simt", w.name, source_digest(kfile)))
+    alg_flops = w.B * w.T * w.H * prefill_flops_per_token_head(w.dk)
+    roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                "frac": achieved / hbm, "traffic": traffic,
+                "kernel": "prefill_simt_kernel", "algorithmic_bytes_per_launch": alg_bytes,
+                "ms_per_launch": ms_launch, "peak_source": peak_src + " HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                "tensor_view": {"algorithmic_flops_per_launch": alg_flops,
+                                "achieved_tflops": alg_flops / (ms_launch / 1e3) / 1e12,
+                                "peak_tflops": tf_burst,
+                                "frac": alg_flops / (ms_launch / 1e3) / 1e12 / tf_burst}}
+
+    e2e = bench_prefill_e2e(w, args.e2e_steps, 1, device, pre["x"])
+    e2e_ms = max_over_ranks(e2e["ms_total"], device)
+    del pre["x"]
+    torch.cuda.empty_cache()
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
+                       "input_dtype": w.dtype, "chunk": 64, "final_state": w.final_state,
+                       "l2": "no flush: inputs %.2f GB per step > 126 MB L2" % (alg_bytes / 1e9),
+                       "per_rank": "independent batch per rank (seed + 1000*rank)",
+                       "inputs": "seeded N(0,1) q,k,v (q,k L2-normalised); log_alpha=logsigmoid(N(%g,%g)); "
+                                 "beta=sigmoid(N(%g,%g))" % (w.alpha_mu, w.alpha_sd, w.beta_mu, w.beta_sd)},
+            "roofline": roofline,
+            "e2e": {"value": tokens_per_step * args.e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
+                    "steps": args.e2e_steps},
+            "gpu_launches": pre["launches"],
+            "clocks": clk}
+
+    if not args.no_decode:
+        wd = rank_workload(I.DECODE_B256, rank)
+        dec = bench_decode(wd, args.decode_steps, args.warmup, device, e2e_steps=64)
+        dms = max_over_ranks(dec["ms"], device)
+        d_e2e = max_over_ranks(dec["e2e_ms"], device)
+        dbytes = wd.B * wd.H * decode_bytes_per_head(wd.dk, wd.dv, 2)
+        d_ach = dbytes * args.decode_steps / (dms / 1e3) / 1e9
+        line["decode"] = {
+            "workload": wd.name, "value": wd.B * args.decode_steps * world / (dms / 1e3),
+            "unit": "tokens/s", "steps": args.decode_steps, "ms_per_step": dms / args.decode_steps,
+            "gpu_launches": dec["launches"],
+            "roofline": {"bound": "hbm", "achieved": d_ach, "peak": hbm, "unit": "GB/s",
+                         "frac": d_ach / hbm, "traffic": None, "kernel": "decode_step_kernel",
+                         "algorithmic_bytes_per_launch": dbytes,
+                         "vs_8TBs_spec": d_ach / 8000.0},
+            "e2e": {"value": wd.B * dec["e2e_steps"] * world / (d_e2e / 1e3), "unit": "tokens/s",
+                    "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"],
+                    "steps": dec["e2e_steps"]}}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        xs = I.make_inputs(I.scaled(w, T=min(w.T, 32768)), device)
+        cb = oracle_sample(w, xs, args.cpu_budget_s)
+        line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],
+                                "kind": "oracle",
+                                "sample": "fp64 oracle on the first %d tokens of all %d heads of the %s "
+                                          "workload (%.1f s)" % (cb["tokens"], w.H, w.name, cb["seconds"])}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    import torch.distributed as dist
+    if dist.is_initialized():
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,184 @@
+"""Python binding of libkda, the B200 Kimi Delta Attention forward library.
+
+Argument marshalling only: every step of the computation runs in libkda's CUDA
+kernels (``csrc/``), reached through its C ABI (``include/kda.h``).  PyTorch
+supplies device memory and the current stream.  There is no fallback: if the
+library is not built, every call raises.
+
+    import gated_delta_rule_109_b200 as kda
+    out, final_state = kda.forward(q, k, v, log_alpha, beta, initial_state)
+    out = kda.decode_step(q, k, v, log_alpha, beta, state)   # state updated in place
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkda.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
+KDA_BF16, KDA_F32 = 0, 1
+
+# every symbol include/kda.h declares
+EXPORTS = ("kda_forward", "kda_decode_step", "kda_status_string", "kda_check_status",
+           "kda_last_cuda_error", "kda_launch_count", "kda_version")
+
+_lib = None
+
+
+class KDAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail: str = ""):
+        self.status = status
+        msg = "%s returned %s" % (where, status_string(status) if _lib else str(status))
+        if detail:
+            msg += " (%s)" % detail
+        super().__init__(msg)
+
+
+def load(path: Optional[str] = None) -> ctypes.CDLL:
+    """Load libkda.so (built in-tree by ``gated_delta_rule_109_b200.build``)."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise RuntimeError("libkda.so is not built (%s); run `python -m gated_delta_rule_109_b200.build`" % p)
+    lib = ctypes.CDLL(p)
+    vp, i, f = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+    lib.kda_forward.restype = i
+    lib.kda_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
+    lib.kda_decode_step.restype = i
+    lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
+    lib.kda_status_string.restype = ctypes.c_char_p
+    lib.kda_status_string.argtypes = [i]
+    lib.kda_check_status.restype = i
+    lib.kda_check_status.argtypes = [vp]
+    lib.kda_last_cuda_error.restype = ctypes.c_char_p
+    lib.kda_last_cuda_error.argtypes = []
+    lib.kda_launch_count.restype = ctypes.c_ulonglong
+    lib.kda_launch_count.argtypes = []
+    lib.kda_version.restype = i
+    lib.kda_version.argtypes = []
+    if path is None:
+        _lib = lib
+    return lib
+
+
+def status_string(status: int) -> str:
+    return load().kda_status_string(int(status)).decode()
+
+
+def _check(status: int, where: str):
+    if status != KDA_OK:
+        detail = load().kda_last_cuda_error().decode() if status == KDA_ERR_CUDA else ""
+        raise KDAError(status, where, detail)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError("q, k, v must be bfloat16 or float32, got %s" % t.dtype)
+
+
+def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None):
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError("%s has shape %s, expected %s" % (name, tuple(t.shape), tuple(shape)))
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError("%s must be %s, got %s" % (name, dtype, t.dtype))
+    if not t.is_contiguous():
+        raise ValueError("%s must be contiguous" % name)
+    if device is not None and t.device != device:
+        raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
+
+
+def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
+            return_final_state=True, scale: float = 0.0):
+    """Chunked KDA prefill (``kda_forward``).
+
+    q, k ``[B,T,H,dk]`` and v ``[B,T,H,dv]`` (bf16 or fp32, one dtype);
+    log_alpha ``[B,T,H,dk]`` fp32; beta ``[B,T,H]`` fp32; initial_state
+    ``[B,H,dk,dv]`` fp32 or None.  Returns ``(out [B,T,H,dv] fp32,
+    final_state [B,H,dk,dv] fp32 or None)``.  ``final_state`` may be passed as
+    the same tensor as ``initial_state`` to carry the state in place.
+    ``scale`` 0 means 1/sqrt(dk).
+    """
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q)
+    _need(q, "q", (B, T, H, dk), q.dtype, dev)
+    _need(k, "k", (B, T, H, dk), q.dtype, dev)
+    _need(v, "v", (B, T, H, dv), q.dtype, dev)
+    _need(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    _need(out, "out", (B, T, H, dv), torch.float32, dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
+    st = lib.kda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                         _ptr(initial_state), _ptr(out), _ptr(final_state),
+                         B, T, H, dk, dv, code, float(scale), _stream(dev))
+    _check(st, "kda_forward")
+    return out, final_state
+
+
+def decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0):
+    """One KDA decode step (``kda_decode_step``); ``state`` is updated in place.
+
+    q, k ``[B,H,dk]``, v ``[B,H,dv]`` (bf16 or fp32); log_alpha ``[B,H,dk]``
+    fp32; beta ``[B,H]`` fp32; state ``[B,H,dk,dv]`` fp32.  Returns
+    ``out [B,H,dv]`` fp32.
+    """
+    lib = load()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q)
+    _need(q, "q", (B, H, dk), q.dtype, dev)
+    _need(k, "k", (B, H, dk), q.dtype, dev)
+    _need(v, "v", (B, H, dv), q.dtype, dev)
+    _need(log_alpha, "log_alpha", (B, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, H), torch.float32, dev)
+    _need(state, "state", (B, H, dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=torch.float32, device=dev)
+    _need(out, "out", (B, H, dv), torch.float32, dev)
+    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                             _ptr(state), _ptr(out), B, H, dk, dv, code, float(scale), _stream(dev))
+    _check(st, "kda_decode_step")
+    return out
+
+
+def check_status(device=None):
+    """Synchronise the current stream and raise on a recorded device-side failure."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(load().kda_check_status(_stream(dev)), "kda_check_status")
+
+
+def launch_count() -> int:
+    """Kernels enqueued through libkda by this process so far."""
+    return int(load().kda_launch_count())
+
+
+def version() -> int:
+    return int(load().kda_version())

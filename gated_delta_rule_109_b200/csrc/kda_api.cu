@@ -1,0 +1,127 @@
+// libkda C ABI: argument validation, dispatch to the kernels, status codes.
+// The contract of every entry point is documented in include/kda.h.
+#include <atomic>
+#include <math.h>
+#include <stdint.h>
+#include <stdio.h>
+#include <string.h>
+
+#include "kda_internal.cuh"
+
+namespace {
+
+thread_local char g_last_cuda_error[256] = "";
+std::atomic<unsigned long long> g_launches{0};
+
+kda_status cuda_fail(cudaError_t e)
+{
+    snprintf(g_last_cuda_error, sizeof(g_last_cuda_error), "%s: %s",
+             cudaGetErrorName(e), cudaGetErrorString(e));
+    return KDA_ERR_CUDA;
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+}  // namespace
+
+void kda::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+extern "C" {
+
+unsigned long long kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+
+int kda_version(void) { return 100; }   // 0.1.0
+
+const char *kda_status_string(kda_status s)
+{
+    switch (s) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_MISALIGNED: return "KDA_ERR_MISALIGNED";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    }
+    return "KDA_ERR_UNKNOWN";
+}
+
+const char *kda_last_cuda_error(void) { return g_last_cuda_error; }
+
+kda_status kda_forward(const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       const float *initial_state, float *out, float *final_state,
+                       int B, int T, int H, int dk, int dv,
+                       kda_dtype dtype, float scale, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    // ---- validation: nothing is enqueued unless every check passes
+    if (B <= 0 || H <= 0 || T < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H > (int64_t)INT32_MAX / 4) return KDA_ERR_INVALID_ARG;
+    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
+                  !aligned16(out) || !aligned4(beta)))
+        return KDA_ERR_MISALIGNED;
+    if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
+        return KDA_ERR_MISALIGNED;
+
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
+    if (T == 0) {
+        // no tokens: the final state is the initial state (or zeros)
+        if (!final_state || final_state == initial_state) return KDA_OK;
+        cudaError_t e = initial_state
+            ? cudaMemcpyAsync(final_state, initial_state, state_bytes, cudaMemcpyDeviceToDevice, st)
+            : cudaMemsetAsync(final_state, 0, state_bytes, st);
+        return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+    }
+
+    kda::ForwardArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.s0 = initial_state; a.out = out; a.sT = final_state;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
+    a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
+    cudaError_t e = kda::launch_prefill_simt(a, st);
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           float *state_inout, float *out,
+                           int B, int H, int dk, int dv,
+                           kda_dtype dtype, float scale, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
+    if (!q || !k || !v || !log_alpha || !beta || !state_inout || !out) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
+        !aligned16(state_inout) || !aligned16(out) || !aligned4(beta))
+        return KDA_ERR_MISALIGNED;
+
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.state = state_inout; a.out = out;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
+    a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
+    cudaError_t e = kda::launch_decode(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_check_status(void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_fail(e);
+    return KDA_OK;
+}
+
+}  // extern "C"

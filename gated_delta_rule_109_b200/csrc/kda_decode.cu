@@ -1,0 +1,147 @@
+// Single-token KDA decode step (one token per sequence, state updated in place).
+//
+// "KDA Technical Deep Dive", §Systems and implementation tradeoffs, Decoding:
+// each new token costs one state update plus one query-state product,
+// independent of the context length; the state is updated in place
+// (§How the Kimi gate changes memory).  Step order as in "Kimi Delta
+// Attention: The Linear Attention Behind Kimi K2 and Qwen3", §How Kimi Delta
+// Attention works step by step: decay per key channel, predict, error, write,
+// read after the write.
+//
+// Per head the whole update is one pass over the fp32 state held in
+// registers:
+//     S~ = Diag(alpha) S
+//     p  = S~^T k,  r = S~^T q          (both reductions over key channels)
+//     d  = beta (v - p)
+//     S  = S~ + k d^T                   (written back in place)
+//     o  = scale (r + (k.q) d)          (= scale S^T q after the write)
+// The state (dk*dv*4 bytes read and written per head) is all the traffic that
+// matters, so the kernel is shaped for HBM: 16-byte coalesced loads issued
+// up front, every state element touched once, reductions through shuffles
+// and a small shared-memory table.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kDecodeThreads = 256;
+
+template <int DK, int DV, typename InT>
+__global__ void __launch_bounds__(kDecodeThreads, 2)
+decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
+                   const InT *__restrict__ v, const float *__restrict__ log_alpha,
+                   const float *__restrict__ beta, float *__restrict__ state,
+                   float *__restrict__ out, float scale)
+{
+    constexpr int CG = DV / 4;                 // float4 column groups per state row
+    constexpr int RS = kDecodeThreads / CG;    // row stride between a thread's rows
+    constexpr int RPT = DK / RS;               // state rows held per thread
+    static_assert(RPT * RS == DK && CG * RS == kDecodeThreads, "shape");
+
+    __shared__ float4 red_p[RS][CG];
+    __shared__ float4 red_r[RS][CG];
+    __shared__ float s_kq;
+
+    const int bh = blockIdx.x;                 // b * H + h
+    const int tid = threadIdx.x;
+    const int cg = tid % CG;
+    const int r0 = tid / CG;
+
+    float4 *S = reinterpret_cast<float4 *>(state) + (size_t)bh * DK * CG;
+    float4 s[RPT];
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(&S[(r0 + i * RS) * CG + cg]);
+
+    const InT *qh = q + (size_t)bh * DK;
+    const InT *kh = k + (size_t)bh * DK;
+    const float *lah = log_alpha + (size_t)bh * DK;
+
+    // k.q for the read after the write (warp 0)
+    if (tid < 32) {
+        float acc = 0.f;
+        for (int c = tid; c < DK; c += 32) acc += to_f32(kh[c]) * to_f32(qh[c]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+        if (tid == 0) s_kq = acc;
+    }
+
+    float kr[RPT];
+    float4 pp = make_float4(0.f, 0.f, 0.f, 0.f), rr = pp;
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const int r = r0 + i * RS;
+        const float a = expf(lah[r]);
+        const float kc = to_f32(kh[r]);
+        const float qc = to_f32(qh[r]);
+        kr[i] = kc;
+        s[i].x *= a; s[i].y *= a; s[i].z *= a; s[i].w *= a;
+        pp.x += kc * s[i].x; pp.y += kc * s[i].y; pp.z += kc * s[i].z; pp.w += kc * s[i].w;
+        rr.x += qc * s[i].x; rr.y += qc * s[i].y; rr.z += qc * s[i].z; rr.w += qc * s[i].w;
+    }
+    red_p[r0][cg] = pp;
+    red_r[r0][cg] = rr;
+    __syncthreads();
+
+    float4 p = make_float4(0.f, 0.f, 0.f, 0.f), r = p;
+#pragma unroll
+    for (int j = 0; j < RS; ++j) {
+        const float4 a = red_p[j][cg], b = red_r[j][cg];
+        p.x += a.x; p.y += a.y; p.z += a.z; p.w += a.w;
+        r.x += b.x; r.y += b.y; r.z += b.z; r.w += b.w;
+    }
+    const InT *vh = v + (size_t)bh * DV + 4 * cg;
+    const float bt = beta[bh];
+    float4 d;
+    d.x = bt * (to_f32(vh[0]) - p.x);
+    d.y = bt * (to_f32(vh[1]) - p.y);
+    d.z = bt * (to_f32(vh[2]) - p.z);
+    d.w = bt * (to_f32(vh[3]) - p.w);
+
+#pragma unroll
+    for (int i = 0; i < RPT; ++i) {
+        const float kc = kr[i];
+        s[i].x += kc * d.x; s[i].y += kc * d.y; s[i].z += kc * d.z; s[i].w += kc * d.w;
+        __stcs(&S[(r0 + i * RS) * CG + cg], s[i]);
+    }
+    if (r0 == 0) {
+        const float kq = s_kq;
+        float4 o;
+        o.x = scale * (r.x + kq * d.x);
+        o.y = scale * (r.y + kq * d.y);
+        o.z = scale * (r.z + kq * d.z);
+        o.w = scale * (r.w + kq * d.w);
+        reinterpret_cast<float4 *>(out)[(size_t)bh * CG + cg] = o;
+    }
+}
+
+template <int DK, int DV, typename InT>
+cudaError_t launch_typed(const DecodeArgs &a, cudaStream_t stream)
+{
+    const unsigned grid = (unsigned)((size_t)a.B * a.H);
+    decode_step_kernel<DK, DV, InT><<<grid, kDecodeThreads, 0, stream>>>(
+        static_cast<const InT *>(a.q), static_cast<const InT *>(a.k),
+        static_cast<const InT *>(a.v), a.log_alpha, a.beta, a.state, a.out, a.scale);
+    cudaError_t e2 = cudaGetLastError();
+    if (e2 == cudaSuccess) note_launch();
+    return e2;
+}
+
+template <typename InT>
+cudaError_t launch_dims(const DecodeArgs &a, cudaStream_t stream)
+{
+    if (a.dk == 128 && a.dv == 128) return launch_typed<128, 128, InT>(a, stream);
+    if (a.dk == 64 && a.dv == 64) return launch_typed<64, 64, InT>(a, stream);
+    if (a.dk == 128 && a.dv == 64) return launch_typed<128, 64, InT>(a, stream);
+    if (a.dk == 64 && a.dv == 128) return launch_typed<64, 128, InT>(a, stream);
+    return cudaErrorInvalidValue;
+}
+
+}  // namespace
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream)
+{
+    if (a.dtype == KDA_BF16) return launch_dims<__nv_bfloat16>(a, stream);
+    return launch_dims<float>(a, stream);
+}
+
+}  // namespace kda

@@ -1,0 +1,47 @@
+// Internal declarations shared by libkda's translation units (not installed).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+constexpr int kChunk = 64;   // tokens per chunk of the prefill
+
+struct ForwardArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    const float *s0;          // may be null (zero state)
+    float *out;
+    float *sT;                // may be null
+    int B, T, H, dk, dv;
+    kda_dtype dtype;
+    float scale;
+};
+
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    float *state;
+    float *out;
+    int B, H, dk, dv;
+    kda_dtype dtype;
+    float scale;
+};
+
+// Each launcher enqueues its kernel(s) on `stream` and returns the launch
+// status.  Arguments are already validated by the C-ABI layer.
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t stream);
+
+// Counts one kernel enqueued through the library (see kda_launch_count).
+void note_launch();
+
+// Loads of the two input dtypes as fp32 (bf16 -> fp32 is exact).
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+}  // namespace kda

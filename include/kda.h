@@ -1,0 +1,144 @@
+/*
+ * kda.h -- C ABI of libkda, the B200 (sm_100a) Kimi Delta Attention forward.
+ *
+ * KDA keeps, per head, a fixed-size state S and updates it once per token t:
+ *
+ *     S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = scale * S_t^T q_t
+ *
+ * i.e. decay each key channel of the state by alpha_t, predict the value the
+ * decayed state holds for k_t, write beta_t times the prediction error along
+ * k_t, and read the updated state with the query scaled by 1/sqrt(d_k).
+ * Source: "Kimi Delta Attention: The Linear Attention Behind Kimi K2 and
+ * Qwen3", §How Kimi Delta Attention works step by step (prose, `kda_step`
+ * code and flowchart); "KDA Technical Deep Dive", §From attention to
+ * recurrent state (delta rule) and §How the Kimi gate changes memory (gate).
+ *
+ * Conventions shared by every call
+ * --------------------------------
+ * - All tensor arguments are DEVICE pointers to dense, contiguous, row-major
+ *   arrays on the current CUDA device.  The caller owns and allocates every
+ *   buffer; the library allocates no device memory.
+ * - The state is stored as [dk, dv] per head (key channels are rows, the value
+ *   axis is contiguous).  The pages write the same matrix as (d_v, d_k); this
+ *   is its transpose, so the per-channel decay scales rows.
+ * - The gate is passed as log_alpha = log(alpha), fp32, alpha in (0, 1).
+ *   beta is fp32; any finite value is accepted (the pages use (0, 1)).
+ * - Keys (and queries) are expected L2-normalised by the caller, as the pages
+ *   require for stability; the library does not renormalise.
+ * - `scale` multiplies the query on the read.  Pass 0.0f for the pages'
+ *   default 1/sqrt(dk).  A non-finite scale is KDA_ERR_INVALID_ARG.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *   asynchronous: a KDA_OK return means the work was validated and enqueued.
+ *   Launch failures are reported as KDA_ERR_CUDA; a device-side wait that ran
+ *   out of its iteration limit is reported by kda_check_status().
+ * - Every argument is validated on the host before anything is enqueued; on
+ *   any error status nothing is launched and no output is touched.
+ * - Calls never throw and never abort; they are safe to call from several
+ *   host threads on different streams.
+ * - Outputs are fp32 for both input dtypes (bf16 output would already exceed
+ *   the 2e-3 relative error the bf16 path is held to).
+ */
+#ifndef KDA_H
+#define KDA_H
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum kda_status {
+    KDA_OK = 0,
+    KDA_ERR_INVALID_ARG = 1,   /* null required pointer, bad size, non-finite scale, bad dtype */
+    KDA_ERR_UNSUPPORTED = 2,   /* head dimensions this build has no kernel for */
+    KDA_ERR_MISALIGNED = 3,    /* a tensor pointer is not 16-byte aligned */
+    KDA_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed (see kda_last_cuda_error) */
+    KDA_ERR_TIMEOUT = 5        /* a device-side wait gave up after its iteration limit */
+} kda_status;
+
+typedef enum kda_dtype {
+    KDA_BF16 = 0,              /* q, k, v are bfloat16 */
+    KDA_F32 = 1                /* q, k, v are float32 */
+} kda_dtype;
+
+/*
+ * kda_forward -- chunked prefill over a whole sequence batch.
+ *
+ * Computes o_t for every token and, optionally, the state after the last
+ * token, processing the sequence in chunks of 64 tokens whose boundary state
+ * is the initial condition of the next chunk ("KDA Technical Deep Dive",
+ * §Systems and implementation tradeoffs, Training; the chunkwise mode noted
+ * under §How Kimi Delta Attention works step by step of the other page).
+ *
+ *   q, k          [B, T, H, dk]  dtype            (16-byte aligned)
+ *   v             [B, T, H, dv]  dtype            (16-byte aligned)
+ *   log_alpha     [B, T, H, dk]  float32          (16-byte aligned)
+ *   beta          [B, T, H]      float32          (4-byte aligned)
+ *   initial_state [B, H, dk, dv] float32 or NULL  (NULL = zero state)
+ *   out           [B, T, H, dv]  float32          (16-byte aligned)
+ *   final_state   [B, H, dk, dv] float32 or NULL  (NULL = not written)
+ *
+ * final_state may be the same pointer as initial_state (in-place carry); any
+ * other overlap between inputs and outputs is undefined.  B, H >= 1, T >= 0.
+ * Supported head dimensions: dk, dv in {64, 128} for both dtypes.  T = 0
+ * writes no output and sets final_state to initial_state (or zeros).
+ * q, k, v, log_alpha, beta and out may be NULL only when T = 0.
+ */
+kda_status kda_forward(const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       const float *initial_state, float *out, float *final_state,
+                       int B, int T, int H, int dk, int dv,
+                       kda_dtype dtype, float scale, void *stream);
+
+/*
+ * kda_decode_step -- one token per sequence, state updated in place.
+ *
+ * The per-token update and query-state product of the decode path, whose cost
+ * does not depend on how many tokens came before ("KDA Technical Deep Dive",
+ * §Systems and implementation tradeoffs, Decoding; the state is updated in
+ * place, §How the Kimi gate changes memory).
+ *
+ *   q, k          [B, H, dk]     dtype     (16-byte aligned)
+ *   v             [B, H, dv]     dtype     (16-byte aligned)
+ *   log_alpha     [B, H, dk]     float32   (16-byte aligned)
+ *   beta          [B, H]         float32
+ *   state_inout   [B, H, dk, dv] float32   (16-byte aligned), read and overwritten
+ *   out           [B, H, dv]     float32   (16-byte aligned)
+ *
+ * Equivalent to kda_forward with T = 1 and final_state == initial_state.
+ * Supported head dimensions: dk, dv in {64, 128}.  All pointers are required.
+ */
+kda_status kda_decode_step(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           float *state_inout, float *out,
+                           int B, int H, int dk, int dv,
+                           kda_dtype dtype, float scale, void *stream);
+
+/* Static, human-readable name of a status code (never NULL). */
+const char *kda_status_string(kda_status status);
+
+/*
+ * kda_check_status -- synchronise `stream`, then report (and clear) any
+ * device-side failure the library's kernels recorded on the current device:
+ * KDA_ERR_TIMEOUT if a bounded wait gave up, KDA_ERR_CUDA if the stream
+ * reports an error, else KDA_OK.
+ */
+kda_status kda_check_status(void *stream);
+
+/* Text of the last CUDA error seen by a kda_* call on this host thread
+ * ("" if none).  The pointer stays valid until the next kda_* call on the
+ * same thread. */
+const char *kda_last_cuda_error(void);
+
+/* Number of kernels this process has enqueued through libkda so far (all
+ * devices, all threads).  Meant for accounting: a caller reads it before and
+ * after a region to count the library's launches inside it. */
+unsigned long long kda_launch_count(void);
+
+/* Library ABI version: major * 10000 + minor * 100 + patch. */
+int kda_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KDA_H */
