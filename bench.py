@@ -316,7 +316,7 @@ def oracle_sample(w, x, budget_s, max_tokens=None, chunk_tokens=2048):
     """Time the fp64 oracle on the first tokens of every head until ``budget_s``."""
     import numpy as np
     import oracle
-    T = w.T if max_tokens is None else min(w.T, max_tokens)
+    T = x["q"].shape[1] if max_tokens is None else min(x["q"].shape[1], max_tokens)
     state = None if x["initial_state"] is None else x["initial_state"].cpu().double().numpy()
     done, elapsed = 0, 0.0
     threads = min(os.cpu_count() or 1, w.B * w.H)
@@ -443,6 +443,9 @@ def main(argv=None):
 
     e2e = bench_prefill_e2e(w, args.e2e_steps, 1, device, pre["x"])
     e2e_ms = max_over_ranks(e2e["ms_total"], device)
+    cb = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cb = oracle_sample(w, pre["x"], args.cpu_budget_s)
     del pre["x"]
     torch.cuda.empty_cache()
 
@@ -482,9 +485,7 @@ def main(argv=None):
                     "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"],
                     "steps": dec["e2e_steps"]}}
 
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        xs = I.make_inputs(I.scaled(w, T=min(w.T, 32768)), device)
-        cb = oracle_sample(w, xs, args.cpu_budget_s)
+    if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],
                                 "kind": "oracle",
                                 "sample": "fp64 oracle on the first %d tokens of all %d heads of the %s "

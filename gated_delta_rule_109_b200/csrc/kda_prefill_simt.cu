@@ -54,11 +54,9 @@ struct SimtSmem {
     static constexpr int off_o = off_d + kC * PV;
     static constexpr int off_b = off_o + kC * PV;
     static constexpr int off_gl = off_b + kC;
-    static constexpr int off_gm = off_gl + DK;
-    static constexpr int off_em = off_gm + DK;
-    static constexpr int off_el = off_em + DK;
-    static constexpr int off_red = off_el + DK;           // [8][DVS] reduction table
-    static constexpr int total = off_red + 2 * 8 * kDVS;
+    static constexpr int off_red = off_gl + DK;           // [2][8][DVS] reduction tables
+    static constexpr int off_g64 = (off_red + 2 * 8 * kDVS + 1) & ~1;   // [2][DK] doubles
+    static constexpr int total = off_g64 + 4 * DK;
     static constexpr size_t bytes = sizeof(float) * (size_t)total;
 };
 
@@ -77,8 +75,8 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
     float *sQ = sm + L::off_q, *sK = sm + L::off_k, *sX = sm + L::off_x, *sY = sm + L::off_y;
     float *sV = sm + L::off_v, *sA = sm + L::off_a, *sM = sm + L::off_m, *sS = sm + L::off_s;
     float *sD = sm + L::off_d, *sO = sm + L::off_o, *sB = sm + L::off_b;
-    float *sGl = sm + L::off_gl, *sGm = sm + L::off_gm, *sEm = sm + L::off_em, *sEl = sm + L::off_el;
-    float *sRed = sm + L::off_red;
+    float *sGl = sm + L::off_gl, *sRed = sm + L::off_red;
+    double *sGl64 = reinterpret_cast<double *>(sm + L::off_g64), *sGm64 = sGl64 + DK;
 
     const int tid = threadIdx.x;
     const int slice = blockIdx.x % NS;
@@ -98,61 +96,49 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
         const int c = min(kC, T - t0);
         __syncthreads();   // previous chunk fully consumed
 
-        // ---- stage the chunk (rows past c are zero: they change nothing)
-        for (int idx = tid; idx < kC * DK; idx += kThreads) {
-            const int t = idx / DK, ch = idx % DK;
-            float qq = 0.f, kk = 0.f, la = 0.f;
-            if (t < c) {
-                const size_t g = (((size_t)b * T + t0 + t) * H + h) * DK + ch;
-                qq = to_f32(q[g]); kk = to_f32(k[g]); la = log_alpha[g];
-            }
-            sQ[t * P + ch] = qq; sK[t * P + ch] = kk; sX[t * P + ch] = la;
-        }
+        // ---- stage v and beta (rows past c are zero: they change nothing)
         for (int idx = tid; idx < kC * kDVS; idx += kThreads) {
             const int t = idx / kDVS, x = idx % kDVS;
             sV[t * PV + x] = (t < c) ? to_f32(v[(((size_t)b * T + t0 + t) * H + h) * DV + col0 + x]) : 0.f;
         }
         if (tid < kC) sB[tid] = (tid < c) ? beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
-        __syncthreads();
+        // global index of (token t of this chunk, key channel ch)
+        auto gk = [&](int t, int ch) { return (((size_t)b * T + t0 + t) * H + h) * DK + ch; };
 
-        // ---- per-channel log-decay range: decides the factored or the token path
+        // ---- pass 1, one thread per key channel: the in-chunk log-decay sums in
+        // fp64 (so each exponent argument below carries a single rounding) and
+        // their range, which decides between the factored and the token path
         bool wide = false;
         if (tid < DK) {
-            float run = 0.f, lo = 0.f, hi = 0.f;
-            for (int t = 0; t < kC; ++t) {
-                run += sX[t * P + tid];
-                lo = (t == 0) ? run : fminf(lo, run);
-                hi = (t == 0) ? run : fmaxf(hi, run);
+            double run = 0.0, lo = 0.0, hi = 0.0;
+            for (int t = 0; t < c; ++t) {
+                run += (double)log_alpha[gk(t, tid)];
+                lo = (t == 0) ? run : fmin(lo, run);
+                hi = (t == 0) ? run : fmax(hi, run);
             }
-            wide = !(0.5f * (hi - lo) <= kGMax && fabsf(hi) <= 2.f * kGMax && fabsf(lo) <= 2.f * kGMax);
+            sGl64[tid] = run;
+            sGm64[tid] = 0.5 * (hi + lo);
+            wide = !(0.5 * (hi - lo) <= (double)kGMax && fabs(hi) <= 2.0 * kGMax && fabs(lo) <= 2.0 * kGMax);
         }
         const bool token_path = __syncthreads_or(wide) != 0;
 
         if (!token_path) {
-            // ---- G (in place) and the split exponentials
+            // ---- pass 2: split exponentials around the per-channel midpoint m
             if (tid < DK) {
-                float run = 0.f, lo = 0.f, hi = 0.f;
+                const double m = sGm64[tid];
+                double run = 0.0;
                 for (int t = 0; t < kC; ++t) {
-                    run += sX[t * P + tid];
-                    sX[t * P + tid] = run;
-                    lo = (t == 0) ? run : fminf(lo, run);
-                    hi = (t == 0) ? run : fmaxf(hi, run);
+                    float kk = 0.f, qq = 0.f;
+                    if (t < c) {
+                        run += (double)log_alpha[gk(t, tid)];
+                        kk = to_f32(k[gk(t, tid)]);
+                        qq = to_f32(q[gk(t, tid)]);
+                    }
+                    const float up = expf((float)(run - m)), dn = expf((float)(m - run));
+                    sX[t * P + tid] = kk * up;            // k exp(G - m)
+                    sY[t * P + tid] = kk * dn;            // k exp(m - G)
+                    sQ[t * P + tid] = qq * up;            // q exp(G - m)
                 }
-                const float m = 0.5f * (hi + lo);
-                sGl[tid] = run;
-                sGm[tid] = m;
-                sEm[tid] = expf(m);
-                sEl[tid] = expf(run - m);
-            }
-            __syncthreads();
-            for (int idx = tid; idx < kC * DK; idx += kThreads) {
-                const int t = idx / DK, ch = idx % DK;
-                const float g = sX[t * P + ch], m = sGm[ch];
-                const float kk = sK[t * P + ch];
-                const float up = expf(g - m), dn = expf(m - g);
-                sX[t * P + ch] = kk * up;                 // k exp(G - m)
-                sY[t * P + ch] = kk * dn;                 // k exp(m - G)
-                sQ[t * P + ch] *= up;                     // q exp(G - m)
             }
             __syncthreads();
 
@@ -190,13 +176,24 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
             }
             __syncthreads();
 
-            // ---- right-hand sides: beta*k*exp(G) (into sK), scale*q*exp(G) (sQ),
-            //      k*exp(G_last - G) (sY), beta*v (sV)
-            for (int idx = tid; idx < kC * DK; idx += kThreads) {
-                const int t = idx / DK, ch = idx % DK;
-                sK[t * P + ch] = sB[t] * sX[t * P + ch] * sEm[ch];
-                sQ[t * P + ch] *= scale * sEm[ch];
-                sY[t * P + ch] *= sEl[ch];
+            // ---- pass 3: right-hand sides beta*k*exp(G) (into sK), scale*q*exp(G)
+            //      (sQ), k*exp(G_last - G) (sY), beta*v (sV); Gamma = exp(G_last)
+            if (tid < DK) {
+                const double gl = sGl64[tid];
+                double run = 0.0;
+                for (int t = 0; t < kC; ++t) {
+                    float kk = 0.f, qq = 0.f;
+                    if (t < c) {
+                        run += (double)log_alpha[gk(t, tid)];
+                        kk = to_f32(k[gk(t, tid)]);
+                        qq = to_f32(q[gk(t, tid)]);
+                    }
+                    const float eg = expf((float)run), el = expf((float)(gl - run));
+                    sK[t * P + tid] = sB[t] * kk * eg;
+                    sQ[t * P + tid] = scale * qq * eg;
+                    sY[t * P + tid] = kk * el;
+                }
+                sGl[tid] = (float)exp(gl);
             }
             for (int idx = tid; idx < kC * kDVS; idx += kThreads) {
                 const int t = idx / kDVS, x = idx % kDVS;
@@ -259,7 +256,7 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
                     const int ch = ti * RPT + r;
-                    sacc[r] = expf(sGl[ch]) * sS[ch * PV + x];
+                    sacc[r] = sGl[ch] * sS[ch * PV + x];
                 }
                 for (int j = 0; j < kC; ++j) {
                     const float dj = sD[j * PV + x];
@@ -273,7 +270,14 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
             __syncthreads();
         } else {
             // ---- token-by-token path for a chunk with a very wide decay range.
-            // sX still holds raw log_alpha.  Thread (rg, x): rows rg*RPT..+RPT-1, column x.
+            // Stage raw q, k, log_alpha; thread (rg, x) owns rows rg*RPT..+RPT-1, column x.
+            for (int idx = tid; idx < kC * DK; idx += kThreads) {
+                const int t = idx / DK, ch = idx % DK;
+                float qq = 0.f, kk = 0.f, la = 0.f;
+                if (t < c) { qq = to_f32(q[gk(t, ch)]); kk = to_f32(k[gk(t, ch)]); la = log_alpha[gk(t, ch)]; }
+                sQ[t * P + ch] = qq; sK[t * P + ch] = kk; sX[t * P + ch] = la;
+            }
+            __syncthreads();
             constexpr int RG = kThreads / kDVS;                  // row groups (8)
             constexpr int RPT = DK / RG;
             const int x = tid % kDVS, rg = tid / kDVS;
