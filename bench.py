@@ -65,9 +65,20 @@ def decode_bytes_per_head(dk, dv, in_bytes):
     return 2 * 4 * dk * dv + (2 * dk + dv) * in_bytes + 4 * dk + 4 + 4 * dv
 
 
-# ncu DRAM traffic of the dominant kernel, per launch, keyed by the kernel
-# source it was measured on; reported only while that source is unchanged.
-MEASURED_TRAFFIC = {}
+# ncu DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch,
+# keyed by (kernel source, workload) -> (source digest at capture, bytes).
+# Reported only while the kernel source is unchanged (profiles/ holds the captures).
+MEASURED_TRAFFIC = {
+    ("kda_decode.cu", "decode_bf16_b256_h32_d128_1024steps"): ("a2103952ead4a8e9", 1.0332e9),
+}
+
+
+def measured_traffic(src, workload):
+    ent = MEASURED_TRAFFIC.get((src, workload))
+    if ent is None:
+        return None
+    path = os.path.join(ROOT, "gated_delta_rule_109_b200", "csrc", src)
+    return ent[1] if source_digest(path) == ent[0] else None
 
 
 def source_digest(path):
@@ -377,6 +388,28 @@ def run_reference(args):
     return 0
 
 
+def _add_decode(line, args, rank, world, device, hbm):
+    from gated_delta_rule_109_b200 import inputs as I
+    wd = rank_workload(I.DECODE_B256, rank)
+    dec = bench_decode(wd, args.decode_steps, args.warmup, device, e2e_steps=64)
+    dms = max_over_ranks(dec["ms"], device)
+    d_e2e = max_over_ranks(dec["e2e_ms"], device)
+    dbytes = wd.B * wd.H * decode_bytes_per_head(wd.dk, wd.dv, 2)
+    d_ach = dbytes * args.decode_steps / (dms / 1e3) / 1e9
+    line["decode"] = {
+        "workload": wd.name, "value": wd.B * args.decode_steps * world / (dms / 1e3),
+        "unit": "tokens/s", "steps": args.decode_steps, "ms_per_step": dms / args.decode_steps,
+        "gpu_launches": dec["launches"],
+        "roofline": {"bound": "hbm", "achieved": d_ach, "peak": hbm, "unit": "GB/s",
+                     "frac": d_ach / hbm, "traffic": measured_traffic("kda_decode.cu", wd.name),
+                     "kernel": "decode_step_kernel",
+                     "algorithmic_bytes_per_launch": dbytes,
+                     "vs_8TBs_spec": d_ach / 8000.0},
+        "e2e": {"value": wd.B * dec["e2e_steps"] * world / (d_e2e / 1e3), "unit": "tokens/s",
+                "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"],
+                "steps": dec["e2e_steps"]}}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -391,6 +424,8 @@ def main(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-tokens-per-step", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+                    help="time only one kernel (profiling runs); the default times both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
@@ -415,6 +450,13 @@ def main(argv=None):
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
     in_bytes = 2 if w.dtype == "bf16" else 4
 
+    if args.only == "decode":
+        line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "impl": "kda", "only": "decode"}
+        _add_decode(line, args, rank, world, device, hbm)
+        if rank == 0:
+            print(json.dumps(line), flush=True)
+        return 0
+
     clocks = ClockSampler(device)
     clocks.start()
     pre = bench_prefill(w, args.steps, args.warmup, device)
@@ -429,8 +471,7 @@ def main(argv=None):
                  + (4 * w.B * w.H * w.dk * w.dv if w.final_state else 0)
                  + (4 * w.B * w.H * w.dk * w.dv if w.state_sd is not None else 0))
     achieved = alg_bytes / (ms_launch / 1e3) / 1e9
-    kfile = os.path.join(ROOT, "gated_delta_rule_109_b200", "csrc", "kda_prefill_simt.cu")
-    traffic = MEASURED_TRAFFIC.get(("kda_prefill_simt", w.name, source_digest(kfile)))
+    traffic = measured_traffic("kda_prefill_simt.cu", w.name)
     alg_flops = w.B * w.T * w.H * prefill_flops_per_token_head(w.dk)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,
@@ -466,24 +507,8 @@ def main(argv=None):
             "gpu_launches": pre["launches"],
             "clocks": clk}
 
-    if not args.no_decode:
-        wd = rank_workload(I.DECODE_B256, rank)
-        dec = bench_decode(wd, args.decode_steps, args.warmup, device, e2e_steps=64)
-        dms = max_over_ranks(dec["ms"], device)
-        d_e2e = max_over_ranks(dec["e2e_ms"], device)
-        dbytes = wd.B * wd.H * decode_bytes_per_head(wd.dk, wd.dv, 2)
-        d_ach = dbytes * args.decode_steps / (dms / 1e3) / 1e9
-        line["decode"] = {
-            "workload": wd.name, "value": wd.B * args.decode_steps * world / (dms / 1e3),
-            "unit": "tokens/s", "steps": args.decode_steps, "ms_per_step": dms / args.decode_steps,
-            "gpu_launches": dec["launches"],
-            "roofline": {"bound": "hbm", "achieved": d_ach, "peak": hbm, "unit": "GB/s",
-                         "frac": d_ach / hbm, "traffic": None, "kernel": "decode_step_kernel",
-                         "algorithmic_bytes_per_launch": dbytes,
-                         "vs_8TBs_spec": d_ach / 8000.0},
-            "e2e": {"value": wd.B * dec["e2e_steps"] * world / (d_e2e / 1e3), "unit": "tokens/s",
-                    "h2d_bytes_per_step": dec["h2d"], "d2h_bytes_per_step": dec["d2h"],
-                    "steps": dec["e2e_steps"]}}
+    if not args.no_decode and args.only == "all":
+        _add_decode(line, args, rank, world, device, hbm)
 
     if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],
