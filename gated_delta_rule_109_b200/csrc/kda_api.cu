@@ -86,7 +86,8 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
     a.s0 = initial_state; a.out = out; a.sT = final_state;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
     a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
-    cudaError_t e = kda::launch_prefill_simt(a, st);
+    cudaError_t e = kda::prefill_tc_supported(a) ? kda::launch_prefill_tc(a, st)
+                                                 : kda::launch_prefill_simt(a, st);
     return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
@@ -121,7 +122,10 @@ kda_status kda_check_status(void *stream)
     g_last_cuda_error[0] = '\0';
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
-    return KDA_OK;
+    unsigned int dev_status = 0;
+    e = kda::take_device_status(&dev_status);
+    if (e != cudaSuccess) return cuda_fail(e);
+    return dev_status ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
 }  // extern "C"

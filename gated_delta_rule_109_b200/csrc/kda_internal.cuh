@@ -36,6 +36,12 @@ struct DecodeArgs {
 // status.  Arguments are already validated by the C-ABI layer.
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t stream);
 cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t stream);
+// Tensor-core (tcgen05) prefill: bf16 inputs with dk = dv = 128.
+bool prefill_tc_supported(const ForwardArgs &a);
+cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t stream);
+// Reads and clears the device status word the tensor-core kernels set when a
+// bounded wait gives up (bit 0).  Synchronous.
+cudaError_t take_device_status(unsigned int *status);
 
 // Counts one kernel enqueued through the library (see kda_launch_count).
 void note_launch();
