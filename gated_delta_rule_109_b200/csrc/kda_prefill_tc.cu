@@ -6,37 +6,38 @@
 // the sequence is processed chunkwise with the chunk-boundary state as the
 // next chunk's initial condition ("KDA Technical Deep Dive", §Systems and
 // implementation tradeoffs, Training).  Per (b, h), chunk of c <= 64 tokens,
-// entering state S (dk x dv), G_t = in-chunk inclusive sum of log_alpha,
+// entering state S (dk x dv), G_t = in-chunk inclusive sum of log_alpha and
 // m = per-channel midpoint of G over the chunk:
 //
-//   D_AM = [k e^{G-m} ; q e^{G-m}] (k e^{m-G})^T            (128 x 64)
-//   A    = Diag(beta) strictly_lower(D_AM[0:64])            A_ij = beta_i k_i.(Gam_i/Gam_j) k_j
-//   M    = scale lower(D_AM[64:128])
-//   T    = (I + A)^-1  (blocked 16x16 forward substitution, fp32)
-//   R    = T Diag(beta),   W = R (k e^G),   Qt = scale q e^G,   Kh = k e^{G_last - G}
-//   D1   = [-W ; Qt] S + [R ; M] V          rows 0..63  = Delta = R V - W S
-//   D2   = Kh^T Delta,   D1 += [R ; M] (Delta - V)
-//                                           rows 64..127 = Qt S + M Delta = O
-//   S   <- Diag(e^{G_last}) S + D2
+//   Kr = k e^{G-m},  Qr = scale q e^{G-m},  Kb = k e^{m-G},  S' = Diag(e^m) S
+//   D    = [Kr ; Qr] [Kb | S']                                     (128 x 96, one product)
+//          columns 0..63:  A = Diag(beta) strictly_lower(D[0:64]),  M = lower(D[64:128])
+//          columns 64..95: rows 0..63 = k e^G S (= K~ S),  rows 64..127 = scale q e^G S (= Q~ S)
+//   T    = (I + A)^-1  (blocked forward substitution, fp32),  R = T Diag(beta)
+//   E    = V - K~ S,   Delta = R E       (row t of Delta is the delta-rule error e_t)
+//   O    = Q~ S + M Delta,   with M Delta = M E + M (Delta - E)
+//   S   <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta
 //
-// (the M V that the first [R ; M] V product puts into rows 64..127 is cancelled
-// by M (Delta - V); both stacked operands stay 128 rows tall, the tcgen05 M).
+// A_ij = beta_i k_i.(Gamma_i/Gamma_j) k_j and (I + A)^-1 are the WY/UT
+// quantities of the chunkwise delta rule.  Three tensor-core round trips per
+// chunk: D; [R; M] E; and (Kb^T Delta, [R; M] (Delta - E)).  The stacked [R; M]
+// keeps every product 128 rows tall (the tcgen05 M); its M E half is cancelled
+// by the M (Delta - E) of the last round trip.
 //
 // Precision: the non-input operands need fp32-level accuracy (a single bf16
 // rounding of any of them already exceeds a 2e-3 max-abs/rms bar), so every
 // fp32 operand X is split X = hi + lo with hi = bf16(X), lo = bf16(X - hi) and
-// a product is hi*hi + lo*hi + hi*lo (the lo*lo term is below fp32 rounding);
-// V is an exact bf16 input, so its products take two terms.  All MMAs
-// accumulate in fp32 in tensor memory.
+// a product is hi*hi + lo*hi + hi*lo (lo*lo is below fp32 rounding).
+// Accumulation is fp32 in tensor memory.
 //
-// One CTA (256 threads) owns one (b, h, 32-column value slice): value columns of
-// the state evolve independently.  The state slice lives in registers (thread
-// (lane dk, half) holds 16 columns of row dk) and is re-split into shared memory
-// each chunk as the B operand of the next product.  A chunk whose log-decay
-// range is too wide for the split exponentials takes an exact token-by-token
-// path on CUDA cores instead.  Every mbarrier wait is bounded; a wait that runs
-// out records KDA_ERR_TIMEOUT in a device status word and the CTA exits after
-// freeing its tensor memory.
+// One CTA (256 threads) owns one (b, h, 32-column value slice): value columns
+// of the state evolve independently.  The state slice stays in registers
+// (thread (lane dk, half) holds 16 columns of row dk).  Each chunk's q, k and
+// log_alpha rows are staged in shared memory by cp.async.bulk copies issued
+// one chunk ahead.  A chunk whose log-decay range is too wide for the split
+// exponentials takes an exact token-by-token path on CUDA cores.  Every
+// mbarrier wait is bounded; a wait that runs out records KDA_ERR_TIMEOUT in a
+// device status word and the CTA exits after freeing its tensor memory.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -46,6 +47,7 @@ __device__ unsigned int g_kda_device_status;   // bit 0: a bounded wait gave up
 namespace {
 
 constexpr int kC = 64, kDK = 128, kDV = 128, kDVS = 32, kNSL = kDV / kDVS, kNT = 256;
+constexpr int kNB = 64 + kDVS;                     // N of the first product
 constexpr float kGMaxTc = 40.f;
 constexpr long long kWaitCycles = 4000000000ll;   // ~2 s at 2 GHz
 
@@ -53,41 +55,41 @@ constexpr long long kWaitCycles = 4000000000ll;   // ~2 s at 2 GHz
 // No-swizzle UMMA tiles: core matrices of 8 rows x 16 bytes.  For a tile indexed
 // (outer, inner) the byte offset is core_off(); K-major tiles have outer = M/N,
 // inner = K; MN-major tiles have outer = K, inner = M/N.
-constexpr uint32_t SM_P = 0;             // [k e^{G-m}; q e^{G-m}] then [-W; Qt]: MN-major 128(K) x 128(M)
+constexpr uint32_t SM_P = 0;             // [Kr; Qr]: outer dk, inner row 0..127
 constexpr uint32_t SM_P_LO = 32768;
-constexpr uint32_t SM_Q = 65536;         // k e^{m-G} (MN-major 128 x 64) then Kh^T (K-major 128 x 64)
-constexpr uint32_t SM_Q_LO = SM_Q + 16384;
-constexpr uint32_t SM_RM = 98304;        // [R; M] K-major 128(M) x 64(K)
+constexpr uint32_t SM_B = 65536;         // [Kb | S']: outer dk, inner 0..63 token, 64..95 state column
+constexpr uint32_t SM_B_LO = SM_B + 24576;
+constexpr uint32_t SM_RM = SM_B_LO + 24576;   // [R; M]: outer row 0..127, inner token 0..63
 constexpr uint32_t SM_RM_LO = SM_RM + 16384;
-constexpr uint32_t SM_W = 131072;        // (k e^G)^T K-major 128 x 64, or fp32 A and T of the solve
-constexpr uint32_t SM_W_LO = SM_W + 16384;
-constexpr uint32_t SM_AMAT = SM_W;                 // fp32 [64][65]
-constexpr uint32_t SM_TMAT = SM_W + 64 * 65 * 4;   // fp32 [64][65]
-constexpr uint32_t SM_S = SM_W + 33792;  // state slice, MN-major 128(K) x 32(N)
-constexpr uint32_t SM_S_LO = SM_S + 8192;
-constexpr uint32_t SM_V = SM_S + 16384;  // value slice, MN-major 64(K) x 32(N), exact bf16
-constexpr uint32_t SM_D = SM_V + 4096;   // Delta, MN-major 64 x 32
-constexpr uint32_t SM_D_LO = SM_D + 4096;
-constexpr uint32_t SM_E = SM_D_LO + 4096;  // Delta - V
+constexpr uint32_t SM_STG = SM_RM_LO + 16384; // staged chunk rows: q bf16 [64][128], k bf16, log_alpha fp32
+constexpr uint32_t SM_STG_K = SM_STG + 16384;
+constexpr uint32_t SM_STG_A = SM_STG + 32768;
+constexpr uint32_t SM_E = SM_STG + 65536;     // E, then Delta - E: outer token, inner column 0..31
 constexpr uint32_t SM_E_LO = SM_E + 4096;
-constexpr uint32_t SM_BETA = SM_E_LO + 4096;   // fp32 [64]
-constexpr uint32_t SM_GAMMA = SM_BETA + 256;    // fp32 [128]
-constexpr uint32_t SM_G64 = SM_GAMMA + 512;     // fp64 [2][128]: G_last, midpoint
-constexpr uint32_t SM_MBAR = SM_G64 + 2048;     // mbarrier (8 B)
-constexpr uint32_t SM_TMEMP = SM_MBAR + 8;      // tensor-memory base address (4 B)
-constexpr uint32_t SM_TOTAL = SM_TMEMP + 8;
-static_assert(SM_TOTAL <= 227 * 1024, "shared memory");
-// token path (wide chunks) reuses [0, SM_W) for fp32 q, k, log_alpha [64][129]
-// and the SM_W region for the fp32 state [128][33], v [64][33] and two [8][32] tables.
-constexpr int kTP = kDK + 1;
+constexpr uint32_t SM_D = SM_E_LO + 4096;     // Delta
+constexpr uint32_t SM_D_LO = SM_D + 4096;
+constexpr uint32_t SM_BETA = SM_D_LO + 4096;  // fp32 [64]
+constexpr uint32_t SM_EM = SM_BETA + 256;     // fp32 [128] e^{m}
+constexpr uint32_t SM_GAM = SM_EM + 512;      // fp32 [128] e^{G_last}
+constexpr uint32_t SM_EL = SM_GAM + 512;      // fp32 [128] e^{G_last - m}
+constexpr uint32_t SM_MBAR = SM_EL + 512;     // two mbarriers: MMA completion, staged loads
+constexpr uint32_t SM_TMEMP = SM_MBAR + 16;   // tensor-memory base address
+constexpr uint32_t SM_TOTAL = SM_TMEMP + 16;
+static_assert(SM_TOTAL <= 232448, "shared memory");
+// After the first product the [Kr; Qr] region is free: it holds the solve's fp32
+// A and T ([64][68] each, 16-byte aligned rows) and the token path's scratch.
+// The pass-1 exchange (fp32 [3][2][128]) uses the [R; M] region, free until then.
+constexpr int kPitch = 68;
+constexpr uint32_t SM_AMAT = SM_P, SM_TMAT = SM_P + 64 * kPitch * 4;
 
 // tile strides (bytes): s_outer, s_inner
-constexpr uint32_t P_SO = 2048, P_SI = 128;     // 128 x 128
-constexpr uint32_t H_SO = 1024, H_SI = 128;     // 128 x 64  (Q, RM, W tiles)
-constexpr uint32_t S_SO = 512, S_SI = 128;      // 128 x 32 / 64 x 32
+constexpr uint32_t P_SO = 2048, P_SI = 128;
+constexpr uint32_t B_SO = (kNB / 8) * 128, B_SI = 128;
+constexpr uint32_t H_SO = 1024, H_SI = 128;
+constexpr uint32_t S_SO = 512, S_SI = 128;
 
 // tensor-memory columns
-constexpr uint32_t TM_AM = 0, TM_W = 64, TM_D1 = 128, TM_D2 = 160, TM_COLS = 256;
+constexpr uint32_t TM_D = 0, TM_D3 = 96, TM_D2 = 128, TM_COLS = 256;
 
 __device__ __forceinline__ uint32_t core_off(int outer, int inner, uint32_t so, uint32_t si)
 {
@@ -126,35 +128,35 @@ __device__ __forceinline__ void umma_commit(uint32_t mbar)
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
 {
     uint32_t r[16];
     asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
-                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
                  : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
                    "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
                    "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr));
-    tmem_wait_ld();
+                 : "r"(taddr) : "memory");
 #pragma unroll
     for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
-
-__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float (&v)[32])
-{
-    float a[16], b[16];
-    tmem_ld16(taddr, a);
-    tmem_ld16(taddr + 16, b);
-#pragma unroll
-    for (int i = 0; i < 16; ++i) { v[i] = a[i]; v[16 + i] = b[i]; }
 }
 
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(mbar), "r"(count) : "memory");
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(mbar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
 }
 
 // Bounded wait for the phase with the given parity; false if it never completed.
@@ -195,7 +197,7 @@ __device__ __forceinline__ void st_split8(uint8_t *smem, uint32_t off_hi, uint32
 }
 
 // One product D (+)= A B on split operands.  Terms hi*hi, lo*hi, hi*lo (the last
-// only when B has a lo part).  Each term walks K in steps of 16.
+// only when B has a lo part).  Each term walks K in steps of 16 (2 core matrices).
 __device__ __forceinline__ void mma_split(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t a_lbo,
                                           uint32_t a_sbo, uint32_t b_hi, uint32_t b_lo, uint32_t b_lbo,
                                           uint32_t b_sbo, int ksteps, uint32_t idesc, bool accumulate)
@@ -212,6 +214,7 @@ __device__ __forceinline__ void mma_split(uint32_t d, uint32_t a_hi, uint32_t a_
     }
 }
 
+
 // ---------------------------------------------------------------- the kernel
 __global__ void __launch_bounds__(kNT, 1)
 prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -222,10 +225,13 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
     float *sBeta = reinterpret_cast<float *>(smem + SM_BETA);
-    float *sGamma = reinterpret_cast<float *>(smem + SM_GAMMA);
-    double *sGl = reinterpret_cast<double *>(smem + SM_G64);
-    double *sGm = sGl + kDK;
-    const uint32_t mbar = sbase + SM_MBAR;
+    float *sEm = reinterpret_cast<float *>(smem + SM_EM);
+    float *sGam = reinterpret_cast<float *>(smem + SM_GAM);
+    float *sEl = reinterpret_cast<float *>(smem + SM_EL);
+    const __nv_bfloat16 *stq = reinterpret_cast<const __nv_bfloat16 *>(smem + SM_STG);
+    const __nv_bfloat16 *stk = reinterpret_cast<const __nv_bfloat16 *>(smem + SM_STG_K);
+    const float *sta = reinterpret_cast<const float *>(smem + SM_STG_A);
+    const uint32_t mbar = sbase + SM_MBAR, mbar_ld = sbase + SM_MBAR + 8;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x % kNSL;
@@ -234,129 +240,200 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
     const int col0 = slice * kDVS;
     const int lrow = 32 * (warp & 3) + lane;     // tensor-memory lane this thread reads
     const int half = warp >> 2;                  // which half of the columns it reads
+    const int ch = tid & (kDK - 1);              // key channel of the per-channel passes
+    const int th = tid >> 7;                     // token half (0: 0..31, 1: 32..63) of those passes
+    const int nchunks = (T + kC - 1) / kC;
+    bool ld_pending = false;                     // a staged copy is armed and not yet waited for
 
-    // ---- tensor memory and the MMA barrier
+    auto row_q = [&](int chunk, int t) { return (((size_t)b * T + (size_t)chunk * kC + t) * H + h); };
+
+    // ---- stage chunk `chunk`'s q, k, log_alpha rows (thread 0 arms the barrier)
+    auto issue_stage = [&](int chunk) {
+        const int cc = min(kC, T - chunk * kC);
+        ld_pending = true;
+        if (tid == 0) mbar_expect_tx(mbar_ld, (uint32_t)cc * 1024u);
+        __syncthreads();
+        if (tid < 3 * cc) {
+            const int which = tid / cc, t = tid % cc;
+            const size_t r = row_q(chunk, t);
+            if (which == 0) bulk_g2s(sbase + SM_STG + t * 256, q + r * kDK, 256, mbar_ld);
+            else if (which == 1) bulk_g2s(sbase + SM_STG_K + t * 256, k + r * kDK, 256, mbar_ld);
+            else bulk_g2s(sbase + SM_STG_A + t * 512, log_alpha + r * kDK, 512, mbar_ld);
+        }
+    };
+    // value slice (threads of rows 0..63: 16 columns each) and beta go through registers
+    auto load_vb = [&](int chunk, uint4 (&vr)[2], float &br) {
+        const int cc = min(kC, T - chunk * kC);
+        vr[0] = vr[1] = make_uint4(0u, 0u, 0u, 0u);
+        if (lrow < cc) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(v + row_q(chunk, lrow) * kDV + col0 + 16 * half);
+            vr[0] = src[0];
+            vr[1] = src[1];
+        }
+        br = (tid < cc) ? beta[row_q(chunk, tid)] : 0.f;
+    };
+
+    // ---- tensor memory and barriers
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      :: "r"(sbase + SM_TMEMP), "r"(TM_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
-    if (tid == 0) mbar_init(mbar, 1);
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_init(mbar_ld, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + SM_TMEMP);
     const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
-    uint32_t phase = 0;
+    uint32_t phase = 0, ld_phase = 0;
     bool failed = false;
 
     // ---- state slice: thread holds row lrow, columns 16*half .. +15
     float S[16];
-    {
-        const int n0 = 16 * half;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-            S[j] = s0 ? s0[((size_t)bh * kDK + lrow) * kDV + col0 + n0 + j] : 0.f;
-    }
-    auto write_state_tile = [&]() {
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            float x[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = S[8 * g + e];
-            const uint32_t off = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
-            st_split8(smem, SM_S + off, SM_S_LO + off, x);
-        }
-    };
-    write_state_tile();
+    for (int j = 0; j < 16; ++j)
+        S[j] = s0 ? s0[((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half + j] : 0.f;
 
-    const int nchunks = (T + kC - 1) / kC;
+    uint4 vreg[2];
+    float breg;
+    if (nchunks > 0) {
+        issue_stage(0);
+        load_vb(0, vreg, breg);
+    }
+
     for (int n = 0; n < nchunks && !failed; ++n) {
         const int t0 = n * kC;
         const int c = min(kC, T - t0);
-        auto gk = [&](int t, int ch) { return (((size_t)b * T + t0 + t) * H + h) * kDK + ch; };
-        auto gv = [&](int t) { return (((size_t)b * T + t0 + t) * H + h) * kDV + col0; };
+        auto gv = [&](int t) { return row_q(n, t) * kDV + col0; };
 
-        // ---- stage beta and the value slice (exact bf16, MN-major 64 x 32)
-        if (tid < kC) sBeta[tid] = (tid < c) ? beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
+        // ---- the staged rows of this chunk and beta
+        failed = __syncthreads_or(!mbar_wait(mbar_ld, ld_phase)) != 0;
+        if (failed) break;
+        ld_phase ^= 1;
+        ld_pending = false;
+        if (tid < kC) sBeta[tid] = breg;
+
+        // ---- pass 1 (two threads per key channel, fp32): log-decay sums and range
+        float *xch = reinterpret_cast<float *>(smem + SM_RM);   // [3][2][128]
         {
-            const int t = tid >> 2, g = tid & 3;
-            uint4 val = make_uint4(0u, 0u, 0u, 0u);
-            if (t < c) val = *reinterpret_cast<const uint4 *>(v + gv(t) + 8 * g);
-            *reinterpret_cast<uint4 *>(smem + SM_V + core_off(t, 8 * g, S_SO, S_SI)) = val;
-        }
-
-        // ---- pass 1 (thread per key channel): fp64 log-decay sums, range, path choice
-        bool wide = false;
-        if (tid < kDK) {
-            double run = 0.0, lo = 0.0, hi = 0.0;
-            for (int t = 0; t < c; ++t) {
-                run += (double)log_alpha[gk(t, tid)];
-                lo = (t == 0) ? run : fmin(lo, run);
-                hi = (t == 0) ? run : fmax(hi, run);
+            float run = 0.f, lo = INFINITY, hi = -INFINITY;
+            for (int i = 0; i < 32; ++i) {
+                const int t = 32 * th + i;
+                if (t < c) {
+                    run += sta[t * kDK + ch];
+                    lo = fminf(lo, run);
+                    hi = fmaxf(hi, run);
+                }
             }
-            sGl[tid] = run;
-            sGm[tid] = 0.5 * (hi + lo);
-            wide = !(0.5 * (hi - lo) <= (double)kGMaxTc && fabs(hi) <= 2.0 * kGMaxTc &&
-                     fabs(lo) <= 2.0 * kGMaxTc);
+            xch[th * kDK + ch] = run;
+            xch[256 + th * kDK + ch] = lo;
+            xch[512 + th * kDK + ch] = hi;
+        }
+        __syncthreads();
+        float g_start, g_mid;
+        bool wide;
+        {
+            const float tot0 = xch[ch], tot1 = xch[kDK + ch];
+            const float lo = fminf(xch[256 + ch], tot0 + xch[256 + kDK + ch]);
+            const float hi = fmaxf(xch[512 + ch], tot0 + xch[512 + kDK + ch]);
+            const float gl = tot0 + tot1;
+            g_mid = 0.5f * (lo + hi);
+            g_start = th ? tot0 : 0.f;
+            wide = !(0.5f * (hi - lo) <= kGMaxTc && fabsf(hi) <= 2.f * kGMaxTc && fabsf(lo) <= 2.f * kGMaxTc);
+            if (th == 0) {
+                sEm[ch] = __expf(g_mid);
+                sGam[ch] = __expf(gl);
+                sEl[ch] = __expf(gl - g_mid);
+            }
         }
         const bool token_path = __syncthreads_or(wide) != 0;
 
         if (!token_path) {
-            // ---- pass 2: [k e^{G-m}; q e^{G-m}] (SM_P) and k e^{m-G} (SM_Q), hi/lo
-            if (tid < kDK) {
-                const int ch = tid;
-                const double m = sGm[ch];
-                double run = 0.0;
-                for (int g = 0; g < 8; ++g) {
+            // ---- pass 2: Kr, Qr (rows t and 64+t of SM_P), Kb and S' (SM_B)
+            {
+                float run = g_start;
+#pragma unroll 1
+                for (int g = 0; g < 4; ++g) {
                     float kr[8], qr[8], kb[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
-                        const int t = 8 * g + e;
+                        const int t = 32 * th + 8 * g + e;
                         float kk = 0.f, qq = 0.f;
                         if (t < c) {
-                            run += (double)log_alpha[gk(t, ch)];
-                            kk = __bfloat162float(k[gk(t, ch)]);
-                            qq = __bfloat162float(q[gk(t, ch)]);
+                            run += sta[t * kDK + ch];
+                            kk = __bfloat162float(stk[t * kDK + ch]);
+                            qq = __bfloat162float(stq[t * kDK + ch]);
                         }
-                        const float x = (float)(run - m);
+                        const float x = run - g_mid;
                         const float up = __expf(x), dn = __expf(-x);
-                        kr[e] = kk * up; qr[e] = qq * up; kb[e] = kk * dn;
+                        kr[e] = kk * up; qr[e] = scale * qq * up; kb[e] = kk * dn;
                     }
-                    const uint32_t o1 = core_off(ch, 8 * g, P_SO, P_SI);
-                    const uint32_t o2 = core_off(ch, 64 + 8 * g, P_SO, P_SI);
-                    const uint32_t o3 = core_off(ch, 8 * g, H_SO, H_SI);
+                    const int t8 = 32 * th + 8 * g;
+                    const uint32_t o1 = core_off(ch, t8, P_SO, P_SI);
+                    const uint32_t o2 = core_off(ch, 64 + t8, P_SO, P_SI);
+                    const uint32_t o3 = core_off(ch, t8, B_SO, B_SI);
                     st_split8(smem, SM_P + o1, SM_P_LO + o1, kr);
                     st_split8(smem, SM_P + o2, SM_P_LO + o2, qr);
-                    st_split8(smem, SM_Q + o3, SM_Q_LO + o3, kb);
+                    st_split8(smem, SM_B + o3, SM_B_LO + o3, kb);
+                }
+                const float em = sEm[lrow];
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    float x[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) x[e] = em * S[8 * g + e];
+                    const uint32_t off = core_off(lrow, 64 + 16 * half + 8 * g, B_SO, B_SI);
+                    st_split8(smem, SM_B + off, SM_B_LO + off, x);
                 }
             }
             proxy_fence();
             __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
-                mma_split(tmem + TM_AM, sbase + SM_P, sbase + SM_P_LO, P_SO, P_SI,
-                          sbase + SM_Q, sbase + SM_Q_LO, H_SO, H_SI, kDK / 16,
-                          idesc_bf16(128, 64, 1, 1), false);
+                // D = [Kr; Qr] [Kb | S']
+                mma_split(tmem + TM_D, sbase + SM_P, sbase + SM_P_LO, P_SO, P_SI,
+                          sbase + SM_B, sbase + SM_B_LO, B_SO, B_SI, kDK / 16,
+                          idesc_bf16(128, kNB, 1, 1), false);
                 umma_commit(mbar);
             }
+            // the staging area is free: prefetch the next chunk's rows
+            if (n + 1 < nchunks) issue_stage(n + 1);
             failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
             phase ^= 1;
             if (failed) break;
             tc_fence_after();
 
-            // ---- A (fp32, rows 0..63) to the solve; M (rows 64..127) into [R; M]
+            // ---- A (fp32) and E = V - K~S (rows 0..63); M into [R; M] (rows 64..127)
+            float e_reg[16];
             {
                 float x[32];
-                tmem_ld32(tmem + tlane + TM_AM + 32 * half, x);
+                tmem_ld16(tmem + tlane + TM_D + 32 * half, *reinterpret_cast<float (*)[16]>(x));
+                tmem_ld16(tmem + tlane + TM_D + 32 * half + 16, *reinterpret_cast<float (*)[16]>(x + 16));
                 if (lrow < 64) {
                     const int i = lrow;
-                    float *Am = reinterpret_cast<float *>(smem + SM_AMAT) + i * 65;
+                    float *Am = reinterpret_cast<float *>(smem + SM_AMAT) + i * kPitch;
                     const float bi = sBeta[i];
 #pragma unroll
                     for (int e = 0; e < 32; ++e) {
                         const int j = 32 * half + e;
                         Am[j] = (j < i) ? bi * x[e] : 0.f;
+                    }
+                    float ks[16];
+                    tmem_ld16(tmem + tlane + TM_D + 64 + 16 * half, ks);
+                    const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(vreg);
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) e_reg[e] = __bfloat162float(vb[e]) - ks[e];
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = e_reg[8 * g + e];
+                        const uint32_t o = core_off(i, 16 * half + 8 * g, S_SO, S_SI);
+                        st_split8(smem, SM_E + o, SM_E_LO + o, y);
                     }
                 } else {
                     const int i = lrow - 64;
@@ -366,7 +443,7 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
 #pragma unroll
                         for (int e = 0; e < 8; ++e) {
                             const int j = 32 * half + 8 * g + e;
-                            y[e] = (j <= i) ? scale * x[8 * g + e] : 0.f;
+                            y[e] = (j <= i) ? x[8 * g + e] : 0.f;
                         }
                         const uint32_t o = core_off(lrow, 32 * half + 8 * g, H_SO, H_SI);
                         st_split8(smem, SM_RM + o, SM_RM_LO + o, y);
@@ -375,135 +452,110 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             }
             __syncthreads();
 
-            // ---- T = (I + A)^-1, blocked 16 x 16, fp32
+            // ---- T = (I + A)^-1 by recursive doubling 16 -> 32 -> 64, fp32
             {
-                const float *Am = reinterpret_cast<const float *>(smem + SM_AMAT);
+                float *Am = reinterpret_cast<float *>(smem + SM_AMAT);
                 float *Tm = reinterpret_cast<float *>(smem + SM_TMAT);
                 if (tid < 64) {
-                    // diagonal blocks by forward substitution, one column per thread
+                    // 16 x 16 diagonal blocks by forward substitution, one column per thread
+                    // (x_l = 0 for l < j, so every term can be summed unconditionally and
+                    // the A loads hoisted ahead of the dependent chain)
                     const int blk = tid >> 4, j = tid & 15, o = 16 * blk;
                     float x[16];
 #pragma unroll
                     for (int i = 0; i < 16; ++i) {
                         float s = (i == j) ? 1.f : 0.f;
-                        if (i > j) {
 #pragma unroll
-                            for (int l = 0; l < i; ++l)
-                                if (l >= j) s -= Am[(o + i) * 65 + o + l] * x[l];
-                        }
+                        for (int l = 0; l < i; ++l) s -= Am[(o + i) * kPitch + o + l] * x[l];
                         x[i] = s;
                     }
 #pragma unroll
-                    for (int i = 0; i < 16; ++i) Tm[(o + i) * 65 + o + j] = x[i];
+                    for (int i = 0; i < 16; ++i) Tm[(o + i) * kPitch + o + j] = x[i];
+                } else {
+                    // the six strictly-upper 16 x 16 blocks of T are zero
+                    for (int e = tid - 64; e < 6 * 256; e += kNT - 64) {
+                        const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
+                        const int rb = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
+                        const int cb = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                        Tm[(16 * rb + i) * kPitch + 16 * cb + j] = 0.f;
+                    }
                 }
                 __syncthreads();
-                for (int dd = 1; dd < 4; ++dd) {
-                    // Y_ab = sum_{c=b}^{a-1} A_ac T_cb, kept in the unused upper block (b, a)
-                    for (int e = tid; e < (4 - dd) * 256; e += kNT) {
-                        const int a = dd + e / 256, bb = a - dd;
-                        const int i = (e & 255) >> 4, j = e & 15;
-                        float s = 0.f;
-                        for (int cb = bb; cb < a; ++cb)
+                // 16 -> 32: T_ab = -T_aa (A_ab T_bb) for (a, b) = (1, 0), (3, 2)
+                const int p = tid >> 6, i16 = (tid >> 2) & 15, jq = tid & 3;
+                if (tid < 128) {
+                    const int a = 2 * p + 1, bb = 2 * p;
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-                            for (int l = 0; l < 16; ++l)
-                                s += Am[(16 * a + i) * 65 + 16 * cb + l] * Tm[(16 * cb + l) * 65 + 16 * bb + j];
-                        Tm[(16 * bb + i) * 65 + 16 * a + j] = s;
+                    for (int l = 0; l < 16; ++l) {
+                        const float av = Am[(16 * a + i16) * kPitch + 16 * bb + l];
+                        const float4 tv = *reinterpret_cast<const float4 *>(Tm + (16 * bb + l) * kPitch + 16 * bb + 4 * jq);
+                        y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
                     }
-                    __syncthreads();
-                    // T_ab = -T_aa Y_ab
-                    for (int e = tid; e < (4 - dd) * 256; e += kNT) {
-                        const int a = dd + e / 256, bb = a - dd;
-                        const int i = (e & 255) >> 4, j = e & 15;
-                        float s = 0.f;
-#pragma unroll
-                        for (int l = 0; l < 16; ++l)
-                            if (l <= i) s += Tm[(16 * a + i) * 65 + 16 * a + l] * Tm[(16 * bb + l) * 65 + 16 * a + j];
-                        Tm[(16 * a + i) * 65 + 16 * bb + j] = -s;
-                    }
-                    __syncthreads();
+                    *reinterpret_cast<float4 *>(Am + (16 * bb + i16) * kPitch + 16 * a + 4 * jq) = y;
                 }
+                __syncthreads();
+                if (tid < 128) {
+                    const int a = 2 * p + 1, bb = 2 * p;
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+                    for (int l = 0; l < 16; ++l) {
+                        const float tv = Tm[(16 * a + i16) * kPitch + 16 * a + l];
+                        const float4 yv = *reinterpret_cast<const float4 *>(Am + (16 * bb + l) * kPitch + 16 * a + 4 * jq);
+                        y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
+                    }
+                    *reinterpret_cast<float4 *>(Tm + (16 * a + i16) * kPitch + 16 * bb + 4 * jq) =
+                        make_float4(-y.x, -y.y, -y.z, -y.w);
+                }
+                __syncthreads();
+                // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (A[32:64, 0:32] T[0:32, 0:32])
+                const int i32 = tid >> 3, jq8 = tid & 7;
+                {
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+                    for (int l = 0; l < 32; ++l) {
+                        const float av = Am[(32 + i32) * kPitch + l];
+                        const float4 tv = *reinterpret_cast<const float4 *>(Tm + l * kPitch + 4 * jq8);
+                        y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
+                    }
+                    *reinterpret_cast<float4 *>(Am + i32 * kPitch + 32 + 4 * jq8) = y;
+                }
+                __syncthreads();
+                {
+                    float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+                    for (int l = 0; l < 32; ++l) {
+                        const float tv = Tm[(32 + i32) * kPitch + 32 + l];
+                        const float4 yv = *reinterpret_cast<const float4 *>(Am + l * kPitch + 32 + 4 * jq8);
+                        y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
+                    }
+                    *reinterpret_cast<float4 *>(Tm + (32 + i32) * kPitch + 4 * jq8) =
+                        make_float4(-y.x, -y.y, -y.z, -y.w);
+                }
+                __syncthreads();
                 // R = T Diag(beta) into rows 0..63 of [R; M]
                 for (int id = tid; id < 512; id += kNT) {
                     const int i = id >> 3, jg = id & 7;
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int j = 8 * jg + e;
-                        y[e] = (j <= i) ? Tm[i * 65 + j] * sBeta[j] : 0.f;
-                    }
+                    const float4 t0v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg);
+                    const float4 t1v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg + 4);
+                    const float *bj = sBeta + 8 * jg;
+                    float y[8] = {t0v.x * bj[0], t0v.y * bj[1], t0v.z * bj[2], t0v.w * bj[3],
+                                  t1v.x * bj[4], t1v.y * bj[5], t1v.z * bj[6], t1v.w * bj[7]};
                     const uint32_t o = core_off(i, 8 * jg, H_SO, H_SI);
                     st_split8(smem, SM_RM + o, SM_RM_LO + o, y);
                 }
             }
-            __syncthreads();
-
-            // ---- pass 3: (k e^G)^T (SM_W), scale q e^G (SM_P rows 64..), Kh^T (SM_Q), Gamma
-            if (tid < kDK) {
-                const int ch = tid;
-                const double gl = sGl[ch];
-                double run = 0.0;
-                for (int g = 0; g < 8; ++g) {
-                    float kt[8], qt[8], kh[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) {
-                        const int t = 8 * g + e;
-                        float kk = 0.f, qq = 0.f;
-                        if (t < c) {
-                            run += (double)log_alpha[gk(t, ch)];
-                            kk = __bfloat162float(k[gk(t, ch)]);
-                            qq = __bfloat162float(q[gk(t, ch)]);
-                        }
-                        const float eg = __expf((float)run), el = __expf((float)(gl - run));
-                        kt[e] = kk * eg; qt[e] = scale * qq * eg; kh[e] = kk * el;
-                    }
-                    const uint32_t ow = core_off(ch, 8 * g, H_SO, H_SI);
-                    const uint32_t oq = core_off(ch, 64 + 8 * g, P_SO, P_SI);
-                    st_split8(smem, SM_W + ow, SM_W_LO + ow, kt);
-                    st_split8(smem, SM_P + oq, SM_P_LO + oq, qt);
-                    st_split8(smem, SM_Q + ow, SM_Q_LO + ow, kh);
-                }
-                sGamma[ch] = (float)exp(gl);
-            }
-            proxy_fence();
-            __syncthreads();
-            if (tid == 0) {
-                tc_fence_after();
-                // W^T = (k e^G)^T R^T  -> TM_W (rows dk, columns token)
-                mma_split(tmem + TM_W, sbase + SM_W, sbase + SM_W_LO, H_SI, H_SO,
-                          sbase + SM_RM, sbase + SM_RM_LO, H_SI, H_SO, kC / 16,
-                          idesc_bf16(128, 64, 0, 0), false);
-                umma_commit(mbar);
-            }
-            failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
-            phase ^= 1;
-            if (failed) break;
-            tc_fence_after();
-
-            // ---- -W into rows 0..63 of SM_P (MN-major: outer dk, inner token)
-            {
-                float x[32];
-                tmem_ld32(tmem + tlane + TM_W + 32 * half, x);
-#pragma unroll
-                for (int g = 0; g < 4; ++g) {
-                    float y[8];
-#pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = -x[8 * g + e];
-                    const uint32_t o = core_off(lrow, 32 * half + 8 * g, P_SO, P_SI);
-                    st_split8(smem, SM_P + o, SM_P_LO + o, y);
-                }
-            }
+            // the value slice and beta of the next chunk (this chunk's are consumed)
+            if (n + 1 < nchunks) load_vb(n + 1, vreg, breg);
             proxy_fence();
             tc_fence_before();
             __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
-                // D1 = [-W; Qt] S + [R; M] V
-                mma_split(tmem + TM_D1, sbase + SM_P, sbase + SM_P_LO, P_SO, P_SI,
-                          sbase + SM_S, sbase + SM_S_LO, S_SO, S_SI, kDK / 16,
-                          idesc_bf16(128, kDVS, 1, 1), false);
-                mma_split(tmem + TM_D1, sbase + SM_RM, sbase + SM_RM_LO, H_SI, H_SO,
-                          sbase + SM_V, 0u, S_SO, S_SI, kC / 16,
-                          idesc_bf16(128, kDVS, 0, 1), true);
+                // D3 = [R; M] E
+                mma_split(tmem + TM_D3, sbase + SM_RM, sbase + SM_RM_LO, H_SI, H_SO,
+                          sbase + SM_E, sbase + SM_E_LO, S_SO, S_SI, kC / 16,
+                          idesc_bf16(128, kDVS, 0, 1), false);
                 umma_commit(mbar);
             }
             failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
@@ -511,24 +563,21 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             if (failed) break;
             tc_fence_after();
 
-            // ---- Delta (rows 0..63 of D1) and Delta - V as split B operands
+            // ---- Delta = rows 0..63 of D3, and Delta - E, as B operands
             if (lrow < 64) {
                 float x[16];
-                tmem_ld16(tmem + tlane + TM_D1 + 16 * half, x);
-                const int t = lrow;
+                tmem_ld16(tmem + tlane + TM_D3 + 16 * half, x);
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
-                    const uint32_t o = core_off(t, 16 * half + 8 * g, S_SO, S_SI);
-                    const uint4 vv = *reinterpret_cast<const uint4 *>(smem + SM_V + o);
-                    const __nv_bfloat16 *vb = reinterpret_cast<const __nv_bfloat16 *>(&vv);
-                    float d[8], ev[8];
+                    float d[8], de[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         d[e] = x[8 * g + e];
-                        ev[e] = d[e] - __bfloat162float(vb[e]);
+                        de[e] = d[e] - e_reg[8 * g + e];
                     }
+                    const uint32_t o = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
                     st_split8(smem, SM_D + o, SM_D_LO + o, d);
-                    st_split8(smem, SM_E + o, SM_E_LO + o, ev);
+                    st_split8(smem, SM_E + o, SM_E_LO + o, de);
                 }
             }
             proxy_fence();
@@ -536,11 +585,11 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             __syncthreads();
             if (tid == 0) {
                 tc_fence_after();
-                // D2 = Kh^T Delta;  D1 += [R; M] (Delta - V)
-                mma_split(tmem + TM_D2, sbase + SM_Q, sbase + SM_Q_LO, H_SI, H_SO,
+                // D2 = Kb^T Delta (Kb read K-major from SM_B);  D3 += [R; M] (Delta - E)
+                mma_split(tmem + TM_D2, sbase + SM_B, sbase + SM_B_LO, B_SI, B_SO,
                           sbase + SM_D, sbase + SM_D_LO, S_SO, S_SI, kC / 16,
                           idesc_bf16(128, kDVS, 0, 1), false);
-                mma_split(tmem + TM_D1, sbase + SM_RM, sbase + SM_RM_LO, H_SI, H_SO,
+                mma_split(tmem + TM_D3, sbase + SM_RM, sbase + SM_RM_LO, H_SI, H_SO,
                           sbase + SM_E, sbase + SM_E_LO, S_SO, S_SI, kC / 16,
                           idesc_bf16(128, kDVS, 0, 1), true);
                 umma_commit(mbar);
@@ -550,51 +599,32 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             if (failed) break;
             tc_fence_after();
 
-            // ---- state update and outputs
+            // ---- state update and outputs (O = Q~S + M Delta, rows 64..127)
             {
                 float x[16];
                 tmem_ld16(tmem + tlane + TM_D2 + 16 * half, x);
-                const float gm = sGamma[lrow];
+                const float gm = sGam[lrow], el = sEl[lrow];
 #pragma unroll
-                for (int j = 0; j < 16; ++j) S[j] = gm * S[j] + x[j];
-                write_state_tile();
+                for (int j = 0; j < 16; ++j) S[j] = gm * S[j] + el * x[j];
                 if (lrow >= 64) {
                     const int t = lrow - 64;
-                    float o[16];
-                    tmem_ld16(tmem + tlane + TM_D1 + 16 * half, o);
+                    float o1[16], o2[16];
+                    tmem_ld16(tmem + tlane + TM_D + 64 + 16 * half, o1);
+                    tmem_ld16(tmem + tlane + TM_D3 + 16 * half, o2);
                     if (t < c) {
                         float4 *dst = reinterpret_cast<float4 *>(out + gv(t) + 16 * half);
 #pragma unroll
                         for (int g = 0; g < 4; ++g)
-                            dst[g] = make_float4(o[4 * g], o[4 * g + 1], o[4 * g + 2], o[4 * g + 3]);
+                            dst[g] = make_float4(o1[4 * g] + o2[4 * g], o1[4 * g + 1] + o2[4 * g + 1],
+                                                 o1[4 * g + 2] + o2[4 * g + 2], o1[4 * g + 3] + o2[4 * g + 3]);
                     }
                 }
             }
-            proxy_fence();
             tc_fence_before();
-            __syncthreads();
         } else {
             // ---- exact token-by-token path for a chunk with a very wide decay range
-            float *fq = reinterpret_cast<float *>(smem);
-            float *fk = fq + kC * kTP;
-            float *fa = fk + kC * kTP;
-            float *fS = reinterpret_cast<float *>(smem + SM_W);     // [128][33]
-            float *fv = fS + kDK * 33;                                // [64][33]
-            float *red = fv + kC * 33;                                // [2][8][32]
-            for (int idx = tid; idx < kC * kDK; idx += kNT) {
-                const int t = idx / kDK, ch = idx % kDK;
-                float qq = 0.f, kk = 0.f, la = 0.f;
-                if (t < c) {
-                    qq = __bfloat162float(q[gk(t, ch)]);
-                    kk = __bfloat162float(k[gk(t, ch)]);
-                    la = log_alpha[gk(t, ch)];
-                }
-                fq[t * kTP + ch] = qq; fk[t * kTP + ch] = kk; fa[t * kTP + ch] = la;
-            }
-            for (int idx = tid; idx < kC * kDVS; idx += kNT) {
-                const int t = idx / kDVS, x = idx % kDVS;
-                fv[t * 33 + x] = (t < c) ? __bfloat162float(v[gv(t) + x]) : 0.f;
-            }
+            float *fS = reinterpret_cast<float *>(smem + SM_P);      // [128][33]
+            float *red = fS + kDK * 33;                               // [2][8][32]
 #pragma unroll
             for (int j = 0; j < 16; ++j) fS[lrow * 33 + 16 * half + j] = S[j];
             __syncthreads();
@@ -607,22 +637,22 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
                 float pk = 0.f;
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
-                    const int ch = rg * RPT + r;
-                    sreg[r] *= expf(fa[t * kTP + ch]);
-                    pk += sreg[r] * fk[t * kTP + ch];
+                    const int cr = rg * RPT + r;
+                    sreg[r] *= expf(sta[t * kDK + cr]);
+                    pk += sreg[r] * __bfloat162float(stk[t * kDK + cr]);
                 }
                 red[rg * kDVS + x] = pk;
                 __syncthreads();
                 float p = 0.f;
 #pragma unroll
                 for (int j = 0; j < RG; ++j) p += red[j * kDVS + x];
-                const float d = sBeta[t] * (fv[t * 33 + x] - p);
+                const float d = sBeta[t] * (__bfloat162float(v[gv(t) + x]) - p);
                 float pq = 0.f;
 #pragma unroll
                 for (int r = 0; r < RPT; ++r) {
-                    const int ch = rg * RPT + r;
-                    sreg[r] += fk[t * kTP + ch] * d;
-                    pq += sreg[r] * fq[t * kTP + ch];
+                    const int cr = rg * RPT + r;
+                    sreg[r] += __bfloat162float(stk[t * kDK + cr]) * d;
+                    pq += sreg[r] * __bfloat162float(stq[t * kDK + cr]);
                 }
                 red[RG * kDVS + rg * kDVS + x] = pq;
                 __syncthreads();
@@ -639,13 +669,20 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
             __syncthreads();
 #pragma unroll
             for (int j = 0; j < 16; ++j) S[j] = fS[lrow * 33 + 16 * half + j];
-            write_state_tile();
             proxy_fence();
-            __syncthreads();
+            if (n + 1 < nchunks) {
+                issue_stage(n + 1);
+                load_vb(n + 1, vreg, breg);
+            }
         }
+        proxy_fence();
+        __syncthreads();
     }
 
     if (failed) {
+        // a bounded wait gave up: let any staged copy still in flight land before
+        // this CTA's shared memory is released (itself bounded), then report
+        if (ld_pending) mbar_wait(mbar_ld, ld_phase);
         if (tid == 0) atomicOr(&g_kda_device_status, 1u);
     } else if (sT) {
         float4 *dst = reinterpret_cast<float4 *>(sT + ((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half);
