@@ -320,11 +320,14 @@ prefill_tc_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__re
         // ---- pass 1 (two threads per key channel, fp32): log-decay sums and range
         float *xch = reinterpret_cast<float *>(smem + SM_RM);   // [3][2][128]
         {
+            float la_r[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) la_r[i] = (32 * th + i < c) ? sta[(32 * th + i) * kDK + ch] : 0.f;
             float run = 0.f, lo = INFINITY, hi = -INFINITY;
-            for (int i = 0; i < 32; ++i) {
-                const int t = 32 * th + i;
-                if (t < c) {
-                    run += sta[t * kDK + ch];
+            if (32 * th < c) {
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    run += la_r[i];
                     lo = fminf(lo, run);
                     hi = fmaxf(hi, run);
                 }
