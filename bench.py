@@ -70,6 +70,10 @@ def decode_bytes_per_head(dk, dv, in_bytes):
 # Reported only while the kernel source is unchanged (profiles/ holds the captures).
 MEASURED_TRAFFIC = {
     ("kda_decode.cu", "decode_bf16_b256_h32_d128_1024steps"): ("a2103952ead4a8e9", 1.0332e9),
+    # captured on B4 H32 T4096 (938.4 MB = 0.979 of its algorithmic bytes) and scaled to
+    # the long-context launch by token-heads processed (the kernel streams its inputs once)
+    ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
+    ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
 }
 
 
@@ -419,6 +423,8 @@ def main(argv=None):
     ap.add_argument("--impl", choices=["kda", "reference"], default="kda")
     ap.add_argument("--workload", default="prefill_bf16_b1_h32_t65536_d128",
                     help="prefill workload to time (name from gated_delta_rule_109_b200.inputs)")
+    ap.add_argument("--seq-len", type=int, default=0,
+                    help="override T of the prefill workload (profiling runs on a shorter case)")
     ap.add_argument("--decode-steps", type=int, default=1024)
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
@@ -447,6 +453,8 @@ def main(argv=None):
 
     byname = {w.name: w for w in I.WORKLOADS}
     w = rank_workload(byname[args.workload], rank)
+    if args.seq_len > 0:
+        w = I.scaled(w, T=args.seq_len, name=w.name + "_T%d" % args.seq_len)
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
     in_bytes = 2 if w.dtype == "bf16" else 4
 
@@ -471,11 +479,13 @@ def main(argv=None):
                  + (4 * w.B * w.H * w.dk * w.dv if w.final_state else 0)
                  + (4 * w.B * w.H * w.dk * w.dv if w.state_sd is not None else 0))
     achieved = alg_bytes / (ms_launch / 1e3) / 1e9
-    traffic = measured_traffic("kda_prefill_simt.cu", w.name)
+    tc = (w.dtype == "bf16" and w.dk == 128 and w.dv == 128)   # the library's dispatch rule
+    kname, ksrc = ("prefill_tc_kernel", "kda_prefill_tc.cu") if tc else ("prefill_simt_kernel", "kda_prefill_simt.cu")
+    traffic = measured_traffic(ksrc, w.name)
     alg_flops = w.B * w.T * w.H * prefill_flops_per_token_head(w.dk)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,
-                "kernel": "prefill_simt_kernel", "algorithmic_bytes_per_launch": alg_bytes,
+                "kernel": kname, "algorithmic_bytes_per_launch": alg_bytes,
                 "ms_per_launch": ms_launch, "peak_source": peak_src + " HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                 "tensor_view": {"algorithmic_flops_per_launch": alg_flops,
                                 "achieved_tflops": alg_flops / (ms_launch / 1e3) / 1e12,
@@ -493,7 +503,9 @@ def main(argv=None):
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_total / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "f32", "data": "synthetic",
+            "dtype": "bf16" if tc else "f32", "data": "synthetic",
+            "arithmetic": ("tcgen05 bf16 products of hi/lo-split operands (3 terms), fp32 accumulation "
+                           "in tensor memory, fp32 CUDA-core solve and scans") if tc else "fp32 CUDA cores",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "input_dtype": w.dtype, "chunk": 64, "final_state": w.final_state,
                        "l2": "no flush: inputs %.2f GB per step > 126 MB L2" % (alg_bytes / 1e9),
