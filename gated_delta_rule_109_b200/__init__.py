@@ -8,6 +8,8 @@ library is not built, every call raises.
     import gated_delta_rule_109_b200 as kda
     out, final_state = kda.forward(q, k, v, log_alpha, beta, initial_state)
     out = kda.decode_step(q, k, v, log_alpha, beta, state)   # state updated in place
+    # scalar-gate variants: Gated DeltaNet (log_alpha [B,T,H]) and DeltaNet (None)
+    out, final_state = kda.gdn_forward(q, k, v, g, beta, initial_state)
 """
 from __future__ import annotations
 
@@ -24,8 +26,9 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED, KDA_ERR_CU
 KDA_BF16, KDA_F32 = 0, 1
 
 # every symbol include/kda.h declares
-EXPORTS = ("kda_forward", "kda_decode_step", "kda_status_string", "kda_check_status",
-           "kda_last_cuda_error", "kda_launch_count", "kda_version")
+EXPORTS = ("kda_forward", "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
+           "kda_status_string", "kda_check_status", "kda_last_cuda_error", "kda_launch_count",
+           "kda_version")
 
 _lib = None
 
@@ -53,6 +56,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
+    lib.kda_gdn_forward.restype = i
+    lib.kda_gdn_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
+    lib.kda_gdn_decode_step.restype = i
+    lib.kda_gdn_decode_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
     lib.kda_status_string.restype = ctypes.c_char_p
     lib.kda_status_string.argtypes = [i]
     lib.kda_check_status.restype = i
@@ -105,6 +112,59 @@ def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None):
         raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
 
 
+def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, final_state,
+             return_final_state, scale):
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q)
+    _need(q, "q", (B, T, H, dk), q.dtype, dev)
+    _need(k, "k", (B, T, H, dk), q.dtype, dev)
+    _need(v, "v", (B, T, H, dv), q.dtype, dev)
+    if log_alpha is not None or gate_shape is not None:
+        _need(log_alpha, "log_alpha", gate_shape(B, T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    _need(out, "out", (B, T, H, dv), torch.float32, dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
+    fn = getattr(lib, entry)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+            _ptr(initial_state), _ptr(out), _ptr(final_state),
+            B, T, H, dk, dv, code, float(scale), _stream(dev))
+    _check(st, entry)
+    return out, final_state
+
+
+def _decode(entry, gate_shape, q, k, v, log_alpha, beta, state, out, scale):
+    lib = load()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q)
+    _need(q, "q", (B, H, dk), q.dtype, dev)
+    _need(k, "k", (B, H, dk), q.dtype, dev)
+    _need(v, "v", (B, H, dv), q.dtype, dev)
+    if log_alpha is not None or gate_shape is not None:
+        _need(log_alpha, "log_alpha", gate_shape(B, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, H), torch.float32, dev)
+    _need(state, "state", (B, H, dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=torch.float32, device=dev)
+    _need(out, "out", (B, H, dv), torch.float32, dev)
+    fn = getattr(lib, entry)
+    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+            _ptr(state), _ptr(out), B, H, dk, dv, code, float(scale), _stream(dev))
+    _check(st, entry)
+    return out
+
+
 def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
             return_final_state=True, scale: float = 0.0):
     """Chunked KDA prefill (``kda_forward``).
@@ -116,30 +176,8 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_sta
     the same tensor as ``initial_state`` to carry the state in place.
     ``scale`` 0 means 1/sqrt(dk).
     """
-    lib = load()
-    B, T, H, dk = q.shape
-    dv = v.shape[-1]
-    dev = q.device
-    code = _dtype_code(q)
-    _need(q, "q", (B, T, H, dk), q.dtype, dev)
-    _need(k, "k", (B, T, H, dk), q.dtype, dev)
-    _need(v, "v", (B, T, H, dv), q.dtype, dev)
-    _need(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
-    _need(beta, "beta", (B, T, H), torch.float32, dev)
-    if initial_state is not None:
-        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
-    if out is None:
-        out = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
-    _need(out, "out", (B, T, H, dv), torch.float32, dev)
-    if final_state is None and return_final_state:
-        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
-    if final_state is not None:
-        _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
-    st = lib.kda_forward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                         _ptr(initial_state), _ptr(out), _ptr(final_state),
-                         B, T, H, dk, dv, code, float(scale), _stream(dev))
-    _check(st, "kda_forward")
-    return out, final_state
+    return _forward("kda_forward", lambda B, T, H, dk: (B, T, H, dk), q, k, v, log_alpha, beta,
+                    initial_state, out, final_state, return_final_state, scale)
 
 
 def decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0):
@@ -149,24 +187,29 @@ def decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0
     fp32; beta ``[B,H]`` fp32; state ``[B,H,dk,dv]`` fp32.  Returns
     ``out [B,H,dv]`` fp32.
     """
-    lib = load()
-    B, H, dk = q.shape
-    dv = v.shape[-1]
-    dev = q.device
-    code = _dtype_code(q)
-    _need(q, "q", (B, H, dk), q.dtype, dev)
-    _need(k, "k", (B, H, dk), q.dtype, dev)
-    _need(v, "v", (B, H, dv), q.dtype, dev)
-    _need(log_alpha, "log_alpha", (B, H, dk), torch.float32, dev)
-    _need(beta, "beta", (B, H), torch.float32, dev)
-    _need(state, "state", (B, H, dk, dv), torch.float32, dev)
-    if out is None:
-        out = torch.empty((B, H, dv), dtype=torch.float32, device=dev)
-    _need(out, "out", (B, H, dv), torch.float32, dev)
-    st = lib.kda_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                             _ptr(state), _ptr(out), B, H, dk, dv, code, float(scale), _stream(dev))
-    _check(st, "kda_decode_step")
-    return out
+    return _decode("kda_decode_step", lambda B, H, dk: (B, H, dk), q, k, v, log_alpha, beta, state,
+                   out, scale)
+
+
+def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
+                return_final_state=True, scale: float = 0.0):
+    """Chunked prefill of Gated DeltaNet / DeltaNet (``kda_gdn_forward``).
+
+    As :func:`forward`, with one decay per token and head: log_alpha
+    ``[B,T,H]`` fp32 (<= 0), or None for DeltaNet (no decay).
+    """
+    shape = None if log_alpha is None else (lambda B, T, H, dk: (B, T, H))
+    return _forward("kda_gdn_forward", shape, q, k, v, log_alpha, beta, initial_state, out,
+                    final_state, return_final_state, scale)
+
+
+def gdn_decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0):
+    """One Gated DeltaNet / DeltaNet decode step (``kda_gdn_decode_step``).
+
+    As :func:`decode_step`, with log_alpha ``[B,H]`` fp32 or None.
+    """
+    shape = None if log_alpha is None else (lambda B, H, dk: (B, H))
+    return _decode("kda_gdn_decode_step", shape, q, k, v, log_alpha, beta, state, out, scale)
 
 
 def check_status(device=None):

@@ -33,7 +33,7 @@ extern "C" {
 unsigned long long kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 
-int kda_version(void) { return 100; }   // 0.1.0
+int kda_version(void) { return 200; }   // 0.2.0
 
 const char *kda_status_string(kda_status s)
 {
@@ -50,11 +50,16 @@ const char *kda_status_string(kda_status s)
 
 const char *kda_last_cuda_error(void) { return g_last_cuda_error; }
 
-kda_status kda_forward(const void *q, const void *k, const void *v,
-                       const float *log_alpha, const float *beta,
-                       const float *initial_state, float *out, float *final_state,
-                       int B, int T, int H, int dk, int dv,
-                       kda_dtype dtype, float scale, void *stream)
+}  // extern "C"
+
+namespace {
+
+// Shared by the per-channel (KDA) and scalar-gate (Gated DeltaNet / DeltaNet)
+// entry points: they differ only in the shape of log_alpha.
+kda_status forward_impl(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *initial_state, float *out, float *final_state,
+                        int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
+                        void *stream, kda::GateKind gate)
 {
     g_last_cuda_error[0] = '\0';
     // ---- validation: nothing is enqueued unless every check passes
@@ -62,9 +67,12 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
     if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
     if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
     if ((int64_t)B * H > (int64_t)INT32_MAX / 4) return KDA_ERR_INVALID_ARG;
-    if (T > 0 && (!q || !k || !v || !log_alpha || !beta || !out)) return KDA_ERR_INVALID_ARG;
+    const bool need_gate = gate != kda::KDA_GATE_NONE;
+    if (T > 0 && (!q || !k || !v || (need_gate && !log_alpha) || !beta || !out)) return KDA_ERR_INVALID_ARG;
     if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
+    const bool gate_aligned = gate == kda::KDA_GATE_CHANNEL ? aligned16(log_alpha)
+                              : gate == kda::KDA_GATE_SCALAR ? aligned4(log_alpha) : true;
+    if (T > 0 && (!aligned16(q) || !aligned16(k) || !aligned16(v) || !gate_aligned ||
                   !aligned16(out) || !aligned4(beta)))
         return KDA_ERR_MISALIGNED;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
@@ -82,13 +90,59 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
     }
 
     kda::ForwardArgs a;
-    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = need_gate ? log_alpha : nullptr; a.beta = beta;
     a.s0 = initial_state; a.out = out; a.sT = final_state;
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
     a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
-    cudaError_t e = kda::prefill_tc_supported(a) ? kda::launch_prefill_tc(a, st)
-                                                 : kda::launch_prefill_simt(a, st);
+    a.gate = gate;
+    cudaError_t e;
+    if (!kda::prefill_tc_supported(a)) e = kda::launch_prefill_simt(a, st);
+    else if (gate == kda::KDA_GATE_CHANNEL) e = kda::launch_prefill_tc(a, st);
+    else e = kda::launch_prefill_gdn_tc(a, st);
     return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status decode_impl(const void *q, const void *k, const void *v, const float *log_alpha,
+                       const float *beta, float *state_inout, float *out, int B, int H, int dk, int dv,
+                       kda_dtype dtype, float scale, void *stream, kda::GateKind gate)
+{
+    g_last_cuda_error[0] = '\0';
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
+    const bool need_gate = gate != kda::KDA_GATE_NONE;
+    if (!q || !k || !v || (need_gate && !log_alpha) || !beta || !state_inout || !out)
+        return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    const bool gate_aligned = gate == kda::KDA_GATE_CHANNEL ? aligned16(log_alpha)
+                              : gate == kda::KDA_GATE_SCALAR ? aligned4(log_alpha) : true;
+    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !gate_aligned ||
+        !aligned16(state_inout) || !aligned16(out) || !aligned4(beta))
+        return KDA_ERR_MISALIGNED;
+
+    kda::DecodeArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = need_gate ? log_alpha : nullptr; a.beta = beta;
+    a.state = state_inout; a.out = out;
+    a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
+    a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
+    a.gate = gate;
+    cudaError_t e = kda::launch_decode(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+}  // namespace
+
+extern "C" {
+
+kda_status kda_forward(const void *q, const void *k, const void *v,
+                       const float *log_alpha, const float *beta,
+                       const float *initial_state, float *out, float *final_state,
+                       int B, int T, int H, int dk, int dv,
+                       kda_dtype dtype, float scale, void *stream)
+{
+    return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                        dtype, scale, stream, kda::KDA_GATE_CHANNEL);
 }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v,
@@ -97,24 +151,28 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            int B, int H, int dk, int dv,
                            kda_dtype dtype, float scale, void *stream)
 {
-    g_last_cuda_error[0] = '\0';
-    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
-    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
-    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
-    if ((int64_t)B * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
-    if (!q || !k || !v || !log_alpha || !beta || !state_inout || !out) return KDA_ERR_INVALID_ARG;
-    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
-    if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) ||
-        !aligned16(state_inout) || !aligned16(out) || !aligned4(beta))
-        return KDA_ERR_MISALIGNED;
+    return decode_impl(q, k, v, log_alpha, beta, state_inout, out, B, H, dk, dv, dtype, scale, stream,
+                       kda::KDA_GATE_CHANNEL);
+}
 
-    kda::DecodeArgs a;
-    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
-    a.state = state_inout; a.out = out;
-    a.B = B; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
-    a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
-    cudaError_t e = kda::launch_decode(a, static_cast<cudaStream_t>(stream));
-    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *initial_state, float *out, float *final_state,
+                           int B, int T, int H, int dk, int dv,
+                           kda_dtype dtype, float scale, void *stream)
+{
+    return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                        dtype, scale, stream, log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
+}
+
+kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               float *state_inout, float *out,
+                               int B, int H, int dk, int dv,
+                               kda_dtype dtype, float scale, void *stream)
+{
+    return decode_impl(q, k, v, log_alpha, beta, state_inout, out, B, H, dk, dv, dtype, scale, stream,
+                       log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
 }
 
 kda_status kda_check_status(void *stream)
@@ -122,10 +180,11 @@ kda_status kda_check_status(void *stream)
     g_last_cuda_error[0] = '\0';
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
-    unsigned int dev_status = 0;
+    unsigned int dev_status = 0, gdn_status = 0;
     e = kda::take_device_status(&dev_status);
+    if (e == cudaSuccess) e = kda::take_gdn_device_status(&gdn_status);
     if (e != cudaSuccess) return cuda_fail(e);
-    return dev_status ? KDA_ERR_TIMEOUT : KDA_OK;
+    return (dev_status | gdn_status) ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
 }  // extern "C"

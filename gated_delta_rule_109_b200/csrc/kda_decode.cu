@@ -26,7 +26,9 @@ namespace {
 
 constexpr int kDecodeThreads = 256;
 
-template <int DK, int DV, typename InT>
+// PER_CHANNEL: log_alpha is [B, H, dk] (KDA); otherwise [B, H] or null (one
+// decay for all channels, or none).
+template <int DK, int DV, typename InT, bool PER_CHANNEL>
 __global__ void __launch_bounds__(kDecodeThreads, 2)
 decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
                    const InT *__restrict__ v, const float *__restrict__ log_alpha,
@@ -54,7 +56,9 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
 
     const InT *qh = q + (size_t)bh * DK;
     const InT *kh = k + (size_t)bh * DK;
+    // decay of this head: per key channel (lah), or one value for all channels
     const float *lah = log_alpha + (size_t)bh * DK;
+    const float a_all = (!PER_CHANNEL && log_alpha) ? expf(log_alpha[bh]) : 1.f;
 
     // k.q for the read after the write (warp 0)
     if (tid < 32) {
@@ -70,7 +74,7 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
 #pragma unroll
     for (int i = 0; i < RPT; ++i) {
         const int r = r0 + i * RS;
-        const float a = expf(lah[r]);
+        const float a = PER_CHANNEL ? expf(lah[r]) : a_all;
         const float kc = to_f32(kh[r]);
         const float qc = to_f32(qh[r]);
         kr[i] = kc;
@@ -118,7 +122,9 @@ template <int DK, int DV, typename InT>
 cudaError_t launch_typed(const DecodeArgs &a, cudaStream_t stream)
 {
     const unsigned grid = (unsigned)((size_t)a.B * a.H);
-    decode_step_kernel<DK, DV, InT><<<grid, kDecodeThreads, 0, stream>>>(
+    auto kernel = (a.gate == KDA_GATE_CHANNEL) ? decode_step_kernel<DK, DV, InT, true>
+                                               : decode_step_kernel<DK, DV, InT, false>;
+    kernel<<<grid, kDecodeThreads, 0, stream>>>(
         static_cast<const InT *>(a.q), static_cast<const InT *>(a.k),
         static_cast<const InT *>(a.v), a.log_alpha, a.beta, a.state, a.out, a.scale);
     cudaError_t e2 = cudaGetLastError();

@@ -11,6 +11,10 @@ namespace kda {
 
 constexpr int kChunk = 64;   // tokens per chunk of the prefill
 
+// How the decay is given: one log_alpha per key channel (KDA), one per token and
+// head (Gated DeltaNet), or none (DeltaNet, alpha = 1).
+enum GateKind { KDA_GATE_NONE = 0, KDA_GATE_SCALAR = 1, KDA_GATE_CHANNEL = 2 };
+
 struct ForwardArgs {
     const void *q, *k, *v;
     const float *log_alpha, *beta;
@@ -20,6 +24,7 @@ struct ForwardArgs {
     int B, T, H, dk, dv;
     kda_dtype dtype;
     float scale;
+    int gate;                 // GateKind
 };
 
 struct DecodeArgs {
@@ -30,6 +35,7 @@ struct DecodeArgs {
     int B, H, dk, dv;
     kda_dtype dtype;
     float scale;
+    int gate;                 // GateKind
 };
 
 // Each launcher enqueues its kernel(s) on `stream` and returns the launch
@@ -39,6 +45,9 @@ cudaError_t launch_prefill_simt(const ForwardArgs &a, cudaStream_t stream);
 // Tensor-core (tcgen05) prefill: bf16 inputs with dk = dv = 128.
 bool prefill_tc_supported(const ForwardArgs &a);
 cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t stream);
+// Tensor-core prefill with one decay per token and head (or none): bf16, dk = dv = 128.
+cudaError_t launch_prefill_gdn_tc(const ForwardArgs &a, cudaStream_t stream);
+cudaError_t take_gdn_device_status(unsigned int *status);
 // Reads and clears the device status word the tensor-core kernels set when a
 // bounded wait gives up (bit 0).  Synchronous.
 cudaError_t take_device_status(unsigned int *status);

@@ -66,7 +66,7 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
                     const InT *__restrict__ v, const float *__restrict__ log_alpha,
                     const float *__restrict__ beta, const float *__restrict__ s0,
                     float *__restrict__ out, float *__restrict__ sT,
-                    int T, int H, float scale)
+                    int T, int H, float scale, int gate)
 {
     using L = SimtSmem<DK>;
     constexpr int P = L::P, PV = L::PV, PC = L::PC;
@@ -104,6 +104,12 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
         if (tid < kC) sB[tid] = (tid < c) ? beta[((size_t)b * T + t0 + tid) * H + h] : 0.f;
         // global index of (token t of this chunk, key channel ch)
         auto gk = [&](int t, int ch) { return (((size_t)b * T + t0 + t) * H + h) * DK + ch; };
+        // log_alpha of (token t, key channel ch): per channel, one per token and head, or none
+        auto la_at = [&](int t, int ch) -> float {
+            if (gate == KDA_GATE_CHANNEL) return log_alpha[gk(t, ch)];
+            if (gate == KDA_GATE_SCALAR) return log_alpha[((size_t)b * T + t0 + t) * H + h];
+            return 0.f;
+        };
 
         // ---- pass 1, one thread per key channel: the in-chunk log-decay sums in
         // fp64 (so each exponent argument below carries a single rounding) and
@@ -112,7 +118,7 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
         if (tid < DK) {
             double run = 0.0, lo = 0.0, hi = 0.0;
             for (int t = 0; t < c; ++t) {
-                run += (double)log_alpha[gk(t, tid)];
+                run += (double)la_at(t, tid);
                 lo = (t == 0) ? run : fmin(lo, run);
                 hi = (t == 0) ? run : fmax(hi, run);
             }
@@ -130,7 +136,7 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
                 for (int t = 0; t < kC; ++t) {
                     float kk = 0.f, qq = 0.f;
                     if (t < c) {
-                        run += (double)log_alpha[gk(t, tid)];
+                        run += (double)la_at(t, tid);
                         kk = to_f32(k[gk(t, tid)]);
                         qq = to_f32(q[gk(t, tid)]);
                     }
@@ -184,7 +190,7 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
                 for (int t = 0; t < kC; ++t) {
                     float kk = 0.f, qq = 0.f;
                     if (t < c) {
-                        run += (double)log_alpha[gk(t, tid)];
+                        run += (double)la_at(t, tid);
                         kk = to_f32(k[gk(t, tid)]);
                         qq = to_f32(q[gk(t, tid)]);
                     }
@@ -274,7 +280,7 @@ prefill_simt_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
             for (int idx = tid; idx < kC * DK; idx += kThreads) {
                 const int t = idx / DK, ch = idx % DK;
                 float qq = 0.f, kk = 0.f, la = 0.f;
-                if (t < c) { qq = to_f32(q[gk(t, ch)]); kk = to_f32(k[gk(t, ch)]); la = log_alpha[gk(t, ch)]; }
+                if (t < c) { qq = to_f32(q[gk(t, ch)]); kk = to_f32(k[gk(t, ch)]); la = la_at(t, ch); }
                 sQ[t * P + ch] = qq; sK[t * P + ch] = kk; sX[t * P + ch] = la;
             }
             __syncthreads();
@@ -347,7 +353,7 @@ cudaError_t launch_typed(const ForwardArgs &a, cudaStream_t stream)
     kern<<<grid, kThreads, smem, stream>>>(
         static_cast<const InT *>(a.q), static_cast<const InT *>(a.k),
         static_cast<const InT *>(a.v), a.log_alpha, a.beta, a.s0, a.out, a.sT,
-        a.T, a.H, a.scale);
+        a.T, a.H, a.scale, a.gate);
     cudaError_t e2 = cudaGetLastError();
     if (e2 == cudaSuccess) note_launch();
     return e2;

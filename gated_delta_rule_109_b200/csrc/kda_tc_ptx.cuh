@@ -1,0 +1,147 @@
+// Inline-PTX wrappers and shared-memory tile helpers of libkda's tcgen05 kernels
+// (internal header, sm_100a only).
+//
+// Shared-memory operands use the no-swizzle canonical layout: core matrices of
+// 8 rows x 16 bytes (8 bf16).  A tile indexed (outer, inner) puts element
+// (outer, inner) at core_off(outer, inner, s_outer, s_inner).  K-major tiles have
+// outer = M (or N) and inner = K; MN-major tiles have outer = K and inner = M (or N).
+// In the matrix descriptor, LBO is the byte stride between core matrices along K
+// and SBO the stride along M/N.
+#pragma once
+
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace tcx {
+
+constexpr long long kWaitCycles = 4000000000ll;   // bounded mbarrier waits: ~2 s at 2 GHz
+
+__device__ __forceinline__ uint32_t core_off(int outer, int inner, uint32_t so, uint32_t si)
+{
+    return (uint32_t)(outer >> 3) * so + (uint32_t)(inner >> 3) * si + (uint32_t)(outer & 7) * 16u +
+           (uint32_t)(inner & 7) * 2u;
+}
+
+// ---------------------------------------------------------------- PTX wrappers
+__device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo)
+{
+    // no-swizzle shared-memory matrix descriptor (sm_100 format, version 1)
+    return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
+           ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | ((uint64_t)1 << 46);
+}
+
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn)
+{
+    // D fp32, A bf16, B bf16, dense, no negation
+    return (1u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)a_mn << 15) | ((uint32_t)b_mn << 16) |
+           ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n"
+                 :: "r"(d_tmem), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t mbar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 :: "r"(mbar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float (&v)[16])
+{
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+                 "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+                   "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr) : "memory");
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
+{
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(mbar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint32_t mbar, uint32_t bytes)
+{
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(mbar), "r"(bytes) : "memory");
+}
+
+__device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t bytes, uint32_t mbar)
+{
+    asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+                 :: "r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
+}
+
+// Bounded wait for the phase with the given parity; false if it never completed.
+__device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity)
+{
+    const long long t0 = clock64();
+    for (;;) {
+        uint32_t ok;
+        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                     "selp.u32 %0, 1, 0, p;\n\t}\n" : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+        if (ok) return true;
+        if (clock64() - t0 > kWaitCycles) return false;
+    }
+}
+
+// Split 8 fp32 values into bf16 hi / lo parts packed as two 16-byte vectors.
+__device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo)
+{
+    uint32_t h[4], l[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        const __nv_bfloat162 hv = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+        const float2 hf = __bfloat1622float2(hv);
+        const __nv_bfloat162 lv = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
+        h[i] = *reinterpret_cast<const uint32_t *>(&hv);
+        l[i] = *reinterpret_cast<const uint32_t *>(&lv);
+    }
+    hi = make_uint4(h[0], h[1], h[2], h[3]);
+    lo = make_uint4(l[0], l[1], l[2], l[3]);
+}
+
+__device__ __forceinline__ void st_split8(uint8_t *smem, uint32_t off_hi, uint32_t off_lo, const float (&x)[8])
+{
+    uint4 hi, lo;
+    split8(x, hi, lo);
+    *reinterpret_cast<uint4 *>(smem + off_hi) = hi;
+    *reinterpret_cast<uint4 *>(smem + off_lo) = lo;
+}
+
+// One product D (+)= A B on bf16 hi/lo split operands: hi*hi, plus lo*hi when A has
+// a lo part and hi*lo when B has one (an operand without a lo part is an exact
+// bf16 input).  Each term walks K in `ksteps` steps of 16 (two core matrices).
+__device__ __forceinline__ void mma_split(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t a_lbo,
+                                          uint32_t a_sbo, uint32_t b_hi, uint32_t b_lo, uint32_t b_lbo,
+                                          uint32_t b_sbo, int ksteps, uint32_t idesc, bool accumulate,
+                                          bool a_has_lo = true, bool b_has_lo = true)
+{
+    bool acc = accumulate;
+    for (int tt = 0; tt < 3; ++tt) {
+        if ((tt == 1 && !a_has_lo) || (tt == 2 && !b_has_lo)) continue;
+        const uint32_t a = (tt == 1) ? a_lo : a_hi;
+        const uint32_t b = (tt == 2) ? b_lo : b_hi;
+        for (int ks = 0; ks < ksteps; ++ks) {
+            const uint64_t ad = smem_desc(a + 2u * a_lbo * ks, a_lbo, a_sbo);
+            const uint64_t bd = smem_desc(b + 2u * b_lbo * ks, b_lbo, b_sbo);
+            umma_bf16(d, ad, bd, idesc, acc ? 1u : 0u);
+            acc = true;
+        }
+    }
+}
+
+}  // namespace tcx
+}  // namespace kda

@@ -113,6 +113,48 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            int B, int H, int dk, int dv,
                            kda_dtype dtype, float scale, void *stream);
 
+/*
+ * kda_gdn_forward -- chunked prefill of the scalar-gate members of the family:
+ * Gated DeltaNet (one decay per token and head) and DeltaNet (no decay).
+ *
+ * The token step is KDA's with Diag(alpha_t) replaced by a scalar alpha_t that
+ * decays every key channel alike ("Kimi Delta Attention: The Linear Attention
+ * Behind Kimi K2 and Qwen3", §DeltaNet, Gated DeltaNet, and KDA, comparison
+ * table, and the FAQ entry on how Gated DeltaNet and KDA differ), or with no
+ * decay at all (the delta rule of "KDA Technical Deep Dive", §From attention
+ * to recurrent state (delta rule)).  KDA with every channel of log_alpha equal
+ * to the scalar gives the same result.
+ *
+ *   q, k          [B, T, H, dk]  dtype            (16-byte aligned)
+ *   v             [B, T, H, dv]  dtype            (16-byte aligned)
+ *   log_alpha     [B, T, H]      float32 or NULL  (4-byte aligned; NULL = DeltaNet, alpha = 1)
+ *   beta          [B, T, H]      float32          (4-byte aligned)
+ *   initial_state, out, final_state: as for kda_forward.
+ *
+ * log_alpha must be finite and <= 0 (alpha in (0, 1]).  Everything else --
+ * sizes, head dimensions, aliasing, T = 0, statuses -- is as for kda_forward.
+ */
+kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
+                           const float *log_alpha, const float *beta,
+                           const float *initial_state, float *out, float *final_state,
+                           int B, int T, int H, int dk, int dv,
+                           kda_dtype dtype, float scale, void *stream);
+
+/*
+ * kda_gdn_decode_step -- one token per sequence of the scalar-gate variants,
+ * state updated in place.
+ *
+ *   log_alpha     [B, H]  float32 or NULL  (4-byte aligned; NULL = DeltaNet)
+ *   every other argument as for kda_decode_step.
+ *
+ * Equivalent to kda_gdn_forward with T = 1 and final_state == initial_state.
+ */
+kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               float *state_inout, float *out,
+                               int B, int H, int dk, int dv,
+                               kda_dtype dtype, float scale, void *stream);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *kda_status_string(kda_status status);
 

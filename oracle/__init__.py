@@ -14,6 +14,8 @@ delta-rule write, read with the query scaled by 1/sqrt(d_k)):
                      parity at realistic sizes and for the timed CPU baseline.
 * ``forward_np``  -- plain numpy, a loop over tokens vectorised over (B, H);
                      used for small cases and to cross-check ``forward``.
+* ``gdn_forward`` -- the scalar-gate variants (Gated DeltaNet, DeltaNet) as
+                     ``forward`` with the gate repeated over key channels.
 
 Both store the state as ``[B, H, dk, dv]`` (the transpose of the page's
 (d_v, d_k) matrix), so the per-channel decay scales rows and the page's
@@ -125,6 +127,29 @@ def forward_np(q, k, v, log_alpha, beta, initial_state=None, scale=None):
         S = S + kf[:, t][..., :, None] * e[..., None, :]   # S~ + k e^T
         out[:, t] = scale * np.einsum("bhcx,bhc->bhx", S, qf[:, t])
     return out, S
+
+
+def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, scale=None, nthreads=0):
+    """fp64 forward of the scalar-gate members of the family.
+
+    Gated DeltaNet decays every key channel of the state by the same alpha_t;
+    KDA's gate is the per-channel refinement of it ("Kimi Delta Attention: The
+    Linear Attention Behind Kimi K2 and Qwen3", §DeltaNet, Gated DeltaNet, and
+    KDA, comparison table).  DeltaNet has no decay (alpha = 1; "KDA Technical
+    Deep Dive", §From attention to recurrent state (delta rule)).  So this is
+    :func:`forward` with ``log_alpha [B,T,H]`` repeated over the dk key
+    channels, or zeros when ``log_alpha`` is None.
+    """
+    qf = _as_f32(q)
+    B, T, H, dk = qf.shape
+    if log_alpha is None:
+        la = np.zeros((B, T, H, dk), dtype=np.float32)
+    else:
+        g = _as_f32(log_alpha)
+        if g.shape != (B, T, H):
+            raise ValueError("log_alpha has shape %s, expected %s" % (g.shape, (B, T, H)))
+        la = np.ascontiguousarray(np.repeat(g[..., None], dk, axis=-1))
+    return forward(qf, k, v, la, beta, initial_state, scale=scale, nthreads=nthreads)
 
 
 def parity_error(x_gpu, x_ref) -> float:

@@ -75,3 +75,43 @@ def test_unmutated_copy_passes_every_pin():
     fwd = _make("none")
     for t in PIN_TESTS:
         t(fwd)
+
+
+def _make_gdn(mutation):
+    """oracle.gdn_forward with one slip in how the [B,T,H] gate reaches the channels."""
+    def gdn(q, k, v, log_alpha, beta, initial_state=None, scale=None, nthreads=0):
+        qf = oracle._as_f32(q)
+        B, T, H, dk = qf.shape
+        g = np.zeros((B, T, H), np.float32) if log_alpha is None else oracle._as_f32(log_alpha)
+        if mutation == "first_channel_only":
+            la = np.zeros((B, T, H, dk), np.float32)
+            la[..., 0] = g
+        elif mutation == "token_head_swapped":
+            la = np.repeat(g.reshape(B, H, T).transpose(0, 2, 1)[..., None], dk, axis=-1)
+        elif mutation == "gate_not_applied":
+            la = np.zeros((B, T, H, dk), np.float32)
+        else:
+            la = np.repeat(g[..., None], dk, axis=-1)
+        return oracle.forward(qf, k, v, np.ascontiguousarray(la), beta, initial_state, scale=scale)
+    return gdn
+
+
+GDN_PINS = [pins.test_gdn_forward_is_the_gated_deltanet_recurrence, pins.test_gdn_forward_rotation_invariance]
+
+
+@pytest.mark.parametrize("mutation", ["first_channel_only", "token_head_swapped", "gate_not_applied"])
+def test_some_gdn_pin_fails_on_planted_mistake(mutation, monkeypatch):
+    monkeypatch.setattr(oracle, "gdn_forward", _make_gdn(mutation))
+    failed = 0
+    for pin in GDN_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, "no scalar-gate pin caught %s" % mutation
+
+
+def test_unmutated_gdn_copy_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(oracle, "gdn_forward", _make_gdn("none"))
+    for pin in GDN_PINS:
+        pin()

@@ -235,3 +235,55 @@ def test_parity_metric():
     ref = np.array([1.0, -1.0, 1.0, -1.0])
     assert oracle.parity_error(ref + np.array([0, 0, 0.002, 0]), ref) == pytest.approx(0.002)
     assert oracle.parity_error(np.zeros(0), np.zeros(0)) == 0.0
+
+
+# ---------------------------------------------------------------- O9 scalar-gate entry
+def test_gdn_forward_is_the_gated_deltanet_recurrence():
+    """oracle.gdn_forward with a [B,T,H] gate against the textbook Gated DeltaNet
+    step S <- alpha_t (I - beta k k^T) S + beta k v^T, read S^T q / sqrt(dk); with
+    no gate, against the DeltaNet step (alpha = 1)."""
+    q, k, v, la, beta, S0 = _rand(21, T=17, dk=8, dv=5)
+    g = np.ascontiguousarray(la[..., 0] - 0.5)            # [B,T,H], distinct per token and head
+    B, T, H, dk = q.shape
+    for gate in (g, None):
+        out, sT = oracle.gdn_forward(q, k, v, gate, beta, S0)
+        for b in range(B):
+            for h in range(H):
+                S = S0[b, h].copy()
+                for t in range(T):
+                    kt = k[b, t, h].astype(np.float64)
+                    a = 1.0 if gate is None else math.exp(float(gate[b, t, h]))
+                    bt = float(beta[b, t, h])
+                    S = a * (np.eye(dk) - bt * np.outer(kt, kt)) @ S + bt * np.outer(kt, v[b, t, h].astype(np.float64))
+                    np.testing.assert_allclose(out[b, t, h], S.T @ q[b, t, h].astype(np.float64) / math.sqrt(dk),
+                                               rtol=1e-11, atol=1e-12)
+                np.testing.assert_allclose(sT[b, h], S, rtol=1e-11, atol=1e-12)
+
+
+def test_gdn_forward_rotation_invariance():
+    """A decay shared by all key channels commutes with any rotation U of key
+    space: (U q, U k, U S0) gives the same outputs and U S_T.  A per-channel
+    decay does not, so this fails if the scalar gate reaches the channels
+    unevenly."""
+    q, k, v, la, beta, S0 = _rand(22, T=24, dk=8, dv=4)
+    g = np.ascontiguousarray(-0.2 - la[..., 0])
+    U, _ = np.linalg.qr(np.random.default_rng(7).standard_normal((8, 8)))
+    rot = lambda x: np.einsum("ij,bthj->bthi", U, x.astype(np.float64)).astype(np.float32)
+    out, sT = oracle.gdn_forward(q, k, v, g, beta, S0)
+    out_r, sT_r = oracle.gdn_forward(rot(q), rot(k), v, g, beta, np.einsum("ij,bhjx->bhix", U, S0))
+    # the rotated q, k are rounded to fp32: agreement to fp32 input precision
+    assert oracle.parity_error(out_r, out) < 2e-5
+    assert oracle.parity_error(sT_r, np.einsum("ij,bhjx->bhix", U, sT)) < 2e-5
+    # the same property fails for KDA's per-channel gate
+    out_c, _ = oracle.forward(q, k, v, la * 8, beta, S0)
+    out_cr, _ = oracle.forward(rot(q), rot(k), v, la * 8, beta, np.einsum("ij,bhjx->bhix", U, S0))
+    assert oracle.parity_error(out_cr, out_c) > 1e-2
+
+
+def test_gdn_forward_empty_and_shape_check():
+    q, k, v, la, beta, S0 = _rand(23, T=0)
+    o, s = oracle.gdn_forward(q, k, v, la[..., 0], beta, S0)
+    assert o.shape == (2, 0, 3, 6)
+    np.testing.assert_array_equal(s, S0)
+    with pytest.raises(ValueError):
+        oracle.gdn_forward(q, k, v, la, beta, S0)          # a per-channel gate is not accepted
