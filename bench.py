@@ -193,16 +193,22 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- prefill
-def bench_prefill(w, K, W, device):
+def bench_prefill(w, K, W, device, gate="channel"):
+    """K timed launches of the prefill.  gate="channel": KDA (kda_forward);
+    "scalar": Gated DeltaNet (kda_gdn_forward) with channel 0 of the draw as the gate."""
     import torch
     import gated_delta_rule_109_b200 as kda
     from gated_delta_rule_109_b200 import inputs as I
     x = I.make_inputs(w, device)
     out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
     sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device) if w.final_state else None
+    fwd = kda.forward
+    if gate == "scalar":
+        x["log_alpha"] = x["log_alpha"][..., 0].contiguous()
+        fwd = kda.gdn_forward
     args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
     for _ in range(W):
-        kda.forward(*args, out=out, final_state=sT, return_final_state=sT is not None)
+        fwd(*args, out=out, final_state=sT, return_final_state=sT is not None)
     torch.cuda.synchronize(device)
     kda.check_status(device)
     stream = torch.cuda.current_stream(device)
@@ -212,7 +218,7 @@ def bench_prefill(w, K, W, device):
     n0 = kda.launch_count()
     evs[0].record(stream)
     for i in range(K):
-        kda.forward(*args, out=out, final_state=sT, return_final_state=sT is not None)
+        fwd(*args, out=out, final_state=sT, return_final_state=sT is not None)
         evs[i + 1].record(stream)
     torch.cuda.synchronize(device)
     launches = kda.launch_count() - n0
@@ -414,6 +420,29 @@ def _add_decode(line, args, rank, world, device, hbm):
                 "steps": dec["e2e_steps"]}}
 
 
+def _add_gdn(line, args, w, world, device, hbm):
+    """The Gated DeltaNet specialisation timed on the same workload shape."""
+    pre = bench_prefill(w, args.steps, args.warmup, device, gate="scalar")
+    del pre["x"]
+    ms_total = max_over_ranks(pre["ms_total"], device)
+    ms_launch = statistics.mean(pre["ms_per_launch"])
+    in_bytes = 2 if w.dtype == "bf16" else 4
+    per_tok_head = (2 * w.dk + w.dv) * in_bytes + 4 + 4 + 4 * w.dv
+    alg_bytes = (w.B * w.T * w.H * per_tok_head
+                 + (4 * w.B * w.H * w.dk * w.dv if w.final_state else 0)
+                 + (4 * w.B * w.H * w.dk * w.dv if w.state_sd is not None else 0))
+    ach = alg_bytes / (ms_launch / 1e3) / 1e9
+    tc = (w.dtype == "bf16" and w.dk == 128 and w.dv == 128)
+    line["gated_deltanet_prefill"] = {
+        "workload": w.name, "gate": "one log_alpha per token and head (channel 0 of the KDA draw)",
+        "value": w.B * w.T * args.steps * world / (ms_total / 1e3), "unit": "tokens/s",
+        "ms_per_step": ms_total / args.steps, "gpu_launches": pre["launches"],
+        "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                     "traffic": None,
+                     "kernel": "prefill_gdn_tc_kernel" if tc else "prefill_simt_kernel",
+                     "algorithmic_bytes_per_launch": alg_bytes}}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -433,6 +462,8 @@ def main(argv=None):
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time only one kernel (profiling runs); the default times both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-variants", action="store_true",
+                    help="skip the Gated DeltaNet timing on the prefill workload")
     args = ap.parse_args(argv)
     args.warmup = max(3, args.warmup)
 
@@ -521,6 +552,8 @@ def main(argv=None):
 
     if not args.no_decode and args.only == "all":
         _add_decode(line, args, rank, world, device, hbm)
+    if not args.no_variants and args.only == "all":
+        _add_gdn(line, args, w, world, device, hbm)
 
     if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],
