@@ -26,7 +26,8 @@ KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED, KDA_ERR_CU
 KDA_BF16, KDA_F32 = 0, 1
 
 # every symbol include/kda.h declares
-EXPORTS = ("kda_forward", "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
+EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
+           "kda_forward_workspace_min_bytes", "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_last_cuda_error", "kda_launch_count",
            "kda_version")
 
@@ -56,6 +57,11 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_decode_step.restype = i
     lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
+    lib.kda_forward_ws.restype = i
+    lib.kda_forward_ws.argtypes = [vp] * 8 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
+    for name in ("kda_forward_workspace_bytes", "kda_forward_workspace_min_bytes"):
+        getattr(lib, name).restype = ctypes.c_size_t
+        getattr(lib, name).argtypes = [i] * 6
     lib.kda_gdn_forward.restype = i
     lib.kda_gdn_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_gdn_decode_step.restype = i
@@ -113,7 +119,7 @@ def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None):
 
 
 def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, final_state,
-             return_final_state, scale):
+             return_final_state, scale, workspace=None):
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -134,10 +140,19 @@ def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, fi
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     if final_state is not None:
         _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
-    fn = getattr(lib, entry)
-    st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-            _ptr(initial_state), _ptr(out), _ptr(final_state),
-            B, T, H, dk, dv, code, float(scale), _stream(dev))
+    if workspace is not None:
+        if workspace.device != dev or not workspace.is_contiguous():
+            raise ValueError("workspace must be a contiguous tensor on %s" % dev)
+        entry = "kda_forward_ws"
+        st = lib.kda_forward_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                _ptr(initial_state), _ptr(out), _ptr(final_state),
+                                B, T, H, dk, dv, code, float(scale), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(dev))
+    else:
+        fn = getattr(lib, entry)
+        st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                _ptr(initial_state), _ptr(out), _ptr(final_state),
+                B, T, H, dk, dv, code, float(scale), _stream(dev))
     _check(st, entry)
     return out, final_state
 
@@ -166,18 +181,36 @@ def _decode(entry, gate_shape, q, k, v, log_alpha, beta, state, out, scale):
 
 
 def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
-            return_final_state=True, scale: float = 0.0):
-    """Chunked KDA prefill (``kda_forward``).
+            return_final_state=True, scale: float = 0.0, workspace=None):
+    """Chunked KDA prefill (``kda_forward``, or ``kda_forward_ws`` with a workspace).
 
     q, k ``[B,T,H,dk]`` and v ``[B,T,H,dv]`` (bf16 or fp32, one dtype);
     log_alpha ``[B,T,H,dk]`` fp32; beta ``[B,T,H]`` fp32; initial_state
     ``[B,H,dk,dv]`` fp32 or None.  Returns ``(out [B,T,H,dv] fp32,
     final_state [B,H,dk,dv] fp32 or None)``.  ``final_state`` may be passed as
     the same tensor as ``initial_state`` to carry the state in place.
-    ``scale`` 0 means 1/sqrt(dk).
+    ``scale`` 0 means 1/sqrt(dk).  ``workspace``: a contiguous device tensor
+    (see :func:`workspace_bytes` / :func:`make_workspace`) enabling the
+    two-kernel prefill for bf16 inputs with dk = dv = 128.
     """
     return _forward("kda_forward", lambda B, T, H, dk: (B, T, H, dk), q, k, v, log_alpha, beta,
-                    initial_state, out, final_state, return_final_state, scale)
+                    initial_state, out, final_state, return_final_state, scale, workspace)
+
+
+def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, minimum=False) -> int:
+    """Workspace size for :func:`forward` (``kda_forward_workspace_bytes`` /
+    ``..._min_bytes``); 0 when the two-kernel prefill does not apply."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    fn = load().kda_forward_workspace_min_bytes if minimum else load().kda_forward_workspace_bytes
+    return int(fn(int(B), int(T), int(H), int(dk), int(dv), code))
+
+
+def make_workspace(B, T, H, dk, dv, dtype=torch.bfloat16, device="cuda", nbytes=None):
+    """A workspace tensor of ``workspace_bytes(...)`` bytes (or ``nbytes``), or None if not needed."""
+    n = workspace_bytes(B, T, H, dk, dv, dtype) if nbytes is None else int(nbytes)
+    if n == 0:
+        return None
+    return torch.empty(n, dtype=torch.uint8, device=device)
 
 
 def decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0):

@@ -59,7 +59,8 @@ namespace {
 kda_status forward_impl(const void *q, const void *k, const void *v, const float *log_alpha,
                         const float *beta, const float *initial_state, float *out, float *final_state,
                         int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
-                        void *stream, kda::GateKind gate)
+                        void *stream, kda::GateKind gate, void *workspace = nullptr,
+                        size_t workspace_bytes = 0)
 {
     g_last_cuda_error[0] = '\0';
     // ---- validation: nothing is enqueued unless every check passes
@@ -77,6 +78,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
         return KDA_ERR_MISALIGNED;
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_MISALIGNED;
+    if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDA_ERR_MISALIGNED;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
@@ -96,7 +98,10 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
     a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
     a.gate = gate;
     cudaError_t e;
-    if (!kda::prefill_tc_supported(a)) e = kda::launch_prefill_simt(a, st);
+    if (workspace && kda::prefill_split_supported(a) &&
+        workspace_bytes >= kda::prefill_split_workspace_min(B, T, H))
+        e = kda::launch_prefill_split(a, static_cast<uint8_t *>(workspace), workspace_bytes, st);
+    else if (!kda::prefill_tc_supported(a)) e = kda::launch_prefill_simt(a, st);
     else if (gate == kda::KDA_GATE_CHANNEL) e = kda::launch_prefill_tc(a, st);
     else e = kda::launch_prefill_gdn_tc(a, st);
     return e == cudaSuccess ? KDA_OK : cuda_fail(e);
@@ -145,6 +150,29 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
                         dtype, scale, stream, kda::KDA_GATE_CHANNEL);
 }
 
+size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (B <= 0 || H <= 0 || T <= 0 || dtype != KDA_BF16 || dk != 128 || dv != 128) return 0;
+    return kda::prefill_split_workspace_full(B, T, H);
+}
+
+size_t kda_forward_workspace_min_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (B <= 0 || H <= 0 || T <= 0 || dtype != KDA_BF16 || dk != 128 || dv != 128) return 0;
+    return kda::prefill_split_workspace_min(B, T, H);
+}
+
+kda_status kda_forward_ws(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta,
+                          const float *initial_state, float *out, float *final_state,
+                          int B, int T, int H, int dk, int dv,
+                          kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes,
+                          void *stream)
+{
+    return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                        dtype, scale, stream, kda::KDA_GATE_CHANNEL, workspace, workspace_bytes);
+}
+
 kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,
                            float *state_inout, float *out,
@@ -180,11 +208,12 @@ kda_status kda_check_status(void *stream)
     g_last_cuda_error[0] = '\0';
     cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) return cuda_fail(e);
-    unsigned int dev_status = 0, gdn_status = 0;
+    unsigned int dev_status = 0, gdn_status = 0, split_status = 0;
     e = kda::take_device_status(&dev_status);
     if (e == cudaSuccess) e = kda::take_gdn_device_status(&gdn_status);
+    if (e == cudaSuccess) e = kda::take_split_device_status(&split_status);
     if (e != cudaSuccess) return cuda_fail(e);
-    return (dev_status | gdn_status) ? KDA_ERR_TIMEOUT : KDA_OK;
+    return (dev_status | gdn_status | split_status) ? KDA_ERR_TIMEOUT : KDA_OK;
 }
 
 }  // extern "C"

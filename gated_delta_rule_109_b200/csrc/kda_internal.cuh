@@ -48,6 +48,13 @@ cudaError_t launch_prefill_tc(const ForwardArgs &a, cudaStream_t stream);
 // Tensor-core prefill with one decay per token and head (or none): bf16, dk = dv = 128.
 cudaError_t launch_prefill_gdn_tc(const ForwardArgs &a, cudaStream_t stream);
 cudaError_t take_gdn_device_status(unsigned int *status);
+// Two-kernel tensor-core prefill (chunk-local kernel, then the state chain) with a
+// caller-provided workspace: bf16, dk = dv = 128, per-channel gate.
+bool prefill_split_supported(const ForwardArgs &a);
+size_t prefill_split_workspace_full(int B, int T, int H);   // whole sequence in one block
+size_t prefill_split_workspace_min(int B, int T, int H);    // one chunk per block + state carry
+cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream);
+cudaError_t take_split_device_status(unsigned int *status);
 // Reads and clears the device status word the tensor-core kernels set when a
 // bounded wait gives up (bit 0).  Synchronous.
 cudaError_t take_device_status(unsigned int *status);

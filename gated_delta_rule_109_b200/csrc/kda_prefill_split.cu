@@ -1,0 +1,791 @@
+// Two-kernel chunked KDA prefill on the sm_100a tensor cores, bf16 inputs,
+// dk = dv = 128, fp32 state and outputs: the chunk-local work of every chunk
+// runs in parallel (prefill_prep_kernel), and only the short state chain runs
+// in sequence (prefill_chain_kernel).
+//
+// The token step is the one of "Kimi Delta Attention: The Linear Attention
+// Behind Kimi K2 and Qwen3", §How Kimi Delta Attention works step by step; the
+// sequence is processed chunkwise with the chunk-boundary state as the next
+// chunk's initial condition ("KDA Technical Deep Dive", §Systems and
+// implementation tradeoffs, Training).  Per (b, h) and chunk of c <= 64 tokens
+// with entering state S, G_t = in-chunk inclusive sum of log_alpha:
+//
+//   A = Diag(beta) strictly_lower([k_i . (e^{G_i - G_j}) k_j]),  M = scale lower([q_i . (e^{G_i - G_j}) k_j])
+//   R = (I + A)^-1 Diag(beta),  W = R (k e^G),  U = R V
+//   Delta = R (V - (k e^G) S) = U - W S          (row t = the token step's error e_t)
+//   O     = (scale q e^G) S + M Delta
+//   S    <- Diag(e^{G_last}) S + (k e^{G_last - G})^T Delta
+//
+// Nothing on the right of the first three lines depends on S, so
+// prefill_prep_kernel computes them for all chunks at once (one CTA per
+// (b, h, chunk)) and writes one record per chunk to a caller-provided
+// workspace; prefill_chain_kernel then walks the chunks of each (b, h) with two
+// tensor-core round trips per chunk:  D1 = [W ; Q~] S  ->  Delta = U - D1[0:64];
+// D2 = K^^T Delta, D3 = M Delta  ->  S update and O = D1[64:128] + D3.
+//
+// A and M come from one product [Kr ; Qr] Kb^T of the split exponentials
+// Kr = k e^{G-m}, Qr = scale q e^{G-m}, Kb = k e^{m-G} (m = the per-channel
+// midpoint of G over the chunk, so every factor is at most e^{range/2}); a chunk
+// whose decay range is too wide for that computes A and M pair by pair with
+// e^{G_i - G_j} <= 1 instead.  Every other exponential is at most 1.
+//
+// Precision: every derived fp32 operand X is split X = hi + lo (bf16 each) and a
+// product takes hi*hi + lo*hi + hi*lo (an exact bf16 input needs no lo part);
+// accumulation is fp32 in tensor memory.
+//
+// Records hold their tiles in the byte order of the no-swizzle canonical
+// operand layout (core matrices of 8 rows x 16 bytes), so the chain kernel
+// brings them into shared memory with plain cp.async.bulk copies.  Every
+// mbarrier wait is bounded; a wait that runs out records KDA_ERR_TIMEOUT in a
+// device status word and the CTA stops after its copies in flight have landed.
+#include "kda_tc_ptx.cuh"
+
+namespace kda {
+
+__device__ unsigned int g_split_device_status;   // bit 0: a bounded wait gave up
+
+namespace {
+
+using namespace tcx;
+
+constexpr int kC = 64, kDK = 128, kDV = 128, kDVS = 32, kNSL = kDV / kDVS, kNT = 256;
+constexpr float kGMaxTc = 40.f;
+constexpr int kPitch = 68;
+
+// ---------------------------------------------------------------- chunk record (bytes)
+// [W ; Q~]: K-major A tile (outer row 0..127, inner dk; rows 0..63 W, 64..127 Q~)
+constexpr uint32_t R_WQ = 0, R_WQ_LO = 32768;
+// K^ = k e^{G_last - G} read as the MN-major A tile of K^^T (outer token, inner dk)
+constexpr uint32_t R_KT = 65536, R_KT_LO = 81920;
+// M: rows 64..127 of a K-major A tile (outer row, inner token)
+constexpr uint32_t R_M = 98304, R_M_LO = 106496;
+// U fp32 [value slice][token][32];  e^{G_last} fp32 [dk]
+constexpr uint32_t R_U = 114688, R_GAM = 147456;
+constexpr uint32_t kRec = 147968;
+
+constexpr uint32_t RW_SO = 2048, RW_SI = 128;   // outer row or token (8 per group), inner dk (128)
+constexpr uint32_t H_SO = 1024, H_SI = 128;     // outer row, inner token (64)
+constexpr uint32_t S_SO = 512, S_SI = 128;      // outer dk or token (K), inner column (N = 32)
+
+// ---------------------------------------------------------------- prep kernel smem
+// Tiles are K-major with outer = token/row and inner = key channel (RW_SO/RW_SI):
+// [Kr; Qr] is the A of the first product, Kb its B, and the Kr rows are read
+// again (MN-major) as the B of W = R Kr.  Layout chosen so that what is free after
+// the first product (Qr, Kb) is contiguous enough for the solve.
+constexpr uint32_t PP_P = 0;            // [Kr hi ; Qr hi]  (Kr hi 0..16K, Qr hi 16K..32K)
+constexpr uint32_t PP_KB = 32768;       // Kb hi, Kb lo
+constexpr uint32_t PP_KB_LO = 49152;
+constexpr uint32_t PP_P_LO = 65536;     // [Kr lo ; Qr lo]
+constexpr uint32_t PP_V = 98304;        // V: MN-major B (outer token, inner column)
+constexpr uint32_t PP_BETA = 114688;    // fp32 [64]
+constexpr uint32_t PP_EM = PP_BETA + 256;   // fp32 [128]: e^{m} (1 on the wide path)
+constexpr uint32_t PP_MBAR = PP_EM + 512;
+constexpr uint32_t PP_TMEMP = PP_MBAR + 8;
+constexpr uint32_t PP_TOTAL = PP_TMEMP + 8;
+static_assert(PP_TOTAL <= 115712, "two CTAs per SM");
+// after the first product: fp32 A and T of the solve over Qr hi and Kb; R (K-major,
+// outer row, inner token) over Qr lo; a 128-row view of R hi or R lo stays in smem
+constexpr uint32_t PP_AMAT = 16384, PP_TMAT = PP_AMAT + 64 * kPitch * 4;
+constexpr uint32_t PP_R = 81920, PP_R_LO = PP_R + 8192;
+static_assert(PP_TMAT + 64 * kPitch * 4 <= PP_P_LO, "solve scratch");
+// wide-range path: G fp32 [64][128] over Qr hi and Kb hi, pairwise A (pitch 64) over Kb lo
+constexpr uint32_t PP_G = 16384, PP_AW = 49152;
+
+constexpr uint32_t TMP_AM = 0, TMP_W = 0, TMP_U = 128, TMP_COLS = 256;
+
+__global__ void __launch_bounds__(kNT, 2)
+prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                    const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
+                    const float *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
+                    int n0, int nb, float scale)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    float *sBeta = reinterpret_cast<float *>(smem + PP_BETA);
+    float *sEm = reinterpret_cast<float *>(smem + PP_EM);
+    const uint32_t mbar = sbase + PP_MBAR;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nloc = blockIdx.x % nb;                 // chunk within this block
+    const int bh = blockIdx.x / nb;
+    const int b = bh / H, h = bh % H;
+    const int t0 = (n0 + nloc) * kC;
+    const int c = min(kC, T - t0);
+    const int lrow = 32 * (warp & 3) + lane;          // tensor-memory lane of the readouts
+    const int half = warp >> 2;
+    const int ch0 = 16 * warp;                        // pass 1/2: channels ch0..ch0+15, tokens lane, lane+32
+    uint8_t *rec = ws + ((size_t)bh * nb + nloc) * kRec;
+    auto row = [&](int t) { return ((size_t)b * T + t0 + t) * H + h; };
+
+    // ---- loads: log_alpha of (token, 8 channels) (the scan needs it) and beta; V follows
+    // by cp.async once the V region has served as scratch for the per-channel scalars
+    float G[2][16];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const int t = lane + 32 * hf;
+        const bool ok = t < c;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            const size_t o = row(ok ? t : 0) * kDK + ch0 + 8 * g;
+            const float4 a0 = ok ? *reinterpret_cast<const float4 *>(log_alpha + o) : make_float4(0.f, 0.f, 0.f, 0.f);
+            const float4 a1 = ok ? *reinterpret_cast<const float4 *>(log_alpha + o + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
+            G[hf][8 * g + 0] = a0.x; G[hf][8 * g + 1] = a0.y; G[hf][8 * g + 2] = a0.z; G[hf][8 * g + 3] = a0.w;
+            G[hf][8 * g + 4] = a1.x; G[hf][8 * g + 5] = a1.y; G[hf][8 * g + 6] = a1.z; G[hf][8 * g + 7] = a1.w;
+        }
+    }
+    if (tid < kC) sBeta[tid] = (tid < c) ? beta[row(tid)] : 0.f;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(sbase + PP_TMEMP), "r"(TMP_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+
+    // ---- in-chunk inclusive sums over tokens (lanes), per channel; padded tokens add 0.
+    // Per channel: G_last (the sum up to the chunk's last token) and the reference
+    // point m midway between the first and last G (the extremes when the decay is
+    // monotone; every token is checked against it in the split pass).  Both go to
+    // shared memory (the V region, before V arrives).
+    float *sGm = reinterpret_cast<float *>(smem + PP_V);
+    float *sGl = sGm + kDK;
+#pragma unroll
+    for (int e = 0; e < 16; ++e) {
+        float a = G[0][e], bb = G[1][e];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float ua = __shfl_up_sync(0xffffffffu, a, o);
+            const float ub = __shfl_up_sync(0xffffffffu, bb, o);
+            if (lane >= o) { a += ua; bb += ub; }
+        }
+        bb += __shfl_sync(0xffffffffu, a, 31);
+        G[0][e] = a;
+        G[1][e] = bb;
+        const float g_l = __shfl_sync(0xffffffffu, bb, 31);
+        const float g_m = 0.5f * (__shfl_sync(0xffffffffu, a, 0) + g_l);
+        if (lane == e) {
+            sGm[ch0 + e] = g_m;
+            sGl[ch0 + e] = g_l;
+            sEm[ch0 + e] = __expf(g_m);
+            reinterpret_cast<float *>(rec + R_GAM)[ch0 + e] = __expf(g_l);
+        }
+    }
+    __syncwarp();
+
+    bool wide = false;      // some |G - m| > 40 (or |m| > 80): the split exponentials could overflow
+    // ---- split operands: [Kr; Qr], Kb (smem); Q~ rows of [W; Q~] and K^ (record).
+    // The wide path puts k e^G where Kr would be and keeps G for the pairwise sums.
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const int t = lane + 32 * hf;
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            // keep each item's loads inside its item (hoisting all of them costs 32 registers)
+            asm volatile("" ::: "memory");
+            float kk[8], qq[8], up[8], y[8];
+            {
+                const bool okt = t < c;
+                const size_t o = row(okt ? t : 0) * kDK + ch0 + 8 * g;
+                const uint4 kv = okt ? *reinterpret_cast<const uint4 *>(k + o) : make_uint4(0u, 0u, 0u, 0u);
+                const uint4 qv = okt ? *reinterpret_cast<const uint4 *>(q + o) : make_uint4(0u, 0u, 0u, 0u);
+                const __nv_bfloat16 *kb16 = reinterpret_cast<const __nv_bfloat16 *>(&kv);
+                const __nv_bfloat16 *qb16 = reinterpret_cast<const __nv_bfloat16 *>(&qv);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    kk[i] = __bfloat162float(kb16[i]);
+                    qq[i] = __bfloat162float(qb16[i]);
+                }
+            }
+            const uint32_t ok = core_off(t, ch0 + 8 * g, RW_SO, RW_SI);
+            const uint32_t oq = core_off(64 + t, ch0 + 8 * g, RW_SO, RW_SI);
+            uint4 hv, lv;
+            // Q~ = scale q e^G -> record
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = scale * qq[i] * __expf(G[hf][8 * g + i]);
+            split8(y, hv, lv);
+            *reinterpret_cast<uint4 *>(rec + R_WQ + oq) = hv;
+            *reinterpret_cast<uint4 *>(rec + R_WQ_LO + oq) = lv;
+            // K^ = k e^{G_last - G} -> record
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = kk[i] * __expf(sGl[ch0 + 8 * g + i] - G[hf][8 * g + i]);
+            split8(y, hv, lv);
+            *reinterpret_cast<uint4 *>(rec + R_KT + ok) = hv;
+            *reinterpret_cast<uint4 *>(rec + R_KT_LO + ok) = lv;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float g_m = sGm[ch0 + 8 * g + i];
+                const float x = G[hf][8 * g + i] - g_m;
+                wide |= !(fabsf(x) <= kGMaxTc && fabsf(g_m) <= 2.f * kGMaxTc);
+                up[i] = __expf(x);
+                y[i] = kk[i] * up[i];
+            }
+            st_split8(smem, PP_P + ok, PP_P_LO + ok, y);                       // Kr
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = scale * qq[i] * up[i];
+            st_split8(smem, PP_P + oq, PP_P_LO + oq, y);                       // Qr
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = kk[i] * __expf(sGm[ch0 + 8 * g + i] - G[hf][8 * g + i]);
+            st_split8(smem, PP_KB + ok, PP_KB_LO + ok, y);                     // Kb
+        }
+    }
+    const bool wide_path = __syncthreads_or(wide) != 0;
+    // V (exact bf16; rows past the chunk's end zero-filled) into its operand tile
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int id = tid + kNT * r, t = id >> 4, g = id & 15;
+        const bool okt = t < c;
+        cp_async16(sbase + PP_V + core_off(t, 8 * g, RW_SO, RW_SI), v + row(okt ? t : 0) * kDV + 8 * g,
+                   okt ? 16u : 0u);
+    }
+    cp_async_commit();
+    if (wide_path) {
+        // rare: redo the scan from the inputs, keep G for the pairwise sums and put
+        // k e^G where Kr was (W then needs no e^m factor)
+#pragma unroll 1
+        for (int hf = 0; hf < 2; ++hf) {
+            const int t = lane + 32 * hf;
+#pragma unroll 1
+            for (int e = 0; e < 16; ++e) {
+                const int chn = ch0 + e;
+                float a = (t < c) ? log_alpha[row(t) * kDK + chn] : 0.f;
+                float a0 = (lane < c) ? log_alpha[row(lane) * kDK + chn] : 0.f;
+#pragma unroll
+                for (int o = 1; o < 32; o <<= 1) {
+                    const float ua = __shfl_up_sync(0xffffffffu, a, o);
+                    const float u0 = __shfl_up_sync(0xffffffffu, a0, o);
+                    if (lane >= o) { a += ua; a0 += u0; }
+                }
+                if (hf) a += __shfl_sync(0xffffffffu, a0, 31);
+                reinterpret_cast<float *>(smem + PP_G)[t * kDK + chn] = a;
+            }
+        }
+        if (lane < 16) sEm[ch0 + lane] = 1.f;
+        __syncthreads();
+        for (int id = tid; id < kC * 16; id += kNT) {
+            const int t = id >> 4, cg = id & 15;
+            float y[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const float kk = (t < c) ? __bfloat162float(k[row(t) * kDK + 8 * cg + i]) : 0.f;
+                y[i] = kk * __expf(reinterpret_cast<const float *>(smem + PP_G)[t * kDK + 8 * cg + i]);
+            }
+            const uint32_t ok = core_off(t, 8 * cg, RW_SO, RW_SI);
+            st_split8(smem, PP_P + ok, PP_P_LO + ok, y);
+        }
+    }
+    proxy_fence();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + PP_TMEMP);
+    const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+    uint32_t phase = 0;
+    bool failed = false;
+
+    float *Am = reinterpret_cast<float *>(smem + PP_AMAT);
+    if (!wide_path) {
+        if (tid == 0) {
+            // [Kr; Qr] Kb^T: rows 0..63 -> A, rows 64..127 -> M
+            mma_split(tmem + TMP_AM, sbase + PP_P, sbase + PP_P_LO, RW_SI, RW_SO,
+                      sbase + PP_KB, sbase + PP_KB_LO, RW_SI, RW_SO, kDK / 16,
+                      idesc_bf16(128, 64, 0, 0), false);
+            umma_commit(mbar);
+        }
+        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
+        phase ^= 1;
+        if (!failed) {
+            tc_fence_after();
+            float x[32];
+            tmem_ld16(tmem + tlane + TMP_AM + 32 * half, *reinterpret_cast<float (*)[16]>(x));
+            tmem_ld16(tmem + tlane + TMP_AM + 32 * half + 16, *reinterpret_cast<float (*)[16]>(x + 16));
+            if (lrow < 64) {
+                const int i = lrow;
+                const float bi = sBeta[i];
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int j = 32 * half + e;
+                    Am[i * kPitch + j] = (j < i) ? bi * x[e] : 0.f;
+                }
+            } else {
+                const int i = lrow - 64;
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 32 * half + 8 * g + e;
+                        y[e] = (j <= i) ? x[8 * g + e] : 0.f;
+                    }
+                    uint4 hv, lv;
+                    split8(y, hv, lv);
+                    const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
+                    *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
+                    *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
+                }
+            }
+        }
+    } else {
+        // wide decay range: A and M pair by pair, every factor e^{G_i - G_j} <= 1
+        const float *sG = reinterpret_cast<const float *>(smem + PP_G);
+        float *Aw = reinterpret_cast<float *>(smem + PP_AW);
+        for (int item = tid; item < 2 * 64 * 8; item += kNT) {
+            const int isM = item >> 9, i = (item >> 3) & 63, jg = item & 7;
+            float y[8];
+#pragma unroll 1
+            for (int e = 0; e < 8; ++e) {
+                const int j = 8 * jg + e;
+                float acc = 0.f;
+                if (i < c && j < c && (isM ? j <= i : j < i)) {
+                    const __nv_bfloat16 *xi = (isM ? q : k) + row(i) * kDK;
+                    const __nv_bfloat16 *kj = k + row(j) * kDK;
+                    for (int cc = 0; cc < kDK; ++cc)
+                        acc += __bfloat162float(xi[cc]) * __bfloat162float(kj[cc]) *
+                               __expf(sG[i * kDK + cc] - sG[j * kDK + cc]);
+                }
+                y[e] = isM ? scale * acc : sBeta[i] * acc;
+            }
+            if (isM) {
+                uint4 hv, lv;
+                split8(y, hv, lv);
+                const uint32_t o = core_off(i, 8 * jg, H_SO, H_SI);
+                *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
+                *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e) Aw[i * 64 + 8 * jg + e] = y[e];
+            }
+        }
+        __syncthreads();
+        for (int id = tid; id < 64 * 64; id += kNT) Am[(id >> 6) * kPitch + (id & 63)] = Aw[id];
+    }
+    __syncthreads();
+
+    if (!failed) {
+        // ---- T = (I + A)^-1 by recursive doubling 16 -> 32 -> 64, fp32; R = T Diag(beta)
+        float *Tm = reinterpret_cast<float *>(smem + PP_TMAT);
+        if (tid < 64) {
+            const int blk = tid >> 4, j = tid & 15, o = 16 * blk;
+            float xs[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+                float s = (i == j) ? 1.f : 0.f;
+#pragma unroll
+                for (int l = 0; l < i; ++l) s -= Am[(o + i) * kPitch + o + l] * xs[l];
+                xs[i] = s;
+            }
+#pragma unroll
+            for (int i = 0; i < 16; ++i) Tm[(o + i) * kPitch + o + j] = xs[i];
+        } else {
+            for (int e = tid - 64; e < 6 * 256; e += kNT - 64) {
+                const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
+                const int rb = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
+                const int cb = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+                Tm[(16 * rb + i) * kPitch + 16 * cb + j] = 0.f;
+            }
+        }
+        __syncthreads();
+        const int p = tid >> 6, i16 = (tid >> 2) & 15, jq = tid & 3;
+        if (tid < 128) {
+            const int a = 2 * p + 1, bb = 2 * p;
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int l = 0; l < 16; ++l) {
+                const float av = Am[(16 * a + i16) * kPitch + 16 * bb + l];
+                const float4 tv = *reinterpret_cast<const float4 *>(Tm + (16 * bb + l) * kPitch + 16 * bb + 4 * jq);
+                y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
+            }
+            *reinterpret_cast<float4 *>(Am + (16 * bb + i16) * kPitch + 16 * a + 4 * jq) = y;
+        }
+        __syncthreads();
+        if (tid < 128) {
+            const int a = 2 * p + 1, bb = 2 * p;
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int l = 0; l < 16; ++l) {
+                const float tv = Tm[(16 * a + i16) * kPitch + 16 * a + l];
+                const float4 yv = *reinterpret_cast<const float4 *>(Am + (16 * bb + l) * kPitch + 16 * a + 4 * jq);
+                y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
+            }
+            *reinterpret_cast<float4 *>(Tm + (16 * a + i16) * kPitch + 16 * bb + 4 * jq) =
+                make_float4(-y.x, -y.y, -y.z, -y.w);
+        }
+        __syncthreads();
+        const int i32 = tid >> 3, jq8 = tid & 7;
+        {
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int l = 0; l < 32; ++l) {
+                const float av = Am[(32 + i32) * kPitch + l];
+                const float4 tv = *reinterpret_cast<const float4 *>(Tm + l * kPitch + 4 * jq8);
+                y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
+            }
+            *reinterpret_cast<float4 *>(Am + i32 * kPitch + 32 + 4 * jq8) = y;
+        }
+        __syncthreads();
+        {
+            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+            for (int l = 0; l < 32; ++l) {
+                const float tv = Tm[(32 + i32) * kPitch + 32 + l];
+                const float4 yv = *reinterpret_cast<const float4 *>(Am + l * kPitch + 32 + 4 * jq8);
+                y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
+            }
+            *reinterpret_cast<float4 *>(Tm + (32 + i32) * kPitch + 4 * jq8) =
+                make_float4(-y.x, -y.y, -y.z, -y.w);
+        }
+        __syncthreads();
+        for (int id = tid; id < 512; id += kNT) {
+            const int i = id >> 3, jg = id & 7;
+            const float4 t0v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg);
+            const float4 t1v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg + 4);
+            const float *bj = sBeta + 8 * jg;
+            float y[8] = {t0v.x * bj[0], t0v.y * bj[1], t0v.z * bj[2], t0v.w * bj[3],
+                          t1v.x * bj[4], t1v.y * bj[5], t1v.z * bj[6], t1v.w * bj[7]};
+            const uint32_t o = core_off(i, 8 * jg, H_SO, H_SI);
+            st_split8(smem, PP_R + o, PP_R_LO + o, y);
+        }
+        cp_async_wait_all();
+        proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // [R; .] Kr (Kr rows read MN-major as B) and [R; .] V; rows 0..63 are R Kr and U
+            mma_split(tmem + TMP_W, sbase + PP_R, sbase + PP_R_LO, H_SI, H_SO,
+                      sbase + PP_P, sbase + PP_P_LO, RW_SO, RW_SI, kC / 16,
+                      idesc_bf16(128, kDK, 0, 1), false);
+            mma_split(tmem + TMP_U, sbase + PP_R, sbase + PP_R_LO, H_SI, H_SO,
+                      sbase + PP_V, 0u, RW_SO, RW_SI, kC / 16,
+                      idesc_bf16(128, kDV, 0, 1), false, true, false);
+            umma_commit(mbar);
+        }
+        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
+        phase ^= 1;
+        if (!failed && lrow < 64) {
+            tc_fence_after();
+            // W = (R Kr) Diag(e^m): lane = row i, 64 key channels per thread
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                float x[16];
+                const int c0 = 64 * half + 16 * r;
+                tmem_ld16(tmem + tlane + TMP_W + c0, x);
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = x[8 * g + e] * sEm[c0 + 8 * g + e];
+                    uint4 hv, lv;
+                    split8(y, hv, lv);
+                    const uint32_t o = core_off(lrow, c0 + 8 * g, RW_SO, RW_SI);
+                    *reinterpret_cast<uint4 *>(rec + R_WQ + o) = hv;
+                    *reinterpret_cast<uint4 *>(rec + R_WQ_LO + o) = lv;
+                }
+            }
+            // U: 64 value columns per thread = two slices
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                float *dst = reinterpret_cast<float *>(rec + R_U + (2 * half + s2) * 8192) + lrow * kDVS;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[16];
+                    tmem_ld16(tmem + tlane + TMP_U + 64 * half + 32 * s2 + 16 * hh, x);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        reinterpret_cast<float4 *>(dst + 16 * hh)[g] =
+                            make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
+                }
+            }
+        }
+    }
+
+    if (failed && tid == 0) atomicOr(&g_split_device_status, 1u);
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMP_COLS) : "memory");
+    }
+}
+
+// ---------------------------------------------------------------- chain kernel smem
+constexpr uint32_t CH_WQ = 0;                        // two [W; Q~] slots, 64 KB each (hi, lo)
+constexpr uint32_t CH_KTM = 131072;                  // K^ hi, K^ lo, M hi, M lo (48 KB)
+constexpr uint32_t CH_MA = CH_KTM + 24576;           // 128-row view whose rows 64..127 are M hi
+constexpr uint32_t CH_MA_LO = CH_KTM + 32768;        //   ... and M lo
+constexpr uint32_t CH_U = CH_KTM + 49152;            // fp32 [64][32]
+constexpr uint32_t CH_GAM = CH_U + 8192;             // fp32 [128]
+constexpr uint32_t CH_S = CH_GAM + 512, CH_S_LO = CH_S + 8192;     // S: MN-major B (outer dk, inner column)
+constexpr uint32_t CH_DL = CH_S + 16384, CH_DL_LO = CH_DL + 4096;  // Delta: MN-major B (outer token)
+constexpr uint32_t CH_MBAR = CH_DL + 8192;           // mma, wq[2], ktm
+constexpr uint32_t CH_TMEMP = CH_MBAR + 32;
+constexpr uint32_t CH_TOTAL = CH_TMEMP + 16;
+static_assert(CH_TOTAL <= 232448, "shared memory");
+static_assert(R_KT_LO + 16384 == R_M && R_M + 16384 == R_U, "K^ and M are one contiguous copy");
+
+constexpr uint32_t TMC_D1 = 0, TMC_D2 = 32, TMC_D3 = 64, TMC_COLS = 128;
+
+__global__ void __launch_bounds__(kNT, 1)
+prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
+                     float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    const float *sU = reinterpret_cast<const float *>(smem + CH_U);
+    const float *sGam = reinterpret_cast<const float *>(smem + CH_GAM);
+    const uint32_t mbar = sbase + CH_MBAR, mbar_wq0 = mbar + 8, mbar_ktm = mbar + 24;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int slice = blockIdx.x % kNSL;
+    const int bh = blockIdx.x / kNSL;
+    const int b = bh / H, h = bh % H;
+    const int col0 = slice * kDVS;
+    const int lrow = 32 * (warp & 3) + lane;
+    const int half = warp >> 2;
+    const uint8_t *recs = ws + (size_t)bh * nb * kRec;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(sbase + CH_TMEMP), "r"(TMC_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        mbar_init(mbar_wq0, 1);
+        mbar_init(mbar_wq0 + 8, 1);
+        mbar_init(mbar_ktm, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + CH_TMEMP);
+    const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+
+    // copies of the streamed operands (thread 0); pending flags are kept by every thread
+    // pending copies: bit s of wq_pend = slot s armed and not yet waited for, bit s
+    // of wq_par = the parity that copy completes
+    uint32_t wq_pend = 0u, wq_par = 0u, ktm_par = 0u;
+    bool ktm_pending = false, failed = false;
+    auto load_wq = [&](int kk) {
+        const uint32_t mb = mbar_wq0 + 8u * (kk & 1);
+        const uint32_t bit = 1u << (kk & 1);
+        wq_pend |= bit;
+        wq_par = ((kk >> 1) & 1) ? (wq_par | bit) : (wq_par & ~bit);
+        if (tid == 0) {
+            mbar_expect_tx(mb, 65536u);
+            bulk_g2s(sbase + CH_WQ + 65536u * (kk & 1), recs + (size_t)kk * kRec + R_WQ, 65536u, mb);
+        }
+    };
+    auto load_ktm = [&](int kk) {
+        ktm_pending = true;
+        ktm_par = (uint32_t)kk & 1u;
+        if (tid == 0) {
+            const uint8_t *r = recs + (size_t)kk * kRec;
+            mbar_expect_tx(mbar_ktm, 49152u + 8192u + 512u);
+            bulk_g2s(sbase + CH_KTM, r + R_KT, 49152u, mbar_ktm);
+            bulk_g2s(sbase + CH_U, r + R_U + slice * 8192u, 8192u, mbar_ktm);
+            bulk_g2s(sbase + CH_GAM, r + R_GAM, 512u, mbar_ktm);
+        }
+    };
+
+    float S[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+        S[j] = s_in ? s_in[((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half + j] : 0.f;
+
+    uint32_t phase = 0;
+    load_wq(0);
+    if (nb > 1) load_wq(1);
+    load_ktm(0);
+
+    for (int kk = 0; kk < nb; ++kk) {
+        const int buf = kk & 1;
+        // ---- S as a split B operand; wait for this chunk's [W; Q~]
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+            float xv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) xv[e] = S[8 * g + e];
+            const uint32_t off = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
+            st_split8(smem, CH_S + off, CH_S_LO + off, xv);
+        }
+        failed = __syncthreads_or(!mbar_wait(mbar_wq0 + 8u * buf, (uint32_t)(kk >> 1) & 1u)) != 0;
+        if (failed) break;
+        wq_pend &= ~(1u << buf);
+        proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // D1 = [W; Q~] S
+            const uint32_t wq = sbase + CH_WQ + 65536u * buf;
+            mma_split(tmem + TMC_D1, wq, wq + 32768u, RW_SI, RW_SO, sbase + CH_S, sbase + CH_S_LO,
+                      S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
+            umma_commit(mbar);
+        }
+        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
+        phase ^= 1;
+        if (failed) break;
+        if (kk + 2 < nb) load_wq(kk + 2);   // this slot is free again: fetch two chunks ahead
+        tc_fence_after();
+        failed = __syncthreads_or(!mbar_wait(mbar_ktm, (uint32_t)kk & 1u)) != 0;
+        if (failed) break;
+        ktm_pending = false;
+
+        // ---- Delta = U - W S (rows 0..63); Q~ S kept for the output (rows 64..127)
+        float qs[16];
+        {
+            float x[16];
+            tmem_ld16(tmem + tlane + TMC_D1 + 16 * half, x);
+            if (lrow < 64) {
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    float d[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) d[e] = sU[lrow * kDVS + 16 * half + 8 * g + e] - x[8 * g + e];
+                    const uint32_t o = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
+                    st_split8(smem, CH_DL + o, CH_DL_LO + o, d);
+                }
+            }
+#pragma unroll
+            for (int e = 0; e < 16; ++e) qs[e] = x[e];
+        }
+        const float gam = sGam[lrow];
+        proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // D2 = K^^T Delta;  D3 = [. ; M] Delta
+            mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
+                      sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 1, 1), false);
+            mma_split(tmem + TMC_D3, sbase + CH_MA, sbase + CH_MA_LO, H_SI, H_SO,
+                      sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 0, 1), false);
+            umma_commit(mbar);
+        }
+        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
+        phase ^= 1;
+        if (failed) break;
+        if (kk + 1 < nb) load_ktm(kk + 1);
+        tc_fence_after();
+
+        // ---- S <- Diag(e^{G_last}) S + K^^T Delta;  O = Q~ S + M Delta
+        {
+            float x[16];
+            tmem_ld16(tmem + tlane + TMC_D2 + 16 * half, x);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + x[j];
+            if (lrow >= 64) {
+                float o2[16];
+                tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
+                const int t = (n0 + kk) * kC + lrow - 64;
+                if (t < T) {
+                    float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_float4(qs[4 * g] + o2[4 * g], qs[4 * g + 1] + o2[4 * g + 1],
+                                             qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
+                }
+            }
+        }
+        tc_fence_before();
+    }
+
+    if (failed) {
+        // let the copies still in flight land before shared memory is released (bounded)
+        if (tid == 0) {
+            for (int sl = 0; sl < 2; ++sl)
+                if ((wq_pend >> sl) & 1u) mbar_wait(mbar_wq0 + 8u * sl, (wq_par >> sl) & 1u);
+            if (ktm_pending) mbar_wait(mbar_ktm, ktm_par);
+            atomicOr(&g_split_device_status, 1u);
+        }
+    } else if (s_out) {
+        float4 *dst = reinterpret_cast<float4 *>(s_out + ((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half);
+#pragma unroll
+        for (int g = 0; g < 4; ++g) dst[g] = make_float4(S[4 * g], S[4 * g + 1], S[4 * g + 2], S[4 * g + 3]);
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMC_COLS) : "memory");
+    }
+}
+
+}  // namespace
+
+bool prefill_split_supported(const ForwardArgs &a)
+{
+    return a.dtype == KDA_BF16 && a.dk == kDK && a.dv == kDV && a.gate == KDA_GATE_CHANNEL;
+}
+
+size_t prefill_split_workspace_full(int B, int T, int H)
+{
+    const size_t nchunks = ((size_t)T + kC - 1) / kC;
+    return (size_t)B * H * nchunks * kRec;
+}
+
+size_t prefill_split_workspace_min(int B, int T, int H)
+{
+    const size_t bh = (size_t)B * H;
+    const size_t one = bh * kRec;
+    const size_t full = prefill_split_workspace_full(B, T, H);
+    return full <= one ? full : one + bh * kDK * kDV * sizeof(float);
+}
+
+// The sequence is processed in blocks of L chunks, L as large as the workspace
+// allows: prep over the block's chunks of every head, then the chain over them.
+// When L < the number of chunks, the state between blocks is carried in the
+// workspace after the records.
+cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream)
+{
+    const int nchunks = (a.T + kC - 1) / kC;
+    const size_t bh = (size_t)a.B * a.H;
+    const size_t per_chunk = bh * kRec;
+    const size_t state_bytes = bh * kDK * kDV * sizeof(float);
+    int L;
+    if (ws_bytes >= per_chunk * (size_t)nchunks) {
+        L = nchunks;
+    } else {
+        if (ws_bytes < per_chunk + state_bytes) return cudaErrorInvalidValue;
+        L = (int)((ws_bytes - state_bytes) / per_chunk);
+    }
+    float *carry = (L < nchunks) ? reinterpret_cast<float *>(ws + per_chunk * (size_t)L) : nullptr;
+    cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PP_TOTAL);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)CH_TOTAL);
+    if (e != cudaSuccess) return e;
+    for (int n0 = 0; n0 < nchunks; n0 += L) {
+        const int nb = min(L, nchunks - n0);
+        prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
+            static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
+            static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        note_launch();
+        const float *s_in = (n0 == 0) ? a.s0 : carry;
+        float *s_out = (n0 + nb >= nchunks) ? a.sT : carry;
+        prefill_chain_kernel<<<(unsigned)(bh * kNSL), kNT, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
+                                                                             a.H, n0, nb);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return e;
+        note_launch();
+    }
+    return cudaSuccess;
+}
+
+cudaError_t take_split_device_status(unsigned int *status)
+{
+    unsigned int zero = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(status, g_split_device_status, sizeof(unsigned int));
+    if (e != cudaSuccess) return e;
+    if (*status) e = cudaMemcpyToSymbol(g_split_device_status, &zero, sizeof(unsigned int));
+    return e;
+}
+
+}  // namespace kda

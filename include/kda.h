@@ -42,6 +42,8 @@
 #ifndef KDA_H
 #define KDA_H
 
+#include <stddef.h>
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -88,6 +90,49 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
                        const float *initial_state, float *out, float *final_state,
                        int B, int T, int H, int dk, int dv,
                        kda_dtype dtype, float scale, void *stream);
+
+/*
+ * kda_forward_ws -- kda_forward with a caller-provided device workspace.
+ *
+ * Same computation, arguments and results as kda_forward.  With bf16 inputs and
+ * dk = dv = 128 and a workspace of at least kda_forward_workspace_min_bytes(),
+ * the prefill runs as two kernels per block of chunks: one computes every
+ * chunk's chunk-local quantities in parallel (the in-chunk decay sums, A and
+ * its UT inverse, and the products that do not involve the state), writing one
+ * record per chunk into the workspace; the other walks the chunks of each
+ * (b, h) in order, carrying the state through them ("KDA Technical Deep
+ * Dive", §Systems and implementation tradeoffs, Training: chunk-local work in
+ * parallel, the boundary state seeding the next chunk).  With
+ * kda_forward_workspace_bytes() the whole sequence is one block; with less
+ * (but at least the minimum) the sequence is processed in blocks of as many
+ * chunks as fit, the state between blocks kept in the workspace.
+ *
+ *   workspace        device memory, 256-byte aligned, owned by the caller; its
+ *                    contents on entry do not matter and on return are
+ *                    unspecified.  It must not be used by another call that
+ *                    may run at the same time.
+ *   workspace_bytes  its size in bytes.
+ *
+ * With a NULL or too small workspace, or for other dtypes and head dimensions,
+ * the call is exactly kda_forward.  A workspace not 256-byte aligned is
+ * KDA_ERR_MISALIGNED.
+ */
+kda_status kda_forward_ws(const void *q, const void *k, const void *v,
+                          const float *log_alpha, const float *beta,
+                          const float *initial_state, float *out, float *final_state,
+                          int B, int T, int H, int dk, int dv,
+                          kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes,
+                          void *stream);
+
+/*
+ * Workspace sizes for kda_forward_ws: the size at which the whole sequence is
+ * one block (the fastest), and the smallest size that still takes the
+ * two-kernel path (one chunk per block plus the carried state).  Both are 0
+ * when the two-kernel path does not apply (dtype, head dimensions, T = 0 or
+ * bad sizes).  About 145 KB per chunk of 64 tokens per (b, h).
+ */
+size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
+size_t kda_forward_workspace_min_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 
 /*
  * kda_decode_step -- one token per sequence, state updated in place.

@@ -132,3 +132,56 @@ def test_binding_raises_when_library_missing(tmp_path):
 def test_binding_error_carries_status(lib):
     err = kda.KDAError(kda.KDA_ERR_UNSUPPORTED, "kda_forward")
     assert err.status == kda.KDA_ERR_UNSUPPORTED and "KDA_ERR_UNSUPPORTED" in str(err)
+
+
+def _gdn(lib, q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, out=FAKE, sT=None,
+         B=1, T=8, H=2, dk=128, dv=128, dtype=kda.KDA_BF16, scale=0.0):
+    return lib.kda_gdn_forward(q, k, v, la, beta, s0, out, sT, B, T, H, dk, dv, dtype,
+                               ctypes.c_float(scale), None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(beta=None), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=0), kda.KDA_ERR_INVALID_ARG),
+    (dict(dk=96), kda.KDA_ERR_UNSUPPORTED),
+    (dict(la=FAKE + 2), kda.KDA_ERR_MISALIGNED),      # the scalar gate needs 4-byte alignment only
+    (dict(v=FAKE + 8), kda.KDA_ERR_MISALIGNED),
+])
+def test_gdn_forward_rejects_bad_arguments_before_launch(lib, kw, code):
+    assert _gdn(lib, **kw) == code
+
+
+def test_gdn_decode_rejects_bad_arguments_before_launch(lib):
+    call = lambda **kw: lib.kda_gdn_decode_step(kw.get("q", FAKE), FAKE, FAKE, kw.get("la", FAKE), FAKE,
+                                                kw.get("st", FAKE), FAKE, 1, 2, 128, 128, kda.KDA_BF16,
+                                                ctypes.c_float(0.0), None)
+    assert call(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert call(st=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+    assert call(la=FAKE + 1) == kda.KDA_ERR_MISALIGNED
+
+
+def test_workspace_sizes(lib):
+    rec = 147968                                     # bytes per chunk record (b, h, chunk)
+    full = lambda *a: lib.kda_forward_workspace_bytes(*a)
+    mini = lambda *a: lib.kda_forward_workspace_min_bytes(*a)
+    assert full(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec
+    assert full(4, 16384, 32, 128, 128, kda.KDA_BF16) == 128 * 256 * rec
+    assert full(2, 65, 3, 128, 128, kda.KDA_BF16) == 6 * 2 * rec             # ragged tail: 2 chunks
+    assert mini(2, 65, 3, 128, 128, kda.KDA_BF16) == 6 * rec + 6 * 128 * 128 * 4
+    assert mini(2, 64, 3, 128, 128, kda.KDA_BF16) == full(2, 64, 3, 128, 128, kda.KDA_BF16) == 6 * rec
+    for args in [(1, 100, 2, 64, 64, kda.KDA_BF16), (1, 100, 2, 128, 128, kda.KDA_F32),
+                 (1, 0, 2, 128, 128, kda.KDA_BF16), (0, 10, 2, 128, 128, kda.KDA_BF16)]:
+        assert full(*args) == 0 and mini(*args) == 0
+    assert kda.workspace_bytes(1, 65536, 32, 128, 128) == 32 * 1024 * rec
+
+
+def test_forward_ws_validates_like_forward(lib):
+    def fws(ws=FAKE * 16, nbytes=1 << 30, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, out=FAKE, sT=None)
+        a.update(kw)
+        return lib.kda_forward_ws(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["out"], a["sT"],
+                                  1, 8, 2, 128, 128, kda.KDA_BF16, ctypes.c_float(0.0), ws, nbytes, None)
+    assert fws(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert fws(ws=FAKE + 16) == kda.KDA_ERR_MISALIGNED    # workspace must be 256-byte aligned
+    assert fws(la=FAKE + 4) == kda.KDA_ERR_MISALIGNED
