@@ -193,9 +193,10 @@ class ClockSampler:
 
 
 # ---------------------------------------------------------------- prefill
-def bench_prefill(w, K, W, device, gate="channel"):
-    """K timed launches of the prefill.  gate="channel": KDA (kda_forward);
-    "scalar": Gated DeltaNet (kda_gdn_forward) with channel 0 of the draw as the gate."""
+def bench_prefill(w, K, W, device, gate="channel", workspace=None):
+    """K timed launches of the prefill.  gate="channel": KDA (kda_forward, or
+    kda_forward_ws when a workspace is given); "scalar": Gated DeltaNet
+    (kda_gdn_forward) with channel 0 of the draw as the gate."""
     import torch
     import gated_delta_rule_109_b200 as kda
     from gated_delta_rule_109_b200 import inputs as I
@@ -203,6 +204,8 @@ def bench_prefill(w, K, W, device, gate="channel"):
     out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
     sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device) if w.final_state else None
     fwd = kda.forward
+    if workspace is not None:
+        fwd = lambda *a, **kw: kda.forward(*a, workspace=workspace, **kw)
     if gate == "scalar":
         x["log_alpha"] = x["log_alpha"][..., 0].contiguous()
         fwd = kda.gdn_forward
@@ -228,7 +231,7 @@ def bench_prefill(w, K, W, device, gate="channel"):
     return {"ms_total": sum(per), "ms_per_launch": per, "launches": launches, "x": x}
 
 
-def bench_prefill_e2e(w, K, W, device, x):
+def bench_prefill_e2e(w, K, W, device, x, workspace=None):
     """Same metric through the public API with pinned host inputs, copies inside the timed region."""
     import torch
     import gated_delta_rule_109_b200 as kda
@@ -250,7 +253,7 @@ def bench_prefill_e2e(w, K, W, device, x):
         if s0h is not None:
             s0d.copy_(s0h, non_blocking=True)
         kda.forward(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], s0d,
-                    out=out, final_state=sT, return_final_state=sT is not None)
+                    out=out, final_state=sT, return_final_state=sT is not None, workspace=workspace)
         out_h.copy_(out, non_blocking=True)
         if sT is not None:
             sT_h.copy_(sT, non_blocking=True)
@@ -462,6 +465,8 @@ def main(argv=None):
     ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
                     help="time only one kernel (profiling runs); the default times both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="time kda_forward without a workspace (the one-kernel prefill)")
     ap.add_argument("--no-variants", action="store_true",
                     help="skip the Gated DeltaNet timing on the prefill workload")
     args = ap.parse_args(argv)
@@ -496,9 +501,14 @@ def main(argv=None):
             print(json.dumps(line), flush=True)
         return 0
 
+    # the two-kernel prefill's workspace, allocated once outside every timed region
+    ws_bytes = 0 if args.no_workspace else kda.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=device) if ws_bytes else None
+    split = ws is not None
+
     clocks = ClockSampler(device)
     clocks.start()
-    pre = bench_prefill(w, args.steps, args.warmup, device)
+    pre = bench_prefill(w, args.steps, args.warmup, device, workspace=ws)
     clk = clocks.stop()
     ms_total = max_over_ranks(pre["ms_total"], device)
     tokens_per_step = w.B * w.T
@@ -512,23 +522,27 @@ def main(argv=None):
     achieved = alg_bytes / (ms_launch / 1e3) / 1e9
     tc = (w.dtype == "bf16" and w.dk == 128 and w.dv == 128)   # the library's dispatch rule
     kname, ksrc = ("prefill_tc_kernel", "kda_prefill_tc.cu") if tc else ("prefill_simt_kernel", "kda_prefill_simt.cu")
+    if split:
+        kname, ksrc = "prefill_prep_kernel + prefill_chain_kernel", "kda_prefill_split.cu"
     traffic = measured_traffic(ksrc, w.name)
     alg_flops = w.B * w.T * w.H * prefill_flops_per_token_head(w.dk)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                 "frac": achieved / hbm, "traffic": traffic,
                 "kernel": kname, "algorithmic_bytes_per_launch": alg_bytes,
-                "ms_per_launch": ms_launch, "peak_source": peak_src + " HBM copy (MEASURED_PEAKS.json hbm_gbs)",
+                "ms_per_launch": ms_launch,
+                "launch": "one kda_forward_ws call (both kernels)" if split else "one kernel launch", "peak_source": peak_src + " HBM copy (MEASURED_PEAKS.json hbm_gbs)",
                 "tensor_view": {"algorithmic_flops_per_launch": alg_flops,
                                 "achieved_tflops": alg_flops / (ms_launch / 1e3) / 1e12,
                                 "peak_tflops": tf_burst,
                                 "frac": alg_flops / (ms_launch / 1e3) / 1e12 / tf_burst}}
 
-    e2e = bench_prefill_e2e(w, args.e2e_steps, 1, device, pre["x"])
+    e2e = bench_prefill_e2e(w, args.e2e_steps, 1, device, pre["x"], workspace=ws)
     e2e_ms = max_over_ranks(e2e["ms_total"], device)
     cb = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cb = oracle_sample(w, pre["x"], args.cpu_budget_s)
     del pre["x"]
+    del ws
     torch.cuda.empty_cache()
 
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
@@ -537,6 +551,8 @@ def main(argv=None):
             "dtype": "bf16" if tc else "f32", "data": "synthetic",
             "arithmetic": ("tcgen05 bf16 products of hi/lo-split operands (3 terms), fp32 accumulation "
                            "in tensor memory, fp32 CUDA-core solve and scans") if tc else "fp32 CUDA cores",
+            "path": ("two kernels per call (chunk-local records in a %.2f GB caller workspace, then the "
+                     "state chain)" % (ws_bytes / 1e9)) if split else "one fused kernel per call",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "input_dtype": w.dtype, "chunk": 64, "final_state": w.final_state,
                        "l2": "no flush: inputs %.2f GB per step > 126 MB L2" % (alg_bytes / 1e9),

@@ -10,24 +10,25 @@
 // implementation tradeoffs, Training).  Per (b, h) and chunk of c <= 64 tokens
 // with entering state S, G_t = in-chunk inclusive sum of log_alpha:
 //
-//   A = Diag(beta) strictly_lower([k_i . (e^{G_i - G_j}) k_j]),  M = scale lower([q_i . (e^{G_i - G_j}) k_j])
-//   R = (I + A)^-1 Diag(beta),  W = R (k e^G),  U = R V
-//   Delta = R (V - (k e^G) S) = U - W S          (row t = the token step's error e_t)
-//   O     = (scale q e^G) S + M Delta
-//   S    <- Diag(e^{G_last}) S + (k e^{G_last - G})^T Delta
+//   Kr = k e^{G-m},  Qr = scale q e^{G-m},  Kb = k e^{m-G}      (m: per-channel reference point)
+//   A = Diag(beta) strictly_lower(Kr Kb^T),  M = lower(Qr Kb^T)
+//   R = (I + A)^-1 Diag(beta),  Wr = R Kr,  U = R V
+//   S'    = Diag(e^m) S
+//   Delta = R (V - (k e^G) S) = U - Wr S'         (row t = the token step's error e_t)
+//   O     = Qr S' + M Delta
+//   S    <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta
 //
-// Nothing on the right of the first three lines depends on S, so
-// prefill_prep_kernel computes them for all chunks at once (one CTA per
+// Nothing above except S', Delta, O and the update depends on S, so
+// prefill_prep_kernel computes it for all chunks at once (one CTA per
 // (b, h, chunk)) and writes one record per chunk to a caller-provided
 // workspace; prefill_chain_kernel then walks the chunks of each (b, h) with two
-// tensor-core round trips per chunk:  D1 = [W ; Q~] S  ->  Delta = U - D1[0:64];
-// D2 = K^^T Delta, D3 = M Delta  ->  S update and O = D1[64:128] + D3.
+// tensor-core round trips per chunk:  D1 = [Wr ; Qr] S'  ->  Delta = U - D1[0:64];
+// D2 = Kb^T Delta, D3 = M Delta  ->  S update and O = D1[64:128] + D3.
 //
-// A and M come from one product [Kr ; Qr] Kb^T of the split exponentials
-// Kr = k e^{G-m}, Qr = scale q e^{G-m}, Kb = k e^{m-G} (m = the per-channel
-// midpoint of G over the chunk, so every factor is at most e^{range/2}); a chunk
-// whose decay range is too wide for that computes A and M pair by pair with
-// e^{G_i - G_j} <= 1 instead.  Every other exponential is at most 1.
+// m is the midpoint of the chunk's first and last G, so each split factor is at
+// most e^{range/2} for a monotone decay; a chunk where some |G - m| > 40 instead
+// computes A and M pair by pair with e^{G_i - G_j} <= 1 and stores k e^G, scale
+// q e^G and k e^{G_last - G} in place of Kr, Qr and Kb (with e^m = e^{G_last - m} = 1).
 //
 // Precision: every derived fp32 operand X is split X = hi + lo (bf16 each) and a
 // product takes hi*hi + lo*hi + hi*lo (an exact bf16 input needs no lo part);
@@ -53,15 +54,17 @@ constexpr float kGMaxTc = 40.f;
 constexpr int kPitch = 68;
 
 // ---------------------------------------------------------------- chunk record (bytes)
-// [W ; Q~]: K-major A tile (outer row 0..127, inner dk; rows 0..63 W, 64..127 Q~)
-constexpr uint32_t R_WQ = 0, R_WQ_LO = 32768;
-// K^ = k e^{G_last - G} read as the MN-major A tile of K^^T (outer token, inner dk)
-constexpr uint32_t R_KT = 65536, R_KT_LO = 81920;
+// [Wr ; Qr]: K-major A tile (outer row 0..127, inner dk), then e^m fp32 [dk]
+constexpr uint32_t R_WQ = 0, R_WQ_LO = 32768, R_EM = 65536;
+constexpr uint32_t kWqBytes = 65536 + 512;
+// Kb read as the MN-major A tile of Kb^T (outer token, inner dk)
+constexpr uint32_t R_KT = R_WQ + kWqBytes, R_KT_LO = R_KT + 16384;
 // M: rows 64..127 of a K-major A tile (outer row, inner token)
-constexpr uint32_t R_M = 98304, R_M_LO = 106496;
-// U fp32 [value slice][token][32];  e^{G_last} fp32 [dk]
-constexpr uint32_t R_U = 114688, R_GAM = 147456;
-constexpr uint32_t kRec = 147968;
+constexpr uint32_t R_M = R_KT + 32768, R_M_LO = R_M + 8192;
+// U fp32 [value slice][token][32];  e^{G_last} and e^{G_last - m} fp32 [dk] each
+constexpr uint32_t R_U = R_M + 16384, R_GAM = R_U + 32768, R_EL = R_GAM + 512;
+constexpr uint32_t kRec = R_EL + 512;
+static_assert(kRec % 16 == 0 && R_KT % 16 == 0, "bulk-copy alignment");
 
 constexpr uint32_t RW_SO = 2048, RW_SI = 128;   // outer row or token (8 per group), inner dk (128)
 constexpr uint32_t H_SO = 1024, H_SI = 128;     // outer row, inner token (64)
@@ -78,8 +81,7 @@ constexpr uint32_t PP_KB_LO = 49152;
 constexpr uint32_t PP_P_LO = 65536;     // [Kr lo ; Qr lo]
 constexpr uint32_t PP_V = 98304;        // V: MN-major B (outer token, inner column)
 constexpr uint32_t PP_BETA = 114688;    // fp32 [64]
-constexpr uint32_t PP_EM = PP_BETA + 256;   // fp32 [128]: e^{m} (1 on the wide path)
-constexpr uint32_t PP_MBAR = PP_EM + 512;
+constexpr uint32_t PP_MBAR = PP_BETA + 256;
 constexpr uint32_t PP_TMEMP = PP_MBAR + 8;
 constexpr uint32_t PP_TOTAL = PP_TMEMP + 8;
 static_assert(PP_TOTAL <= 115712, "two CTAs per SM");
@@ -102,7 +104,6 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
     float *sBeta = reinterpret_cast<float *>(smem + PP_BETA);
-    float *sEm = reinterpret_cast<float *>(smem + PP_EM);
     const uint32_t mbar = sbase + PP_MBAR;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -169,15 +170,15 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         if (lane == e) {
             sGm[ch0 + e] = g_m;
             sGl[ch0 + e] = g_l;
-            sEm[ch0 + e] = __expf(g_m);
+            reinterpret_cast<float *>(rec + R_EM)[ch0 + e] = __expf(g_m);
             reinterpret_cast<float *>(rec + R_GAM)[ch0 + e] = __expf(g_l);
+            reinterpret_cast<float *>(rec + R_EL)[ch0 + e] = __expf(g_l - g_m);
         }
     }
     __syncwarp();
 
     bool wide = false;      // some |G - m| > 40 (or |m| > 80): the split exponentials could overflow
-    // ---- split operands: [Kr; Qr], Kb (smem); Q~ rows of [W; Q~] and K^ (record).
-    // The wide path puts k e^G where Kr would be and keeps G for the pairwise sums.
+    // ---- split operands: Kr (smem), Qr and Kb (smem and record)
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
         const int t = lane + 32 * hf;
@@ -202,18 +203,6 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             const uint32_t ok = core_off(t, ch0 + 8 * g, RW_SO, RW_SI);
             const uint32_t oq = core_off(64 + t, ch0 + 8 * g, RW_SO, RW_SI);
             uint4 hv, lv;
-            // Q~ = scale q e^G -> record
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = scale * qq[i] * __expf(G[hf][8 * g + i]);
-            split8(y, hv, lv);
-            *reinterpret_cast<uint4 *>(rec + R_WQ + oq) = hv;
-            *reinterpret_cast<uint4 *>(rec + R_WQ_LO + oq) = lv;
-            // K^ = k e^{G_last - G} -> record
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = kk[i] * __expf(sGl[ch0 + 8 * g + i] - G[hf][8 * g + i]);
-            split8(y, hv, lv);
-            *reinterpret_cast<uint4 *>(rec + R_KT + ok) = hv;
-            *reinterpret_cast<uint4 *>(rec + R_KT_LO + ok) = lv;
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const float g_m = sGm[ch0 + 8 * g + i];
@@ -225,10 +214,18 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             st_split8(smem, PP_P + ok, PP_P_LO + ok, y);                       // Kr
 #pragma unroll
             for (int i = 0; i < 8; ++i) y[i] = scale * qq[i] * up[i];
-            st_split8(smem, PP_P + oq, PP_P_LO + oq, y);                       // Qr
+            split8(y, hv, lv);                                                 // Qr
+            *reinterpret_cast<uint4 *>(smem + PP_P + oq) = hv;
+            *reinterpret_cast<uint4 *>(smem + PP_P_LO + oq) = lv;
+            *reinterpret_cast<uint4 *>(rec + R_WQ + oq) = hv;
+            *reinterpret_cast<uint4 *>(rec + R_WQ_LO + oq) = lv;
 #pragma unroll
             for (int i = 0; i < 8; ++i) y[i] = kk[i] * __expf(sGm[ch0 + 8 * g + i] - G[hf][8 * g + i]);
-            st_split8(smem, PP_KB + ok, PP_KB_LO + ok, y);                     // Kb
+            split8(y, hv, lv);                                                 // Kb
+            *reinterpret_cast<uint4 *>(smem + PP_KB + ok) = hv;
+            *reinterpret_cast<uint4 *>(smem + PP_KB_LO + ok) = lv;
+            *reinterpret_cast<uint4 *>(rec + R_KT + ok) = hv;
+            *reinterpret_cast<uint4 *>(rec + R_KT_LO + ok) = lv;
         }
     }
     const bool wide_path = __syncthreads_or(wide) != 0;
@@ -242,8 +239,9 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
     cp_async_commit();
     if (wide_path) {
-        // rare: redo the scan from the inputs, keep G for the pairwise sums and put
-        // k e^G where Kr was (W then needs no e^m factor)
+        // rare: redo the scan from the inputs and keep G for the pairwise sums; put
+        // k e^G, scale q e^G and k e^{G_last - G} where Kr, Qr and Kb were, and set
+        // e^m = e^{G_last - m} = 1 in the record
 #pragma unroll 1
         for (int hf = 0; hf < 2; ++hf) {
             const int t = lane + 32 * hf;
@@ -262,18 +260,36 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 reinterpret_cast<float *>(smem + PP_G)[t * kDK + chn] = a;
             }
         }
-        if (lane < 16) sEm[ch0 + lane] = 1.f;
+        if (lane < 16) {
+            reinterpret_cast<float *>(rec + R_EM)[ch0 + lane] = 1.f;
+            reinterpret_cast<float *>(rec + R_EL)[ch0 + lane] = 1.f;
+        }
         __syncthreads();
+        const float *sG = reinterpret_cast<const float *>(smem + PP_G);
         for (int id = tid; id < kC * 16; id += kNT) {
             const int t = id >> 4, cg = id & 15;
-            float y[8];
+            float y1[8], y2[8], y3[8];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float kk = (t < c) ? __bfloat162float(k[row(t) * kDK + 8 * cg + i]) : 0.f;
-                y[i] = kk * __expf(reinterpret_cast<const float *>(smem + PP_G)[t * kDK + 8 * cg + i]);
+                const int chn = 8 * cg + i;
+                const float kk = (t < c) ? __bfloat162float(k[row(t) * kDK + chn]) : 0.f;
+                const float qq = (t < c) ? __bfloat162float(q[row(t) * kDK + chn]) : 0.f;
+                const float gg = sG[t * kDK + chn];
+                const float eg = __expf(gg);
+                y1[i] = kk * eg;
+                y2[i] = scale * qq * eg;
+                y3[i] = kk * __expf(sG[(kC - 1) * kDK + chn] - gg);
             }
             const uint32_t ok = core_off(t, 8 * cg, RW_SO, RW_SI);
-            st_split8(smem, PP_P + ok, PP_P_LO + ok, y);
+            const uint32_t oq = core_off(64 + t, 8 * cg, RW_SO, RW_SI);
+            st_split8(smem, PP_P + ok, PP_P_LO + ok, y1);
+            uint4 hv, lv;
+            split8(y2, hv, lv);
+            *reinterpret_cast<uint4 *>(rec + R_WQ + oq) = hv;
+            *reinterpret_cast<uint4 *>(rec + R_WQ_LO + oq) = lv;
+            split8(y3, hv, lv);
+            *reinterpret_cast<uint4 *>(rec + R_KT + ok) = hv;
+            *reinterpret_cast<uint4 *>(rec + R_KT_LO + ok) = lv;
         }
     }
     proxy_fence();
@@ -305,9 +321,14 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 const int i = lrow;
                 const float bi = sBeta[i];
 #pragma unroll
-                for (int e = 0; e < 32; ++e) {
-                    const int j = 32 * half + e;
-                    Am[i * kPitch + j] = (j < i) ? bi * x[e] : 0.f;
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    float y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 32 * half + 4 * e4 + e;
+                        y[e] = (j < i) ? bi * x[4 * e4 + e] : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(Am + i * kPitch + 32 * half + 4 * e4) = make_float4(y[0], y[1], y[2], y[3]);
                 }
             } else {
                 const int i = lrow - 64;
@@ -466,7 +487,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         phase ^= 1;
         if (!failed && lrow < 64) {
             tc_fence_after();
-            // W = (R Kr) Diag(e^m): lane = row i, 64 key channels per thread
+            // Wr = R Kr: lane = row i, 64 key channels per thread
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 float x[16];
@@ -476,7 +497,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 for (int g = 0; g < 2; ++g) {
                     float y[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) y[e] = x[8 * g + e] * sEm[c0 + 8 * g + e];
+                    for (int e = 0; e < 8; ++e) y[e] = x[8 * g + e];
                     uint4 hv, lv;
                     split8(y, hv, lv);
                     const uint32_t o = core_off(lrow, c0 + 8 * g, RW_SO, RW_SI);
@@ -511,19 +532,20 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 }
 
 // ---------------------------------------------------------------- chain kernel smem
-constexpr uint32_t CH_WQ = 0;                        // two [W; Q~] slots, 64 KB each (hi, lo)
-constexpr uint32_t CH_KTM = 131072;                  // K^ hi, K^ lo, M hi, M lo (48 KB)
+constexpr uint32_t CH_WQ = 0;                        // two slots of [Wr; Qr] (hi, lo) and e^m
+constexpr uint32_t CH_KTM = 2 * kWqBytes;            // Kb hi, Kb lo, M hi, M lo (48 KB)
 constexpr uint32_t CH_MA = CH_KTM + 24576;           // 128-row view whose rows 64..127 are M hi
 constexpr uint32_t CH_MA_LO = CH_KTM + 32768;        //   ... and M lo
 constexpr uint32_t CH_U = CH_KTM + 49152;            // fp32 [64][32]
-constexpr uint32_t CH_GAM = CH_U + 8192;             // fp32 [128]
-constexpr uint32_t CH_S = CH_GAM + 512, CH_S_LO = CH_S + 8192;     // S: MN-major B (outer dk, inner column)
+constexpr uint32_t CH_GAM = CH_U + 8192;             // fp32 [128] e^{G_last}, then [128] e^{G_last - m}
+constexpr uint32_t CH_S = CH_GAM + 1024, CH_S_LO = CH_S + 8192;    // S': MN-major B (outer dk, inner column)
 constexpr uint32_t CH_DL = CH_S + 16384, CH_DL_LO = CH_DL + 4096;  // Delta: MN-major B (outer token)
 constexpr uint32_t CH_MBAR = CH_DL + 8192;           // mma, wq[2], ktm
 constexpr uint32_t CH_TMEMP = CH_MBAR + 32;
 constexpr uint32_t CH_TOTAL = CH_TMEMP + 16;
 static_assert(CH_TOTAL <= 232448, "shared memory");
-static_assert(R_KT_LO + 16384 == R_M && R_M + 16384 == R_U, "K^ and M are one contiguous copy");
+static_assert(R_KT_LO + 16384 == R_M && R_M + 16384 == R_U, "Kb and M are one contiguous copy");
+static_assert(R_GAM + 512 == R_EL, "e^{G_last} and e^{G_last - m} are one contiguous copy");
 
 constexpr uint32_t TMC_D1 = 0, TMC_D2 = 32, TMC_D3 = 64, TMC_COLS = 128;
 
@@ -575,8 +597,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
         wq_pend |= bit;
         wq_par = ((kk >> 1) & 1) ? (wq_par | bit) : (wq_par & ~bit);
         if (tid == 0) {
-            mbar_expect_tx(mb, 65536u);
-            bulk_g2s(sbase + CH_WQ + 65536u * (kk & 1), recs + (size_t)kk * kRec + R_WQ, 65536u, mb);
+            mbar_expect_tx(mb, kWqBytes);
+            bulk_g2s(sbase + CH_WQ + kWqBytes * (kk & 1), recs + (size_t)kk * kRec + R_WQ, kWqBytes, mb);
         }
     };
     auto load_ktm = [&](int kk) {
@@ -584,10 +606,10 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
         ktm_par = (uint32_t)kk & 1u;
         if (tid == 0) {
             const uint8_t *r = recs + (size_t)kk * kRec;
-            mbar_expect_tx(mbar_ktm, 49152u + 8192u + 512u);
+            mbar_expect_tx(mbar_ktm, 49152u + 8192u + 1024u);
             bulk_g2s(sbase + CH_KTM, r + R_KT, 49152u, mbar_ktm);
             bulk_g2s(sbase + CH_U, r + R_U + slice * 8192u, 8192u, mbar_ktm);
-            bulk_g2s(sbase + CH_GAM, r + R_GAM, 512u, mbar_ktm);
+            bulk_g2s(sbase + CH_GAM, r + R_GAM, 1024u, mbar_ktm);
         }
     };
 
@@ -601,41 +623,47 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     if (nb > 1) load_wq(1);
     load_ktm(0);
 
-    for (int kk = 0; kk < nb; ++kk) {
+    // S' = Diag(e^m) S as a split B operand, then D1 = [Wr; Qr] S' for chunk kk
+    // (thread 0 issues)
+    auto issue_rt1 = [&](int kk) -> bool {
         const int buf = kk & 1;
-        // ---- S as a split B operand; wait for this chunk's [W; Q~]
+        const bool bad = !mbar_wait(mbar_wq0 + 8u * buf, (uint32_t)(kk >> 1) & 1u);
+        const float em = bad ? 0.f : reinterpret_cast<const float *>(smem + CH_WQ + kWqBytes * buf + 65536u)[lrow];
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
             float xv[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) xv[e] = S[8 * g + e];
+            for (int e = 0; e < 8; ++e) xv[e] = em * S[8 * g + e];
             const uint32_t off = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
             st_split8(smem, CH_S + off, CH_S_LO + off, xv);
         }
-        failed = __syncthreads_or(!mbar_wait(mbar_wq0 + 8u * buf, (uint32_t)(kk >> 1) & 1u)) != 0;
-        if (failed) break;
-        wq_pend &= ~(1u << buf);
         proxy_fence();
         tc_fence_before();
-        __syncthreads();
+        if (__syncthreads_or(bad)) return false;
+        wq_pend &= ~(1u << buf);
         if (tid == 0) {
             tc_fence_after();
-            // D1 = [W; Q~] S
-            const uint32_t wq = sbase + CH_WQ + 65536u * buf;
+            const uint32_t wq = sbase + CH_WQ + kWqBytes * buf;
             mma_split(tmem + TMC_D1, wq, wq + 32768u, RW_SI, RW_SO, sbase + CH_S, sbase + CH_S_LO,
                       S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
             umma_commit(mbar);
         }
-        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
-        phase ^= 1;
-        if (failed) break;
-        if (kk + 2 < nb) load_wq(kk + 2);   // this slot is free again: fetch two chunks ahead
-        tc_fence_after();
-        failed = __syncthreads_or(!mbar_wait(mbar_ktm, (uint32_t)kk & 1u)) != 0;
-        if (failed) break;
-        ktm_pending = false;
+        return true;
+    };
 
-        // ---- Delta = U - W S (rows 0..63); Q~ S kept for the output (rows 64..127)
+    failed = !issue_rt1(0);
+    for (int kk = 0; kk < nb && !failed; ++kk) {
+        // ---- D1 of chunk kk and its K^, M, U, e^{G_last}
+        {
+            const bool bad = !mbar_wait(mbar, phase) || !mbar_wait(mbar_ktm, (uint32_t)kk & 1u);
+            phase ^= 1;
+            if (__syncthreads_or(bad)) { failed = true; break; }
+        }
+        ktm_pending = false;
+        if (kk + 2 < nb) load_wq(kk + 2);   // slot kk & 1 is free again: fetch two chunks ahead
+        tc_fence_after();
+
+        // ---- Delta = U - Wr S' (rows 0..63); Qr S' kept for the output (rows 64..127)
         float qs[16];
         {
             float x[16];
@@ -653,42 +681,48 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
 #pragma unroll
             for (int e = 0; e < 16; ++e) qs[e] = x[e];
         }
-        const float gam = sGam[lrow];
+        const float gam = sGam[lrow], el = sGam[kDK + lrow];
         proxy_fence();
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            // D2 = K^^T Delta;  D3 = [. ; M] Delta
+            // D2 = Kb^T Delta;  D3 = [. ; M] Delta
             mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
                       sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 1, 1), false);
             mma_split(tmem + TMC_D3, sbase + CH_MA, sbase + CH_MA_LO, H_SI, H_SO,
                       sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 0, 1), false);
             umma_commit(mbar);
         }
-        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
-        phase ^= 1;
-        if (failed) break;
+        {
+            const bool bad = !mbar_wait(mbar, phase);
+            phase ^= 1;
+            if (__syncthreads_or(bad)) { failed = true; break; }
+        }
         if (kk + 1 < nb) load_ktm(kk + 1);
         tc_fence_after();
 
-        // ---- S <- Diag(e^{G_last}) S + K^^T Delta;  O = Q~ S + M Delta
+        // ---- S <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta, and the next
+        // chunk's first product
         {
             float x[16];
             tmem_ld16(tmem + tlane + TMC_D2 + 16 * half, x);
 #pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + x[j];
-            if (lrow >= 64) {
-                float o2[16];
-                tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
-                const int t = (n0 + kk) * kC + lrow - 64;
-                if (t < T) {
-                    float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
+            for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + el * x[j];
+        }
+        if (kk + 1 < nb && !issue_rt1(kk + 1)) { failed = true; break; }
+
+        // ---- O = Qr S' + M Delta of chunk kk, while the tensor cores run chunk kk + 1
+        if (lrow >= 64) {
+            float o2[16];
+            tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
+            const int t = (n0 + kk) * kC + lrow - 64;
+            if (t < T) {
+                float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_float4(qs[4 * g] + o2[4 * g], qs[4 * g + 1] + o2[4 * g + 1],
-                                             qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
-                }
+                for (int g = 0; g < 4; ++g)
+                    dst[g] = make_float4(qs[4 * g] + o2[4 * g], qs[4 * g + 1] + o2[4 * g + 1],
+                                         qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
             }
         }
         tc_fence_before();

@@ -132,22 +132,29 @@ __device__ __forceinline__ void st_split8(uint8_t *smem, uint32_t off_hi, uint32
 
 // One product D (+)= A B on bf16 hi/lo split operands: hi*hi, plus lo*hi when A has
 // a lo part and hi*lo when B has one (an operand without a lo part is an exact
-// bf16 input).  Each term walks K in `ksteps` steps of 16 (two core matrices).
+// bf16 input).  Each term walks K in `ksteps` steps of 16 (two core matrices,
+// 2 * LBO bytes).  The descriptors are built once; a K step adds 2 * LBO / 16 to
+// their address field (every operand lies below 256 KB, so the 14-bit field
+// never carries into the LBO field).
 __device__ __forceinline__ void mma_split(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t a_lbo,
                                           uint32_t a_sbo, uint32_t b_hi, uint32_t b_lo, uint32_t b_lbo,
                                           uint32_t b_sbo, int ksteps, uint32_t idesc, bool accumulate,
                                           bool a_has_lo = true, bool b_has_lo = true)
 {
+    const uint64_t da[2] = {smem_desc(a_hi, a_lbo, a_sbo), smem_desc(a_lo, a_lbo, a_sbo)};
+    const uint64_t db[2] = {smem_desc(b_hi, b_lbo, b_sbo), smem_desc(b_lo, b_lbo, b_sbo)};
+    const uint64_t sa = (2u * a_lbo) >> 4, sb = (2u * b_lbo) >> 4;
     bool acc = accumulate;
+#pragma unroll
     for (int tt = 0; tt < 3; ++tt) {
         if ((tt == 1 && !a_has_lo) || (tt == 2 && !b_has_lo)) continue;
-        const uint32_t a = (tt == 1) ? a_lo : a_hi;
-        const uint32_t b = (tt == 2) ? b_lo : b_hi;
+        uint64_t ad = da[tt == 1 ? 1 : 0], bd = db[tt == 2 ? 1 : 0];
+#pragma unroll
         for (int ks = 0; ks < ksteps; ++ks) {
-            const uint64_t ad = smem_desc(a + 2u * a_lbo * ks, a_lbo, a_sbo);
-            const uint64_t bd = smem_desc(b + 2u * b_lbo * ks, b_lbo, b_sbo);
             umma_bf16(d, ad, bd, idesc, acc ? 1u : 0u);
             acc = true;
+            ad += sa;
+            bd += sb;
         }
     }
 }

