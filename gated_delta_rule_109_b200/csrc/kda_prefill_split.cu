@@ -531,7 +531,15 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
 }
 
-// ---------------------------------------------------------------- chain kernel smem
+// ---------------------------------------------------------------- chain kernel
+// Warp roles: warps 0..7 hold the state slice (thread (lane dk, half) owns 16
+// columns of row dk), split the B operands and read the accumulators; warp 8
+// issues the tensor-core products and the bulk copies.  Handoffs go through
+// mbarriers, never a CTA-wide barrier:
+//   bar_s  (8 arrivals)  S' of chunk kk is in shared memory, D1/D2 of chunk kk-1 read
+//   bar_d  (8 arrivals)  Delta of chunk kk is in shared memory, D1 of kk and D3 of kk-1 read
+//   mma1 / mma2 (commit) the first / second product of chunk kk is complete
+constexpr int kChainThreads = 288;
 constexpr uint32_t CH_WQ = 0;                        // two slots of [Wr; Qr] (hi, lo) and e^m
 constexpr uint32_t CH_KTM = 2 * kWqBytes;            // Kb hi, Kb lo, M hi, M lo (48 KB)
 constexpr uint32_t CH_MA = CH_KTM + 24576;           // 128-row view whose rows 64..127 are M hi
@@ -540,8 +548,9 @@ constexpr uint32_t CH_U = CH_KTM + 49152;            // fp32 [64][32]
 constexpr uint32_t CH_GAM = CH_U + 8192;             // fp32 [128] e^{G_last}, then [128] e^{G_last - m}
 constexpr uint32_t CH_S = CH_GAM + 1024, CH_S_LO = CH_S + 8192;    // S': MN-major B (outer dk, inner column)
 constexpr uint32_t CH_DL = CH_S + 16384, CH_DL_LO = CH_DL + 4096;  // Delta: MN-major B (outer token)
-constexpr uint32_t CH_MBAR = CH_DL + 8192;           // mma, wq[2], ktm
-constexpr uint32_t CH_TMEMP = CH_MBAR + 32;
+constexpr uint32_t CH_MBAR = CH_DL + 8192;           // mma1, mma2, wq[2], ktm, bar_s, bar_d
+constexpr uint32_t CH_FAIL = CH_MBAR + 56;           // a wait gave up somewhere in the CTA
+constexpr uint32_t CH_TMEMP = CH_MBAR + 64;
 constexpr uint32_t CH_TOTAL = CH_TMEMP + 16;
 static_assert(CH_TOTAL <= 232448, "shared memory");
 static_assert(R_KT_LO + 16384 == R_M && R_M + 16384 == R_U, "Kb and M are one contiguous copy");
@@ -549,7 +558,7 @@ static_assert(R_GAM + 512 == R_EL, "e^{G_last} and e^{G_last - m} are one contig
 
 constexpr uint32_t TMC_D1 = 0, TMC_D2 = 32, TMC_D3 = 64, TMC_COLS = 128;
 
-__global__ void __launch_bounds__(kNT, 1)
+__global__ void __launch_bounds__(kChainThreads, 1)
 prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
                      float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb)
 {
@@ -557,7 +566,9 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
     const float *sU = reinterpret_cast<const float *>(smem + CH_U);
     const float *sGam = reinterpret_cast<const float *>(smem + CH_GAM);
-    const uint32_t mbar = sbase + CH_MBAR, mbar_wq0 = mbar + 8, mbar_ktm = mbar + 24;
+    volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + CH_FAIL);
+    const uint32_t mbar1 = sbase + CH_MBAR, mbar2 = mbar1 + 8, mbar_wq0 = mbar1 + 16, mbar_ktm = mbar1 + 32;
+    const uint32_t bar_s = mbar1 + 40, bar_d = mbar1 + 48;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x % kNSL;
@@ -565,7 +576,7 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     const int b = bh / H, h = bh % H;
     const int col0 = slice * kDVS;
     const int lrow = 32 * (warp & 3) + lane;
-    const int half = warp >> 2;
+    const int half = (warp >> 2) & 1;
     const uint8_t *recs = ws + (size_t)bh * nb * kRec;
 
     if (warp == 0) {
@@ -574,149 +585,169 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
-        mbar_init(mbar, 1);
+        mbar_init(mbar1, 1);
+        mbar_init(mbar2, 1);
         mbar_init(mbar_wq0, 1);
         mbar_init(mbar_wq0 + 8, 1);
         mbar_init(mbar_ktm, 1);
+        mbar_init(bar_s, 8);
+        mbar_init(bar_d, 8);
+        *sFail = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + CH_TMEMP);
-    const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
-
-    // copies of the streamed operands (thread 0); pending flags are kept by every thread
-    // pending copies: bit s of wq_pend = slot s armed and not yet waited for, bit s
-    // of wq_par = the parity that copy completes
-    uint32_t wq_pend = 0u, wq_par = 0u, ktm_par = 0u;
-    bool ktm_pending = false, failed = false;
-    auto load_wq = [&](int kk) {
-        const uint32_t mb = mbar_wq0 + 8u * (kk & 1);
-        const uint32_t bit = 1u << (kk & 1);
-        wq_pend |= bit;
-        wq_par = ((kk >> 1) & 1) ? (wq_par | bit) : (wq_par & ~bit);
-        if (tid == 0) {
-            mbar_expect_tx(mb, kWqBytes);
-            bulk_g2s(sbase + CH_WQ + kWqBytes * (kk & 1), recs + (size_t)kk * kRec + R_WQ, kWqBytes, mb);
-        }
-    };
-    auto load_ktm = [&](int kk) {
-        ktm_pending = true;
-        ktm_par = (uint32_t)kk & 1u;
-        if (tid == 0) {
-            const uint8_t *r = recs + (size_t)kk * kRec;
-            mbar_expect_tx(mbar_ktm, 49152u + 8192u + 1024u);
-            bulk_g2s(sbase + CH_KTM, r + R_KT, 49152u, mbar_ktm);
-            bulk_g2s(sbase + CH_U, r + R_U + slice * 8192u, 8192u, mbar_ktm);
-            bulk_g2s(sbase + CH_GAM, r + R_GAM, 1024u, mbar_ktm);
-        }
+    // a wait that gives up marks the CTA failed; the others then stop at their next wait
+    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (*sFail) return false;
+        if (mbar_wait(bar, parity)) return true;
+        *sFail = 1u;
+        return false;
     };
 
-    float S[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-        S[j] = s_in ? s_in[((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half + j] : 0.f;
-
-    uint32_t phase = 0;
-    load_wq(0);
-    if (nb > 1) load_wq(1);
-    load_ktm(0);
-
-    // S' = Diag(e^m) S as a split B operand, then D1 = [Wr; Qr] S' for chunk kk
-    // (thread 0 issues)
-    auto issue_rt1 = [&](int kk) -> bool {
-        const int buf = kk & 1;
-        const bool bad = !mbar_wait(mbar_wq0 + 8u * buf, (uint32_t)(kk >> 1) & 1u);
-        const float em = bad ? 0.f : reinterpret_cast<const float *>(smem + CH_WQ + kWqBytes * buf + 65536u)[lrow];
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            float xv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) xv[e] = em * S[8 * g + e];
-            const uint32_t off = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
-            st_split8(smem, CH_S + off, CH_S_LO + off, xv);
+    if (warp == 8) {
+        // ---------------- issuer: products and copies (lane 0)
+        if (lane == 0) {
+            uint32_t wq_pend = 0u, wq_par = 0u, ktm_par = 0u;
+            bool ktm_pending = false;
+            auto load_wq = [&](int kk) {
+                const uint32_t mb = mbar_wq0 + 8u * (kk & 1);
+                const uint32_t bit = 1u << (kk & 1);
+                wq_pend |= bit;
+                wq_par = ((kk >> 1) & 1) ? (wq_par | bit) : (wq_par & ~bit);
+                mbar_expect_tx(mb, kWqBytes);
+                bulk_g2s(sbase + CH_WQ + kWqBytes * (kk & 1), recs + (size_t)kk * kRec + R_WQ, kWqBytes, mb);
+            };
+            auto load_ktm = [&](int kk) {
+                const uint8_t *r = recs + (size_t)kk * kRec;
+                ktm_pending = true;
+                ktm_par = (uint32_t)kk & 1u;
+                mbar_expect_tx(mbar_ktm, 49152u + 8192u + 1024u);
+                bulk_g2s(sbase + CH_KTM, r + R_KT, 49152u, mbar_ktm);
+                bulk_g2s(sbase + CH_U, r + R_U + slice * 8192u, 8192u, mbar_ktm);
+                bulk_g2s(sbase + CH_GAM, r + R_GAM, 1024u, mbar_ktm);
+            };
+            load_wq(0);
+            if (nb > 1) load_wq(1);
+            load_ktm(0);
+            for (int kk = 0; kk < nb; ++kk) {
+                const uint32_t par = (uint32_t)kk & 1u;
+                // the compute warps have waited for this chunk's [Wr; Qr] before arriving
+                if (!wait(bar_s, par)) break;
+                wq_pend &= ~(1u << (kk & 1));
+                tc_fence_after();
+                const uint32_t wq = sbase + CH_WQ + kWqBytes * (kk & 1);
+                mma_split(tmem + TMC_D1, wq, wq + 32768u, RW_SI, RW_SO, sbase + CH_S, sbase + CH_S_LO,
+                          S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
+                umma_commit(mbar1);
+                if (!wait(mbar1, par)) break;
+                if (kk + 2 < nb) load_wq(kk + 2);
+                // ... and for this chunk's Kb, M, U before arriving
+                if (!wait(bar_d, par)) break;
+                ktm_pending = false;
+                tc_fence_after();
+                mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
+                          sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 1, 1), false);
+                mma_split(tmem + TMC_D3, sbase + CH_MA, sbase + CH_MA_LO, H_SI, H_SO,
+                          sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 0, 1), false);
+                umma_commit(mbar2);
+                if (!wait(mbar2, par)) break;
+                if (kk + 1 < nb) load_ktm(kk + 1);
+            }
+            if (*sFail) {
+                // let the copies still in flight land before shared memory is released
+                for (int sl = 0; sl < 2; ++sl)
+                    if ((wq_pend >> sl) & 1u) mbar_wait(mbar_wq0 + 8u * sl, (wq_par >> sl) & 1u);
+                if (ktm_pending) mbar_wait(mbar_ktm, ktm_par);
+            }
         }
-        proxy_fence();
-        tc_fence_before();
-        if (__syncthreads_or(bad)) return false;
-        wq_pend &= ~(1u << buf);
-        if (tid == 0) {
-            tc_fence_after();
-            const uint32_t wq = sbase + CH_WQ + kWqBytes * buf;
-            mma_split(tmem + TMC_D1, wq, wq + 32768u, RW_SI, RW_SO, sbase + CH_S, sbase + CH_S_LO,
-                      S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
-            umma_commit(mbar);
-        }
-        return true;
-    };
-
-    failed = !issue_rt1(0);
-    for (int kk = 0; kk < nb && !failed; ++kk) {
-        // ---- D1 of chunk kk and its K^, M, U, e^{G_last}
-        {
-            const bool bad = !mbar_wait(mbar, phase) || !mbar_wait(mbar_ktm, (uint32_t)kk & 1u);
-            phase ^= 1;
-            if (__syncthreads_or(bad)) { failed = true; break; }
-        }
-        ktm_pending = false;
-        if (kk + 2 < nb) load_wq(kk + 2);   // slot kk & 1 is free again: fetch two chunks ahead
-        tc_fence_after();
-
-        // ---- Delta = U - Wr S' (rows 0..63); Qr S' kept for the output (rows 64..127)
+    } else {
+        // ---------------- state slice: S' and Delta operands, updates, outputs
+        const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+        float S[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+            S[j] = s_in ? s_in[((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half + j] : 0.f;
         float qs[16];
-        {
-            float x[16];
-            tmem_ld16(tmem + tlane + TMC_D1 + 16 * half, x);
-            if (lrow < 64) {
+        bool ok = true;
+        for (int kk = 0; kk < nb && ok; ++kk) {
+            const uint32_t par = (uint32_t)kk & 1u;
+            // ---- S' = Diag(e^m) S of chunk kk as a split B operand
+            if (!(ok = wait(mbar_wq0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u))) break;
+            {
+                const float em = reinterpret_cast<const float *>(smem + CH_WQ + kWqBytes * (kk & 1) + 65536u)[lrow];
 #pragma unroll
                 for (int g = 0; g < 2; ++g) {
-                    float d[8];
+                    float xv[8];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e) d[e] = sU[lrow * kDVS + 16 * half + 8 * g + e] - x[8 * g + e];
-                    const uint32_t o = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
-                    st_split8(smem, CH_DL + o, CH_DL_LO + o, d);
+                    for (int e = 0; e < 8; ++e) xv[e] = em * S[8 * g + e];
+                    const uint32_t off = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
+                    st_split8(smem, CH_S + off, CH_S_LO + off, xv);
                 }
             }
+            proxy_fence();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s);
+
+            // ---- O = Qr S' + M Delta of chunk kk - 1 while the first product of kk runs
+            if (kk > 0 && lrow >= 64) {
+                float o2[16];
+                tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
+                const int t = (n0 + kk - 1) * kC + lrow - 64;
+                if (t < T) {
+                    float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
 #pragma unroll
-            for (int e = 0; e < 16; ++e) qs[e] = x[e];
-        }
-        const float gam = sGam[lrow], el = sGam[kDK + lrow];
-        proxy_fence();
-        tc_fence_before();
-        __syncthreads();
-        if (tid == 0) {
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_float4(qs[4 * g] + o2[4 * g], qs[4 * g + 1] + o2[4 * g + 1],
+                                             qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
+                }
+            }
+
+            // ---- Delta = U - Wr S' (rows 0..63); Qr S' kept for the output (rows 64..127)
+            if (!(ok = wait(mbar1, par) && wait(mbar_ktm, par))) break;
             tc_fence_after();
-            // D2 = Kb^T Delta;  D3 = [. ; M] Delta
-            mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
-                      sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 1, 1), false);
-            mma_split(tmem + TMC_D3, sbase + CH_MA, sbase + CH_MA_LO, H_SI, H_SO,
-                      sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 0, 1), false);
-            umma_commit(mbar);
-        }
-        {
-            const bool bad = !mbar_wait(mbar, phase);
-            phase ^= 1;
-            if (__syncthreads_or(bad)) { failed = true; break; }
-        }
-        if (kk + 1 < nb) load_ktm(kk + 1);
-        tc_fence_after();
-
-        // ---- S <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta, and the next
-        // chunk's first product
-        {
-            float x[16];
-            tmem_ld16(tmem + tlane + TMC_D2 + 16 * half, x);
+            {
+                float x[16];
+                tmem_ld16(tmem + tlane + TMC_D1 + 16 * half, x);
+                if (lrow < 64) {
 #pragma unroll
-            for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + el * x[j];
-        }
-        if (kk + 1 < nb && !issue_rt1(kk + 1)) { failed = true; break; }
+                    for (int g = 0; g < 2; ++g) {
+                        float d[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) d[e] = sU[lrow * kDVS + 16 * half + 8 * g + e] - x[8 * g + e];
+                        const uint32_t o = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
+                        st_split8(smem, CH_DL + o, CH_DL_LO + o, d);
+                    }
+                }
+#pragma unroll
+                for (int e = 0; e < 16; ++e) qs[e] = x[e];
+            }
+            const float gam = sGam[lrow], el = sGam[kDK + lrow];
+            proxy_fence();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_d);
 
-        // ---- O = Qr S' + M Delta of chunk kk, while the tensor cores run chunk kk + 1
-        if (lrow >= 64) {
+            // ---- S <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta
+            if (!(ok = wait(mbar2, par))) break;
+            tc_fence_after();
+            {
+                float x[16];
+                tmem_ld16(tmem + tlane + TMC_D2 + 16 * half, x);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) S[j] = gam * S[j] + el * x[j];
+            }
+            tc_fence_before();
+        }
+        if (ok && nb > 0 && lrow >= 64) {
+            // the last chunk's output
+            tc_fence_after();
             float o2[16];
             tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
-            const int t = (n0 + kk) * kC + lrow - 64;
+            const int t = (n0 + nb - 1) * kC + lrow - 64;
             if (t < T) {
                 float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
 #pragma unroll
@@ -725,24 +756,16 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
                                          qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
             }
         }
-        tc_fence_before();
+        if (ok && s_out) {
+            float4 *dst = reinterpret_cast<float4 *>(s_out + ((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half);
+#pragma unroll
+            for (int g = 0; g < 4; ++g) dst[g] = make_float4(S[4 * g], S[4 * g + 1], S[4 * g + 2], S[4 * g + 3]);
+        }
     }
 
-    if (failed) {
-        // let the copies still in flight land before shared memory is released (bounded)
-        if (tid == 0) {
-            for (int sl = 0; sl < 2; ++sl)
-                if ((wq_pend >> sl) & 1u) mbar_wait(mbar_wq0 + 8u * sl, (wq_par >> sl) & 1u);
-            if (ktm_pending) mbar_wait(mbar_ktm, ktm_par);
-            atomicOr(&g_split_device_status, 1u);
-        }
-    } else if (s_out) {
-        float4 *dst = reinterpret_cast<float4 *>(s_out + ((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half);
-#pragma unroll
-        for (int g = 0; g < 4; ++g) dst[g] = make_float4(S[4 * g], S[4 * g + 1], S[4 * g + 2], S[4 * g + 3]);
-    }
     tc_fence_before();
     __syncthreads();
+    if (tid == 0 && *sFail) atomicOr(&g_split_device_status, 1u);
     if (warp == 0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMC_COLS) : "memory");
@@ -804,7 +827,7 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
         note_launch();
         const float *s_in = (n0 == 0) ? a.s0 : carry;
         float *s_out = (n0 + nb >= nchunks) ? a.sT : carry;
-        prefill_chain_kernel<<<(unsigned)(bh * kNSL), kNT, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
+        prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
                                                                              a.H, n0, nb);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
