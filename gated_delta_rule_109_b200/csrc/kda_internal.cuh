@@ -53,6 +53,8 @@ cudaError_t take_gdn_device_status(unsigned int *status);
 bool prefill_split_supported(const ForwardArgs &a);
 size_t prefill_split_workspace_full(int B, int T, int H);   // whole sequence in one block
 size_t prefill_split_workspace_min(int B, int T, int H);    // one chunk per block + state carry
+// The chain runs one CTA per (b, h, 32-column slice) while 4 B H CTAs fit on the
+// SMs, else one CTA per (b, h).
 cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t take_split_device_status(unsigned int *status);
 // Reads and clears the device status word the tensor-core kernels set when a

@@ -772,6 +772,257 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     }
 }
 
+// ---------------------------------------------------------------- full-head chain kernel
+// The chain of one (b, h) with all 128 value columns in one CTA: each tensor-core
+// instruction is N = 128 wide (four times the columns per instruction of the
+// slice kernel), so a CTA per head walks a chunk in about the time a slice CTA
+// does.  Used when the heads alone fill the GPU.  The fp32 state lives in tensor
+// memory (columns 384..511, lane = key channel); warp w of warps 0..15 owns TMEM
+// lane quadrant w % 4 and value columns 32 (w / 4) .. +31 of it and of the
+// accumulators; warp 16 issues the products and the copies.  U rows are fetched
+// into registers (rows 0..63) while the first product runs; Qr S' rows 64..127
+// share those registers.
+constexpr int kHeadThreads = 17 * 32;
+constexpr uint32_t HC_WQ = 0;                                  // [Wr; Qr] hi, lo, e^m (one slot)
+constexpr uint32_t HC_KTM = kWqBytes;                          // Kb hi, Kb lo, M hi, M lo
+constexpr uint32_t HC_MA = HC_KTM + 24576, HC_MA_LO = HC_KTM + 32768;
+constexpr uint32_t HC_GAM = HC_KTM + 49152;                    // e^{G_last} [128], e^{G_last - m} [128]
+constexpr uint32_t HC_S = HC_GAM + 1024, HC_S_LO = HC_S + 32768;     // S': MN-major B, outer dk, inner column
+constexpr uint32_t HC_DL = HC_S + 65536, HC_DL_LO = HC_DL + 16384;   // Delta: MN-major B, outer token
+constexpr uint32_t HC_MBAR = HC_DL + 32768;                    // mma1, mma2, wq, ktm, bar_s, bar_d
+constexpr uint32_t HC_FAIL = HC_MBAR + 48;
+constexpr uint32_t HC_TMEMP = HC_MBAR + 64;
+constexpr uint32_t HC_TOTAL = HC_TMEMP + 16;
+static_assert(HC_TOTAL <= 232448, "shared memory");
+constexpr uint32_t HS_SO = 2048, HS_SI = 128;                  // N = 128 B-operand strides
+constexpr uint32_t TMH_D1 = 0, TMH_D2 = 128, TMH_D3 = 256, TMH_S = 384, TMH_COLS = 512;
+
+__global__ void __launch_bounds__(kHeadThreads, 1)
+prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
+                          float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + HC_FAIL);
+    const float *sEm = reinterpret_cast<const float *>(smem + HC_WQ + 65536u);
+    const float *sGam = reinterpret_cast<const float *>(smem + HC_GAM);
+    const uint32_t mbar1 = sbase + HC_MBAR, mbar2 = mbar1 + 8, mbar_wq = mbar1 + 16, mbar_ktm = mbar1 + 24;
+    const uint32_t bar_s = mbar1 + 32, bar_d = mbar1 + 40;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int bh = blockIdx.x;
+    const int b = bh / H, h = bh % H;
+    const int r = 32 * (warp & 3) + lane;          // TMEM lane: key channel (S, D2) or row (D1, D3)
+    const int cg = (warp >> 2) & 3;                // value columns 32 cg .. 32 cg + 31
+    const uint8_t *recs = ws + (size_t)bh * nb * kRec;
+
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(sbase + HC_TMEMP), "r"(TMH_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(mbar1, 1);
+        mbar_init(mbar2, 1);
+        mbar_init(mbar_wq, 1);
+        mbar_init(mbar_ktm, 1);
+        mbar_init(bar_s, 16);
+        mbar_init(bar_d, 16);
+        *sFail = 0u;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + HC_TMEMP);
+    auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (*sFail) return false;
+        if (mbar_wait(bar, parity)) return true;
+        *sFail = 1u;
+        return false;
+    };
+
+    if (warp == 16) {
+        // ---------------- issuer (lane 0): products and record copies
+        if (lane == 0) {
+            bool wq_pending = false, ktm_pending = false;
+            uint32_t wq_par = 0u, ktm_par = 0u;
+            auto load_wq = [&](int kk) {
+                wq_pending = true;
+                wq_par = (uint32_t)kk & 1u;
+                mbar_expect_tx(mbar_wq, kWqBytes);
+                bulk_g2s(sbase + HC_WQ, recs + (size_t)kk * kRec + R_WQ, kWqBytes, mbar_wq);
+            };
+            auto load_ktm = [&](int kk) {
+                const uint8_t *rc = recs + (size_t)kk * kRec;
+                ktm_pending = true;
+                ktm_par = (uint32_t)kk & 1u;
+                mbar_expect_tx(mbar_ktm, 49152u + 1024u);
+                bulk_g2s(sbase + HC_KTM, rc + R_KT, 49152u, mbar_ktm);
+                bulk_g2s(sbase + HC_GAM, rc + R_GAM, 1024u, mbar_ktm);
+            };
+            load_wq(0);
+            load_ktm(0);
+            for (int kk = 0; kk < nb; ++kk) {
+                const uint32_t par = (uint32_t)kk & 1u;
+                if (!wait(bar_s, par)) break;          // S' written; [Wr; Qr] of kk seen by all
+                wq_pending = false;
+                tc_fence_after();
+                mma_split(tmem + TMH_D1, sbase + HC_WQ, sbase + HC_WQ + 32768u, RW_SI, RW_SO,
+                          sbase + HC_S, sbase + HC_S_LO, HS_SO, HS_SI, kDK / 16, idesc_bf16(128, kDV, 0, 1), false);
+                umma_commit(mbar1);
+                if (!wait(mbar1, par)) break;
+                if (kk + 1 < nb) load_wq(kk + 1);
+                if (!wait(bar_d, par)) break;          // Delta written; Kb, M of kk seen by all
+                ktm_pending = false;
+                tc_fence_after();
+                mma_split(tmem + TMH_D2, sbase + HC_KTM, sbase + HC_KTM + 16384u, RW_SO, RW_SI,
+                          sbase + HC_DL, sbase + HC_DL_LO, HS_SO, HS_SI, kC / 16, idesc_bf16(128, kDV, 1, 1), false);
+                mma_split(tmem + TMH_D3, sbase + HC_MA, sbase + HC_MA_LO, H_SI, H_SO,
+                          sbase + HC_DL, sbase + HC_DL_LO, HS_SO, HS_SI, kC / 16, idesc_bf16(128, kDV, 0, 1), false);
+                umma_commit(mbar2);
+                if (!wait(mbar2, par)) break;
+                if (kk + 1 < nb) load_ktm(kk + 1);
+            }
+            if (*sFail) {
+                if (wq_pending) mbar_wait(mbar_wq, wq_par);
+                if (ktm_pending) mbar_wait(mbar_ktm, ktm_par);
+            }
+        }
+    } else {
+        // ---------------- state: row r, columns 32 cg .. +31
+        const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+        const uint32_t tS = tmem + tlane + TMH_S + 32 * cg;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float x[16];
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+                x[j] = s_in ? s_in[((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh + j] : 0.f;
+            tmem_st16(tS + 16 * hh, x);
+        }
+        tmem_wait_st();
+        float aux[32];            // rows 0..63: U of this chunk; rows 64..127: Qr S' of the last one
+        auto store_out = [&](int kk) {
+            const int t = (n0 + kk) * kC + r - 64;
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float o2[16];
+                tmem_ld16(tmem + tlane + TMH_D3 + 32 * cg + 16 * hh, o2);
+                if (t < T) {
+                    float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + 32 * cg + 16 * hh);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        dst[g] = make_float4(aux[16 * hh + 4 * g] + o2[4 * g], aux[16 * hh + 4 * g + 1] + o2[4 * g + 1],
+                                             aux[16 * hh + 4 * g + 2] + o2[4 * g + 2], aux[16 * hh + 4 * g + 3] + o2[4 * g + 3]);
+                }
+            }
+        };
+        bool ok = true;
+        for (int kk = 0; kk < nb && ok; ++kk) {
+            const uint32_t par = (uint32_t)kk & 1u;
+            // ---- S' = Diag(e^m) S as a split B operand
+            if (!(ok = wait(mbar_wq, par))) break;
+            {
+                const float em = sEm[r];
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[16];
+                    tmem_ld16(tS + 16 * hh, x);
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        float xv[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) xv[e] = em * x[8 * g + e];
+                        const uint32_t off = core_off(r, 32 * cg + 16 * hh + 8 * g, HS_SO, HS_SI);
+                        st_split8(smem, HC_S + off, HC_S_LO + off, xv);
+                    }
+                }
+            }
+            proxy_fence();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_s);
+
+            // ---- the previous chunk's output while this chunk's first product runs
+            if (kk > 0 && r >= 64) store_out(kk - 1);
+            // ---- this chunk's U rows (read while the first product runs)
+            if (r < 64) {
+                const float4 *src = reinterpret_cast<const float4 *>(recs + (size_t)kk * kRec + R_U + cg * 8192u) + r * 8;
+#pragma unroll
+                for (int g = 0; g < 8; ++g) {
+                    const float4 u4 = src[g];
+                    aux[4 * g] = u4.x; aux[4 * g + 1] = u4.y; aux[4 * g + 2] = u4.z; aux[4 * g + 3] = u4.w;
+                }
+            }
+
+            // ---- Delta = U - Wr S' (rows 0..63); Qr S' kept for the output (rows 64..127)
+            if (!(ok = wait(mbar1, par) && wait(mbar_ktm, par))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[16];
+                tmem_ld16(tmem + tlane + TMH_D1 + 32 * cg + 16 * hh, x);
+                if (r < 64) {
+#pragma unroll
+                    for (int g = 0; g < 2; ++g) {
+                        float d[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) d[e] = aux[16 * hh + 8 * g + e] - x[8 * g + e];
+                        const uint32_t o = core_off(r, 32 * cg + 16 * hh + 8 * g, HS_SO, HS_SI);
+                        st_split8(smem, HC_DL + o, HC_DL_LO + o, d);
+                    }
+                } else {
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) aux[16 * hh + e] = x[e];
+                }
+            }
+            const float gam = sGam[r], el = sGam[kDK + r];
+            proxy_fence();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_d);
+
+            // ---- S <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta
+            if (!(ok = wait(mbar2, par))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float x[16], sv[16];
+                tmem_ld16(tmem + tlane + TMH_D2 + 32 * cg + 16 * hh, x);
+                tmem_ld16(tS + 16 * hh, sv);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) sv[j] = gam * sv[j] + el * x[j];
+                tmem_st16(tS + 16 * hh, sv);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+        }
+        if (ok && nb > 0 && r >= 64) {
+            tc_fence_after();
+            store_out(nb - 1);
+        }
+        if (ok && s_out) {
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float sv[16];
+                tmem_ld16(tS + 16 * hh, sv);
+                float4 *dst = reinterpret_cast<float4 *>(s_out + ((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) dst[g] = make_float4(sv[4 * g], sv[4 * g + 1], sv[4 * g + 2], sv[4 * g + 3]);
+            }
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    if (tid == 0 && *sFail) atomicOr(&g_split_device_status, 1u);
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMH_COLS) : "memory");
+    }
+}
+
 }  // namespace
 
 bool prefill_split_supported(const ForwardArgs &a)
@@ -816,7 +1067,16 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
     if (e == cudaSuccess)
         e = cudaFuncSetAttribute(prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)CH_TOTAL);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_chain_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)HC_TOTAL);
+    int dev = 0, sms = 0;
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
+    // value slices while they fit on the SMs in one wave, whole heads once the heads
+    // alone fill them (a head CTA walks a chunk in about the time a slice CTA does)
+    const bool per_head = bh * kNSL > (size_t)sms;
     for (int n0 = 0; n0 < nchunks; n0 += L) {
         const int nb = min(L, nchunks - n0);
         prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
@@ -827,8 +1087,12 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
         note_launch();
         const float *s_in = (n0 == 0) ? a.s0 : carry;
         float *s_out = (n0 + nb >= nchunks) ? a.sT : carry;
-        prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
-                                                                             a.H, n0, nb);
+        if (per_head)
+            prefill_chain_head_kernel<<<(unsigned)bh, kHeadThreads, HC_TOTAL, stream>>>(ws, s_in, s_out, a.out,
+                                                                                      a.T, a.H, n0, nb);
+        else
+            prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out,
+                                                                                         a.T, a.H, n0, nb);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         note_launch();

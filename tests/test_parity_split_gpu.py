@@ -63,6 +63,30 @@ def test_split_shape_sweep(T, B, H, state):
     _compare(x, out, sT)
 
 
+# ------------------------------------------------------------ one chain CTA per head
+# More than SMs / 4 heads (148 SMs: more than 37) take the full-head chain kernel.
+@pytest.mark.parametrize("T,B,H,state", [(1, 2, 19, True), (64, 2, 19, True), (200, 2, 19, True),
+                                         (131, 1, 40, False), (333, 4, 12, True)])
+def test_split_full_head_chain(T, B, H, state):
+    assert B * H * 4 > torch.cuda.get_device_properties(0).multi_processor_count
+    w = I.scaled(I.PREFILL_B4_T16K_STATE if state else I.PREFILL_H16_T4K, B=B, H=H, T=T, seed=4000 + T)
+    x = I.make_inputs(w, "cuda")
+    out, sT = _run(x, _ws(w))
+    _compare(x, out, sT)
+
+
+def test_full_head_chain_blocked_and_extreme():
+    w = I.scaled(I.PREFILL_B4_T16K_STATE, B=2, H=20, T=300, seed=81)
+    x = I.make_inputs(w, "cuda")
+    x["log_alpha"][:, 64:128] = -3.0
+    x["log_alpha"][:, 130:135, :, :9] = -30.0
+    out_f, s_f = _run(x, _ws(w))
+    bh, rec = w.B * w.H, kda.workspace_bytes(1, 64, 1, 128, 128)
+    out_b, s_b = _run(x, _ws(w, bh * rec * 2 + bh * 128 * 128 * 4))
+    assert torch.equal(out_f, out_b) and torch.equal(s_f, s_b)
+    _compare(x, out_f, s_f)
+
+
 # ------------------------------------------------------------ blocked workspaces
 @pytest.mark.parametrize("blocks", [1, 2, 3, 5])
 def test_blocked_workspace_matches_one_block(blocks):
