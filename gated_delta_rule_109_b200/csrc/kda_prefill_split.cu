@@ -92,6 +92,12 @@ constexpr uint32_t PP_R = 81920, PP_R_LO = PP_R + 8192;
 static_assert(PP_TMAT + 64 * kPitch * 4 <= PP_P_LO, "solve scratch");
 // wide-range path: G fp32 [64][128] over Qr hi and Kb hi, pairwise A (pitch 64) over Kb lo
 constexpr uint32_t PP_G = 16384, PP_AW = 49152;
+// the scan: log_alpha transposed through shared memory (row pitch 132 floats keeps the
+// 16-byte row accesses of a quarter warp on distinct banks), over Qr hi and Kb before
+// the split pass writes them; half totals after the per-channel scalars in the V region
+constexpr int kGP = 132;
+constexpr uint32_t PP_GS = 16384;
+static_assert(PP_GS + 64 * kGP * 4 <= PP_P_LO, "scan scratch");
 
 constexpr uint32_t TMP_AM = 0, TMP_W = 0, TMP_U = 128, TMP_COLS = 256;
 
@@ -118,23 +124,40 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     uint8_t *rec = ws + ((size_t)bh * nb + nloc) * kRec;
     auto row = [&](int t) { return ((size_t)b * T + t0 + t) * H + h; };
 
-    // ---- loads: log_alpha of (token, 8 channels) (the scan needs it) and beta; V follows
-    // by cp.async once the V region has served as scratch for the per-channel scalars
-    float G[2][16];
+    // ---- loads, all issued at once (one DRAM latency per CTA): log_alpha rows and beta
+    // by cp.async into shared memory (rows past the chunk's end zero-filled), the k and
+    // q of this thread's four (token, 8 channels) items into registers; V follows by
+    // cp.async once the V region has served as scratch
+    float *Gs = reinterpret_cast<float *>(smem + PP_GS);
 #pragma unroll
-    for (int hf = 0; hf < 2; ++hf) {
-        const int t = lane + 32 * hf;
-        const bool ok = t < c;
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-            const size_t o = row(ok ? t : 0) * kDK + ch0 + 8 * g;
-            const float4 a0 = ok ? *reinterpret_cast<const float4 *>(log_alpha + o) : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float4 a1 = ok ? *reinterpret_cast<const float4 *>(log_alpha + o + 4) : make_float4(0.f, 0.f, 0.f, 0.f);
-            G[hf][8 * g + 0] = a0.x; G[hf][8 * g + 1] = a0.y; G[hf][8 * g + 2] = a0.z; G[hf][8 * g + 3] = a0.w;
-            G[hf][8 * g + 4] = a1.x; G[hf][8 * g + 5] = a1.y; G[hf][8 * g + 6] = a1.z; G[hf][8 * g + 7] = a1.w;
-        }
+    for (int r = 0; r < 8; ++r) {
+        const int id = tid + kNT * r, t = id >> 5, j = id & 31;
+        const bool okt = t < c;
+        cp_async16(sbase + PP_GS + (uint32_t)(t * kGP + 4 * j) * 4u, log_alpha + row(okt ? t : 0) * kDK + 4 * j,
+                   okt ? 16u : 0u);
     }
-    if (tid < kC) sBeta[tid] = (tid < c) ? beta[row(tid)] : 0.f;
+    if (tid < kC / 4) {
+        const bool okt = 4 * tid < c;
+        // beta is [B, T, H]: the chunk's 64 values are H apart, so they come one by one
+        float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (okt) {
+            bv.x = beta[row(4 * tid)];
+            if (4 * tid + 1 < c) bv.y = beta[row(4 * tid + 1)];
+            if (4 * tid + 2 < c) bv.z = beta[row(4 * tid + 2)];
+            if (4 * tid + 3 < c) bv.w = beta[row(4 * tid + 3)];
+        }
+        reinterpret_cast<float4 *>(sBeta)[tid] = bv;
+    }
+    uint4 kv4[4], qv4[4];
+#pragma unroll
+    for (int item = 0; item < 4; ++item) {
+        const int t = lane + 32 * (item >> 1);
+        const bool okt = t < c;
+        const size_t o = row(okt ? t : 0) * kDK + ch0 + 8 * (item & 1);
+        kv4[item] = okt ? *reinterpret_cast<const uint4 *>(k + o) : make_uint4(0u, 0u, 0u, 0u);
+        qv4[item] = okt ? *reinterpret_cast<const uint4 *>(q + o) : make_uint4(0u, 0u, 0u, 0u);
+    }
+    cp_async_commit();
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
@@ -145,37 +168,58 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         mbar_init(mbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
+    cp_async_wait_all();
+    __syncthreads();
 
-    // ---- in-chunk inclusive sums over tokens (lanes), per channel; padded tokens add 0.
-    // Per channel: G_last (the sum up to the chunk's last token) and the reference
-    // point m midway between the first and last G (the extremes when the decay is
-    // monotone; every token is checked against it in the split pass).  Both go to
-    // shared memory (the V region, before V arrives).
+    // ---- in-chunk inclusive sums over tokens, per channel, in shared memory: thread
+    // (channel, token half) sums its 32 tokens in order, the second half then adds the
+    // first half's total.
+    // Padded tokens add 0.  Per channel: G_last (the sum up to the chunk's last token)
+    // and the reference point m midway between the first and last G (the extremes when
+    // the decay is monotone; every token is checked against it in the split pass).
     float *sGm = reinterpret_cast<float *>(smem + PP_V);
     float *sGl = sGm + kDK;
-#pragma unroll
-    for (int e = 0; e < 16; ++e) {
-        float a = G[0][e], bb = G[1][e];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float ua = __shfl_up_sync(0xffffffffu, a, o);
-            const float ub = __shfl_up_sync(0xffffffffu, bb, o);
-            if (lane >= o) { a += ua; bb += ub; }
+    float *sTot = sGm + 2 * kDK;
+    {
+        const int ch = tid & (kDK - 1), th = tid >> 7;
+        float run = 0.f;
+#pragma unroll 8
+        for (int i = 0; i < 32; ++i) {
+            float *gp = Gs + (32 * th + i) * kGP + ch;
+            run += *gp;
+            *gp = run;
         }
-        bb += __shfl_sync(0xffffffffu, a, 31);
-        G[0][e] = a;
-        G[1][e] = bb;
-        const float g_l = __shfl_sync(0xffffffffu, bb, 31);
-        const float g_m = 0.5f * (__shfl_sync(0xffffffffu, a, 0) + g_l);
-        if (lane == e) {
-            sGm[ch0 + e] = g_m;
-            sGl[ch0 + e] = g_l;
-            reinterpret_cast<float *>(rec + R_EM)[ch0 + e] = __expf(g_m);
-            reinterpret_cast<float *>(rec + R_GAM)[ch0 + e] = __expf(g_l);
-            reinterpret_cast<float *>(rec + R_EL)[ch0 + e] = __expf(g_l - g_m);
+        sTot[th * kDK + ch] = run;
+    }
+    __syncthreads();
+    {
+        const int ch = tid & (kDK - 1), th = tid >> 7;
+        const float tot0 = sTot[ch];
+        if (th == 1) {
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) Gs[(32 + i) * kGP + ch] += tot0;
+        } else {
+            const float g_l = tot0 + sTot[kDK + ch];
+            const float g_m = 0.5f * (Gs[ch] + g_l);
+            sGm[ch] = g_m;
+            sGl[ch] = g_l;
+            reinterpret_cast<float *>(rec + R_EM)[ch] = __expf(g_m);
+            reinterpret_cast<float *>(rec + R_GAM)[ch] = __expf(g_l);
+            reinterpret_cast<float *>(rec + R_EL)[ch] = __expf(g_l - g_m);
         }
     }
-    __syncwarp();
+    __syncthreads();
+    float G[2][16];
+#pragma unroll
+    for (int hf = 0; hf < 2; ++hf) {
+        const float4 *src = reinterpret_cast<const float4 *>(Gs + (lane + 32 * hf) * kGP + ch0);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const float4 gv = src[j];
+            G[hf][4 * j] = gv.x; G[hf][4 * j + 1] = gv.y; G[hf][4 * j + 2] = gv.z; G[hf][4 * j + 3] = gv.w;
+        }
+    }
+    __syncthreads();        // the split pass writes over the scratch
 
     bool wide = false;      // some |G - m| > 40 (or |m| > 80): the split exponentials could overflow
     // ---- split operands: Kr (smem), Qr and Kb (smem and record)
@@ -184,14 +228,9 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         const int t = lane + 32 * hf;
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-            // keep each item's loads inside its item (hoisting all of them costs 32 registers)
-            asm volatile("" ::: "memory");
+            const uint4 kv = kv4[2 * hf + g], qv = qv4[2 * hf + g];
             float kk[8], qq[8], up[8], y[8];
             {
-                const bool okt = t < c;
-                const size_t o = row(okt ? t : 0) * kDK + ch0 + 8 * g;
-                const uint4 kv = okt ? *reinterpret_cast<const uint4 *>(k + o) : make_uint4(0u, 0u, 0u, 0u);
-                const uint4 qv = okt ? *reinterpret_cast<const uint4 *>(q + o) : make_uint4(0u, 0u, 0u, 0u);
                 const __nv_bfloat16 *kb16 = reinterpret_cast<const __nv_bfloat16 *>(&kv);
                 const __nv_bfloat16 *qb16 = reinterpret_cast<const __nv_bfloat16 *>(&qv);
 #pragma unroll
@@ -474,19 +513,21 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         __syncthreads();
         if (tid == 0) {
             tc_fence_after();
-            // [R; .] Kr (Kr rows read MN-major as B) and [R; .] V; rows 0..63 are R Kr and U
+            // [R; .] Kr (Kr rows read MN-major as B): rows 0..63 are Wr = R Kr;
+            // [. ; R] V (R viewed as rows 64..127): rows 64..127 are U, so that the
+            // other four warps read it
             mma_split(tmem + TMP_W, sbase + PP_R, sbase + PP_R_LO, H_SI, H_SO,
                       sbase + PP_P, sbase + PP_P_LO, RW_SO, RW_SI, kC / 16,
                       idesc_bf16(128, kDK, 0, 1), false);
-            mma_split(tmem + TMP_U, sbase + PP_R, sbase + PP_R_LO, H_SI, H_SO,
+            mma_split(tmem + TMP_U, sbase + PP_R - 8192u, sbase + PP_R_LO - 8192u, H_SI, H_SO,
                       sbase + PP_V, 0u, RW_SO, RW_SI, kC / 16,
                       idesc_bf16(128, kDV, 0, 1), false, true, false);
             umma_commit(mbar);
         }
         failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
         phase ^= 1;
+        if (!failed) tc_fence_after();
         if (!failed && lrow < 64) {
-            tc_fence_after();
             // Wr = R Kr: lane = row i, 64 key channels per thread
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
@@ -505,10 +546,12 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                     *reinterpret_cast<uint4 *>(rec + R_WQ_LO + o) = lv;
                 }
             }
-            // U: 64 value columns per thread = two slices
+        }
+        if (!failed && lrow >= 64) {
+            // U: lane 64 + token, 64 value columns per thread = two slices
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
-                float *dst = reinterpret_cast<float *>(rec + R_U + (2 * half + s2) * 8192) + lrow * kDVS;
+                float *dst = reinterpret_cast<float *>(rec + R_U + (2 * half + s2) * 8192) + (lrow - 64) * kDVS;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float x[16];
