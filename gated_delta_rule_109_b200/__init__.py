@@ -27,7 +27,8 @@ KDA_BF16, KDA_F32 = 0, 1
 
 # every symbol include/kda.h declares
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
-           "kda_forward_workspace_min_bytes", "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
+           "kda_forward_workspace_min_bytes", "kda_forward_noalloc", "kda_forward_noalloc_scratch_bytes",
+           "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_last_cuda_error", "kda_launch_count",
            "kda_version")
 
@@ -62,6 +63,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     for name in ("kda_forward_workspace_bytes", "kda_forward_workspace_min_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [i] * 6
+    lib.kda_forward_noalloc.restype = i
+    lib.kda_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
+    lib.kda_forward_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.kda_forward_noalloc_scratch_bytes.argtypes = []
     lib.kda_gdn_forward.restype = i
     lib.kda_gdn_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_gdn_decode_step.restype = i
@@ -195,6 +200,18 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_sta
     """
     return _forward("kda_forward", lambda B, T, H, dk: (B, T, H, dk), q, k, v, log_alpha, beta,
                     initial_state, out, final_state, return_final_state, scale, workspace)
+
+
+def forward_noalloc(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
+                    return_final_state=True, scale: float = 0.0):
+    """:func:`forward` through ``kda_forward_noalloc``: the two-kernel prefill on
+    scratch owned by the library (no workspace argument, nothing allocated)."""
+    return _forward("kda_forward_noalloc", lambda B, T, H, dk: (B, T, H, dk), q, k, v, log_alpha, beta,
+                    initial_state, out, final_state, return_final_state, scale)
+
+
+def noalloc_scratch_bytes() -> int:
+    return int(load().kda_forward_noalloc_scratch_bytes())
 
 
 def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, minimum=False) -> int:

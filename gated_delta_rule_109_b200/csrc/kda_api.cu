@@ -2,6 +2,7 @@
 // The contract of every entry point is documented in include/kda.h.
 #include <atomic>
 #include <math.h>
+#include <mutex>
 #include <stdint.h>
 #include <stdio.h>
 #include <string.h>
@@ -23,6 +24,19 @@ kda_status cuda_fail(cudaError_t e)
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+// Scratch of kda_forward_noalloc: part of the library's device image, so a call
+// allocates nothing.  Its address is looked up once per device; an event per
+// device orders the calls that use it, whatever their streams.
+constexpr size_t kScratchBytes = size_t(128) << 20;
+static __device__ __align__(256) uint8_t g_kda_scratch[kScratchBytes];
+constexpr int kMaxDevices = 64;
+struct ScratchSlot {
+    void *ptr = nullptr;
+    cudaEvent_t done = nullptr;
+};
+ScratchSlot g_scratch[kMaxDevices];
+std::mutex g_scratch_mu;
 
 }  // namespace
 
@@ -54,16 +68,12 @@ const char *kda_last_cuda_error(void) { return g_last_cuda_error; }
 
 namespace {
 
-// Shared by the per-channel (KDA) and scalar-gate (Gated DeltaNet / DeltaNet)
-// entry points: they differ only in the shape of log_alpha.
-kda_status forward_impl(const void *q, const void *k, const void *v, const float *log_alpha,
-                        const float *beta, const float *initial_state, float *out, float *final_state,
-                        int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
-                        void *stream, kda::GateKind gate, void *workspace = nullptr,
-                        size_t workspace_bytes = 0)
+// Argument checks of the forward entry points (nothing is enqueued unless all pass).
+kda_status validate_forward(const void *q, const void *k, const void *v, const float *log_alpha,
+                            const float *beta, const float *initial_state, float *out, float *final_state,
+                            int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
+                            kda::GateKind gate, void *workspace)
 {
-    g_last_cuda_error[0] = '\0';
-    // ---- validation: nothing is enqueued unless every check passes
     if (B <= 0 || H <= 0 || T < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
     if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
@@ -79,6 +89,22 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
     if ((initial_state && !aligned16(initial_state)) || (final_state && !aligned16(final_state)))
         return KDA_ERR_MISALIGNED;
     if (workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u)) return KDA_ERR_MISALIGNED;
+    return KDA_OK;
+}
+
+// Shared by the per-channel (KDA) and scalar-gate (Gated DeltaNet / DeltaNet)
+// entry points: they differ only in the shape of log_alpha.
+kda_status forward_impl(const void *q, const void *k, const void *v, const float *log_alpha,
+                        const float *beta, const float *initial_state, float *out, float *final_state,
+                        int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
+                        void *stream, kda::GateKind gate, void *workspace = nullptr,
+                        size_t workspace_bytes = 0)
+{
+    g_last_cuda_error[0] = '\0';
+    const kda_status vs = validate_forward(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H,
+                                           dk, dv, dtype, scale, gate, workspace);
+    if (vs != KDA_OK) return vs;
+    const bool need_gate = gate != kda::KDA_GATE_NONE;
 
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
@@ -172,6 +198,41 @@ kda_status kda_forward_ws(const void *q, const void *k, const void *v,
     return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
                         dtype, scale, stream, kda::KDA_GATE_CHANNEL, workspace, workspace_bytes);
 }
+
+kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               const float *initial_state, float *out, float *final_state,
+                               int B, int T, int H, int dk, int dv,
+                               kda_dtype dtype, float scale, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    const kda_status vs = validate_forward(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H,
+                                           dk, dv, dtype, scale, kda::KDA_GATE_CHANNEL, nullptr);
+    if (vs != KDA_OK) return vs;
+    std::lock_guard<std::mutex> lock(g_scratch_mu);
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+    ScratchSlot &slot = g_scratch[dev];
+    if (!slot.ptr) {
+        void *ptr = nullptr;
+        e = cudaGetSymbolAddress(&ptr, g_kda_scratch);
+        if (e == cudaSuccess && !slot.done) e = cudaEventCreateWithFlags(&slot.done, cudaEventDisableTiming);
+        if (e != cudaSuccess) return cuda_fail(e);
+        slot.ptr = ptr;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    e = cudaStreamWaitEvent(st, slot.done, 0);          // the previous user of the scratch is done
+    if (e != cudaSuccess) return cuda_fail(e);
+    const kda_status rs = forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk,
+                                       dv, dtype, scale, stream, kda::KDA_GATE_CHANNEL, slot.ptr, kScratchBytes);
+    e = cudaEventRecord(slot.done, st);
+    if (rs != KDA_OK) return rs;
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+size_t kda_forward_noalloc_scratch_bytes(void) { return kScratchBytes; }
 
 kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,

@@ -135,6 +135,31 @@ size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtyp
 size_t kda_forward_workspace_min_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 
 /*
+ * kda_forward_noalloc -- kda_forward on the two-kernel prefill with scratch that
+ * belongs to the library, so that the call allocates nothing and needs no
+ * workspace from the caller.
+ *
+ * The pages have no counterpart to this call: they describe no memory
+ * management.  It computes exactly what kda_forward computes, with the same
+ * arguments, layouts, statuses and aliasing rules.  The scratch is a fixed
+ * 128 MiB array in the library's device image (kda_forward_noalloc_scratch_bytes),
+ * so the sequence runs in blocks of as many 64-token chunks as fit it (results
+ * are bit-identical to kda_forward_ws with a workspace of that size).  When a
+ * single chunk of every (b, h) plus the carried state does not fit, and for
+ * other dtypes or head dimensions, the call is kda_forward.  Calls that use the
+ * scratch on one device are ordered by the library (an event per device), on
+ * any streams; they run one after another.
+ */
+kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
+                               const float *log_alpha, const float *beta,
+                               const float *initial_state, float *out, float *final_state,
+                               int B, int T, int H, int dk, int dv,
+                               kda_dtype dtype, float scale, void *stream);
+
+/* Size in bytes of the scratch kda_forward_noalloc uses on each device. */
+size_t kda_forward_noalloc_scratch_bytes(void);
+
+/*
  * kda_decode_step -- one token per sequence, state updated in place.
  *
  * The per-token update and query-state product of the decode path, whose cost
