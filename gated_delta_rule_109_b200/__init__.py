@@ -29,7 +29,8 @@ KDA_BF16, KDA_F32 = 0, 1
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
            "kda_forward_workspace_min_bytes", "kda_forward_noalloc", "kda_forward_noalloc_scratch_bytes",
            "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
-           "kda_status_string", "kda_check_status", "kda_last_cuda_error", "kda_launch_count",
+           "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
+           "kda_launch_count",
            "kda_version")
 
 _lib = None
@@ -75,6 +76,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_status_string.argtypes = [i]
     lib.kda_check_status.restype = i
     lib.kda_check_status.argtypes = [vp]
+    lib.kda_selftest_timeout.restype = i
+    lib.kda_selftest_timeout.argtypes = [ctypes.c_uint, vp]
     lib.kda_last_cuda_error.restype = ctypes.c_char_p
     lib.kda_last_cuda_error.argtypes = []
     lib.kda_launch_count.restype = ctypes.c_ulonglong
@@ -266,6 +269,14 @@ def check_status(device=None):
     """Synchronise the current stream and raise on a recorded device-side failure."""
     dev = torch.device("cuda") if device is None else torch.device(device)
     _check(load().kda_check_status(_stream(dev)), "kda_check_status")
+
+
+def selftest_timeout(wait_ms: int = 50, device=None):
+    """Enqueue the failure-path self-test (``kda_selftest_timeout``): a bounded
+    device-side wait that gives up after ~wait_ms; the next :func:`check_status`
+    raises KDAError with KDA_ERR_TIMEOUT."""
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    _check(load().kda_selftest_timeout(int(wait_ms), _stream(dev)), "kda_selftest_timeout")
 
 
 def launch_count() -> int:

@@ -264,6 +264,14 @@ kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
                        log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
 }
 
+kda_status kda_selftest_timeout(unsigned int wait_ms, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (wait_ms == 0 || wait_ms > 10000) return KDA_ERR_INVALID_ARG;
+    cudaError_t e = kda::launch_selftest_timeout(wait_ms, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
 kda_status kda_check_status(void *stream)
 {
     g_last_cuda_error[0] = '\0';

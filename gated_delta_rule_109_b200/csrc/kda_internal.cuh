@@ -57,6 +57,9 @@ size_t prefill_split_workspace_min(int B, int T, int H);    // one chunk per blo
 // SMs, else one CTA per (b, h).
 cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t take_split_device_status(unsigned int *status);
+// One CTA whose bounded wait on a barrier nothing completes gives up after about
+// wait_ms and records the device status bit (failure-path self-test).
+cudaError_t launch_selftest_timeout(unsigned int wait_ms, cudaStream_t stream);
 // Reads and clears the device status word the tensor-core kernels set when a
 // bounded wait gives up (bit 0).  Synchronous.
 cudaError_t take_device_status(unsigned int *status);

@@ -1066,6 +1066,23 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
     }
 }
 
+// ---------------------------------------------------------------- failure-path self-test
+// One CTA waits on an mbarrier phase that nothing completes, with the bounded wait
+// of the kernels above but a caller-chosen limit; giving up records the same status
+// bit the prefill kernels record.
+__global__ void selftest_timeout_kernel(long long limit_cycles)
+{
+    __shared__ __align__(8) uint64_t bar;
+    const uint32_t addr = (uint32_t)__cvta_generic_to_shared(&bar);
+    if (threadIdx.x == 0) {
+        mbar_init(addr, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    const bool ok = mbar_wait(addr, 0u, limit_cycles);
+    if (!ok && threadIdx.x == 0) atomicOr(&g_split_device_status, 1u);
+}
+
 }  // namespace
 
 bool prefill_split_supported(const ForwardArgs &a)
@@ -1141,6 +1158,18 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
         note_launch();
     }
     return cudaSuccess;
+}
+
+cudaError_t launch_selftest_timeout(unsigned int wait_ms, cudaStream_t stream)
+{
+    int dev = 0, khz = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&khz, cudaDevAttrClockRate, dev);
+    if (e != cudaSuccess) return e;
+    selftest_timeout_kernel<<<1, 32, 0, stream>>>((long long)wait_ms * (long long)khz);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) note_launch();
+    return e;
 }
 
 cudaError_t take_split_device_status(unsigned int *status)

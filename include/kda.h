@@ -236,6 +236,18 @@ const char *kda_status_string(kda_status status);
  */
 kda_status kda_check_status(void *stream);
 
+/*
+ * kda_selftest_timeout -- exercise the failure detection without a fault.
+ *
+ * Enqueues one small kernel whose bounded wait on a barrier that nothing
+ * completes gives up after about wait_ms milliseconds (1..10000; else
+ * KDA_ERR_INVALID_ARG) and records the device-side status that the prefill
+ * kernels record when one of their waits gives up; the next kda_check_status
+ * then returns KDA_ERR_TIMEOUT and clears it.  The device context stays usable.
+ * The pages have no counterpart; this exists to test the failure path.
+ */
+kda_status kda_selftest_timeout(unsigned int wait_ms, void *stream);
+
 /* Text of the last CUDA error seen by a kda_* call on this host thread
  * ("" if none).  The pointer stays valid until the next kda_* call on the
  * same thread. */
