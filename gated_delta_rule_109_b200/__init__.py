@@ -24,10 +24,12 @@ LIB_PATH = os.path.join(_PKG, "libkda.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_MISALIGNED, KDA_ERR_CUDA, KDA_ERR_TIMEOUT = range(6)
 KDA_BF16, KDA_F32 = 0, 1
+KDA_PREP_LOGSIGMOID_GATE, KDA_PREP_L2NORM_QK = 1, 2
 
 # every symbol include/kda.h declares
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
-           "kda_forward_workspace_min_bytes", "kda_forward_noalloc", "kda_forward_noalloc_scratch_bytes",
+           "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_forward_noalloc",
+           "kda_forward_noalloc_scratch_bytes",
            "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
            "kda_launch_count",
@@ -64,6 +66,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     for name in ("kda_forward_workspace_bytes", "kda_forward_workspace_min_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [i] * 6
+    lib.kda_forward_raw.restype = i
+    lib.kda_forward_raw.argtypes = [vp] * 8 + [i] * 6 + [f, ctypes.c_uint, vp, ctypes.c_size_t, vp]
     lib.kda_forward_noalloc.restype = i
     lib.kda_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_forward_noalloc_scratch_bytes.restype = ctypes.c_size_t
@@ -203,6 +207,41 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_sta
     """
     return _forward("kda_forward", lambda B, T, H, dk: (B, T, H, dk), q, k, v, log_alpha, beta,
                     initial_state, out, final_state, return_final_state, scale, workspace)
+
+
+def forward_raw(q, k, v, gate, beta, initial_state=None, *, workspace, logsigmoid_gate=True,
+                normalize_qk=True, out=None, final_state=None, return_final_state=True, scale: float = 0.0):
+    """Prefill on raw activations (``kda_forward_raw``): with ``logsigmoid_gate``
+    the gate ``[B,T,H,dk]`` holds pre-activations x and log alpha = log sigmoid(x);
+    with ``normalize_qk`` q and k rows are L2-normalised.  Both run inside the
+    two-kernel prefill (bf16, dk = dv = 128), which needs ``workspace``."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q)
+    _need(q, "q", (B, T, H, dk), q.dtype, dev)
+    _need(k, "k", (B, T, H, dk), q.dtype, dev)
+    _need(v, "v", (B, T, H, dv), q.dtype, dev)
+    _need(gate, "gate", (B, T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    _need(out, "out", (B, T, H, dv), torch.float32, dev)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    if final_state is not None:
+        _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
+    if workspace is None or workspace.device != dev or not workspace.is_contiguous():
+        raise ValueError("workspace must be a contiguous tensor on %s" % dev)
+    prep = (KDA_PREP_LOGSIGMOID_GATE if logsigmoid_gate else 0) | (KDA_PREP_L2NORM_QK if normalize_qk else 0)
+    st = lib.kda_forward_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(initial_state), _ptr(out),
+                             _ptr(final_state), B, T, H, dk, dv, code, float(scale), prep, _ptr(workspace),
+                             workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(st, "kda_forward_raw")
+    return out, final_state
 
 
 def forward_noalloc(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,

@@ -98,7 +98,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
                         const float *beta, const float *initial_state, float *out, float *final_state,
                         int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
                         void *stream, kda::GateKind gate, void *workspace = nullptr,
-                        size_t workspace_bytes = 0)
+                        size_t workspace_bytes = 0, int prep_flags = 0)
 {
     g_last_cuda_error[0] = '\0';
     const kda_status vs = validate_forward(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H,
@@ -123,6 +123,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
     a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
     a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
     a.gate = gate;
+    a.prep_flags = prep_flags;
     cudaError_t e;
     if (workspace && kda::prefill_split_supported(a) &&
         workspace_bytes >= kda::prefill_split_workspace_min(B, T, H))
@@ -174,6 +175,28 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
 {
     return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
                         dtype, scale, stream, kda::KDA_GATE_CHANNEL);
+}
+
+kda_status kda_forward_raw(const void *q, const void *k, const void *v,
+                           const float *gate, const float *beta,
+                           const float *initial_state, float *out, float *final_state,
+                           int B, int T, int H, int dk, int dv,
+                           kda_dtype dtype, float scale, unsigned int prep,
+                           void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (prep & ~(unsigned)(KDA_PREP_LOGSIGMOID_GATE | KDA_PREP_L2NORM_QK)) return KDA_ERR_INVALID_ARG;
+    const kda_status vs = validate_forward(q, k, v, gate, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                                           dtype, scale, kda::KDA_GATE_CHANNEL, workspace);
+    if (vs != KDA_OK) return vs;
+    if (prep != 0 && T > 0) {
+        // the fused steps live in the two-kernel prefill's first kernel
+        if (dtype != KDA_BF16 || dk != 128 || dv != 128 || !workspace ||
+            workspace_bytes < kda::prefill_split_workspace_min(B, T, H))
+            return KDA_ERR_UNSUPPORTED;
+    }
+    return forward_impl(q, k, v, gate, beta, initial_state, out, final_state, B, T, H, dk, dv, dtype, scale,
+                        stream, kda::KDA_GATE_CHANNEL, workspace, workspace_bytes, (int)prep);
 }
 
 size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype)

@@ -25,7 +25,13 @@ struct ForwardArgs {
     kda_dtype dtype;
     float scale;
     int gate;                 // GateKind
+    int prep_flags;           // kPrep* (two-kernel prefill only)
 };
+
+// Optional steps before the path, fused into the two-kernel prefill's first kernel:
+// log_alpha holds gate pre-activations x and log alpha = log(sigmoid(x)); q and k
+// rows are L2-normalised (a zero row stays zero).
+constexpr int kPrepLogsigmoidGate = 1, kPrepNormalizeQK = 2;
 
 struct DecodeArgs {
     const void *q, *k, *v;

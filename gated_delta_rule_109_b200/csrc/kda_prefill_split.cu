@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kNT, 2)
 prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                     const float *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                    int n0, int nb, float scale)
+                    int n0, int nb, float scale, int prep_flags)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -121,6 +121,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     const int lrow = 32 * (warp & 3) + lane;          // tensor-memory lane of the readouts
     const int half = warp >> 2;
     const int ch0 = 16 * warp;                        // pass 1/2: channels ch0..ch0+15, tokens lane, lane+32
+    const bool gate_act = (prep_flags & kPrepLogsigmoidGate) != 0;   // log_alpha holds gate pre-activations
+    const bool norm_qk = (prep_flags & kPrepNormalizeQK) != 0;       // q, k are L2-normalised here
     uint8_t *rec = ws + ((size_t)bh * nb + nloc) * kRec;
     auto row = [&](int t) { return ((size_t)b * T + t0 + t) * H + h; };
 
@@ -186,7 +188,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 #pragma unroll 8
         for (int i = 0; i < 32; ++i) {
             float *gp = Gs + (32 * th + i) * kGP + ch;
-            run += *gp;
+            const float x = *gp;
+            run += (gate_act && 32 * th + i < c) ? log_sigmoid(x) : x;
             *gp = run;
         }
         sTot[th * kDK + ch] = run;
@@ -219,6 +222,49 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             G[hf][4 * j] = gv.x; G[hf][4 * j + 1] = gv.y; G[hf][4 * j + 2] = gv.z; G[hf][4 * j + 3] = gv.w;
         }
     }
+    __syncthreads();
+    // ---- optional L2 normalisation of q and k rows: squared-norm partials of this
+    // thread's 16 channels, summed over the eight warps through the (now free) scratch
+    float inv_k[2] = {1.f, 1.f}, inv_q[2] = {1.f, 1.f};
+    float *sInv = sGm + 4 * kDK;            // [2][64]: 1/|k_t|, 1/|q_t| (for the wide path)
+    if (norm_qk) {
+        float *part = Gs;                   // [2][8 warps][64 tokens]
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+                const __nv_bfloat16 *kb16 = reinterpret_cast<const __nv_bfloat16 *>(&kv4[2 * hf + g]);
+                const __nv_bfloat16 *qb16 = reinterpret_cast<const __nv_bfloat16 *>(&qv4[2 * hf + g]);
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                    const float kf = __bfloat162float(kb16[i]), qf = __bfloat162float(qb16[i]);
+                    sk += kf * kf;
+                    sq += qf * qf;
+                }
+            }
+            part[warp * kC + lane + 32 * hf] = sk;
+            part[8 * kC + warp * kC + lane + 32 * hf] = sq;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+            float sk = 0.f, sq = 0.f;
+#pragma unroll
+            for (int w = 0; w < 8; ++w) {
+                sk += part[w * kC + lane + 32 * hf];
+                sq += part[8 * kC + w * kC + lane + 32 * hf];
+            }
+            inv_k[hf] = sk > 0.f ? 1.f / sqrtf(sk) : 0.f;
+            inv_q[hf] = sq > 0.f ? 1.f / sqrtf(sq) : 0.f;
+            if (warp == 0) {
+                sInv[lane + 32 * hf] = inv_k[hf];
+                sInv[kC + lane + 32 * hf] = inv_q[hf];
+            }
+        }
+    } else if (warp == 0) {
+        sInv[lane] = sInv[lane + 32] = sInv[kC + lane] = sInv[kC + lane + 32] = 1.f;
+    }
     __syncthreads();        // the split pass writes over the scratch
 
     bool wide = false;      // some |G - m| > 40 (or |m| > 80): the split exponentials could overflow
@@ -235,8 +281,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 const __nv_bfloat16 *qb16 = reinterpret_cast<const __nv_bfloat16 *>(&qv);
 #pragma unroll
                 for (int i = 0; i < 8; ++i) {
-                    kk[i] = __bfloat162float(kb16[i]);
-                    qq[i] = __bfloat162float(qb16[i]);
+                    kk[i] = __bfloat162float(kb16[i]) * inv_k[hf];
+                    qq[i] = __bfloat162float(qb16[i]) * inv_q[hf];
                 }
             }
             const uint32_t ok = core_off(t, ch0 + 8 * g, RW_SO, RW_SI);
@@ -268,15 +314,19 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         }
     }
     const bool wide_path = __syncthreads_or(wide) != 0;
-    // V (exact bf16; rows past the chunk's end zero-filled) into its operand tile
+    // V (exact bf16; rows past the chunk's end zero-filled) into its operand tile; a
+    // wide-range chunk first finishes with the per-token scalars kept in that region
+    auto issue_v = [&]() {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int id = tid + kNT * r, t = id >> 4, g = id & 15;
-        const bool okt = t < c;
-        cp_async16(sbase + PP_V + core_off(t, 8 * g, RW_SO, RW_SI), v + row(okt ? t : 0) * kDV + 8 * g,
-                   okt ? 16u : 0u);
-    }
-    cp_async_commit();
+        for (int r = 0; r < 4; ++r) {
+            const int id = tid + kNT * r, t = id >> 4, g = id & 15;
+            const bool okt = t < c;
+            cp_async16(sbase + PP_V + core_off(t, 8 * g, RW_SO, RW_SI), v + row(okt ? t : 0) * kDV + 8 * g,
+                       okt ? 16u : 0u);
+        }
+        cp_async_commit();
+    };
+    if (!wide_path) issue_v();
     if (wide_path) {
         // rare: redo the scan from the inputs and keep G for the pairwise sums; put
         // k e^G, scale q e^G and k e^{G_last - G} where Kr, Qr and Kb were, and set
@@ -289,6 +339,10 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 const int chn = ch0 + e;
                 float a = (t < c) ? log_alpha[row(t) * kDK + chn] : 0.f;
                 float a0 = (lane < c) ? log_alpha[row(lane) * kDK + chn] : 0.f;
+                if (gate_act) {
+                    a = (t < c) ? log_sigmoid(a) : 0.f;
+                    a0 = (lane < c) ? log_sigmoid(a0) : 0.f;
+                }
 #pragma unroll
                 for (int o = 1; o < 32; o <<= 1) {
                     const float ua = __shfl_up_sync(0xffffffffu, a, o);
@@ -311,8 +365,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
                 const int chn = 8 * cg + i;
-                const float kk = (t < c) ? __bfloat162float(k[row(t) * kDK + chn]) : 0.f;
-                const float qq = (t < c) ? __bfloat162float(q[row(t) * kDK + chn]) : 0.f;
+                const float kk = (t < c) ? __bfloat162float(k[row(t) * kDK + chn]) * sInv[t] : 0.f;
+                const float qq = (t < c) ? __bfloat162float(q[row(t) * kDK + chn]) * sInv[kC + t] : 0.f;
                 const float gg = sG[t * kDK + chn];
                 const float eg = __expf(gg);
                 y1[i] = kk * eg;
@@ -404,6 +458,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                     for (int cc = 0; cc < kDK; ++cc)
                         acc += __bfloat162float(xi[cc]) * __bfloat162float(kj[cc]) *
                                __expf(sG[i * kDK + cc] - sG[j * kDK + cc]);
+                    acc *= sInv[(isM ? kC : 0) + i] * sInv[j];
                 }
                 y[e] = isM ? scale * acc : sBeta[i] * acc;
             }
@@ -419,6 +474,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             }
         }
         __syncthreads();
+        issue_v();                           // the per-token scalars are no longer needed
         for (int id = tid; id < 64 * 64; id += kNT) Am[(id >> 6) * kPitch + (id & 63)] = Aw[id];
     }
     __syncthreads();
@@ -1141,7 +1197,8 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
         const int nb = min(L, nchunks - n0);
         prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
             static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
-            static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale);
+            static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale,
+            a.prep_flags);
         e = cudaGetLastError();
         if (e != cudaSuccess) return e;
         note_launch();

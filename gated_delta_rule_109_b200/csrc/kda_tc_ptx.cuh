@@ -108,6 +108,12 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
 
+// log(sigmoid(x)) without overflow for either sign of x
+__device__ __forceinline__ float log_sigmoid(float x)
+{
+    return x < 0.f ? x - log1pf(expf(x)) : -log1pf(expf(-x));
+}
+
 // Bounded wait for the phase with the given parity; false if it never completed
 // within `limit` SM cycles.
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, long long limit = kWaitCycles)

@@ -22,6 +22,11 @@ Input recipe (one draw order for every workload, from one seeded
 5. ``x_beta``  ~ N(mu_b, sd_b); ``beta = sigmoid(x_beta)`` in fp32.
 6. ``S_0`` ~ N(0, sd_s) in fp32 when the workload carries a state, else absent.
 
+Raw-activation variant (``make_raw_inputs``, for the fused steps before the
+path): the same draws with q and k cast to the input dtype without
+normalisation, and the gate returned as its pre-activation ``x_alpha``
+(fp32) instead of ``logsigmoid(x_alpha)``.
+
 Shapes follow the library's layout: q, k ``[B, T, H, dk]``; v ``[B, T, H, dv]``;
 log_alpha ``[B, T, H, dk]`` fp32; beta ``[B, T, H]`` fp32; state
 ``[B, H, dk, dv]`` fp32.  Decode workloads draw every step at once with a
@@ -127,3 +132,27 @@ def make_inputs(w: Workload, device="cpu", steps: Optional[int] = None) -> dict:
     return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(),
                 log_alpha=log_alpha.contiguous(), beta=beta.contiguous(),
                 initial_state=s0)
+
+
+def make_raw_inputs(w: Workload, device="cpu") -> dict:
+    """The draws of :func:`make_inputs` before the steps the prefill can fuse: q, k
+    cast to the input dtype without L2 normalisation, and ``gate`` = the gate
+    pre-activations x_alpha (fp32).  Prefill workloads only."""
+    if w.is_decode:
+        raise ValueError("prefill workloads only")
+    gen = torch.Generator(device=device)
+    gen.manual_seed(w.seed)
+    lead = (w.B, w.T, w.H)
+    dt = w.torch_dtype
+    q = _normal(lead + (w.dk,), gen, device).to(dt)
+    k = _normal(lead + (w.dk,), gen, device).to(dt)
+    v = _normal(lead + (w.dv,), gen, device).to(dt)
+    xa = _normal(lead + (w.dk,), gen, device, w.alpha_mu, w.alpha_sd)
+    xb = _normal(lead, gen, device, w.beta_mu, w.beta_sd)
+    beta = torch.sigmoid(xb)
+    del xb
+    s0 = None
+    if w.state_sd is not None:
+        s0 = _normal((w.B, w.H, w.dk, w.dv), gen, device, 0.0, w.state_sd)
+    return dict(q=q.contiguous(), k=k.contiguous(), v=v.contiguous(), gate=xa.contiguous(),
+                beta=beta.contiguous(), initial_state=s0)

@@ -134,6 +134,42 @@ kda_status kda_forward_ws(const void *q, const void *k, const void *v,
 size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 size_t kda_forward_workspace_min_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 
+/* Steps before the path that kda_forward_raw can fuse into the prefill. */
+enum {
+    KDA_PREP_LOGSIGMOID_GATE = 1,  /* gate holds pre-activations x; log alpha = log(sigmoid(x)) */
+    KDA_PREP_L2NORM_QK = 2         /* q and k rows are L2-normalised (a zero row stays zero) */
+};
+
+/*
+ * kda_forward_raw -- kda_forward_ws on raw layer activations.
+ *
+ * The step before the path is fused into the prefill's first kernel: with
+ * KDA_PREP_LOGSIGMOID_GATE, `gate` [B, T, H, dk] fp32 holds the gate
+ * pre-activations x and the decay is alpha = sigmoid(x) (the sigmoid-like
+ * retention gate of "KDA Technical Deep Dive", §How the Kimi gate changes
+ * memory); with KDA_PREP_L2NORM_QK, q and k are divided by the L2 norm of
+ * their dk channels per (b, t, h) (the normalised keys and queries that "Kimi
+ * Delta Attention: The Linear Attention Behind Kimi K2 and Qwen3" expects the
+ * path to receive).  Both run in fp32 on the bf16 inputs before the chunk
+ * algebra; nothing is written back.
+ *
+ *   prep       an OR of KDA_PREP_* flags (other bits: KDA_ERR_INVALID_ARG).
+ *              prep = 0 is exactly kda_forward_ws.
+ *   gate       [B, T, H, dk] fp32, 16-byte aligned: log alpha, or x with
+ *              KDA_PREP_LOGSIGMOID_GATE.
+ *   workspace, workspace_bytes  as for kda_forward_ws.
+ *
+ * With prep != 0 the call needs the two-kernel path: bf16 inputs, dk = dv = 128
+ * and a workspace of at least kda_forward_workspace_min_bytes(); otherwise it
+ * returns KDA_ERR_UNSUPPORTED before anything is enqueued.
+ */
+kda_status kda_forward_raw(const void *q, const void *k, const void *v,
+                           const float *gate, const float *beta,
+                           const float *initial_state, float *out, float *final_state,
+                           int B, int T, int H, int dk, int dv,
+                           kda_dtype dtype, float scale, unsigned int prep,
+                           void *workspace, size_t workspace_bytes, void *stream);
+
 /*
  * kda_forward_noalloc -- kda_forward on the two-kernel prefill with scratch that
  * belongs to the library, so that the call allocates nothing and needs no

@@ -16,6 +16,8 @@ delta-rule write, read with the query scaled by 1/sqrt(d_k)):
                      used for small cases and to cross-check ``forward``.
 * ``gdn_forward`` -- the scalar-gate variants (Gated DeltaNet, DeltaNet) as
                      ``forward`` with the gate repeated over key channels.
+* ``forward_raw`` -- raw activations: sigmoid gate pre-activations and
+                     unnormalised q, k, prepared in fp64, then ``forward``.
 
 Both store the state as ``[B, H, dk, dv]`` (the transpose of the page's
 (d_v, d_k) matrix), so the per-channel decay scales rows and the page's
@@ -150,6 +152,27 @@ def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, scale=None, nthrea
             raise ValueError("log_alpha has shape %s, expected %s" % (g.shape, (B, T, H)))
         la = np.ascontiguousarray(np.repeat(g[..., None], dk, axis=-1))
     return forward(qf, k, v, la, beta, initial_state, scale=scale, nthreads=nthreads)
+
+
+def forward_raw(q, k, v, gate, beta, initial_state=None, logsigmoid_gate=True, normalize_qk=True,
+                scale=None, nthreads=0):
+    """fp64 forward of raw layer activations: the steps before the path, then :func:`forward`.
+
+    With ``logsigmoid_gate`` the gate holds pre-activations x of the sigmoid
+    retention gate ("KDA Technical Deep Dive", §How the Kimi gate changes
+    memory: alpha a sigmoid-like value in (0, 1)), so log alpha = log(sigmoid(x))
+    = -log(1 + e^{-x}).  With ``normalize_qk`` q and k are divided by the L2 norm
+    of their dk channels per (b, t, h) (the normalised keys the KDA page says the
+    path receives); a zero row stays zero.  Both in fp64 on the exact inputs.
+    """
+    q64, k64, g64 = (_as_f64(x) for x in (q, k, gate))
+    if normalize_qk:
+        def unit(x):
+            n = np.linalg.norm(x, axis=-1, keepdims=True)
+            return np.where(n > 0, x / np.where(n > 0, n, 1.0), 0.0)
+        q64, k64 = unit(q64), unit(k64)
+    la = -np.logaddexp(0.0, -g64) if logsigmoid_gate else g64
+    return forward(q64, k64, v, la, beta, initial_state, scale=scale, nthreads=nthreads)
 
 
 def parity_error(x_gpu, x_ref) -> float:

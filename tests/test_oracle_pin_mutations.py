@@ -115,3 +115,41 @@ def test_unmutated_gdn_copy_passes_every_pin(monkeypatch):
     monkeypatch.setattr(oracle, "gdn_forward", _make_gdn("none"))
     for pin in GDN_PINS:
         pin()
+
+
+def _make_raw(mutation):
+    """oracle.forward_raw with one slip in the steps before the path."""
+    def raw(q, k, v, gate, beta, initial_state=None, logsigmoid_gate=True, normalize_qk=True, scale=None,
+            nthreads=0):
+        q64, k64, g64 = (oracle._as_f64(x) for x in (q, k, gate))
+        if normalize_qk:
+            axis = 1 if mutation == "norm_over_tokens" else -1
+            q64 = q64 / np.linalg.norm(q64, axis=axis, keepdims=True)
+            k64 = k64 / np.linalg.norm(k64, axis=axis, keepdims=True)
+        if logsigmoid_gate:
+            la = np.log(1.0 / (1.0 + np.exp(-g64))) if mutation != "sigmoid_not_logged" else 1.0 / (1.0 + np.exp(-g64)) - 1.0
+        else:
+            la = g64
+        return oracle.forward(q64, k64, v, la, beta, initial_state, scale=scale)
+    return raw
+
+
+RAW_PINS = [pins.test_raw_gate_is_log_of_sigmoid, pins.test_raw_normalisation_is_per_row_and_scale_free]
+
+
+@pytest.mark.parametrize("mutation", ["norm_over_tokens", "sigmoid_not_logged"])
+def test_some_raw_pin_fails_on_planted_mistake(mutation, monkeypatch):
+    monkeypatch.setattr(oracle, "forward_raw", _make_raw(mutation))
+    failed = 0
+    for pin in RAW_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, "no raw-activation pin caught %s" % mutation
+
+
+def test_unmutated_raw_copy_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(oracle, "forward_raw", _make_raw("none"))
+    for pin in RAW_PINS:
+        pin()

@@ -287,3 +287,63 @@ def test_gdn_forward_empty_and_shape_check():
     np.testing.assert_array_equal(s, S0)
     with pytest.raises(ValueError):
         oracle.gdn_forward(q, k, v, la, beta, S0)          # a per-channel gate is not accepted
+
+
+# ---------------------------------------------------------------- O10 raw activations
+def _raw(seed, B=2, T=19, H=3, dk=8, dv=5):
+    rng = np.random.default_rng(seed)
+    q = (3.0 * rng.standard_normal((B, T, H, dk))).astype(np.float32)
+    k = (0.5 * rng.standard_normal((B, T, H, dk))).astype(np.float32)
+    v = rng.standard_normal((B, T, H, dv)).astype(np.float32)
+    x = (2.0 + rng.standard_normal((B, T, H, dk))).astype(np.float32)
+    beta = rng.random((B, T, H)).astype(np.float32)
+    S0 = rng.standard_normal((B, H, dk, dv))
+    return q, k, v, x, beta, S0
+
+
+def test_raw_gate_is_log_of_sigmoid():
+    """gate pre-activations x give the same result as log alpha = log(1 / (1 + e^-x))
+    written out directly (unit q, k, so normalisation is the identity)."""
+    q, k, v, x, beta, S0 = _raw(31)
+    q = (q / np.linalg.norm(q.astype(np.float64), axis=-1, keepdims=True)).astype(np.float32)
+    k = (k / np.linalg.norm(k.astype(np.float64), axis=-1, keepdims=True)).astype(np.float32)
+    la = np.log(1.0 / (1.0 + np.exp(-x.astype(np.float64))))
+    o_ref, s_ref = oracle.forward(q, k, v, la, beta, S0)
+    o, s = oracle.forward_raw(q, k, v, x, beta, S0, logsigmoid_gate=True, normalize_qk=False)
+    np.testing.assert_allclose(o, o_ref, rtol=0, atol=2e-6 * np.abs(o_ref).max())
+    np.testing.assert_allclose(s, s_ref, rtol=0, atol=2e-6 * np.abs(s_ref).max())
+
+
+def test_raw_normalisation_is_per_row_and_scale_free():
+    """Rescaling each (b, t, h) row of q and k by a positive factor changes nothing;
+    unit rows reproduce forward(); the result depends on q, k only through q/|q|, k/|k|."""
+    q, k, v, x, beta, S0 = _raw(32)
+    la = -np.logaddexp(0.0, -x.astype(np.float64))
+    rng = np.random.default_rng(5)
+    cq = rng.uniform(0.1, 10.0, q.shape[:-1] + (1,)).astype(np.float32)
+    ck = rng.uniform(0.1, 10.0, k.shape[:-1] + (1,)).astype(np.float32)
+    o1, s1 = oracle.forward_raw(q, k, v, la, beta, S0, logsigmoid_gate=False, normalize_qk=True)
+    o2, s2 = oracle.forward_raw(q * cq, k * ck, v, la, beta, S0, logsigmoid_gate=False, normalize_qk=True)
+    assert oracle.parity_error(o2, o1) < 1e-5 and oracle.parity_error(s2, s1) < 1e-5
+    qn = q / np.linalg.norm(q.astype(np.float64), axis=-1, keepdims=True)
+    kn = k / np.linalg.norm(k.astype(np.float64), axis=-1, keepdims=True)
+    o3, s3 = oracle.forward(qn, kn, v, la, beta, S0)
+    assert oracle.parity_error(o3, o1) < 1e-5 and oracle.parity_error(s3, s1) < 1e-5
+    # and the factors matter without normalisation
+    o4, _ = oracle.forward_raw(q * cq, k * ck, v, la, beta, S0, logsigmoid_gate=False, normalize_qk=False)
+    assert oracle.parity_error(o4, o1) > 1e-2
+
+
+def test_raw_zero_key_row_writes_nothing():
+    q, k, v, x, beta, S0 = _raw(33, B=1, H=1, T=6)
+    k[0, 3, 0] = 0.0
+    o, s = oracle.forward_raw(q, k, v, x, beta, S0)
+    assert np.isfinite(o).all() and np.isfinite(s).all()
+    # token 3 with a zero key only decays the state: same as beta = 0 there
+    b2 = beta.copy()
+    b2[0, 3, 0] = 0.0
+    k2 = k.copy()
+    k2[0, 3, 0] = 1.0
+    o2, s2 = oracle.forward_raw(q, k2, v, x, b2, S0)
+    np.testing.assert_allclose(s, s2, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(o[0, 4:], o2[0, 4:], rtol=1e-12, atol=1e-12)
