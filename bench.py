@@ -451,6 +451,56 @@ def _add_gdn(line, args, w, world, device, hbm):
                      "algorithmic_bytes_per_launch": alg_bytes}}
 
 
+def _add_raw(line, args, w, world, device, hbm):
+    """The prefill on raw activations (gate pre-activations, unnormalised q and k):
+    the steps before the path fused (kda_forward_raw) against the same steps as
+    separate torch passes followed by kda_forward_ws."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    x = I.make_raw_inputs(w, device)
+    ws = kda.make_workspace(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, device=device)
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+    sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
+    names = ("q", "k", "v", "gate", "beta")
+
+    def fused():
+        kda.forward_raw(*(x[n] for n in names), x["initial_state"], workspace=ws, out=out, final_state=sT)
+
+    def unfused():
+        la = torch.nn.functional.logsigmoid(x["gate"])
+        qn = torch.nn.functional.normalize(x["q"].float(), dim=-1).to(x["q"].dtype)
+        kn = torch.nn.functional.normalize(x["k"].float(), dim=-1).to(x["k"].dtype)
+        kda.forward(qn, kn, x["v"], la, x["beta"], x["initial_state"], out=out, final_state=sT, workspace=ws)
+
+    res = {}
+    for name, fn in (("fused", fused), ("unfused", unfused)):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        stream = torch.cuda.current_stream(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(device)
+        torch.cuda.synchronize(device)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        res[name] = max_over_ranks(e0.elapsed_time(e1), device) / args.steps
+    kda.check_status(device)
+    del ws
+    tokens = w.B * w.T
+    line["raw_activation_prefill"] = {
+        "workload": w.name,
+        "inputs": "gate pre-activations x ~ N(%g,%g) and unnormalised q, k ~ N(0,1)" % (w.alpha_mu, w.alpha_sd),
+        "value": tokens * world / (res["fused"] / 1e3), "unit": "tokens/s",
+        "ms_per_step": res["fused"],
+        "unfused_ms_per_step": res["unfused"],
+        "unfused": "torch logsigmoid + two normalize passes, then kda_forward_ws",
+        "kernel": "prefill_prep_kernel (with the fused steps) + prefill_chain_kernel"}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -575,6 +625,8 @@ def main(argv=None):
         _add_decode(line, args, rank, world, device, hbm)
     if not args.no_variants and args.only == "all":
         _add_gdn(line, args, w, world, device, hbm)
+        if ws_bytes:
+            _add_raw(line, args, w, world, device, hbm)
 
     if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],
