@@ -28,7 +28,8 @@ KDA_PREP_LOGSIGMOID_GATE, KDA_PREP_L2NORM_QK = 1, 2
 
 # every symbol include/kda.h declares
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
-           "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_forward_noalloc",
+           "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_segment_local",
+           "kda_segment_start_state", "kda_segment_correct", "kda_forward_noalloc",
            "kda_forward_noalloc_scratch_bytes",
            "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
@@ -68,6 +69,12 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
         getattr(lib, name).argtypes = [i] * 6
     lib.kda_forward_raw.restype = i
     lib.kda_forward_raw.argtypes = [vp] * 8 + [i] * 6 + [f, ctypes.c_uint, vp, ctypes.c_size_t, vp]
+    lib.kda_segment_local.restype = i
+    lib.kda_segment_local.argtypes = [vp] * 9 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
+    lib.kda_segment_start_state.restype = i
+    lib.kda_segment_start_state.argtypes = [vp, vp, i, vp, i, i, i, i, vp]
+    lib.kda_segment_correct.restype = i
+    lib.kda_segment_correct.argtypes = [vp] * 4 + [i] * 5 + [vp, ctypes.c_size_t, vp]
     lib.kda_forward_noalloc.restype = i
     lib.kda_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_forward_noalloc_scratch_bytes.restype = ctypes.c_size_t
@@ -242,6 +249,63 @@ def forward_raw(q, k, v, gate, beta, initial_state=None, *, workspace, logsigmoi
                              workspace.numel() * workspace.element_size(), _stream(dev))
     _check(st, "kda_forward_raw")
     return out, final_state
+
+
+def segment_local(q, k, v, log_alpha, beta, initial_state=None, *, workspace, scale: float = 0.0):
+    """Phase 1 of a time-axis split (``kda_segment_local``): returns
+    ``(out, local_final, transfer)`` of one contiguous segment of a sequence."""
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    code = _dtype_code(q)
+    for t, n, shp in ((q, "q", (B, T, H, dk)), (k, "k", (B, T, H, dk)), (v, "v", (B, T, H, dv))):
+        _need(t, n, shp, q.dtype, dev)
+    _need(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    out = torch.empty((B, T, H, dv), dtype=torch.float32, device=dev)
+    local_final = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    transfer = torch.empty((B, H, dk, dk), dtype=torch.float32, device=dev)
+    st = lib.kda_segment_local(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                               _ptr(out), _ptr(local_final), _ptr(transfer), B, T, H, dk, dv, code, float(scale),
+                               _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(st, "kda_segment_local")
+    return out, local_final, transfer
+
+
+def segment_start_state(transfers, local_finals):
+    """The state entering the next segment (``kda_segment_start_state``) from the
+    stacked ``[R, B, H, dk, dk]`` transfers and ``[R, B, H, dk, dv]`` local finals
+    of the earlier segments."""
+    R, B, H, dk, _ = transfers.shape
+    dv = local_finals.shape[-1]
+    dev = transfers.device
+    _need(transfers, "transfers", (R, B, H, dk, dk), torch.float32, dev)
+    _need(local_finals, "local_finals", (R, B, H, dk, dv), torch.float32, dev)
+    start = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    st = load().kda_segment_start_state(_ptr(transfers), _ptr(local_finals), R, _ptr(start), B, H, dk, dv,
+                                        _stream(dev))
+    _check(st, "kda_segment_start_state")
+    return start
+
+
+def segment_correct(start, local_final, out, *, workspace, final_state=None):
+    """Phase 3 (``kda_segment_correct``): ``out`` += the start state's outputs;
+    returns ``final_state`` (= local_final + the propagated start)."""
+    B, T, H, dv = out.shape
+    dk = start.shape[-2]
+    dev = out.device
+    _need(start, "start", (B, H, dk, dv), torch.float32, dev)
+    _need(local_final, "local_final", (B, H, dk, dv), torch.float32, dev)
+    _need(out, "out", (B, T, H, dv), torch.float32, dev)
+    if final_state is None:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
+    st = load().kda_segment_correct(_ptr(start), _ptr(local_final), _ptr(out), _ptr(final_state), B, T, H, dk, dv,
+                                    _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(st, "kda_segment_correct")
+    return final_state
 
 
 def forward_noalloc(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,

@@ -199,6 +199,67 @@ kda_status kda_forward_raw(const void *q, const void *k, const void *v,
                         stream, kda::KDA_GATE_CHANNEL, workspace, workspace_bytes, (int)prep);
 }
 
+kda_status kda_segment_local(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             const float *initial_state, float *out, float *local_final, float *transfer,
+                             int B, int T, int H, int dk, int dv,
+                             kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (T <= 0 || !local_final || !transfer) return KDA_ERR_INVALID_ARG;
+    const kda_status vs = validate_forward(q, k, v, log_alpha, beta, initial_state, out, local_final, B, T, H, dk,
+                                           dv, dtype, scale, kda::KDA_GATE_CHANNEL, workspace);
+    if (vs != KDA_OK) return vs;
+    if (!aligned16(transfer)) return KDA_ERR_MISALIGNED;
+    if (dtype != KDA_BF16 || dk != 128 || dv != 128 || !workspace ||
+        workspace_bytes < kda::prefill_split_workspace_full(B, T, H))
+        return KDA_ERR_UNSUPPORTED;
+    kda::ForwardArgs a;
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta;
+    a.s0 = initial_state; a.out = out; a.sT = local_final;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = dtype;
+    a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
+    a.gate = kda::KDA_GATE_CHANNEL;
+    a.prep_flags = 0;
+    const cudaError_t e = kda::launch_segment_local(a, transfer, static_cast<uint8_t *>(workspace),
+                                                    static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_segment_start_state(const float *transfers, const float *local_finals, int R,
+                                   float *start, int B, int H, int dk, int dv, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (R < 1 || B <= 0 || H <= 0 || !transfers || !local_finals || !start) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H > (int64_t)INT32_MAX / 4) return KDA_ERR_INVALID_ARG;
+    if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(transfers) || !aligned16(local_finals) || !aligned16(start)) return KDA_ERR_MISALIGNED;
+    const cudaError_t e = kda::launch_affine_compose(transfers, local_finals, R, B * H, start,
+                                                     static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+kda_status kda_segment_correct(const float *start, const float *local_final, float *out, float *final_state,
+                               int B, int T, int H, int dk, int dv,
+                               const void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (B <= 0 || H <= 0 || T <= 0 || !start || !local_final || !out || !workspace) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H > (int64_t)INT32_MAX / 4) return KDA_ERR_INVALID_ARG;
+    if (dk != 128 || dv != 128) return KDA_ERR_UNSUPPORTED;
+    if (!aligned16(start) || !aligned16(local_final) || !aligned16(out) ||
+        (final_state && !aligned16(final_state)) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+        return KDA_ERR_MISALIGNED;
+    if (workspace_bytes < kda::prefill_split_workspace_full(B, T, H)) return KDA_ERR_UNSUPPORTED;
+    kda::ForwardArgs a = {};
+    a.out = out; a.sT = final_state;
+    a.B = B; a.T = T; a.H = H; a.dk = dk; a.dv = dv; a.dtype = KDA_BF16;
+    a.gate = kda::KDA_GATE_CHANNEL;
+    const cudaError_t e = kda::launch_segment_correct(a, start, local_final, static_cast<const uint8_t *>(workspace),
+                                                      static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
 size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype)
 {
     if (B <= 0 || H <= 0 || T <= 0 || dtype != KDA_BF16 || dk != 128 || dv != 128) return 0;

@@ -63,6 +63,17 @@ size_t prefill_split_workspace_min(int B, int T, int H);    // one chunk per blo
 // SMs, else one CTA per (b, h).
 cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream);
 cudaError_t take_split_device_status(unsigned int *status);
+// Time-axis split (the chain is linear in (U, S_0)), one contiguous segment of the
+// sequence per call; the workspace holds the whole segment's records:
+//   local:   outputs and final state (a.sT) from a.s0 (zero if null), and the
+//            transfer [B,H,dk,dk] = the state alone propagated from I;
+//   correct: out += outputs of `start` propagated alone; a.sT = local_final + that state;
+//   compose: start = F_0, then F_j + P_j start for j = 1..R-1 (fp32).
+cudaError_t launch_segment_local(const ForwardArgs &a, float *transfer, uint8_t *ws, cudaStream_t stream);
+cudaError_t launch_segment_correct(const ForwardArgs &a, const float *start, const float *local_final,
+                                   const uint8_t *ws, cudaStream_t stream);
+cudaError_t launch_affine_compose(const float *transfers, const float *local_finals, int R, int BH, float *start,
+                                  cudaStream_t stream);
 // One CTA whose bounded wait on a barrier nothing completes gives up after about
 // wait_ms and records the device status bit (failure-path self-test).
 cudaError_t launch_selftest_timeout(unsigned int wait_ms, cudaStream_t stream);

@@ -630,6 +630,29 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
 }
 
+// ---------------------------------------------------------------- chain kernels: modes
+// The chain is linear in (U, S_0), which lets one segment of a sequence be run from
+// a zero state and corrected afterwards (time-axis split):
+constexpr int kChainIdentityS0 = 1;   // start from S = I (dk x dk), ignoring s_in
+constexpr int kChainZeroU = 2;        // treat U as zero (propagate the state alone)
+constexpr int kChainNoOut = 4;        // write no outputs
+constexpr int kChainAccumOut = 8;     // add the outputs to out instead of storing them
+
+// out row slice (16 values) = qs + d3, stored or added
+__device__ __forceinline__ void emit_out(float4 *dst, const float (&qs)[16], const float (&d3)[16], bool accum)
+{
+#pragma unroll
+    for (int g = 0; g < 4; ++g) {
+        float4 o = make_float4(qs[4 * g] + d3[4 * g], qs[4 * g + 1] + d3[4 * g + 1], qs[4 * g + 2] + d3[4 * g + 2],
+                               qs[4 * g + 3] + d3[4 * g + 3]);
+        if (accum) {
+            const float4 p = dst[g];
+            o.x += p.x; o.y += p.y; o.z += p.z; o.w += p.w;
+        }
+        dst[g] = o;
+    }
+}
+
 // ---------------------------------------------------------------- chain kernel
 // Warp roles: warps 0..7 hold the state slice (thread (lane dk, half) owns 16
 // columns of row dk), split the B operands and read the accumulators; warp 8
@@ -659,7 +682,8 @@ constexpr uint32_t TMC_D1 = 0, TMC_D2 = 32, TMC_D3 = 64, TMC_COLS = 128;
 
 __global__ void __launch_bounds__(kChainThreads, 1)
 prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
-                     float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb)
+                     float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb,
+                     int mode, const float *__restrict__ s_add)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -768,7 +792,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
         float S[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j)
-            S[j] = s_in ? s_in[((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half + j] : 0.f;
+            S[j] = (mode & kChainIdentityS0) ? (lrow == col0 + 16 * half + j ? 1.f : 0.f)
+                   : s_in ? s_in[((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half + j] : 0.f;
         float qs[16];
         bool ok = true;
         for (int kk = 0; kk < nb && ok; ++kk) {
@@ -796,13 +821,9 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
                 float o2[16];
                 tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
                 const int t = (n0 + kk - 1) * kC + lrow - 64;
-                if (t < T) {
-                    float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
-#pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_float4(qs[4 * g] + o2[4 * g], qs[4 * g + 1] + o2[4 * g + 1],
-                                             qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
-                }
+                if (t < T && !(mode & kChainNoOut))
+                    emit_out(reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half),
+                             qs, o2, (mode & kChainAccumOut) != 0);
             }
 
             // ---- Delta = U - Wr S' (rows 0..63); Qr S' kept for the output (rows 64..127)
@@ -816,7 +837,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
                     for (int g = 0; g < 2; ++g) {
                         float d[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) d[e] = sU[lrow * kDVS + 16 * half + 8 * g + e] - x[8 * g + e];
+                        for (int e = 0; e < 8; ++e)
+                            d[e] = ((mode & kChainZeroU) ? 0.f : sU[lrow * kDVS + 16 * half + 8 * g + e]) - x[8 * g + e];
                         const uint32_t o = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
                         st_split8(smem, CH_DL + o, CH_DL_LO + o, d);
                     }
@@ -847,16 +869,17 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
             float o2[16];
             tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
             const int t = (n0 + nb - 1) * kC + lrow - 64;
-            if (t < T) {
-                float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half);
-#pragma unroll
-                for (int g = 0; g < 4; ++g)
-                    dst[g] = make_float4(qs[4 * g] + o2[4 * g], qs[4 * g + 1] + o2[4 * g + 1],
-                                         qs[4 * g + 2] + o2[4 * g + 2], qs[4 * g + 3] + o2[4 * g + 3]);
-            }
+            if (t < T && !(mode & kChainNoOut))
+                emit_out(reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + col0 + 16 * half),
+                         qs, o2, (mode & kChainAccumOut) != 0);
         }
         if (ok && s_out) {
-            float4 *dst = reinterpret_cast<float4 *>(s_out + ((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half);
+            const size_t o = ((size_t)bh * kDK + lrow) * kDV + col0 + 16 * half;
+            if (s_add) {
+#pragma unroll
+                for (int j = 0; j < 16; ++j) S[j] += s_add[o + j];
+            }
+            float4 *dst = reinterpret_cast<float4 *>(s_out + o);
 #pragma unroll
             for (int g = 0; g < 4; ++g) dst[g] = make_float4(S[4 * g], S[4 * g + 1], S[4 * g + 2], S[4 * g + 3]);
         }
@@ -898,7 +921,8 @@ constexpr uint32_t TMH_D1 = 0, TMH_D2 = 128, TMH_D3 = 256, TMH_S = 384, TMH_COLS
 
 __global__ void __launch_bounds__(kHeadThreads, 1)
 prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
-                          float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb)
+                          float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb,
+                          int mode, const float *__restrict__ s_add)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -997,7 +1021,8 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
             float x[16];
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-                x[j] = s_in ? s_in[((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh + j] : 0.f;
+                x[j] = (mode & kChainIdentityS0) ? (r == 32 * cg + 16 * hh + j ? 1.f : 0.f)
+                       : s_in ? s_in[((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh + j] : 0.f;
             tmem_st16(tS + 16 * hh, x);
         }
         tmem_wait_st();
@@ -1008,12 +1033,12 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
             for (int hh = 0; hh < 2; ++hh) {
                 float o2[16];
                 tmem_ld16(tmem + tlane + TMH_D3 + 32 * cg + 16 * hh, o2);
-                if (t < T) {
-                    float4 *dst = reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + 32 * cg + 16 * hh);
+                if (t < T && !(mode & kChainNoOut)) {
+                    float qv[16];
 #pragma unroll
-                    for (int g = 0; g < 4; ++g)
-                        dst[g] = make_float4(aux[16 * hh + 4 * g] + o2[4 * g], aux[16 * hh + 4 * g + 1] + o2[4 * g + 1],
-                                             aux[16 * hh + 4 * g + 2] + o2[4 * g + 2], aux[16 * hh + 4 * g + 3] + o2[4 * g + 3]);
+                    for (int e = 0; e < 16; ++e) qv[e] = aux[16 * hh + e];
+                    emit_out(reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + 32 * cg + 16 * hh),
+                             qv, o2, (mode & kChainAccumOut) != 0);
                 }
             }
         };
@@ -1046,7 +1071,10 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
             // ---- the previous chunk's output while this chunk's first product runs
             if (kk > 0 && r >= 64) store_out(kk - 1);
             // ---- this chunk's U rows (read while the first product runs)
-            if (r < 64) {
+            if (r < 64 && (mode & kChainZeroU)) {
+#pragma unroll
+                for (int e = 0; e < 32; ++e) aux[e] = 0.f;
+            } else if (r < 64) {
                 const float4 *src = reinterpret_cast<const float4 *>(recs + (size_t)kk * kRec + R_U + cg * 8192u) + r * 8;
 #pragma unroll
                 for (int g = 0; g < 8; ++g) {
@@ -1106,7 +1134,12 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
             for (int hh = 0; hh < 2; ++hh) {
                 float sv[16];
                 tmem_ld16(tS + 16 * hh, sv);
-                float4 *dst = reinterpret_cast<float4 *>(s_out + ((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh);
+                const size_t o = ((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh;
+                if (s_add) {
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) sv[j] += s_add[o + j];
+                }
+                float4 *dst = reinterpret_cast<float4 *>(s_out + o);
 #pragma unroll
                 for (int g = 0; g < 4; ++g) dst[g] = make_float4(sv[4 * g], sv[4 * g + 1], sv[4 * g + 2], sv[4 * g + 3]);
             }
@@ -1160,6 +1193,98 @@ size_t prefill_split_workspace_min(int B, int T, int H)
     return full <= one ? full : one + bh * kDK * kDV * sizeof(float);
 }
 
+namespace {
+
+cudaError_t split_setup(size_t bh, bool &per_head)
+{
+    cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)PP_TOTAL);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)CH_TOTAL);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_chain_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)HC_TOTAL);
+    int dev = 0, sms = 0;
+    if (e == cudaSuccess) e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    // value slices while they fit on the SMs in one wave, whole heads once the heads
+    // alone fill them (a head CTA walks a chunk in about the time a slice CTA does)
+    per_head = bh * kNSL > (size_t)sms;
+    return e;
+}
+
+cudaError_t run_prep(const ForwardArgs &a, uint8_t *ws, int n0, int nb, cudaStream_t stream)
+{
+    const size_t bh = (size_t)a.B * a.H;
+    prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
+        static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
+        static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale,
+        a.prep_flags);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) note_launch();
+    return e;
+}
+
+cudaError_t run_chain(const ForwardArgs &a, bool per_head, const uint8_t *ws, int n0, int nb, const float *s_in,
+                      float *s_out, int mode, const float *s_add, cudaStream_t stream)
+{
+    const size_t bh = (size_t)a.B * a.H;
+    if (per_head)
+        prefill_chain_head_kernel<<<(unsigned)bh, kHeadThreads, HC_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T, a.H,
+                                                                                  n0, nb, mode, s_add);
+    else
+        prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
+                                                                                     a.H, n0, nb, mode, s_add);
+    const cudaError_t e = cudaGetLastError();
+    if (e == cudaSuccess) note_launch();
+    return e;
+}
+
+// start = fold over the earlier segments: S = F_0; S = F_j + P_j S for j = 1..R-1.
+// One CTA per (b, h, 32-column slice); P_j staged in shared memory with a padded
+// row pitch; thread (row, half) owns 16 columns.  fp32.
+constexpr int kAffPitch = 129;
+constexpr uint32_t kAffSmem = (128 * kAffPitch + 128 * 32) * 4;
+
+__global__ void __launch_bounds__(256, 1)
+affine_compose_kernel(const float *__restrict__ P, const float *__restrict__ F, int R, int BH,
+                      float *__restrict__ start)
+{
+    extern __shared__ __align__(16) float asmem[];
+    float *sP = asmem;                      // [128][129]
+    float *sS = asmem + 128 * kAffPitch;    // [128][32] current state slice
+    const int tid = threadIdx.x;
+    const int slice = blockIdx.x % kNSL, bh = blockIdx.x / kNSL;
+    const int r = tid >> 1, c0 = 16 * (tid & 1);
+    const size_t stride = (size_t)BH * kDK * kDV;
+    const size_t base = ((size_t)bh * kDK + r) * kDV + kDVS * slice + c0;
+#pragma unroll
+    for (int j = 0; j < 16; ++j) sS[r * 32 + c0 + j] = F[base + j];
+    for (int seg = 1; seg < R; ++seg) {
+        const float *Pj = P + (size_t)seg * stride + (size_t)bh * kDK * kDK;
+        __syncthreads();
+        for (int id = tid; id < 128 * 128; id += 256) sP[(id >> 7) * kAffPitch + (id & 127)] = Pj[id];
+        __syncthreads();
+        float acc[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) acc[j] = F[(size_t)seg * stride + base + j];
+        for (int c = 0; c < 128; ++c) {
+            const float pv = sP[r * kAffPitch + c];
+#pragma unroll
+            for (int j = 0; j < 16; ++j) acc[j] += pv * sS[c * 32 + c0 + j];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) sS[r * 32 + c0 + j] = acc[j];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 16; ++j) start[base + j] = sS[r * 32 + c0 + j];
+}
+
+}  // namespace
+
 // The sequence is processed in blocks of L chunks, L as large as the workspace
 // allows: prep over the block's chunks of every head, then the chain over them.
 // When L < the number of chunks, the state between blocks is carried in the
@@ -1178,43 +1303,61 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
         L = (int)((ws_bytes - state_bytes) / per_chunk);
     }
     float *carry = (L < nchunks) ? reinterpret_cast<float *>(ws + per_chunk * (size_t)L) : nullptr;
-    cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)PP_TOTAL);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)CH_TOTAL);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_chain_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)HC_TOTAL);
-    int dev = 0, sms = 0;
-    if (e == cudaSuccess) e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    bool per_head = false;
+    cudaError_t e = split_setup(bh, per_head);
     if (e != cudaSuccess) return e;
-    // value slices while they fit on the SMs in one wave, whole heads once the heads
-    // alone fill them (a head CTA walks a chunk in about the time a slice CTA does)
-    const bool per_head = bh * kNSL > (size_t)sms;
     for (int n0 = 0; n0 < nchunks; n0 += L) {
         const int nb = min(L, nchunks - n0);
-        prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
-            static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
-            static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale,
-            a.prep_flags);
-        e = cudaGetLastError();
+        e = run_prep(a, ws, n0, nb, stream);
         if (e != cudaSuccess) return e;
-        note_launch();
         const float *s_in = (n0 == 0) ? a.s0 : carry;
         float *s_out = (n0 + nb >= nchunks) ? a.sT : carry;
-        if (per_head)
-            prefill_chain_head_kernel<<<(unsigned)bh, kHeadThreads, HC_TOTAL, stream>>>(ws, s_in, s_out, a.out,
-                                                                                      a.T, a.H, n0, nb);
-        else
-            prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out,
-                                                                                         a.T, a.H, n0, nb);
-        e = cudaGetLastError();
+        e = run_chain(a, per_head, ws, n0, nb, s_in, s_out, 0, nullptr, stream);
         if (e != cudaSuccess) return e;
-        note_launch();
     }
     return cudaSuccess;
+}
+
+// Segment phases of a time-axis split: the whole segment is one block (the records
+// stay in the workspace for the correction).
+cudaError_t launch_segment_local(const ForwardArgs &a, float *transfer, uint8_t *ws, cudaStream_t stream)
+{
+    const int nchunks = (a.T + kC - 1) / kC;
+    bool per_head = false;
+    cudaError_t e = split_setup((size_t)a.B * a.H, per_head);
+    if (e == cudaSuccess) e = run_prep(a, ws, 0, nchunks, stream);
+    // outputs and final state of the segment from the given start (zero if none)
+    if (e == cudaSuccess) e = run_chain(a, per_head, ws, 0, nchunks, a.s0, a.sT, 0, nullptr, stream);
+    // the segment's transfer: the state alone, propagated from S = I
+    if (e == cudaSuccess)
+        e = run_chain(a, per_head, ws, 0, nchunks, nullptr, transfer, kChainIdentityS0 | kChainZeroU | kChainNoOut,
+                      nullptr, stream);
+    return e;
+}
+
+cudaError_t launch_segment_correct(const ForwardArgs &a, const float *start, const float *local_final,
+                                   const uint8_t *ws, cudaStream_t stream)
+{
+    const int nchunks = (a.T + kC - 1) / kC;
+    bool per_head = false;
+    cudaError_t e = split_setup((size_t)a.B * a.H, per_head);
+    // out += outputs of the start state propagated alone; final = local final + that state
+    if (e == cudaSuccess)
+        e = run_chain(a, per_head, ws, 0, nchunks, start, a.sT, kChainZeroU | kChainAccumOut, local_final, stream);
+    return e;
+}
+
+cudaError_t launch_affine_compose(const float *transfers, const float *local_finals, int R, int BH, float *start,
+                                  cudaStream_t stream)
+{
+    cudaError_t e = cudaFuncSetAttribute(affine_compose_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)kAffSmem);
+    if (e != cudaSuccess) return e;
+    affine_compose_kernel<<<(unsigned)((size_t)BH * kNSL), 256, kAffSmem, stream>>>(transfers, local_finals, R, BH,
+                                                                                   start);
+    e = cudaGetLastError();
+    if (e == cudaSuccess) note_launch();
+    return e;
 }
 
 cudaError_t launch_selftest_timeout(unsigned int wait_ms, cudaStream_t stream)

@@ -171,6 +171,57 @@ kda_status kda_forward_raw(const void *q, const void *k, const void *v,
                            void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * Time-axis split of one long sequence (context parallelism).
+ *
+ * The chunk-boundary state seeds the next chunk ("KDA Technical Deep Dive",
+ * §Systems and implementation tradeoffs, Training), and the chunked recurrence
+ * is linear in (values, starting state).  So a segment of the sequence run
+ * from a zero state gives its outputs and final state up to the contribution
+ * of the true starting state S_in, which enters as
+ *     final = local_final + P S_in,    out += (outputs of S_in propagated alone),
+ * with P [dk, dk] the segment's transfer (its state map with zero values).  The
+ * associative combination of these affine transfers across segments is the
+ * "associative scan" the deep dive mentions (same section).  With segments
+ * 0..R-1 in time order (on one device or one per rank): run
+ * kda_segment_local on each (segment 0 with the sequence's initial state),
+ * exchange the (transfer, local_final) pairs, then for each segment r >= 1
+ * compute its start with kda_segment_start_state over segments 0..r-1 and
+ * finish it with kda_segment_correct.  bf16 inputs, dk = dv = 128.
+ *
+ * kda_segment_local -- outputs `out` and `local_final` of the segment from
+ *   `initial_state` (NULL = zero), and its `transfer` [B, H, dk, dk] fp32
+ *   (16-byte aligned).  Other arguments as kda_forward_ws; the workspace must
+ *   hold the whole segment (kda_forward_workspace_bytes) and must be passed
+ *   unchanged to kda_segment_correct.  T >= 1.
+ */
+kda_status kda_segment_local(const void *q, const void *k, const void *v,
+                             const float *log_alpha, const float *beta,
+                             const float *initial_state, float *out, float *local_final, float *transfer,
+                             int B, int T, int H, int dk, int dv,
+                             kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes, void *stream);
+
+/*
+ * kda_segment_start_state -- the state entering segment R of a sequence from the
+ * R earlier segments: start = F_0, then start = F_j + P_j start for j = 1..R-1,
+ * where transfers = P [R][B, H, dk, dk] and local_finals = F [R][B, H, dk, dv]
+ * (segment 0's F already includes the sequence's initial state; P_0 is not
+ * read).  fp32; all pointers 16-byte aligned device memory.  R >= 1.
+ */
+kda_status kda_segment_start_state(const float *transfers, const float *local_finals, int R,
+                                   float *start, int B, int H, int dk, int dv, void *stream);
+
+/*
+ * kda_segment_correct -- finish a segment given its true start state: adds the
+ * outputs of `start` propagated through the segment to `out` (the segment's
+ * local outputs) and writes final_state = local_final + the propagated start
+ * (NULL = not written).  Reads the chunk records kda_segment_local left in
+ * `workspace` (same B, T, H); q, k, v are not needed again.
+ */
+kda_status kda_segment_correct(const float *start, const float *local_final, float *out, float *final_state,
+                               int B, int T, int H, int dk, int dv,
+                               const void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * kda_forward_noalloc -- kda_forward on the two-kernel prefill with scratch that
  * belongs to the library, so that the call allocates nothing and needs no
  * workspace from the caller.

@@ -187,3 +187,39 @@ def test_forward_ws_validates_like_forward(lib):
     assert fws(q=None) == kda.KDA_ERR_INVALID_ARG
     assert fws(ws=FAKE + 16) == kda.KDA_ERR_MISALIGNED    # workspace must be 256-byte aligned
     assert fws(la=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+
+
+def test_segment_calls_validate_before_launch(lib):
+    WS = FAKE * 16
+
+    def local(T=8, transfer=FAKE, sT=FAKE, ws=WS, nbytes=1 << 40, dtype=kda.KDA_BF16, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, out=FAKE)
+        a.update(kw)
+        return lib.kda_segment_local(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["out"], sT, transfer,
+                                     1, T, 2, 128, 128, dtype, ctypes.c_float(0.0), ws, nbytes, None)
+    assert local(T=0) == kda.KDA_ERR_INVALID_ARG
+    assert local(transfer=None) == kda.KDA_ERR_INVALID_ARG
+    assert local(sT=None) == kda.KDA_ERR_INVALID_ARG
+    assert local(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert local(transfer=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+    assert local(la=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+    assert local(ws=WS + 16) == kda.KDA_ERR_MISALIGNED
+    assert local(dtype=kda.KDA_F32) == kda.KDA_ERR_UNSUPPORTED
+    assert local(ws=None) == kda.KDA_ERR_UNSUPPORTED
+    assert local(nbytes=kda.workspace_bytes(1, 8, 2, 128, 128) - 1) == kda.KDA_ERR_UNSUPPORTED
+
+    def start(R=2, P=FAKE, F=FAKE, S=FAKE, dk=128):
+        return lib.kda_segment_start_state(P, F, R, S, 1, 2, dk, 128, None)
+    assert start(R=0) == kda.KDA_ERR_INVALID_ARG
+    assert start(P=None) == kda.KDA_ERR_INVALID_ARG
+    assert start(dk=64) == kda.KDA_ERR_UNSUPPORTED
+    assert start(S=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+
+    def correct(T=8, ws=WS, nbytes=1 << 40, sT=FAKE, out=FAKE):
+        return lib.kda_segment_correct(FAKE, FAKE, out, sT, 1, T, 2, 128, 128, ws, nbytes, None)
+    assert correct(T=0) == kda.KDA_ERR_INVALID_ARG
+    assert correct(ws=None) == kda.KDA_ERR_INVALID_ARG
+    assert correct(ws=WS + 16) == kda.KDA_ERR_MISALIGNED
+    assert correct(out=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+    assert correct(sT=FAKE + 8) == kda.KDA_ERR_MISALIGNED
+    assert correct(nbytes=kda.workspace_bytes(1, 8, 2, 128, 128) - 1) == kda.KDA_ERR_UNSUPPORTED
