@@ -501,6 +501,74 @@ def _add_raw(line, args, w, world, device, hbm):
         "kernel": "prefill_prep_kernel (with the fused steps) + prefill_chain_kernel"}
 
 
+def _add_time_split(line, args, w, device, segments=8):
+    """One sequence of the prefill workload cut into `segments` contiguous
+    segments (time-axis split), run one after another on this GPU.  Timed: the
+    phases of the last segment, the one with the most work (its local run and
+    transfer, the fold over all earlier segments, the correction).  Checked: the
+    concatenated outputs and the last final state against one kda_forward_ws
+    call on the whole sequence."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    if w.T % segments or w.dk != w.dv:
+        return
+    Ts = w.T // segments
+    x = I.make_inputs(w, device)
+    names = ("q", "k", "v", "log_alpha", "beta")
+    segs = [{n: x[n][:, r * Ts:(r + 1) * Ts].contiguous() for n in names} for r in range(segments)]
+    ws = kda.make_workspace(w.B, Ts, w.H, w.dk, w.dv, w.torch_dtype, device=device)
+    outs, Ps, Fs, final = [], [], [], None
+    for r in range(segments):
+        o, lf, P = kda.segment_local(*(segs[r][n] for n in names), x["initial_state"] if r == 0 else None,
+                                     workspace=ws)
+        final = lf
+        if r:
+            start = kda.segment_start_state(torch.stack(Ps), torch.stack(Fs))
+            final = kda.segment_correct(start, lf, o, workspace=ws)
+        outs.append(o); Ps.append(P); Fs.append(lf)
+    whole_ws = kda.make_workspace(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, device=device)
+    o_w, s_w = kda.forward(*(x[n] for n in names), x["initial_state"], workspace=whole_ws)
+    del whole_ws
+    out = torch.cat(outs, dim=1)
+    rel = lambda a, b: float((a - b).abs().max() / b.pow(2).mean().sqrt())
+    check = {"out": rel(out, o_w), "final_state": rel(final, s_w)}
+    del out, o_w, outs
+
+    last = segs[-1]
+    Pst, Fst = torch.stack(Ps[:-1]), torch.stack(Fs[:-1])
+    phases = {
+        "local": lambda: kda.segment_local(*(last[n] for n in names), None, workspace=ws),
+        "fold": lambda: kda.segment_start_state(Pst, Fst),
+    }
+    o_l, lf_l, _ = phases["local"]()
+    start = phases["fold"]()
+    phases["correct"] = lambda: kda.segment_correct(start, lf_l, o_l, workspace=ws)
+    ms = {}
+    for name, fn in phases.items():
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize(device)
+        stream = torch.cuda.current_stream(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms[name] = e0.elapsed_time(e1) / args.steps
+    kda.check_status(device)
+    per_rank = ms["local"] + ms["fold"] + ms["correct"]
+    line["time_split"] = {
+        "workload": w.name, "segments": segments, "segment_tokens": Ts,
+        "emulation": "segments run one after another on one GPU; per-rank phases timed on the last segment",
+        "local_ms": ms["local"], "fold_ms": ms["fold"], "correct_ms": ms["correct"],
+        "per_rank_ms_without_exchange": per_rank,
+        "exchange_bytes_per_rank": 2 * w.B * w.H * w.dk * w.dv * 4,
+        "whole_sequence_ms": line.get("ms_per_step"),
+        "max_abs_err_over_rms_vs_whole_sequence": check}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -627,6 +695,8 @@ def main(argv=None):
         _add_gdn(line, args, w, world, device, hbm)
         if ws_bytes:
             _add_raw(line, args, w, world, device, hbm)
+            if world == 1:
+                _add_time_split(line, args, w, device)
 
     if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],

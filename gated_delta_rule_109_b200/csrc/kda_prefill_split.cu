@@ -656,12 +656,17 @@ __device__ __forceinline__ void emit_out(float4 *dst, const float (&qs)[16], con
 // ---------------------------------------------------------------- chain kernel
 // Warp roles: warps 0..7 hold the state slice (thread (lane dk, half) owns 16
 // columns of row dk), split the B operands and read the accumulators; warp 8
-// issues the tensor-core products and the bulk copies.  Handoffs go through
-// mbarriers, never a CTA-wide barrier:
+// issues the tensor-core products; warp 9 issues the record copies (issuing a
+// bulk copy stalls the issuing thread for hundreds of cycles, which must not
+// delay a product).  Handoffs go through mbarriers, never a CTA-wide barrier:
 //   bar_s  (8 arrivals)  S' of chunk kk is in shared memory, D1/D2 of chunk kk-1 read
 //   bar_d  (8 arrivals)  Delta of chunk kk is in shared memory, D1 of kk and D3 of kk-1 read
-//   mma1 / mma2 (commit) the first / second product of chunk kk is complete
-constexpr int kChainThreads = 288;
+//   mma1 / mma2 (commit) the first product / Kb^T Delta of chunk kk is complete
+//   mma3 (commit)        M Delta of chunk kk is complete (the output only: the state
+//                        update does not wait for it, it runs beside the next S');
+//                        also: Kb, M and U of chunk kk are no longer read
+//   wq_free[s] (commit)  the first product has read the [Wr; Qr] in slot s
+constexpr int kChainThreads = 320;
 constexpr uint32_t CH_WQ = 0;                        // two slots of [Wr; Qr] (hi, lo) and e^m
 constexpr uint32_t CH_KTM = 2 * kWqBytes;            // Kb hi, Kb lo, M hi, M lo (48 KB)
 constexpr uint32_t CH_MA = CH_KTM + 24576;           // 128-row view whose rows 64..127 are M hi
@@ -673,7 +678,9 @@ constexpr uint32_t CH_DL = CH_S + 16384, CH_DL_LO = CH_DL + 4096;  // Delta: MN-
 constexpr uint32_t CH_MBAR = CH_DL + 8192;           // mma1, mma2, wq[2], ktm, bar_s, bar_d
 constexpr uint32_t CH_FAIL = CH_MBAR + 56;           // a wait gave up somewhere in the CTA
 constexpr uint32_t CH_TMEMP = CH_MBAR + 64;
-constexpr uint32_t CH_TOTAL = CH_TMEMP + 16;
+constexpr uint32_t CH_MBAR3 = CH_MBAR + 72;          // mma3
+constexpr uint32_t CH_WQFREE = CH_MBAR + 80;         // wq_free[2]
+constexpr uint32_t CH_TOTAL = CH_MBAR + 96;
 static_assert(CH_TOTAL <= 232448, "shared memory");
 static_assert(R_KT_LO + 16384 == R_M && R_M + 16384 == R_U, "Kb and M are one contiguous copy");
 static_assert(R_GAM + 512 == R_EL, "e^{G_last} and e^{G_last - m} are one contiguous copy");
@@ -691,7 +698,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     const float *sGam = reinterpret_cast<const float *>(smem + CH_GAM);
     volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + CH_FAIL);
     const uint32_t mbar1 = sbase + CH_MBAR, mbar2 = mbar1 + 8, mbar_wq0 = mbar1 + 16, mbar_ktm = mbar1 + 32;
-    const uint32_t bar_s = mbar1 + 40, bar_d = mbar1 + 48;
+    const uint32_t bar_s = mbar1 + 40, bar_d = mbar1 + 48, mbar3 = sbase + CH_MBAR3;
+    const uint32_t wq_free0 = sbase + CH_WQFREE;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x % kNSL;
@@ -710,8 +718,11 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     if (tid == 0) {
         mbar_init(mbar1, 1);
         mbar_init(mbar2, 1);
+        mbar_init(mbar3, 1);
         mbar_init(mbar_wq0, 1);
         mbar_init(mbar_wq0 + 8, 1);
+        mbar_init(wq_free0, 1);
+        mbar_init(wq_free0 + 8, 1);
         mbar_init(mbar_ktm, 1);
         mbar_init(bar_s, 8);
         mbar_init(bar_d, 8);
@@ -731,7 +742,35 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     };
 
     if (warp == 8) {
-        // ---------------- issuer: products and copies (lane 0)
+        // ---------------- issuer: the products (lane 0)
+        if (lane == 0) {
+            for (int kk = 0; kk < nb; ++kk) {
+                const uint32_t par = (uint32_t)kk & 1u;
+                // S' written; the compute warps have waited for this chunk's [Wr; Qr]
+                if (!wait(bar_s, par)) break;
+                tc_fence_after();
+                const uint32_t wq = sbase + CH_WQ + kWqBytes * (kk & 1);
+                mma_split(tmem + TMC_D1, wq, wq + 32768u, RW_SI, RW_SO, sbase + CH_S, sbase + CH_S_LO,
+                          S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
+                umma_commit(mbar1);
+                umma_commit(wq_free0 + 8u * (kk & 1));
+                // Delta written; the compute warps have waited for this chunk's Kb, M, U
+                if (!wait(bar_d, par)) break;
+                tc_fence_after();
+                mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
+                          sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 1, 1), false);
+                umma_commit(mbar2);
+                mma_split(tmem + TMC_D3, sbase + CH_MA, sbase + CH_MA_LO, H_SI, H_SO,
+                          sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 0, 1), false);
+                umma_commit(mbar3);
+            }
+        }
+    } else if (warp == 9) {
+        // ---------------- copies (lane 0): [Wr; Qr] and e^m two chunks ahead (two slots,
+        // refilled once the first product has read them), Kb, M, U and the decays one
+        // chunk ahead (one slot, refilled once both products of the chunk have read it).
+        // Every refill waits for the slot's previous use, so no wait here can fall two
+        // phases behind its barrier.
         if (lane == 0) {
             uint32_t wq_pend = 0u, wq_par = 0u, ktm_par = 0u;
             bool ktm_pending = false;
@@ -756,28 +795,15 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
             if (nb > 1) load_wq(1);
             load_ktm(0);
             for (int kk = 0; kk < nb; ++kk) {
-                const uint32_t par = (uint32_t)kk & 1u;
-                // the compute warps have waited for this chunk's [Wr; Qr] before arriving
-                if (!wait(bar_s, par)) break;
-                wq_pend &= ~(1u << (kk & 1));
-                tc_fence_after();
-                const uint32_t wq = sbase + CH_WQ + kWqBytes * (kk & 1);
-                mma_split(tmem + TMC_D1, wq, wq + 32768u, RW_SI, RW_SO, sbase + CH_S, sbase + CH_S_LO,
-                          S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
-                umma_commit(mbar1);
-                if (!wait(mbar1, par)) break;
-                if (kk + 2 < nb) load_wq(kk + 2);
-                // ... and for this chunk's Kb, M, U before arriving
-                if (!wait(bar_d, par)) break;
-                ktm_pending = false;
-                tc_fence_after();
-                mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
-                          sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 1, 1), false);
-                mma_split(tmem + TMC_D3, sbase + CH_MA, sbase + CH_MA_LO, H_SI, H_SO,
-                          sbase + CH_DL, sbase + CH_DL_LO, S_SO, S_SI, kC / 16, idesc_bf16(128, kDVS, 0, 1), false);
-                umma_commit(mbar2);
-                if (!wait(mbar2, par)) break;
-                if (kk + 1 < nb) load_ktm(kk + 1);
+                if (kk + 2 < nb) {
+                    if (!wait(wq_free0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u)) break;
+                    wq_pend &= ~(1u << (kk & 1));
+                    load_wq(kk + 2);
+                }
+                if (kk + 1 < nb) {
+                    if (!wait(mbar3, (uint32_t)kk & 1u)) break;
+                    load_ktm(kk + 1);
+                }
             }
             if (*sFail) {
                 // let the copies still in flight land before shared memory is released
@@ -818,6 +844,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
 
             // ---- O = Qr S' + M Delta of chunk kk - 1 while the first product of kk runs
             if (kk > 0 && lrow >= 64) {
+                if (!(ok = wait(mbar3, par ^ 1u))) break;
+                tc_fence_after();
                 float o2[16];
                 tmem_ld16(tmem + tlane + TMC_D3 + 16 * half, o2);
                 const int t = (n0 + kk - 1) * kC + lrow - 64;
@@ -863,7 +891,7 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
             }
             tc_fence_before();
         }
-        if (ok && nb > 0 && lrow >= 64) {
+        if (ok && nb > 0 && lrow >= 64 && (ok = wait(mbar3, (uint32_t)(nb - 1) & 1u))) {
             // the last chunk's output
             tc_fence_after();
             float o2[16];
@@ -914,6 +942,7 @@ constexpr uint32_t HC_DL = HC_S + 65536, HC_DL_LO = HC_DL + 16384;   // Delta: M
 constexpr uint32_t HC_MBAR = HC_DL + 32768;                    // mma1, mma2, wq, ktm, bar_s, bar_d
 constexpr uint32_t HC_FAIL = HC_MBAR + 48;
 constexpr uint32_t HC_TMEMP = HC_MBAR + 64;
+constexpr uint32_t HC_MBAR3 = HC_MBAR + 72;                    // mma3: M Delta complete (output only)
 constexpr uint32_t HC_TOTAL = HC_TMEMP + 16;
 static_assert(HC_TOTAL <= 232448, "shared memory");
 constexpr uint32_t HS_SO = 2048, HS_SI = 128;                  // N = 128 B-operand strides
@@ -930,7 +959,7 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
     const float *sEm = reinterpret_cast<const float *>(smem + HC_WQ + 65536u);
     const float *sGam = reinterpret_cast<const float *>(smem + HC_GAM);
     const uint32_t mbar1 = sbase + HC_MBAR, mbar2 = mbar1 + 8, mbar_wq = mbar1 + 16, mbar_ktm = mbar1 + 24;
-    const uint32_t bar_s = mbar1 + 32, bar_d = mbar1 + 40;
+    const uint32_t bar_s = mbar1 + 32, bar_d = mbar1 + 40, mbar3 = sbase + HC_MBAR3;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
@@ -947,6 +976,7 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
     if (tid == 0) {
         mbar_init(mbar1, 1);
         mbar_init(mbar2, 1);
+        mbar_init(mbar3, 1);
         mbar_init(mbar_wq, 1);
         mbar_init(mbar_ktm, 1);
         mbar_init(bar_s, 16);
@@ -1001,10 +1031,11 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
                 tc_fence_after();
                 mma_split(tmem + TMH_D2, sbase + HC_KTM, sbase + HC_KTM + 16384u, RW_SO, RW_SI,
                           sbase + HC_DL, sbase + HC_DL_LO, HS_SO, HS_SI, kC / 16, idesc_bf16(128, kDV, 1, 1), false);
+                umma_commit(mbar2);
                 mma_split(tmem + TMH_D3, sbase + HC_MA, sbase + HC_MA_LO, H_SI, H_SO,
                           sbase + HC_DL, sbase + HC_DL_LO, HS_SO, HS_SI, kC / 16, idesc_bf16(128, kDV, 0, 1), false);
-                umma_commit(mbar2);
-                if (!wait(mbar2, par)) break;
+                umma_commit(mbar3);
+                if (!wait(mbar3, par)) break;          // Kb and M read by both products
                 if (kk + 1 < nb) load_ktm(kk + 1);
             }
             if (*sFail) {
@@ -1069,7 +1100,11 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
             if (lane == 0) mbar_arrive(bar_s);
 
             // ---- the previous chunk's output while this chunk's first product runs
-            if (kk > 0 && r >= 64) store_out(kk - 1);
+            if (kk > 0 && r >= 64) {
+                if (!(ok = wait(mbar3, par ^ 1u))) break;
+                tc_fence_after();
+                store_out(kk - 1);
+            }
             // ---- this chunk's U rows (read while the first product runs)
             if (r < 64 && (mode & kChainZeroU)) {
 #pragma unroll
@@ -1125,7 +1160,7 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
             tmem_wait_st();
             tc_fence_before();
         }
-        if (ok && nb > 0 && r >= 64) {
+        if (ok && nb > 0 && r >= 64 && (ok = wait(mbar3, (uint32_t)(nb - 1) & 1u))) {
             tc_fence_after();
             store_out(nb - 1);
         }
