@@ -18,6 +18,9 @@ delta-rule write, read with the query scaled by 1/sqrt(d_k)):
                      ``forward`` with the gate repeated over key channels.
 * ``forward_raw`` -- raw activations: sigmoid gate pre-activations and
                      unnormalised q, k, prepared in fp64, then ``forward``.
+* ``backward``    -- gradients of the forward with respect to every input, by
+                     reverse-mode automatic differentiation (torch.autograd, CPU,
+                     fp64) of the same token recurrence.
 
 Both store the state as ``[B, H, dk, dv]`` (the transpose of the page's
 (d_v, d_k) matrix), so the per-channel decay scales rows and the page's
@@ -109,12 +112,15 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, scale=None, nthreads=0
     return out, sT
 
 
-def forward_np(q, k, v, log_alpha, beta, initial_state=None, scale=None):
+def forward_np(q, k, v, log_alpha, beta, initial_state=None, scale=None, exact64=False):
     """fp64 KDA forward by the token recurrence (numpy implementation).
 
     Same arguments and results as :func:`forward`.  Meant for small inputs.
+    ``exact64`` takes fp64 inputs as they are instead of as their fp32 values
+    (finite differences of the forward need perturbations below fp32 spacing).
     """
-    qf, kf, vf, af, bf = (_as_f32(x).astype(np.float64) for x in (q, k, v, log_alpha, beta))
+    conv = _as_f64 if exact64 else (lambda x: _as_f32(x).astype(np.float64))
+    qf, kf, vf, af, bf = (conv(x) for x in (q, k, v, log_alpha, beta))
     B, T, H, dk = qf.shape
     dv = vf.shape[-1]
     if scale is None:
@@ -173,6 +179,67 @@ def forward_raw(q, k, v, gate, beta, initial_state=None, logsigmoid_gate=True, n
         q64, k64 = unit(q64), unit(k64)
     la = -np.logaddexp(0.0, -g64) if logsigmoid_gate else g64
     return forward(q64, k64, v, la, beta, initial_state, scale=scale, nthreads=nthreads)
+
+
+def backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_state=None, scale=None,
+             segment=64):
+    """fp64 gradients of the KDA forward with respect to every input.
+
+    The loss is L = sum(O * d_out) + sum(S_T * d_final_state): ``d_out`` [B,T,H,dv]
+    and ``d_final_state`` [B,H,dk,dv] (None: zeros) are the cotangents of the
+    outputs and of the final state.  The gradient is the derivative of the token
+    recurrence of "Kimi Delta Attention: The Linear Attention Behind Kimi K2 and
+    Qwen3", §How Kimi Delta Attention works step by step (the same steps as
+    :func:`forward_np`, written in torch ops), taken by torch.autograd in fp64 on
+    the exact input values.  The pages give no gradient formulas ("KDA Technical
+    Deep Dive", §Systems and implementation tradeoffs, Training, names only
+    chunkwise training), so the definition is the derivative itself.  Tokens run in
+    segments of ``segment`` whose states are recomputed during the backward sweep
+    (torch.utils.checkpoint), so memory grows with T / segment.
+
+    Returns a dict of fp64 numpy arrays: ``dq``, ``dk``, ``dv``, ``dlog_alpha``,
+    ``dbeta`` (shapes of the inputs) and ``dinitial_state`` [B,H,dk,dv] (the
+    gradient with respect to the initial state; a zero state when it is None).
+    """
+    import torch
+    from torch.utils.checkpoint import checkpoint
+
+    def exact(x):
+        return torch.from_numpy(_as_f32(x).astype(np.float64))
+
+    qt, kt, vt, at, bt = (exact(x).requires_grad_(True) for x in (q, k, v, log_alpha, beta))
+    B, T, H, dk = qt.shape
+    dv = vt.shape[-1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(dk)
+    s0 = (torch.zeros((B, H, dk, dv), dtype=torch.float64) if initial_state is None
+          else torch.from_numpy(_as_f64(initial_state)).clone())
+    s0.requires_grad_(True)
+    d_o = torch.from_numpy(_as_f64(d_out))
+    d_s = (torch.zeros((B, H, dk, dv), dtype=torch.float64) if d_final_state is None
+           else torch.from_numpy(_as_f64(d_final_state)))
+
+    def run(S, q_, k_, v_, a_, b_):
+        outs = []
+        for t in range(q_.shape[1]):
+            S = S * torch.exp(a_[:, t]).unsqueeze(-1)                   # decay rows (key channels)
+            p = torch.einsum("bhcx,bhc->bhx", S, k_[:, t])               # S~^T k
+            e = b_[:, t].unsqueeze(-1) * (v_[:, t] - p)                  # beta (v - p)
+            S = S + k_[:, t].unsqueeze(-1) * e.unsqueeze(-2)             # S~ + k e^T
+            outs.append(scale * torch.einsum("bhcx,bhc->bhx", S, q_[:, t]))
+        return S, torch.stack(outs, 1)
+
+    S = s0
+    loss = torch.zeros((), dtype=torch.float64)
+    for t0 in range(0, T, segment):
+        sl = slice(t0, min(T, t0 + segment))
+        S, O = checkpoint(run, S, qt[:, sl], kt[:, sl], vt[:, sl], at[:, sl], bt[:, sl], use_reentrant=False)
+        loss = loss + (O * d_o[:, sl]).sum()
+    loss = loss + (S * d_s).sum()
+    g = torch.autograd.grad(loss, [qt, kt, vt, at, bt, s0], allow_unused=True)
+    names = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dinitial_state")
+    ref = (qt, kt, vt, at, bt, s0)
+    return {n: (gi if gi is not None else torch.zeros_like(r)).detach().numpy() for n, gi, r in zip(names, g, ref)}
 
 
 def parity_error(x_gpu, x_ref) -> float:

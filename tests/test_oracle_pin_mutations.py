@@ -153,3 +153,63 @@ def test_unmutated_raw_copy_passes_every_pin(monkeypatch):
     monkeypatch.setattr(oracle, "forward_raw", _make_raw("none"))
     for pin in RAW_PINS:
         pin()
+
+
+def _make_bwd(mutation):
+    """oracle.backward with one slip planted in the differentiated recurrence."""
+    def bwd(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_state=None, scale=None, segment=64):
+        import torch
+        ex = lambda x: torch.from_numpy(oracle._as_f32(x).astype(np.float64))
+        qt, kt, vt, at, bt = (ex(x).requires_grad_(True) for x in (q, k, v, log_alpha, beta))
+        B, T, H, dk = qt.shape
+        dv = vt.shape[-1]
+        sc = 1.0 if mutation == "no_scale" else (1.0 / math.sqrt(dk) if scale is None else scale)
+        s0 = (torch.zeros((B, H, dk, dv), dtype=torch.float64) if initial_state is None
+              else torch.from_numpy(oracle._as_f64(initial_state)).clone()).requires_grad_(True)
+        d_o = torch.from_numpy(oracle._as_f64(d_out))
+        d_s = (torch.zeros((B, H, dk, dv), dtype=torch.float64)
+               if d_final_state is None or mutation == "final_cotangent_dropped"
+               else torch.from_numpy(oracle._as_f64(d_final_state)))
+        S, loss = s0, torch.zeros((), dtype=torch.float64)
+        for t0 in range(0, T, segment):
+            if mutation == "segments_restart":
+                S = s0
+            for t in range(t0, min(T, t0 + segment)):
+                Sd = S * torch.exp(at[:, t]).unsqueeze(-1)
+                p = torch.einsum("bhcx,bhc->bhx", S if mutation == "predict_undecayed" else Sd, kt[:, t])
+                e = bt[:, t].unsqueeze(-1) * (vt[:, t] - p)
+                Sn = Sd + kt[:, t].unsqueeze(-1) * e.unsqueeze(-2)
+                o = sc * torch.einsum("bhcx,bhc->bhx", Sd if mutation == "read_before_write" else Sn, qt[:, t])
+                loss = loss + (o * d_o[:, t]).sum()
+                S = Sn
+        loss = loss + (S * d_s).sum()
+        g = torch.autograd.grad(loss, [qt, kt, vt, at, bt, s0], allow_unused=True)
+        names = ("dq", "dk", "dv", "dlog_alpha", "dbeta", "dinitial_state")
+        ref = (qt, kt, vt, at, bt, s0)
+        return {n: (gi if gi is not None else torch.zeros_like(r)).detach().numpy()
+                for n, gi, r in zip(names, g, ref)}
+    return bwd
+
+
+from tests import test_oracle_backward_pins as bpins  # noqa: E402
+
+BWD_PINS = [bpins.test_backward_matches_finite_differences, bpins.test_backward_beta_zero_closed_form]
+
+
+@pytest.mark.parametrize("mutation", ["final_cotangent_dropped", "predict_undecayed", "segments_restart",
+                                      "read_before_write", "no_scale"])
+def test_some_backward_pin_fails_on_planted_mistake(mutation, monkeypatch):
+    monkeypatch.setattr(oracle, "backward", _make_bwd(mutation))
+    failed = 0
+    for pin in BWD_PINS:
+        try:
+            pin()
+        except AssertionError:
+            failed += 1
+    assert failed > 0, "no backward pin caught %s" % mutation
+
+
+def test_unmutated_backward_copy_passes_every_pin(monkeypatch):
+    monkeypatch.setattr(oracle, "backward", _make_bwd("none"))
+    for pin in BWD_PINS:
+        pin()
