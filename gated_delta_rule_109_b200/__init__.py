@@ -30,7 +30,7 @@ KDA_PREP_LOGSIGMOID_GATE, KDA_PREP_L2NORM_QK = 1, 2
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
            "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_segment_local",
            "kda_segment_start_state", "kda_segment_correct", "kda_forward_noalloc",
-           "kda_forward_noalloc_scratch_bytes",
+           "kda_forward_noalloc_scratch_bytes", "kda_backward", "kda_backward_workspace_bytes",
            "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
            "kda_launch_count",
@@ -78,6 +78,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_forward_noalloc.restype = i
     lib.kda_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_forward_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.kda_backward.restype = i
+    lib.kda_backward.argtypes = [vp] * 14 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
+    lib.kda_backward_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_backward_workspace_bytes.argtypes = [i] * 5
     lib.kda_forward_noalloc_scratch_bytes.argtypes = []
     lib.kda_gdn_forward.restype = i
     lib.kda_gdn_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
@@ -306,6 +310,72 @@ def segment_correct(start, local_final, out, *, workspace, final_state=None):
                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check(st, "kda_segment_correct")
     return final_state
+
+
+def backward_workspace_bytes(B: int, T: int, H: int, dk: int, dv: int) -> int:
+    """Bytes of the workspace ``kda_backward`` needs (0: unsupported shape)."""
+    return int(load().kda_backward_workspace_bytes(B, T, H, dk, dv))
+
+
+def backward(q, k, v, log_alpha, beta, grad_out, initial_state=None, grad_final_state=None, *,
+             workspace=None, scale: float = 0.0, initial_state_grad: bool = True):
+    """Gradients of :func:`forward` (``kda_backward``).
+
+    ``grad_out`` [B,T,H,dv] and ``grad_final_state`` [B,H,dk,dv] (None: zero) are
+    the cotangents of the outputs and of the final state.  Returns a dict of fp32
+    tensors ``dq, dk, dv, dlog_alpha, dbeta`` and ``dinitial_state`` (None unless
+    ``initial_state_grad``).  ``workspace``: a uint8 device tensor of at least
+    :func:`backward_workspace_bytes` bytes (allocated here when None).
+    """
+    lib = load()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    for t, n, shp in ((q, "q", (B, T, H, dk)), (k, "k", (B, T, H, dk)), (v, "v", (B, T, H, dv))):
+        _need(t, n, shp, q.dtype, dev)
+    _need(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
+    _need(beta, "beta", (B, T, H), torch.float32, dev)
+    _need(grad_out, "grad_out", (B, T, H, dv), torch.float32, dev)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, dev)
+    if grad_final_state is not None:
+        _need(grad_final_state, "grad_final_state", (B, H, dk, dv), torch.float32, dev)
+    nbytes = backward_workspace_bytes(B, T, H, dk, dv)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    f32 = dict(dtype=torch.float32, device=dev)
+    g = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
+             dv=torch.empty((B, T, H, dv), **f32), dlog_alpha=torch.empty((B, T, H, dk), **f32),
+             dbeta=torch.empty((B, T, H), **f32),
+             dinitial_state=torch.empty((B, H, dk, dv), **f32) if initial_state_grad else None)
+    st = lib.kda_backward(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                          _ptr(grad_out), _ptr(grad_final_state), _ptr(g["dq"]), _ptr(g["dk"]), _ptr(g["dv"]),
+                          _ptr(g["dlog_alpha"]), _ptr(g["dbeta"]), _ptr(g["dinitial_state"]),
+                          B, T, H, dk, dv, _dtype_code(q), float(scale), _ptr(workspace),
+                          workspace.numel() * workspace.element_size(), _stream(dev))
+    _check(st, "kda_backward")
+    return g
+
+
+class KDAFunction(torch.autograd.Function):
+    """``out, final_state = KDAFunction.apply(q, k, v, log_alpha, beta, initial_state)``
+    with ``kda_forward`` forward and ``kda_backward`` backward (gradients in fp32,
+    cast to each input's dtype)."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, log_alpha, beta, initial_state):
+        out, final_state = forward(q, k, v, log_alpha, beta, initial_state)
+        ctx.save_for_backward(q, k, v, log_alpha, beta, initial_state)
+        return out, final_state
+
+    @staticmethod
+    def backward(ctx, grad_out, grad_final_state):
+        q, k, v, log_alpha, beta, initial_state = ctx.saved_tensors
+        g = backward(q, k, v, log_alpha, beta, grad_out.contiguous().float(),
+                     initial_state, None if grad_final_state is None else grad_final_state.contiguous().float(),
+                     initial_state_grad=initial_state is not None)
+        return (g["dq"].to(q.dtype), g["dk"].to(k.dtype), g["dv"].to(v.dtype), g["dlog_alpha"], g["dbeta"],
+                g["dinitial_state"])
 
 
 def forward_noalloc(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,

@@ -47,7 +47,7 @@ extern "C" {
 unsigned long long kda_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 
-int kda_version(void) { return 200; }   // 0.2.0
+int kda_version(void) { return 300; }   // 0.3.0
 
 const char *kda_status_string(kda_status s)
 {
@@ -346,6 +346,53 @@ kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
 {
     return decode_impl(q, k, v, log_alpha, beta, state_inout, out, B, H, dk, dv, dtype, scale, stream,
                        log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
+}
+
+size_t kda_backward_workspace_bytes(int B, int T, int H, int dk, int dv)
+{
+    if (B <= 0 || H <= 0 || T < 0 || dk != dv || (dk != 64 && dk != 128)) return 0;
+    return kda::backward_workspace_bytes(B, T, H, dk);
+}
+
+kda_status kda_backward(const void *q, const void *k, const void *v,
+                        const float *log_alpha, const float *beta, const float *initial_state,
+                        const float *grad_out, const float *grad_final_state,
+                        float *grad_q, float *grad_k, float *grad_v, float *grad_log_alpha,
+                        float *grad_beta, float *grad_initial_state,
+                        int B, int T, int H, int dk, int dv,
+                        kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes,
+                        void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (B <= 0 || H <= 0 || T < 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if ((int64_t)B * H * ((int64_t)T + 64) > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
+    if (dk != dv || (dk != 64 && dk != 128)) return KDA_ERR_UNSUPPORTED;
+    if (T > 0) {
+        if (!q || !k || !v || !log_alpha || !beta || !grad_out || !grad_q || !grad_k || !grad_v ||
+            !grad_log_alpha || !grad_beta || !workspace)
+            return KDA_ERR_INVALID_ARG;
+        if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(log_alpha) || !aligned16(grad_out) ||
+            !aligned16(grad_q) || !aligned16(grad_k) || !aligned16(grad_v) || !aligned16(grad_log_alpha) ||
+            !aligned4(beta) || !aligned4(grad_beta) || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+            return KDA_ERR_MISALIGNED;
+        if (workspace_bytes < kda::backward_workspace_bytes(B, T, H, dk)) return KDA_ERR_INVALID_ARG;
+    }
+    if ((initial_state && !aligned16(initial_state)) || (grad_final_state && !aligned16(grad_final_state)) ||
+        (grad_initial_state && !aligned16(grad_initial_state)))
+        return KDA_ERR_MISALIGNED;
+    if (T == 0 && !grad_initial_state) return KDA_OK;
+    kda::BackwardArgs a = {};
+    a.q = q; a.k = k; a.v = v; a.log_alpha = log_alpha; a.beta = beta; a.s0 = initial_state;
+    a.d_out = grad_out; a.d_final = grad_final_state;
+    a.dq = grad_q; a.dk = grad_k; a.dv = grad_v; a.dlog_alpha = grad_log_alpha; a.dbeta = grad_beta;
+    a.d_s0 = grad_initial_state;
+    a.B = B; a.T = T; a.H = H; a.Dk = dk; a.Dv = dv; a.dtype = dtype;
+    a.scale = (scale == 0.0f) ? 1.0f / sqrtf((float)dk) : scale;
+    a.workspace = workspace;
+    const cudaError_t e = kda::launch_backward(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
 kda_status kda_selftest_timeout(unsigned int wait_ms, void *stream)

@@ -1,0 +1,451 @@
+// The KDA backward pass: gradients of the forward with respect to q, k, v,
+// log_alpha, beta and the initial state, given the cotangents of the outputs
+// and of the final state.
+//
+// The pages define the forward by its token step ("Kimi Delta Attention: The
+// Linear Attention Behind Kimi K2 and Qwen3", §How Kimi Delta Attention works
+// step by step) and name chunkwise training without giving a gradient ("KDA
+// Technical Deep Dive", §Systems and implementation tradeoffs, Training).  The
+// backward here is the reverse-mode derivative of that step.  Per token, with
+// a = exp(log_alpha_t):
+//
+//   forward   S~ = Diag(a) S,  p = S~^T k,  e = beta (v - p),  S' = S~ + k e^T,  o = scale S'^T q
+//   backward  (dS = dL/dS', swept from the last token to the first)
+//             dS += scale q dO^T;          dq = scale S' dO
+//             de = dS^T k;  dv = beta de;  dbeta = de . (v - p);  dp = -beta de
+//             dk = dS e + S~ dp;           dS~ = dS + k dp^T
+//             dlog_alpha = rowsum(dS~ * S~);  dS <- Diag(a) dS~
+//
+// Value columns of S never mix, so every pass is parallel over columns: warp w of
+// a CTA owns one column, lane l owns the key rows l, l + 32, ...  Sums over rows
+// (p and dS^T k, which feed the recurrence) are warp sums; sums over columns (dq,
+// dk, dlog_alpha) are outputs only and are reduced across warps in shared memory.
+//
+// Three kernels, all fp32 on CUDA cores:
+//   bwd_state_kernel     the forward state at the start of every chunk of 64 tokens
+//   bwd_adjoint_kernel   dS at the end of every chunk (and dL/dS_0), swept backwards
+//   bwd_chunk_grad_kernel  one CTA per (b, h, chunk): the chunk's states recomputed
+//                        from its start (checkpoints every 8 tokens), the backward
+//                        sweep from the chunk's end adjoint, one value-column block
+//                        after another; the chunk's rows of dq, dk, dlog_alpha and
+//                        dbeta belong to this CTA alone, so the blocks accumulate
+//                        into them without atomics.
+#include "kda_internal.cuh"
+
+namespace kda {
+namespace {
+
+constexpr int kBC = 64;              // tokens per chunk
+constexpr int kBW = 8;               // warps per CTA = value columns per block
+constexpr int kBThreads = kBW * 32;
+constexpr int kSub = 8;              // tokens between recomputation checkpoints
+
+__device__ __forceinline__ float warp_sum(float x)
+{
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+__device__ __forceinline__ void cp_async(void *dst, const void *src, int bytes, bool valid)
+{
+    const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
+    if (bytes == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(d), "l"(src), "r"(valid ? 16 : 0)
+                     : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(d), "l"(src), "r"(valid ? 4 : 0)
+                     : "memory");
+}
+__device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
+
+// One chunk's per-token inputs in shared memory (rows past the sequence end are
+// zero-filled): key rows (and query rows) in the input dtype, log_alpha rows,
+// beta, and the block's 8 value (and output-cotangent) columns.
+template <typename Tin, int D>
+struct Stage {
+    Tin k[kBC][D];
+    Tin q[kBC][D];
+    float la[kBC][D];
+    Tin v[kBC][kBW];
+    float dout[kBC][kBW];
+    float beta[kBC];
+};
+
+struct Dims {
+    int T, H, nc;
+    float scale;
+};
+
+__device__ __forceinline__ size_t tok_row(int b, int t, int h, const Dims &d)
+{
+    return ((size_t)b * d.T + t) * d.H + h;
+}
+
+// Copies the chunk's key rows (and query rows), log_alpha rows and beta into a
+// stage (cp.async; rows past the sequence end zero-filled, their source clamped to
+// a valid row).
+template <typename Tin, int D>
+__device__ void stage_rows(Stage<Tin, D> &s, const Tin *k, const Tin *q, const float *la, const float *beta,
+                           int b, int h, int c, bool with_q, const Dims &d)
+{
+    const int tid = threadIdx.x, t0 = c * kBC;
+    constexpr int kPerRowK = D * (int)sizeof(Tin) / 16, kPerRowA = D * 4 / 16;
+    for (int i = tid; i < kBC * kPerRowK; i += kBThreads) {
+        const int t = i / kPerRowK, j = i % kPerRowK;
+        const bool ok = t0 + t < d.T;
+        const size_t row = tok_row(b, ok ? t0 + t : 0, h, d);
+        cp_async(reinterpret_cast<uint8_t *>(&s.k[t][0]) + 16 * j,
+                 reinterpret_cast<const uint8_t *>(k + row * D) + 16 * j, 16, ok);
+        if (with_q)
+            cp_async(reinterpret_cast<uint8_t *>(&s.q[t][0]) + 16 * j,
+                     reinterpret_cast<const uint8_t *>(q + row * D) + 16 * j, 16, ok);
+    }
+    for (int i = tid; i < kBC * kPerRowA; i += kBThreads) {
+        const int t = i / kPerRowA, j = i % kPerRowA;
+        const bool ok = t0 + t < d.T;
+        cp_async(&s.la[t][4 * j], la + tok_row(b, ok ? t0 + t : 0, h, d) * D + 4 * j, 16, ok);
+    }
+    if (tid < kBC) {
+        const bool ok = t0 + tid < d.T;
+        cp_async(&s.beta[tid], beta + tok_row(b, ok ? t0 + tid : 0, h, d), 4, ok);
+    }
+}
+
+// Copies the chunk's value columns col0 .. col0 + 7 (and output-cotangent columns).
+template <typename Tin, int D>
+__device__ void stage_cols(Stage<Tin, D> &s, const Tin *v, const float *dout, int b, int h, int c, int col0,
+                           const Dims &d)
+{
+    const int tid = threadIdx.x, t0 = c * kBC;
+    constexpr int kPerRowV = kBW * (int)sizeof(Tin) / 16;    // 1 (bf16) or 2 (fp32)
+    for (int i = tid; i < kBC * kPerRowV; i += kBThreads) {
+        const int t = i / kPerRowV, j = i % kPerRowV;
+        const bool ok = t0 + t < d.T;
+        cp_async(reinterpret_cast<uint8_t *>(&s.v[t][0]) + 16 * j,
+                 reinterpret_cast<const uint8_t *>(v + tok_row(b, ok ? t0 + t : 0, h, d) * D + col0) + 16 * j, 16, ok);
+    }
+    if (dout) {
+        for (int i = tid; i < kBC * 2; i += kBThreads) {
+            const int t = i >> 1, j = i & 1;
+            const bool ok = t0 + t < d.T;
+            cp_async(&s.dout[t][4 * j], dout + tok_row(b, ok ? t0 + t : 0, h, d) * D + col0 + 4 * j, 16, ok);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- forward states
+// CTA (b, h, block of 8 value columns); writes S at the start of every chunk:
+// states[c][b][h][row][col].
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kBThreads)
+bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ la,
+                 const float *__restrict__ beta, const float *__restrict__ s0, float *__restrict__ states, Dims d)
+{
+    constexpr int R = D / 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    Stage<Tin, D> *st = reinterpret_cast<Stage<Tin, D> *>(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = D / kBW;
+    const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
+    const int b = bh / d.H, h = bh % d.H;
+    const int col = blk * kBW + warp;
+    float S[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) S[i] = s0 ? s0[((size_t)bh * D + lane + 32 * i) * D + col] : 0.f;
+    auto stage = [&](int c) {
+        stage_rows<Tin, D>(st[c & 1], k, nullptr, la, beta, b, h, c, false, d);
+        stage_cols<Tin, D>(st[c & 1], v, nullptr, b, h, c, blk * kBW, d);
+        cp_commit();
+    };
+    if (d.nc > 0) stage(0);
+    for (int c = 0; c < d.nc; ++c) {
+        Stage<Tin, D> &s = st[c & 1];
+        if (c + 1 < d.nc) {
+            stage(c + 1);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        __syncthreads();
+        float *dst = states + ((size_t)c * gridDim.x / nblk + bh) * D * D;
+#pragma unroll
+        for (int i = 0; i < R; ++i) dst[(size_t)(lane + 32 * i) * D + col] = S[i];
+        const int len = min(kBC, d.T - c * kBC);
+        for (int t = 0; t < len; ++t) {
+            float part = 0.f, kk[R];
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                kk[i] = to_f32(s.k[t][lane + 32 * i]);
+                S[i] *= __expf(s.la[t][lane + 32 * i]);
+                part += S[i] * kk[i];
+            }
+            const float p = warp_sum(part);
+            const float e = s.beta[t] * (to_f32(s.v[t][warp]) - p);
+#pragma unroll
+            for (int i = 0; i < R; ++i) S[i] += kk[i] * e;
+        }
+        __syncthreads();      // the stage is refilled two chunks later
+    }
+}
+
+// ---------------------------------------------------------------- adjoint states
+// CTA (b, h, block of 8 value columns); sweeps the tokens backwards from dS =
+// d_final (or 0) and writes dS at the end of every chunk: dstates[c][b][h][row][col];
+// at the start of the sequence, dL/dS_0 into d_s0 (if given).
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kBThreads)
+bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                   const float *__restrict__ la, const float *__restrict__ beta, const float *__restrict__ dout,
+                   const float *__restrict__ d_final, float *__restrict__ dstates, float *__restrict__ d_s0, Dims d)
+{
+    constexpr int R = D / 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    Stage<Tin, D> *st = reinterpret_cast<Stage<Tin, D> *>(smem);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nblk = D / kBW;
+    const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
+    const int b = bh / d.H, h = bh % d.H;
+    const int col = blk * kBW + warp;
+    float dS[R];
+#pragma unroll
+    for (int i = 0; i < R; ++i) dS[i] = d_final ? d_final[((size_t)bh * D + lane + 32 * i) * D + col] : 0.f;
+    auto stage = [&](int c) {
+        stage_rows<Tin, D>(st[c & 1], k, q, la, beta, b, h, c, true, d);
+        stage_cols<Tin, D>(st[c & 1], v, dout, b, h, c, blk * kBW, d);
+        cp_commit();
+    };
+    if (d.nc > 0) stage(d.nc - 1);
+    for (int c = d.nc - 1; c >= 0; --c) {
+        Stage<Tin, D> &s = st[c & 1];
+        if (c > 0) {
+            stage(c - 1);
+            cp_wait<1>();
+        } else {
+            cp_wait<0>();
+        }
+        __syncthreads();
+        float *dst = dstates + ((size_t)c * gridDim.x / nblk + bh) * D * D;
+#pragma unroll
+        for (int i = 0; i < R; ++i) dst[(size_t)(lane + 32 * i) * D + col] = dS[i];
+        const int len = min(kBC, d.T - c * kBC);
+        for (int t = len - 1; t >= 0; --t) {
+            const float go = d.scale * s.dout[t][warp];
+            float part = 0.f, kk[R];
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                kk[i] = to_f32(s.k[t][lane + 32 * i]);
+                dS[i] += to_f32(s.q[t][lane + 32 * i]) * go;
+                part += dS[i] * kk[i];
+            }
+            const float dp = -s.beta[t] * warp_sum(part);
+#pragma unroll
+            for (int i = 0; i < R; ++i) dS[i] = __expf(s.la[t][lane + 32 * i]) * (dS[i] + kk[i] * dp);
+        }
+        __syncthreads();
+    }
+    if (d_s0) {
+#pragma unroll
+        for (int i = 0; i < R; ++i) d_s0[((size_t)bh * D + lane + 32 * i) * D + col] = dS[i];
+    }
+}
+
+// ---------------------------------------------------------------- per-chunk gradients
+template <typename Tin, int D>
+struct GradSmem {
+    Stage<Tin, D> s;                       // k, q, log_alpha, beta of the chunk; v, dO of the block
+    float ckpt[kBC / kSub][D][kBW];        // state before tokens 0, 8, 16, ... of the chunk
+    float red[kBW][3][D];                  // per-warp partials of dq, dk, dlog_alpha for one token
+    float redb[kBW];                       // ... and of dbeta
+};
+
+template <typename Tin, int D>
+__global__ void __launch_bounds__(kBThreads, 2)
+bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
+                      const float *__restrict__ la, const float *__restrict__ beta, const float *__restrict__ dout,
+                      const float *__restrict__ states, const float *__restrict__ dstates,
+                      float *__restrict__ dq, float *__restrict__ dk, float *__restrict__ dv,
+                      float *__restrict__ dla, float *__restrict__ dbeta, Dims d)
+{
+    constexpr int R = D / 32;
+    extern __shared__ __align__(16) uint8_t smem[];
+    GradSmem<Tin, D> &g = *reinterpret_cast<GradSmem<Tin, D> *>(smem);
+    Stage<Tin, D> &s = g.s;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int c = blockIdx.x % d.nc, bh = blockIdx.x / d.nc;
+    const int b = bh / d.H, h = bh % d.H;
+    const int t0 = c * kBC, len = min(kBC, d.T - t0);
+    const size_t BH = (size_t)gridDim.x / d.nc;
+    const float *S0 = states + ((size_t)c * BH + bh) * D * D;
+    const float *dSe = dstates + ((size_t)c * BH + bh) * D * D;
+
+    for (int blk = 0; blk < D / kBW; ++blk) {
+        const int col = blk * kBW + warp;
+        // the chunk's rows are staged once, the block's value and cotangent columns every block
+        if (blk == 0) stage_rows<Tin, D>(s, k, q, la, beta, b, h, c, true, d);
+        stage_cols<Tin, D>(s, v, dout, b, h, c, blk * kBW, d);
+        cp_commit();
+        cp_wait<0>();
+        __syncthreads();
+
+        // ---- forward through the chunk from its start, keeping a checkpoint every 8 tokens
+        float S[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) S[i] = S0[(size_t)(lane + 32 * i) * D + col];
+        for (int t = 0; t < len; ++t) {
+            if (t % kSub == 0) {
+#pragma unroll
+                for (int i = 0; i < R; ++i) g.ckpt[t / kSub][lane + 32 * i][warp] = S[i];
+            }
+            float part = 0.f;
+#pragma unroll
+            for (int i = 0; i < R; ++i) {
+                S[i] *= __expf(s.la[t][lane + 32 * i]);
+                part += S[i] * to_f32(s.k[t][lane + 32 * i]);
+            }
+            const float e = s.beta[t] * (to_f32(s.v[t][warp]) - warp_sum(part));
+#pragma unroll
+            for (int i = 0; i < R; ++i) S[i] += to_f32(s.k[t][lane + 32 * i]) * e;
+        }
+
+        // ---- backward sweep, one group of 8 tokens at a time (states recomputed from its checkpoint)
+        float dS[R];
+#pragma unroll
+        for (int i = 0; i < R; ++i) dS[i] = dSe[(size_t)(lane + 32 * i) * D + col];
+        for (int j = (len - 1) / kSub; j >= 0; --j) {
+            float Sb[kSub][R], pb[kSub], eb[kSub];
+            float X[R];
+#pragma unroll
+            for (int i = 0; i < R; ++i) X[i] = g.ckpt[j][lane + 32 * i][warp];
+#pragma unroll
+            for (int u = 0; u < kSub; ++u) {
+                const int t = j * kSub + u;
+#pragma unroll
+                for (int i = 0; i < R; ++i) Sb[u][i] = X[i];
+                pb[u] = eb[u] = 0.f;
+                if (t < len) {
+                    float part = 0.f;
+#pragma unroll
+                    for (int i = 0; i < R; ++i) {
+                        X[i] *= __expf(s.la[t][lane + 32 * i]);
+                        part += X[i] * to_f32(s.k[t][lane + 32 * i]);
+                    }
+                    pb[u] = warp_sum(part);
+                    eb[u] = s.beta[t] * (to_f32(s.v[t][warp]) - pb[u]);
+#pragma unroll
+                    for (int i = 0; i < R; ++i) X[i] += to_f32(s.k[t][lane + 32 * i]) * eb[u];
+                }
+            }
+#pragma unroll
+            for (int u = kSub - 1; u >= 0; --u) {
+                const int t = j * kSub + u;
+                if (t >= len) continue;
+                const float bt = s.beta[t], go = d.scale * s.dout[t][warp];
+                float a[R], kk[R], St[R], part = 0.f;
+#pragma unroll
+                for (int i = 0; i < R; ++i) {
+                    const int r = lane + 32 * i;
+                    a[i] = __expf(s.la[t][r]);
+                    kk[i] = to_f32(s.k[t][r]);
+                    St[i] = a[i] * Sb[u][i];                       // S~
+                    const float Sn = St[i] + kk[i] * eb[u];        // S' (after the write)
+                    dS[i] += to_f32(s.q[t][r]) * go;
+                    g.red[warp][0][r] = Sn * go;                   // dq (this column's share)
+                    part += dS[i] * kk[i];
+                }
+                const float de = warp_sum(part);
+                const float dp = -bt * de;
+#pragma unroll
+                for (int i = 0; i < R; ++i) {
+                    const int r = lane + 32 * i;
+                    g.red[warp][1][r] = dS[i] * eb[u] + St[i] * dp;   // dk
+                    const float dSt = dS[i] + kk[i] * dp;             // dS~
+                    g.red[warp][2][r] = dSt * St[i];                  // dlog_alpha
+                    dS[i] = a[i] * dSt;
+                }
+                if (lane == 0) {
+                    g.redb[warp] = de * (to_f32(s.v[t][warp]) - pb[u]);
+                    dv[(((size_t)b * d.T + t0 + t) * d.H + h) * D + col] = bt * de;
+                }
+                __syncthreads();
+                const size_t row = ((size_t)b * d.T + t0 + t) * d.H + h;
+                for (int idx = tid; idx < 3 * D + 1; idx += kBThreads) {
+                    float sum = 0.f;
+                    if (idx < 3 * D) {
+                        const int qn = idx / D, r = idx % D;
+#pragma unroll
+                        for (int w = 0; w < kBW; ++w) sum += g.red[w][qn][r];
+                        float *dst = (qn == 0 ? dq : qn == 1 ? dk : dla) + row * D + r;
+                        *dst = blk == 0 ? sum : *dst + sum;
+                    } else {
+#pragma unroll
+                        for (int w = 0; w < kBW; ++w) sum += g.redb[w];
+                        dbeta[row] = blk == 0 ? sum : dbeta[row] + sum;
+                    }
+                }
+                __syncthreads();
+            }
+        }
+    }
+}
+
+template <typename Tin, int D>
+cudaError_t launch_backward_t(const BackwardArgs &a, cudaStream_t stream)
+{
+    const Tin *q = static_cast<const Tin *>(a.q), *k = static_cast<const Tin *>(a.k),
+              *v = static_cast<const Tin *>(a.v);
+    Dims d;
+    d.T = a.T;
+    d.H = a.H;
+    d.nc = (a.T + kBC - 1) / kBC;
+    d.scale = a.scale;
+    const size_t BH = (size_t)a.B * a.H;
+    float *states = reinterpret_cast<float *>(a.workspace);
+    float *dstates = states + (size_t)d.nc * BH * D * D;
+    const unsigned col_ctas = (unsigned)(BH * (D / kBW));
+    const size_t stage2 = 2 * sizeof(Stage<Tin, D>);
+    cudaError_t e = cudaSuccess;
+    if (d.nc > 0) {
+        e = cudaFuncSetAttribute(bwd_state_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stage2);
+        if (e != cudaSuccess) return e;
+        bwd_state_kernel<Tin, D><<<col_ctas, kBThreads, stage2, stream>>>(k, v, a.log_alpha, a.beta, a.s0, states, d);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        note_launch();
+    }
+    e = cudaFuncSetAttribute(bwd_adjoint_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stage2);
+    if (e != cudaSuccess) return e;
+    bwd_adjoint_kernel<Tin, D><<<col_ctas, kBThreads, stage2, stream>>>(q, k, v, a.log_alpha, a.beta, a.d_out,
+                                                                          a.d_final, dstates, a.d_s0, d);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    note_launch();
+    if (d.nc > 0) {
+        const size_t sm = sizeof(GradSmem<Tin, D>);
+        e = cudaFuncSetAttribute(bwd_chunk_grad_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)sm);
+        if (e != cudaSuccess) return e;
+        bwd_chunk_grad_kernel<Tin, D><<<(unsigned)(BH * d.nc), kBThreads, sm, stream>>>(
+            q, k, v, a.log_alpha, a.beta, a.d_out, states, dstates, a.dq, a.dk, a.dv, a.dlog_alpha, a.dbeta, d);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        note_launch();
+    }
+    return cudaSuccess;
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int B, int T, int H, int D)
+{
+    const size_t nc = ((size_t)T + kBC - 1) / kBC;
+    return 2 * nc * (size_t)B * H * D * D * sizeof(float);
+}
+
+cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t stream)
+{
+    if (a.dtype == KDA_BF16)
+        return a.Dk == 128 ? launch_backward_t<__nv_bfloat16, 128>(a, stream)
+                           : launch_backward_t<__nv_bfloat16, 64>(a, stream);
+    return a.Dk == 128 ? launch_backward_t<float, 128>(a, stream) : launch_backward_t<float, 64>(a, stream);
+}
+
+}  // namespace kda

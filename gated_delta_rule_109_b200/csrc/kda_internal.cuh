@@ -74,6 +74,24 @@ cudaError_t launch_segment_correct(const ForwardArgs &a, const float *start, con
                                    const uint8_t *ws, cudaStream_t stream);
 cudaError_t launch_affine_compose(const float *transfers, const float *local_finals, int R, int BH, float *start,
                                   cudaStream_t stream);
+// Backward pass (fp32 CUDA cores; bf16 or fp32 inputs; dk = dv = D in {64, 128}).
+// The workspace holds the forward state at the start of every chunk and the adjoint
+// at its end: backward_workspace_bytes(B, T, H, D) bytes.
+struct BackwardArgs {
+    const void *q, *k, *v;
+    const float *log_alpha, *beta;
+    const float *s0;          // may be null (zero initial state)
+    const float *d_out;
+    const float *d_final;     // may be null (no cotangent of the final state)
+    float *dq, *dk, *dv, *dlog_alpha, *dbeta;
+    float *d_s0;              // may be null
+    int B, T, H, Dk, Dv;      // head dims (equal)
+    kda_dtype dtype;
+    float scale;
+    void *workspace;
+};
+size_t backward_workspace_bytes(int B, int T, int H, int D);
+cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t stream);
 // One CTA whose bounded wait on a barrier nothing completes gives up after about
 // wait_ms and records the device status bit (failure-path self-test).
 cudaError_t launch_selftest_timeout(unsigned int wait_ms, cudaStream_t stream);

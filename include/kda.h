@@ -312,6 +312,52 @@ kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
                                int B, int H, int dk, int dv,
                                kda_dtype dtype, float scale, void *stream);
 
+/*
+ * kda_backward -- gradients of kda_forward with respect to every input.
+ *
+ * The pages give the forward's token step ("Kimi Delta Attention: The Linear
+ * Attention Behind Kimi K2 and Qwen3", §How Kimi Delta Attention works step by
+ * step) and name chunkwise training ("KDA Technical Deep Dive", §Systems and
+ * implementation tradeoffs, Training) but print no gradient; this call returns
+ * the exact derivative of that step (no counterpart on the pages).  With the
+ * loss L = sum(out * grad_out) + sum(final_state * grad_final_state):
+ *
+ *   q, k          [B, T, H, dk]  dtype    (16-byte aligned)   forward inputs, as for kda_forward
+ *   v             [B, T, H, dv]  dtype    (16-byte aligned)
+ *   log_alpha     [B, T, H, dk]  float32  (16-byte aligned)
+ *   beta          [B, T, H]      float32  (4-byte aligned)
+ *   initial_state [B, H, dk, dv] float32  (16-byte aligned) or NULL (zero state)
+ *   grad_out      [B, T, H, dv]  float32  (16-byte aligned)   dL/d out
+ *   grad_final_state [B, H, dk, dv] float32 or NULL (zero)    dL/d final_state
+ *   grad_q, grad_k [B, T, H, dk], grad_v [B, T, H, dv], grad_log_alpha [B, T, H, dk]:
+ *                  float32 outputs (16-byte aligned), overwritten
+ *   grad_beta     [B, T, H]      float32 output (4-byte aligned), overwritten
+ *   grad_initial_state [B, H, dk, dv] float32 output or NULL (not wanted)
+ *   workspace     device buffer of kda_backward_workspace_bytes(B, T, H, dk, dv)
+ *                 bytes (256-byte aligned), caller-owned; holds the forward state
+ *                 at the start of every chunk of 64 tokens and the adjoint at its end
+ *
+ * Supported: dk = dv in {64, 128}, bf16 or fp32 inputs; fp32 arithmetic on CUDA
+ * cores (KDA_ERR_UNSUPPORTED otherwise).  Every buffer is caller-owned device
+ * memory; nothing is allocated.  The outputs may not alias the inputs.  T = 0
+ * writes grad_initial_state = grad_final_state (or zeros) and nothing else.
+ * Bad pointers, sizes, dtype or scale -> KDA_ERR_INVALID_ARG; misaligned ->
+ * KDA_ERR_MISALIGNED; a workspace below the size -> KDA_ERR_INVALID_ARG; launch
+ * failures -> KDA_ERR_CUDA.  Asynchronous on `stream`; deterministic.
+ */
+kda_status kda_backward(const void *q, const void *k, const void *v,
+                        const float *log_alpha, const float *beta, const float *initial_state,
+                        const float *grad_out, const float *grad_final_state,
+                        float *grad_q, float *grad_k, float *grad_v, float *grad_log_alpha,
+                        float *grad_beta, float *grad_initial_state,
+                        int B, int T, int H, int dk, int dv,
+                        kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes,
+                        void *stream);
+
+/* Workspace bytes kda_backward needs: 2 * ceil(T / 64) * B * H * dk * dv * 4
+ * (0 for unsupported shapes). */
+size_t kda_backward_workspace_bytes(int B, int T, int H, int dk, int dv);
+
 /* Static, human-readable name of a status code (never NULL). */
 const char *kda_status_string(kda_status status);
 

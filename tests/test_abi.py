@@ -223,3 +223,37 @@ def test_segment_calls_validate_before_launch(lib):
     assert correct(out=FAKE + 4) == kda.KDA_ERR_MISALIGNED
     assert correct(sT=FAKE + 8) == kda.KDA_ERR_MISALIGNED
     assert correct(nbytes=kda.workspace_bytes(1, 8, 2, 128, 128) - 1) == kda.KDA_ERR_UNSUPPORTED
+
+
+def test_backward_validates_before_launch(lib):
+    WS = FAKE * 16
+
+    def bwd(T=8, dk=128, dv=128, dtype=kda.KDA_BF16, ws=WS, nbytes=1 << 40, scale=0.0, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, go=FAKE, gs=None, gq=FAKE, gk=FAKE,
+                 gv=FAKE, gla=FAKE, gb=FAKE, gs0=FAKE)
+        a.update(kw)
+        return lib.kda_backward(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["go"], a["gs"], a["gq"],
+                                a["gk"], a["gv"], a["gla"], a["gb"], a["gs0"], 1, T, 2, dk, dv, dtype,
+                                ctypes.c_float(scale), ws, nbytes, None)
+    assert bwd(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(go=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(gla=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(ws=None) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(T=-1) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dtype=5) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(scale=float("nan")) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(nbytes=kda.backward_workspace_bytes(1, 8, 2, 128, 128) - 1) == kda.KDA_ERR_INVALID_ARG
+    assert bwd(dk=96, dv=96) == kda.KDA_ERR_UNSUPPORTED
+    assert bwd(dk=64, dv=128) == kda.KDA_ERR_UNSUPPORTED
+    assert bwd(q=FAKE + 8) == kda.KDA_ERR_MISALIGNED
+    assert bwd(gk=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+    assert bwd(beta=FAKE + 2) == kda.KDA_ERR_MISALIGNED
+    assert bwd(ws=WS + 16) == kda.KDA_ERR_MISALIGNED
+    assert bwd(s0=FAKE + 4) == kda.KDA_ERR_MISALIGNED
+    # T = 0 without a wanted initial-state gradient: nothing to do, no CUDA call
+    assert bwd(T=0, q=None, k=None, v=None, la=None, beta=None, go=None, gq=None, gk=None, gv=None, gla=None,
+               gb=None, gs0=None, ws=None) == kda.KDA_OK
+    wb = lib.kda_backward_workspace_bytes
+    assert wb(1, 65, 2, 128, 128) == 2 * 2 * 2 * 128 * 128 * 4
+    assert wb(3, 64, 5, 64, 64) == 2 * 1 * 15 * 64 * 64 * 4
+    assert wb(1, 0, 2, 128, 128) == 0 and wb(1, 64, 2, 96, 96) == 0 and wb(1, 64, 2, 64, 128) == 0
