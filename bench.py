@@ -569,6 +569,53 @@ def _add_time_split(line, args, w, device, segments=8):
         "max_abs_err_over_rms_vs_whole_sequence": check}
 
 
+def backward_bytes_per_token_head(dk, dv, in_bytes):
+    """Algorithmic HBM bytes of the backward per token and head: q, k (dk) and v (dv)
+    in the input dtype, log_alpha (dk) and the output cotangent (dv) in fp32, beta,
+    and the fp32 gradients of q, k, v, log_alpha and beta."""
+    return in_bytes * (2 * dk + dv) + 4 * (dk + dv) + 4 + 4 * (3 * dk + dv) + 4
+
+
+def _add_backward(line, args, device, hbm, world=1, w=None):
+    """kda_backward on the short-context prefill workload (B1 H16 T4096 d128 bf16):
+    every gradient, with the forward inputs and the output cotangent resident."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    w = w or I.PREFILL_H16_T4K
+    x = I.make_inputs(w, device)
+    g = torch.Generator(device=device)
+    g.manual_seed(w.seed + 500)
+    d_out = torch.randn((w.B, w.T, w.H, w.dv), generator=g, device=device)
+    ws = torch.empty(kda.backward_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv), dtype=torch.uint8, device=device)
+    names = ("q", "k", "v", "log_alpha", "beta")
+    fn = lambda: kda.backward(*(x[n] for n in names), d_out, x["initial_state"], None, workspace=ws)
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize(device)
+    stream = torch.cuda.current_stream(device)
+    n0 = kda.launch_count()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.steps):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    launches = kda.launch_count() - n0
+    kda.check_status(device)
+    ms = max_over_ranks(e0.elapsed_time(e1), device) / args.steps
+    in_bytes = 2 if w.dtype == "bf16" else 4
+    alg = w.B * w.T * w.H * backward_bytes_per_token_head(w.dk, w.dv, in_bytes)
+    achieved = alg / (ms / 1e3) / 1e9
+    line["backward"] = {
+        "workload": w.name, "value": w.B * w.T * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+        "gpu_launches": launches,
+        "kernels": "bwd_state_kernel + bwd_adjoint_kernel + bwd_chunk_grad_kernel (fp32 CUDA cores)",
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                     "traffic": None, "algorithmic_bytes_per_launch": alg,
+                     "launch": "one kda_backward call (three kernels)"}}
+
+
 # ---------------------------------------------------------------- main
 def main(argv=None):
     ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
@@ -697,6 +744,7 @@ def main(argv=None):
             _add_raw(line, args, w, world, device, hbm)
             if world == 1:
                 _add_time_split(line, args, w, device)
+        _add_backward(line, args, device, hbm, world)
 
     if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],

@@ -36,7 +36,7 @@ namespace kda {
 namespace {
 
 constexpr int kBC = 64;              // tokens per chunk
-constexpr int kBW = 8;               // warps per CTA = value columns per block
+constexpr int kBW = 16;              // warps per CTA = value columns per block
 constexpr int kBThreads = kBW * 32;
 constexpr int kSub = 8;              // tokens between recomputation checkpoints
 
@@ -64,13 +64,13 @@ __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0
 // One chunk's per-token inputs in shared memory (rows past the sequence end are
 // zero-filled): key rows (and query rows) in the input dtype, log_alpha rows,
 // beta, and the block's 8 value (and output-cotangent) columns.
-template <typename Tin, int D>
+template <typename Tin, int D, bool WITH_Q = true>
 struct Stage {
     Tin k[kBC][D];
-    Tin q[kBC][D];
-    float la[kBC][D];
+    Tin q[WITH_Q ? kBC : 1][D];
+    float la[kBC][D];                      // log_alpha as staged, then alpha = exp(log_alpha)
     Tin v[kBC][kBW];
-    float dout[kBC][kBW];
+    float dout[WITH_Q ? kBC : 1][kBW];
     float beta[kBC];
 };
 
@@ -87,9 +87,9 @@ __device__ __forceinline__ size_t tok_row(int b, int t, int h, const Dims &d)
 // Copies the chunk's key rows (and query rows), log_alpha rows and beta into a
 // stage (cp.async; rows past the sequence end zero-filled, their source clamped to
 // a valid row).
-template <typename Tin, int D>
-__device__ void stage_rows(Stage<Tin, D> &s, const Tin *k, const Tin *q, const float *la, const float *beta,
-                           int b, int h, int c, bool with_q, const Dims &d)
+template <typename Tin, int D, bool WITH_Q>
+__device__ void stage_rows(Stage<Tin, D, WITH_Q> &s, const Tin *k, const Tin *q, const float *la,
+                           const float *beta, int b, int h, int c, const Dims &d)
 {
     const int tid = threadIdx.x, t0 = c * kBC;
     constexpr int kPerRowK = D * (int)sizeof(Tin) / 16, kPerRowA = D * 4 / 16;
@@ -99,7 +99,7 @@ __device__ void stage_rows(Stage<Tin, D> &s, const Tin *k, const Tin *q, const f
         const size_t row = tok_row(b, ok ? t0 + t : 0, h, d);
         cp_async(reinterpret_cast<uint8_t *>(&s.k[t][0]) + 16 * j,
                  reinterpret_cast<const uint8_t *>(k + row * D) + 16 * j, 16, ok);
-        if (with_q)
+        if (WITH_Q)
             cp_async(reinterpret_cast<uint8_t *>(&s.q[t][0]) + 16 * j,
                      reinterpret_cast<const uint8_t *>(q + row * D) + 16 * j, 16, ok);
     }
@@ -114,10 +114,10 @@ __device__ void stage_rows(Stage<Tin, D> &s, const Tin *k, const Tin *q, const f
     }
 }
 
-// Copies the chunk's value columns col0 .. col0 + 7 (and output-cotangent columns).
-template <typename Tin, int D>
-__device__ void stage_cols(Stage<Tin, D> &s, const Tin *v, const float *dout, int b, int h, int c, int col0,
-                           const Dims &d)
+// Copies the chunk's value columns col0 .. col0 + kBW - 1 (and output-cotangent columns).
+template <typename Tin, int D, bool WITH_Q>
+__device__ void stage_cols(Stage<Tin, D, WITH_Q> &s, const Tin *v, const float *dout, int b, int h, int c,
+                           int col0, const Dims &d)
 {
     const int tid = threadIdx.x, t0 = c * kBC;
     constexpr int kPerRowV = kBW * (int)sizeof(Tin) / 16;    // 1 (bf16) or 2 (fp32)
@@ -127,13 +127,23 @@ __device__ void stage_cols(Stage<Tin, D> &s, const Tin *v, const float *dout, in
         cp_async(reinterpret_cast<uint8_t *>(&s.v[t][0]) + 16 * j,
                  reinterpret_cast<const uint8_t *>(v + tok_row(b, ok ? t0 + t : 0, h, d) * D + col0) + 16 * j, 16, ok);
     }
-    if (dout) {
-        for (int i = tid; i < kBC * 2; i += kBThreads) {
-            const int t = i >> 1, j = i & 1;
+    if (WITH_Q) {
+        constexpr int kPerRowO = kBW * 4 / 16;
+        for (int i = tid; i < kBC * kPerRowO; i += kBThreads) {
+            const int t = i / kPerRowO, j = i % kPerRowO;
             const bool ok = t0 + t < d.T;
             cp_async(&s.dout[t][4 * j], dout + tok_row(b, ok ? t0 + t : 0, h, d) * D + col0 + 4 * j, 16, ok);
         }
     }
+}
+
+// log_alpha rows of a landed stage -> alpha = exp(log_alpha), once per chunk
+// (every warp of the CTA reads the same rows).
+template <typename Tin, int D, bool WITH_Q>
+__device__ __forceinline__ void stage_exp(Stage<Tin, D, WITH_Q> &s)
+{
+    float *x = &s.la[0][0];
+    for (int i = threadIdx.x; i < kBC * D; i += kBThreads) x[i] = expf(x[i]);
 }
 
 // ---------------------------------------------------------------- forward states
@@ -146,7 +156,8 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
 {
     constexpr int R = D / 32;
     extern __shared__ __align__(16) uint8_t smem[];
-    Stage<Tin, D> *st = reinterpret_cast<Stage<Tin, D> *>(smem);
+    using St = Stage<Tin, D, false>;
+    St *st = reinterpret_cast<St *>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nblk = D / kBW;
     const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
@@ -156,19 +167,21 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
 #pragma unroll
     for (int i = 0; i < R; ++i) S[i] = s0 ? s0[((size_t)bh * D + lane + 32 * i) * D + col] : 0.f;
     auto stage = [&](int c) {
-        stage_rows<Tin, D>(st[c & 1], k, nullptr, la, beta, b, h, c, false, d);
-        stage_cols<Tin, D>(st[c & 1], v, nullptr, b, h, c, blk * kBW, d);
+        stage_rows<Tin, D, false>(st[c & 1], k, nullptr, la, beta, b, h, c, d);
+        stage_cols<Tin, D, false>(st[c & 1], v, nullptr, b, h, c, blk * kBW, d);
         cp_commit();
     };
     if (d.nc > 0) stage(0);
     for (int c = 0; c < d.nc; ++c) {
-        Stage<Tin, D> &s = st[c & 1];
+        St &s = st[c & 1];
         if (c + 1 < d.nc) {
             stage(c + 1);
             cp_wait<1>();
         } else {
             cp_wait<0>();
         }
+        __syncthreads();
+        stage_exp(s);
         __syncthreads();
         float *dst = states + ((size_t)c * gridDim.x / nblk + bh) * D * D;
 #pragma unroll
@@ -179,7 +192,7 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
 #pragma unroll
             for (int i = 0; i < R; ++i) {
                 kk[i] = to_f32(s.k[t][lane + 32 * i]);
-                S[i] *= __expf(s.la[t][lane + 32 * i]);
+                S[i] *= s.la[t][lane + 32 * i];
                 part += S[i] * kk[i];
             }
             const float p = warp_sum(part);
@@ -203,7 +216,8 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 {
     constexpr int R = D / 32;
     extern __shared__ __align__(16) uint8_t smem[];
-    Stage<Tin, D> *st = reinterpret_cast<Stage<Tin, D> *>(smem);
+    using St = Stage<Tin, D, true>;
+    St *st = reinterpret_cast<St *>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nblk = D / kBW;
     const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
@@ -213,19 +227,21 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 #pragma unroll
     for (int i = 0; i < R; ++i) dS[i] = d_final ? d_final[((size_t)bh * D + lane + 32 * i) * D + col] : 0.f;
     auto stage = [&](int c) {
-        stage_rows<Tin, D>(st[c & 1], k, q, la, beta, b, h, c, true, d);
-        stage_cols<Tin, D>(st[c & 1], v, dout, b, h, c, blk * kBW, d);
+        stage_rows<Tin, D, true>(st[c & 1], k, q, la, beta, b, h, c, d);
+        stage_cols<Tin, D, true>(st[c & 1], v, dout, b, h, c, blk * kBW, d);
         cp_commit();
     };
     if (d.nc > 0) stage(d.nc - 1);
     for (int c = d.nc - 1; c >= 0; --c) {
-        Stage<Tin, D> &s = st[c & 1];
+        St &s = st[c & 1];
         if (c > 0) {
             stage(c - 1);
             cp_wait<1>();
         } else {
             cp_wait<0>();
         }
+        __syncthreads();
+        stage_exp(s);
         __syncthreads();
         float *dst = dstates + ((size_t)c * gridDim.x / nblk + bh) * D * D;
 #pragma unroll
@@ -242,7 +258,7 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
             }
             const float dp = -s.beta[t] * warp_sum(part);
 #pragma unroll
-            for (int i = 0; i < R; ++i) dS[i] = __expf(s.la[t][lane + 32 * i]) * (dS[i] + kk[i] * dp);
+            for (int i = 0; i < R; ++i) dS[i] = s.la[t][lane + 32 * i] * (dS[i] + kk[i] * dp);
         }
         __syncthreads();
     }
@@ -255,14 +271,14 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 // ---------------------------------------------------------------- per-chunk gradients
 template <typename Tin, int D>
 struct GradSmem {
-    Stage<Tin, D> s;                       // k, q, log_alpha, beta of the chunk; v, dO of the block
+    Stage<Tin, D, true> s;                 // k, q, log_alpha, beta of the chunk; v, dO of the block
     float ckpt[kBC / kSub][D][kBW];        // state before tokens 0, 8, 16, ... of the chunk
-    float red[kBW][3][D];                  // per-warp partials of dq, dk, dlog_alpha for one token
-    float redb[kBW];                       // ... and of dbeta
+    float red[2][kBW][3][D];               // per-warp partials of dq, dk, dlog_alpha (two tokens in turn)
+    float redb[2][kBW];                    // ... and of dbeta
 };
 
 template <typename Tin, int D>
-__global__ void __launch_bounds__(kBThreads, 2)
+__global__ void __launch_bounds__(kBThreads, 1)
 bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const Tin *__restrict__ v,
                       const float *__restrict__ la, const float *__restrict__ beta, const float *__restrict__ dout,
                       const float *__restrict__ states, const float *__restrict__ dstates,
@@ -272,7 +288,7 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
     constexpr int R = D / 32;
     extern __shared__ __align__(16) uint8_t smem[];
     GradSmem<Tin, D> &g = *reinterpret_cast<GradSmem<Tin, D> *>(smem);
-    Stage<Tin, D> &s = g.s;
+    Stage<Tin, D, true> &s = g.s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int c = blockIdx.x % d.nc, bh = blockIdx.x / d.nc;
     const int b = bh / d.H, h = bh % d.H;
@@ -284,11 +300,15 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
     for (int blk = 0; blk < D / kBW; ++blk) {
         const int col = blk * kBW + warp;
         // the chunk's rows are staged once, the block's value and cotangent columns every block
-        if (blk == 0) stage_rows<Tin, D>(s, k, q, la, beta, b, h, c, true, d);
-        stage_cols<Tin, D>(s, v, dout, b, h, c, blk * kBW, d);
+        if (blk == 0) stage_rows<Tin, D, true>(s, k, q, la, beta, b, h, c, d);
+        stage_cols<Tin, D, true>(s, v, dout, b, h, c, blk * kBW, d);
         cp_commit();
         cp_wait<0>();
         __syncthreads();
+        if (blk == 0) {
+            stage_exp(s);
+            __syncthreads();
+        }
 
         // ---- forward through the chunk from its start, keeping a checkpoint every 8 tokens
         float S[R];
@@ -302,7 +322,7 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
             float part = 0.f;
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                S[i] *= __expf(s.la[t][lane + 32 * i]);
+                S[i] *= s.la[t][lane + 32 * i];
                 part += S[i] * to_f32(s.k[t][lane + 32 * i]);
             }
             const float e = s.beta[t] * (to_f32(s.v[t][warp]) - warp_sum(part));
@@ -329,7 +349,7 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
                     float part = 0.f;
 #pragma unroll
                     for (int i = 0; i < R; ++i) {
-                        X[i] *= __expf(s.la[t][lane + 32 * i]);
+                        X[i] *= s.la[t][lane + 32 * i];
                         part += X[i] * to_f32(s.k[t][lane + 32 * i]);
                     }
                     pb[u] = warp_sum(part);
@@ -342,17 +362,29 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
             for (int u = kSub - 1; u >= 0; --u) {
                 const int t = j * kSub + u;
                 if (t >= len) continue;
+                const int rb = t & 1;                       // partials buffer of this token
+                const size_t row = ((size_t)b * d.T + t0 + t) * d.H + h;
+                // the accumulated sums of the previous column blocks, fetched early
+                float prev[(3 * D + 1 + kBThreads - 1) / kBThreads];
+#pragma unroll
+                for (int m = 0; m < (3 * D + 1 + kBThreads - 1) / kBThreads; ++m) {
+                    const int idx = tid + m * kBThreads;
+                    prev[m] = 0.f;
+                    if (blk > 0 && idx < 3 * D + 1)
+                        prev[m] = idx < 3 * D ? (idx < D ? dq : idx < 2 * D ? dk : dla)[row * D + idx % D]
+                                              : dbeta[row];
+                }
                 const float bt = s.beta[t], go = d.scale * s.dout[t][warp];
                 float a[R], kk[R], St[R], part = 0.f;
 #pragma unroll
                 for (int i = 0; i < R; ++i) {
                     const int r = lane + 32 * i;
-                    a[i] = __expf(s.la[t][r]);
+                    a[i] = s.la[t][r];
                     kk[i] = to_f32(s.k[t][r]);
                     St[i] = a[i] * Sb[u][i];                       // S~
                     const float Sn = St[i] + kk[i] * eb[u];        // S' (after the write)
                     dS[i] += to_f32(s.q[t][r]) * go;
-                    g.red[warp][0][r] = Sn * go;                   // dq (this column's share)
+                    g.red[rb][warp][0][r] = Sn * go;               // dq (this column's share)
                     part += dS[i] * kk[i];
                 }
                 const float de = warp_sum(part);
@@ -360,34 +392,37 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
 #pragma unroll
                 for (int i = 0; i < R; ++i) {
                     const int r = lane + 32 * i;
-                    g.red[warp][1][r] = dS[i] * eb[u] + St[i] * dp;   // dk
-                    const float dSt = dS[i] + kk[i] * dp;             // dS~
-                    g.red[warp][2][r] = dSt * St[i];                  // dlog_alpha
+                    g.red[rb][warp][1][r] = dS[i] * eb[u] + St[i] * dp;   // dk
+                    const float dSt = dS[i] + kk[i] * dp;                 // dS~
+                    g.red[rb][warp][2][r] = dSt * St[i];                  // dlog_alpha
                     dS[i] = a[i] * dSt;
                 }
                 if (lane == 0) {
-                    g.redb[warp] = de * (to_f32(s.v[t][warp]) - pb[u]);
-                    dv[(((size_t)b * d.T + t0 + t) * d.H + h) * D + col] = bt * de;
+                    g.redb[rb][warp] = de * (to_f32(s.v[t][warp]) - pb[u]);
+                    dv[row * D + col] = bt * de;
                 }
+                // one barrier per token: buffer rb is written again two tokens later,
+                // after the next token's barrier, by which time every thread has read it
                 __syncthreads();
-                const size_t row = ((size_t)b * d.T + t0 + t) * d.H + h;
-                for (int idx = tid; idx < 3 * D + 1; idx += kBThreads) {
-                    float sum = 0.f;
+#pragma unroll
+                for (int m = 0; m < (3 * D + 1 + kBThreads - 1) / kBThreads; ++m) {
+                    const int idx = tid + m * kBThreads;
                     if (idx < 3 * D) {
                         const int qn = idx / D, r = idx % D;
+                        float sum = prev[m];
 #pragma unroll
-                        for (int w = 0; w < kBW; ++w) sum += g.red[w][qn][r];
-                        float *dst = (qn == 0 ? dq : qn == 1 ? dk : dla) + row * D + r;
-                        *dst = blk == 0 ? sum : *dst + sum;
-                    } else {
+                        for (int w = 0; w < kBW; ++w) sum += g.red[rb][w][qn][r];
+                        (qn == 0 ? dq : qn == 1 ? dk : dla)[row * D + r] = sum;
+                    } else if (idx == 3 * D) {
+                        float sum = prev[m];
 #pragma unroll
-                        for (int w = 0; w < kBW; ++w) sum += g.redb[w];
-                        dbeta[row] = blk == 0 ? sum : dbeta[row] + sum;
+                        for (int w = 0; w < kBW; ++w) sum += g.redb[rb][w];
+                        dbeta[row] = sum;
                     }
                 }
-                __syncthreads();
             }
         }
+        __syncthreads();      // the next block re-stages v and dO
     }
 }
 
@@ -405,12 +440,12 @@ cudaError_t launch_backward_t(const BackwardArgs &a, cudaStream_t stream)
     float *states = reinterpret_cast<float *>(a.workspace);
     float *dstates = states + (size_t)d.nc * BH * D * D;
     const unsigned col_ctas = (unsigned)(BH * (D / kBW));
-    const size_t stage2 = 2 * sizeof(Stage<Tin, D>);
+    const size_t stage_s = 2 * sizeof(Stage<Tin, D, false>), stage2 = 2 * sizeof(Stage<Tin, D, true>);
     cudaError_t e = cudaSuccess;
     if (d.nc > 0) {
-        e = cudaFuncSetAttribute(bwd_state_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stage2);
+        e = cudaFuncSetAttribute(bwd_state_kernel<Tin, D>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)stage_s);
         if (e != cudaSuccess) return e;
-        bwd_state_kernel<Tin, D><<<col_ctas, kBThreads, stage2, stream>>>(k, v, a.log_alpha, a.beta, a.s0, states, d);
+        bwd_state_kernel<Tin, D><<<col_ctas, kBThreads, stage_s, stream>>>(k, v, a.log_alpha, a.beta, a.s0, states, d);
         if ((e = cudaGetLastError()) != cudaSuccess) return e;
         note_launch();
     }
