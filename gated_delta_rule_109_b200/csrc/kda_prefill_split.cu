@@ -185,12 +185,21 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     {
         const int ch = tid & (kDK - 1), th = tid >> 7;
         float run = 0.f;
+        if (gate_act) {
 #pragma unroll 8
-        for (int i = 0; i < 32; ++i) {
-            float *gp = Gs + (32 * th + i) * kGP + ch;
-            const float x = *gp;
-            run += (gate_act && 32 * th + i < c) ? log_sigmoid(x) : x;
-            *gp = run;
+            for (int i = 0; i < 32; ++i) {
+                float *gp = Gs + (32 * th + i) * kGP + ch;
+                run += (32 * th + i < c) ? log_sigmoid(*gp) : 0.f;
+                *gp = run;
+            }
+        } else {
+            // separate loop: no log-sigmoid evaluated (and discarded) per element
+#pragma unroll 8
+            for (int i = 0; i < 32; ++i) {
+                float *gp = Gs + (32 * th + i) * kGP + ch;
+                run += *gp;
+                *gp = run;
+            }
         }
         sTot[th * kDK + ch] = run;
     }
