@@ -22,14 +22,17 @@
 // dk, dlog_alpha) are outputs only and are reduced across warps in shared memory.
 //
 // Three kernels, all fp32 on CUDA cores:
-//   bwd_state_kernel     the forward state at the start of every chunk of 64 tokens
-//   bwd_adjoint_kernel   dS at the end of every chunk (and dL/dS_0), swept backwards
-//   bwd_chunk_grad_kernel  one CTA per (b, h, chunk): the chunk's states recomputed
-//                        from its start (checkpoints every 8 tokens), the backward
-//                        sweep from the chunk's end adjoint, one value-column block
-//                        after another; the chunk's rows of dq, dk, dlog_alpha and
-//                        dbeta belong to this CTA alone, so the blocks accumulate
-//                        into them without atomics.
+//   bwd_state_kernel     the forward state before every 8th token (checkpoints)
+//   bwd_adjoint_kernel   dS at the end of every chunk of 64 tokens (and dL/dS_0),
+//                        swept backwards
+//   bwd_chunk_grad_kernel  one CTA per (b, h, chunk): per group of 8 tokens, the
+//                        states recomputed from the group's checkpoint and the
+//                        backward swept from the chunk's end adjoint, one
+//                        value-column block after another; the chunk's rows of dq,
+//                        dk, dlog_alpha and dbeta belong to this CTA alone, so the
+//                        blocks accumulate into them without atomics.
+// Saved states and adjoints are column-major per (b, h): [slot][b, h][column][row],
+// so a warp (one column, rows across lanes) reads and writes 128-byte rows.
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -147,8 +150,8 @@ __device__ __forceinline__ void stage_exp(Stage<Tin, D, WITH_Q> &s)
 }
 
 // ---------------------------------------------------------------- forward states
-// CTA (b, h, block of 8 value columns); writes S at the start of every chunk:
-// states[c][b][h][row][col].
+// CTA (b, h, block of value columns); writes S before every 8th token:
+// states[t / 8][b, h][col][row].
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kBThreads)
 bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const float *__restrict__ la,
@@ -183,11 +186,13 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
         __syncthreads();
         stage_exp(s);
         __syncthreads();
-        float *dst = states + ((size_t)c * gridDim.x / nblk + bh) * D * D;
-#pragma unroll
-        for (int i = 0; i < R; ++i) dst[(size_t)(lane + 32 * i) * D + col] = S[i];
         const int len = min(kBC, d.T - c * kBC);
         for (int t = 0; t < len; ++t) {
+            if (t % kSub == 0) {
+                float *dst = states + (((size_t)(c * kBC + t) / kSub * (gridDim.x / nblk) + bh) * D + col) * D;
+#pragma unroll
+                for (int i = 0; i < R; ++i) dst[lane + 32 * i] = S[i];
+            }
             float part = 0.f, kk[R];
 #pragma unroll
             for (int i = 0; i < R; ++i) {
@@ -206,7 +211,7 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
 
 // ---------------------------------------------------------------- adjoint states
 // CTA (b, h, block of 8 value columns); sweeps the tokens backwards from dS =
-// d_final (or 0) and writes dS at the end of every chunk: dstates[c][b][h][row][col];
+// d_final (or 0) and writes dS at the end of every chunk: dstates[c][b, h][col][row];
 // at the start of the sequence, dL/dS_0 into d_s0 (if given).
 template <typename Tin, int D>
 __global__ void __launch_bounds__(kBThreads)
@@ -243,9 +248,9 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
         __syncthreads();
         stage_exp(s);
         __syncthreads();
-        float *dst = dstates + ((size_t)c * gridDim.x / nblk + bh) * D * D;
+        float *dst = dstates + (((size_t)c * (gridDim.x / nblk) + bh) * D + col) * D;
 #pragma unroll
-        for (int i = 0; i < R; ++i) dst[(size_t)(lane + 32 * i) * D + col] = dS[i];
+        for (int i = 0; i < R; ++i) dst[lane + 32 * i] = dS[i];
         const int len = min(kBC, d.T - c * kBC);
         for (int t = len - 1; t >= 0; --t) {
             const float go = d.scale * s.dout[t][warp];
@@ -272,7 +277,6 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
 template <typename Tin, int D>
 struct GradSmem {
     Stage<Tin, D, true> s;                 // k, q, log_alpha, beta of the chunk; v, dO of the block
-    float ckpt[kBC / kSub][D][kBW];        // state before tokens 0, 8, 16, ... of the chunk
     float red[2][kBW][3][D];               // per-warp partials of dq, dk, dlog_alpha (two tokens in turn)
     float redb[2][kBW];                    // ... and of dbeta
 };
@@ -294,7 +298,6 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
     const int b = bh / d.H, h = bh % d.H;
     const int t0 = c * kBC, len = min(kBC, d.T - t0);
     const size_t BH = (size_t)gridDim.x / d.nc;
-    const float *S0 = states + ((size_t)c * BH + bh) * D * D;
     const float *dSe = dstates + ((size_t)c * BH + bh) * D * D;
 
     for (int blk = 0; blk < D / kBW; ++blk) {
@@ -310,35 +313,16 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
             __syncthreads();
         }
 
-        // ---- forward through the chunk from its start, keeping a checkpoint every 8 tokens
-        float S[R];
-#pragma unroll
-        for (int i = 0; i < R; ++i) S[i] = S0[(size_t)(lane + 32 * i) * D + col];
-        for (int t = 0; t < len; ++t) {
-            if (t % kSub == 0) {
-#pragma unroll
-                for (int i = 0; i < R; ++i) g.ckpt[t / kSub][lane + 32 * i][warp] = S[i];
-            }
-            float part = 0.f;
-#pragma unroll
-            for (int i = 0; i < R; ++i) {
-                S[i] *= s.la[t][lane + 32 * i];
-                part += S[i] * to_f32(s.k[t][lane + 32 * i]);
-            }
-            const float e = s.beta[t] * (to_f32(s.v[t][warp]) - warp_sum(part));
-#pragma unroll
-            for (int i = 0; i < R; ++i) S[i] += to_f32(s.k[t][lane + 32 * i]) * e;
-        }
-
         // ---- backward sweep, one group of 8 tokens at a time (states recomputed from its checkpoint)
         float dS[R];
 #pragma unroll
-        for (int i = 0; i < R; ++i) dS[i] = dSe[(size_t)(lane + 32 * i) * D + col];
+        for (int i = 0; i < R; ++i) dS[i] = dSe[(size_t)col * D + lane + 32 * i];
         for (int j = (len - 1) / kSub; j >= 0; --j) {
             float Sb[kSub][R], pb[kSub], eb[kSub];
             float X[R];
+            const float *ck = states + (((size_t)(t0 / kSub + j) * BH + bh) * D + col) * D;
 #pragma unroll
-            for (int i = 0; i < R; ++i) X[i] = g.ckpt[j][lane + 32 * i][warp];
+            for (int i = 0; i < R; ++i) X[i] = ck[lane + 32 * i];
 #pragma unroll
             for (int u = 0; u < kSub; ++u) {
                 const int t = j * kSub + u;
@@ -438,7 +422,7 @@ cudaError_t launch_backward_t(const BackwardArgs &a, cudaStream_t stream)
     d.scale = a.scale;
     const size_t BH = (size_t)a.B * a.H;
     float *states = reinterpret_cast<float *>(a.workspace);
-    float *dstates = states + (size_t)d.nc * BH * D * D;
+    float *dstates = states + (size_t)((a.T + kSub - 1) / kSub) * BH * D * D;
     const unsigned col_ctas = (unsigned)(BH * (D / kBW));
     const size_t stage_s = 2 * sizeof(Stage<Tin, D, false>), stage2 = 2 * sizeof(Stage<Tin, D, true>);
     cudaError_t e = cudaSuccess;
@@ -471,8 +455,8 @@ cudaError_t launch_backward_t(const BackwardArgs &a, cudaStream_t stream)
 
 size_t backward_workspace_bytes(int B, int T, int H, int D)
 {
-    const size_t nc = ((size_t)T + kBC - 1) / kBC;
-    return 2 * nc * (size_t)B * H * D * D * sizeof(float);
+    const size_t nc = ((size_t)T + kBC - 1) / kBC, ns = ((size_t)T + kSub - 1) / kSub;
+    return (ns + nc) * (size_t)B * H * D * D * sizeof(float);
 }
 
 cudaError_t launch_backward(const BackwardArgs &a, cudaStream_t stream)

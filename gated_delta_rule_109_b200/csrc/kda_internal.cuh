@@ -75,8 +75,8 @@ cudaError_t launch_segment_correct(const ForwardArgs &a, const float *start, con
 cudaError_t launch_affine_compose(const float *transfers, const float *local_finals, int R, int BH, float *start,
                                   cudaStream_t stream);
 // Backward pass (fp32 CUDA cores; bf16 or fp32 inputs; dk = dv = D in {64, 128}).
-// The workspace holds the forward state at the start of every chunk and the adjoint
-// at its end: backward_workspace_bytes(B, T, H, D) bytes.
+// The workspace holds the forward state before every 8th token and the adjoint at
+// the end of every chunk: backward_workspace_bytes(B, T, H, D) bytes.
 struct BackwardArgs {
     const void *q, *k, *v;
     const float *log_alpha, *beta;

@@ -335,7 +335,8 @@ kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
  *   grad_initial_state [B, H, dk, dv] float32 output or NULL (not wanted)
  *   workspace     device buffer of kda_backward_workspace_bytes(B, T, H, dk, dv)
  *                 bytes (256-byte aligned), caller-owned; holds the forward state
- *                 at the start of every chunk of 64 tokens and the adjoint at its end
+ *                 before every 8th token and the adjoint at the end of every
+ *                 chunk of 64 tokens
  *
  * Supported: dk = dv in {64, 128}, bf16 or fp32 inputs; fp32 arithmetic on CUDA
  * cores (KDA_ERR_UNSUPPORTED otherwise).  Every buffer is caller-owned device
@@ -354,8 +355,8 @@ kda_status kda_backward(const void *q, const void *k, const void *v,
                         kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes,
                         void *stream);
 
-/* Workspace bytes kda_backward needs: 2 * ceil(T / 64) * B * H * dk * dv * 4
- * (0 for unsupported shapes). */
+/* Workspace bytes kda_backward needs: (ceil(T / 8) + ceil(T / 64)) * B * H *
+ * dk * dv * 4 (0 for unsupported shapes). */
 size_t kda_backward_workspace_bytes(int B, int T, int H, int dk, int dv);
 
 /* Static, human-readable name of a status code (never NULL). */

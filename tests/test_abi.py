@@ -254,6 +254,6 @@ def test_backward_validates_before_launch(lib):
     assert bwd(T=0, q=None, k=None, v=None, la=None, beta=None, go=None, gq=None, gk=None, gv=None, gla=None,
                gb=None, gs0=None, ws=None) == kda.KDA_OK
     wb = lib.kda_backward_workspace_bytes
-    assert wb(1, 65, 2, 128, 128) == 2 * 2 * 2 * 128 * 128 * 4
-    assert wb(3, 64, 5, 64, 64) == 2 * 1 * 15 * 64 * 64 * 4
+    assert wb(1, 65, 2, 128, 128) == (9 + 2) * 2 * 128 * 128 * 4
+    assert wb(3, 64, 5, 64, 64) == (8 + 1) * 15 * 64 * 64 * 4
     assert wb(1, 0, 2, 128, 128) == 0 and wb(1, 64, 2, 96, 96) == 0 and wb(1, 64, 2, 64, 128) == 0
