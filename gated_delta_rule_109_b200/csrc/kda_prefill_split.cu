@@ -673,15 +673,14 @@ __device__ __forceinline__ void emit_out(float4 *dst, const float (&qs)[16], con
 //   mma1 / mma2 (commit) the first product / Kb^T Delta of chunk kk is complete
 //   mma3 (commit)        M Delta of chunk kk is complete (the output only: the state
 //                        update does not wait for it, it runs beside the next S');
-//                        also: Kb, M and U of chunk kk are no longer read
+//                        also: Kb and M of chunk kk are no longer read
 //   wq_free[s] (commit)  the first product has read the [Wr; Qr] in slot s
 constexpr int kChainThreads = 320;
 constexpr uint32_t CH_WQ = 0;                        // two slots of [Wr; Qr] (hi, lo) and e^m
 constexpr uint32_t CH_KTM = 2 * kWqBytes;            // Kb hi, Kb lo, M hi, M lo (48 KB)
 constexpr uint32_t CH_MA = CH_KTM + 24576;           // 128-row view whose rows 64..127 are M hi
 constexpr uint32_t CH_MA_LO = CH_KTM + 32768;        //   ... and M lo
-constexpr uint32_t CH_U = CH_KTM + 49152;            // fp32 [64][32]
-constexpr uint32_t CH_GAM = CH_U + 8192;             // fp32 [128] e^{G_last}, then [128] e^{G_last - m}
+constexpr uint32_t CH_GAM = CH_KTM + 49152;          // fp32 [128] e^{G_last}, then [128] e^{G_last - m}
 constexpr uint32_t CH_S = CH_GAM + 1024, CH_S_LO = CH_S + 8192;    // S': MN-major B (outer dk, inner column)
 constexpr uint32_t CH_DL = CH_S + 16384, CH_DL_LO = CH_DL + 4096;  // Delta: MN-major B (outer token)
 constexpr uint32_t CH_MBAR = CH_DL + 8192;           // mma1, mma2, wq[2], ktm, bar_s, bar_d
@@ -703,7 +702,6 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
-    const float *sU = reinterpret_cast<const float *>(smem + CH_U);
     const float *sGam = reinterpret_cast<const float *>(smem + CH_GAM);
     volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + CH_FAIL);
     const uint32_t mbar1 = sbase + CH_MBAR, mbar2 = mbar1 + 8, mbar_wq0 = mbar1 + 16, mbar_ktm = mbar1 + 32;
@@ -763,7 +761,7 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
                           S_SO, S_SI, kDK / 16, idesc_bf16(128, kDVS, 0, 1), false);
                 umma_commit(mbar1);
                 umma_commit(wq_free0 + 8u * (kk & 1));
-                // Delta written; the compute warps have waited for this chunk's Kb, M, U
+                // Delta written; the compute warps have waited for this chunk's Kb, M, decays
                 if (!wait(bar_d, par)) break;
                 tc_fence_after();
                 mma_split(tmem + TMC_D2, sbase + CH_KTM, sbase + CH_KTM + 16384u, RW_SO, RW_SI,
@@ -776,8 +774,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
         }
     } else if (warp == 9) {
         // ---------------- copies (lane 0): [Wr; Qr] and e^m two chunks ahead (two slots,
-        // refilled once the first product has read them), Kb, M, U and the decays one
-        // chunk ahead (one slot, refilled once both products of the chunk have read it).
+        // refilled once the first product has read them), Kb, M and the decays one chunk
+        // ahead (one slot, refilled once both products of the chunk have read it).
         // Every refill waits for the slot's previous use, so no wait here can fall two
         // phases behind its barrier.
         if (lane == 0) {
@@ -795,9 +793,8 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
                 const uint8_t *r = recs + (size_t)kk * kRec;
                 ktm_pending = true;
                 ktm_par = (uint32_t)kk & 1u;
-                mbar_expect_tx(mbar_ktm, 49152u + 8192u + 1024u);
+                mbar_expect_tx(mbar_ktm, 49152u + 1024u);
                 bulk_g2s(sbase + CH_KTM, r + R_KT, 49152u, mbar_ktm);
-                bulk_g2s(sbase + CH_U, r + R_U + slice * 8192u, 8192u, mbar_ktm);
                 bulk_g2s(sbase + CH_GAM, r + R_GAM, 1024u, mbar_ktm);
             };
             load_wq(0);
@@ -833,6 +830,21 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
         bool ok = true;
         for (int kk = 0; kk < nb && ok; ++kk) {
             const uint32_t par = (uint32_t)kk & 1u;
+            // this thread's 16 values of U (token lrow), read from the record into
+            // registers now and used after the first product
+            float uu[16];
+            if (lrow < 64 && !(mode & kChainZeroU)) {
+                const float4 *src = reinterpret_cast<const float4 *>(recs + (size_t)kk * kRec + R_U + slice * 8192u +
+                                                                     lrow * 128u + half * 64u);
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    const float4 u4 = src[g];
+                    uu[4 * g] = u4.x; uu[4 * g + 1] = u4.y; uu[4 * g + 2] = u4.z; uu[4 * g + 3] = u4.w;
+                }
+            } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) uu[e] = 0.f;
+            }
             // ---- S' = Diag(e^m) S of chunk kk as a split B operand
             if (!(ok = wait(mbar_wq0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u))) break;
             {
@@ -875,7 +887,7 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
                         float d[8];
 #pragma unroll
                         for (int e = 0; e < 8; ++e)
-                            d[e] = ((mode & kChainZeroU) ? 0.f : sU[lrow * kDVS + 16 * half + 8 * g + e]) - x[8 * g + e];
+                            d[e] = uu[8 * g + e] - x[8 * g + e];
                         const uint32_t o = core_off(lrow, 16 * half + 8 * g, S_SO, S_SI);
                         st_split8(smem, CH_DL + o, CH_DL_LO + o, d);
                     }
