@@ -742,6 +742,7 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + CH_TMEMP);
     // a wait that gives up marks the CTA failed; the others then stop at their next wait
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (mbar_try(bar, parity)) return true;        // fast path: no flag read, no clock
         if (*sFail) return false;
         if (mbar_wait(bar, parity)) return true;
         *sFail = 1u;
@@ -1010,6 +1011,7 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restric
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + HC_TMEMP);
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
+        if (mbar_try(bar, parity)) return true;        // fast path: no flag read, no clock
         if (*sFail) return false;
         if (mbar_wait(bar, parity)) return true;
         *sFail = 1u;

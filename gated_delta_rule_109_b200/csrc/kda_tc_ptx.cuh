@@ -114,16 +114,24 @@ __device__ __forceinline__ float log_sigmoid(float x)
     return x < 0.f ? x - log1pf(expf(x)) : -log1pf(expf(-x));
 }
 
+// One try at the phase with the given parity (true if it has completed).
+__device__ __forceinline__ bool mbar_try(uint32_t mbar, uint32_t parity)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}\n" : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
+    return ok != 0;
+}
+
 // Bounded wait for the phase with the given parity; false if it never completed
-// within `limit` SM cycles.
+// within `limit` SM cycles.  The first try reads no clock (most waits on a hot path
+// find the phase complete or complete while the try suspends the thread).
 __device__ __forceinline__ bool mbar_wait(uint32_t mbar, uint32_t parity, long long limit = kWaitCycles)
 {
+    if (mbar_try(mbar, parity)) return true;
     const long long t0 = clock64();
     for (;;) {
-        uint32_t ok;
-        asm volatile("{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-                     "selp.u32 %0, 1, 0, p;\n\t}\n" : "=r"(ok) : "r"(mbar), "r"(parity) : "memory");
-        if (ok) return true;
+        if (mbar_try(mbar, parity)) return true;
         if (clock64() - t0 > limit) return false;
     }
 }
