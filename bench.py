@@ -75,10 +75,10 @@ MEASURED_TRAFFIC = {
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
     ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
     # two-kernel prefill, one kda_forward_ws call (prep + chain), captured on B1 H32 T8192
-    # (prep 339.6 + 574.1 MB, chain 610.3 + 119.2 MB) and scaled by 8 to T = 65536: every
+    # (prep 339.7 + 577.3 MB, chain 610.3 + 118.8 MB) and scaled by 8 to T = 65536: every
     # term (inputs, chunk records, outputs) grows with the token count
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("574d1f65745b22df", 8 * 1643.3e6),
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("574d1f65745b22df", 1643.3e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("56dce53a347229e1", 8 * 1646.1e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("56dce53a347229e1", 1646.1e6),
 }
 
 
