@@ -201,7 +201,7 @@ class ClockSampler:
 def bench_prefill(w, K, W, device, gate="channel", workspace=None):
     """K timed launches of the prefill.  gate="channel": KDA (kda_forward, or
     kda_forward_ws when a workspace is given); "scalar": Gated DeltaNet
-    (kda_gdn_forward) with channel 0 of the draw as the gate."""
+    (kda_gdn_forward, or kda_gdn_forward_ws) with channel 0 of the draw as the gate."""
     import torch
     import gated_delta_rule_109_b200 as kda
     from gated_delta_rule_109_b200 import inputs as I
@@ -214,6 +214,8 @@ def bench_prefill(w, K, W, device, gate="channel", workspace=None):
     if gate == "scalar":
         x["log_alpha"] = x["log_alpha"][..., 0].contiguous()
         fwd = kda.gdn_forward
+        if workspace is not None:
+            fwd = lambda *a, **kw: kda.gdn_forward(*a, workspace=workspace, **kw)
     args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
     for _ in range(W):
         fwd(*args, out=out, final_state=sT, return_final_state=sT is not None)
@@ -428,10 +430,16 @@ def _add_decode(line, args, rank, world, device, hbm):
                 "steps": dec["e2e_steps"]}}
 
 
-def _add_gdn(line, args, w, world, device, hbm):
-    """The Gated DeltaNet specialisation timed on the same workload shape."""
-    pre = bench_prefill(w, args.steps, args.warmup, device, gate="scalar")
+def _add_gdn(line, args, w, world, device, hbm, use_workspace=True):
+    """The Gated DeltaNet specialisation timed on the same workload shape (the
+    two-kernel path with a workspace when the shape has one)."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    ws = kda.make_workspace(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, device=device) if use_workspace else None
+    pre = bench_prefill(w, args.steps, args.warmup, device, gate="scalar", workspace=ws)
     del pre["x"]
+    del ws
+    torch.cuda.empty_cache()
     ms_total = max_over_ranks(pre["ms_total"], device)
     ms_launch = statistics.mean(pre["ms_per_launch"])
     in_bytes = 2 if w.dtype == "bf16" else 4
@@ -447,7 +455,8 @@ def _add_gdn(line, args, w, world, device, hbm):
         "ms_per_step": ms_total / args.steps, "gpu_launches": pre["launches"],
         "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                      "traffic": None,
-                     "kernel": "prefill_gdn_tc_kernel" if tc else "prefill_simt_kernel",
+                     "kernel": ("prefill_prep_kernel + prefill_chain_kernel" if tc and use_workspace
+                                else "prefill_gdn_tc_kernel" if tc else "prefill_simt_kernel"),
                      "algorithmic_bytes_per_launch": alg_bytes}}
 
 

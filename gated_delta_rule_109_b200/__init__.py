@@ -31,7 +31,7 @@ EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
            "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_segment_local",
            "kda_segment_start_state", "kda_segment_correct", "kda_forward_noalloc",
            "kda_forward_noalloc_scratch_bytes", "kda_backward", "kda_backward_workspace_bytes",
-           "kda_decode_step", "kda_gdn_forward", "kda_gdn_decode_step",
+           "kda_decode_step", "kda_gdn_forward", "kda_gdn_forward_ws", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
            "kda_launch_count",
            "kda_version")
@@ -64,6 +64,8 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_decode_step.argtypes = [vp] * 7 + [i] * 5 + [f, vp]
     lib.kda_forward_ws.restype = i
     lib.kda_forward_ws.argtypes = [vp] * 8 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
+    lib.kda_gdn_forward_ws.restype = i
+    lib.kda_gdn_forward_ws.argtypes = [vp] * 8 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
     for name in ("kda_forward_workspace_bytes", "kda_forward_workspace_min_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [i] * 6
@@ -166,11 +168,11 @@ def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, fi
     if workspace is not None:
         if workspace.device != dev or not workspace.is_contiguous():
             raise ValueError("workspace must be a contiguous tensor on %s" % dev)
-        entry = "kda_forward_ws"
-        st = lib.kda_forward_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
-                                _ptr(initial_state), _ptr(out), _ptr(final_state),
-                                B, T, H, dk, dv, code, float(scale), _ptr(workspace),
-                                workspace.numel() * workspace.element_size(), _stream(dev))
+        entry = entry + "_ws"
+        st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
+                                 _ptr(initial_state), _ptr(out), _ptr(final_state),
+                                 B, T, H, dk, dv, code, float(scale), _ptr(workspace),
+                                 workspace.numel() * workspace.element_size(), _stream(dev))
     else:
         fn = getattr(lib, entry)
         st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
@@ -418,15 +420,16 @@ def decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0
 
 
 def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
-                return_final_state=True, scale: float = 0.0):
-    """Chunked prefill of Gated DeltaNet / DeltaNet (``kda_gdn_forward``).
+                return_final_state=True, scale: float = 0.0, workspace=None):
+    """Chunked prefill of Gated DeltaNet / DeltaNet (``kda_gdn_forward``, or
+    ``kda_gdn_forward_ws`` with a workspace).
 
     As :func:`forward`, with one decay per token and head: log_alpha
     ``[B,T,H]`` fp32 (<= 0), or None for DeltaNet (no decay).
     """
     shape = None if log_alpha is None else (lambda B, T, H, dk: (B, T, H))
     return _forward("kda_gdn_forward", shape, q, k, v, log_alpha, beta, initial_state, out,
-                    final_state, return_final_state, scale)
+                    final_state, return_final_state, scale, workspace)
 
 
 def gdn_decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0):

@@ -338,6 +338,17 @@ kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
                         dtype, scale, stream, log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
 }
 
+kda_status kda_gdn_forward_ws(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta,
+                              const float *initial_state, float *out, float *final_state,
+                              int B, int T, int H, int dk, int dv,
+                              kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes, void *stream)
+{
+    return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                        dtype, scale, stream, log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE,
+                        workspace, workspace_bytes);
+}
+
 kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
                                const float *log_alpha, const float *beta,
                                float *state_inout, float *out,

@@ -105,7 +105,7 @@ __global__ void __launch_bounds__(kNT, 2)
 prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                     const float *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                    int n0, int nb, float scale, int prep_flags)
+                    int n0, int nb, float scale, int prep_flags, int gate)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -125,18 +125,32 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     const bool norm_qk = (prep_flags & kPrepNormalizeQK) != 0;       // q, k are L2-normalised here
     uint8_t *rec = ws + ((size_t)bh * nb + nloc) * kRec;
     auto row = [&](int t) { return ((size_t)b * T + t0 + t) * H + h; };
+    auto la_at = [&](int t, int chn) -> float {
+        return gate == KDA_GATE_CHANNEL ? log_alpha[row(t) * kDK + chn]
+               : gate == KDA_GATE_SCALAR ? log_alpha[row(t)] : 0.f;
+    };
 
     // ---- loads, all issued at once (one DRAM latency per CTA): log_alpha rows and beta
     // by cp.async into shared memory (rows past the chunk's end zero-filled), the k and
     // q of this thread's four (token, 8 channels) items into registers; V follows by
     // cp.async once the V region has served as scratch
     float *Gs = reinterpret_cast<float *>(smem + PP_GS);
+    if (gate == KDA_GATE_CHANNEL) {
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int id = tid + kNT * r, t = id >> 5, j = id & 31;
-        const bool okt = t < c;
-        cp_async16(sbase + PP_GS + (uint32_t)(t * kGP + 4 * j) * 4u, log_alpha + row(okt ? t : 0) * kDK + 4 * j,
-                   okt ? 16u : 0u);
+        for (int r = 0; r < 8; ++r) {
+            const int id = tid + kNT * r, t = id >> 5, j = id & 31;
+            const bool okt = t < c;
+            cp_async16(sbase + PP_GS + (uint32_t)(t * kGP + 4 * j) * 4u, log_alpha + row(okt ? t : 0) * kDK + 4 * j,
+                       okt ? 16u : 0u);
+        }
+    } else {
+        // one decay per token and head (Gated DeltaNet) or none (DeltaNet): the
+        // token's value repeated over the key channels, so the rest is unchanged
+        const int t = tid >> 2, c0 = 32 * (tid & 3);
+        const float g = (gate == KDA_GATE_SCALAR && t < c) ? log_alpha[row(t)] : 0.f;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4)
+            *reinterpret_cast<float4 *>(Gs + t * kGP + c0 + j) = make_float4(g, g, g, g);
     }
     if (tid < kC / 4) {
         const bool okt = 4 * tid < c;
@@ -346,8 +360,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
 #pragma unroll 1
             for (int e = 0; e < 16; ++e) {
                 const int chn = ch0 + e;
-                float a = (t < c) ? log_alpha[row(t) * kDK + chn] : 0.f;
-                float a0 = (lane < c) ? log_alpha[row(lane) * kDK + chn] : 0.f;
+                float a = (t < c) ? la_at(t, chn) : 0.f;
+                float a0 = (lane < c) ? la_at(lane, chn) : 0.f;
                 if (gate_act) {
                     a = (t < c) ? log_sigmoid(a) : 0.f;
                     a0 = (lane < c) ? log_sigmoid(a0) : 0.f;
@@ -1234,7 +1248,9 @@ __global__ void selftest_timeout_kernel(long long limit_cycles)
 
 bool prefill_split_supported(const ForwardArgs &a)
 {
-    return a.dtype == KDA_BF16 && a.dk == kDK && a.dv == kDV && a.gate == KDA_GATE_CHANNEL;
+    // any gate: a scalar decay (or none) is staged as the same value in every channel
+    return a.dtype == KDA_BF16 && a.dk == kDK && a.dv == kDV &&
+           (a.gate == KDA_GATE_CHANNEL || a.prep_flags == 0);
 }
 
 size_t prefill_split_workspace_full(int B, int T, int H)
@@ -1278,7 +1294,7 @@ cudaError_t run_prep(const ForwardArgs &a, uint8_t *ws, int n0, int nb, cudaStre
     prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
         static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale,
-        a.prep_flags);
+        a.prep_flags, a.gate);
     const cudaError_t e = cudaGetLastError();
     if (e == cudaSuccess) note_launch();
     return e;

@@ -298,6 +298,21 @@ kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
                            kda_dtype dtype, float scale, void *stream);
 
 /*
+ * kda_gdn_forward_ws -- kda_gdn_forward with a caller-provided device workspace,
+ * as kda_forward_ws is to kda_forward: bf16 with dk = dv = 128 and a workspace of
+ * at least kda_forward_workspace_min_bytes(B, T, H, dk, dv, dtype) bytes (256-byte
+ * aligned) take the two-kernel prefill, with each token's scalar decay (or none)
+ * staged in every key channel; anything else is kda_gdn_forward.  Same arguments,
+ * statuses and results as kda_gdn_forward.
+ */
+kda_status kda_gdn_forward_ws(const void *q, const void *k, const void *v,
+                              const float *log_alpha, const float *beta,
+                              const float *initial_state, float *out, float *final_state,
+                              int B, int T, int H, int dk, int dv,
+                              kda_dtype dtype, float scale, void *workspace, size_t workspace_bytes,
+                              void *stream);
+
+/*
  * kda_gdn_decode_step -- one token per sequence of the scalar-gate variants,
  * state updated in place.
  *

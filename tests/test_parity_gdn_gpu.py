@@ -191,3 +191,42 @@ def test_gdn_binding_rejects_per_channel_gate():
     x = I.make_inputs(I.scaled(I.PREFILL_H16_T4K, H=2, T=10), "cuda")
     with pytest.raises(ValueError):
         kda.gdn_forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"])
+
+
+# ------------------------------------------------------------ two-kernel path with a workspace
+@pytest.mark.parametrize("gate,T,B,H,state", [("scalar", 1, 1, 2, True), ("scalar", 65, 2, 3, True),
+                                              ("scalar", 200, 1, 4, False), ("none", 130, 2, 2, True),
+                                              ("scalar", 333, 2, 20, True), ("none", 64, 1, 40, False)])
+def test_gdn_workspace_path(gate, T, B, H, state):
+    """kda_gdn_forward_ws: the scalar decay (or none) staged in every key channel of
+    the two-kernel prefill; slice and full-head chain kernels both covered."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE if state else I.PREFILL_H16_T4K, B=B, H=H, T=T, seed=9000 + T + H)
+    x = _inputs(w, gate)
+    ws = kda.make_workspace(w.B, w.T, w.H, 128, 128)
+    out, sT = _run(x, workspace=ws)
+    _compare("bf16", x, out, sT)
+
+
+def test_gdn_workspace_path_strong_decay_and_blocks():
+    w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=3, T=300, seed=9100)
+    x = _inputs(w)
+    x["g"][:, 64:128] = -3.0          # range 192 per chunk: the wide-range (pairwise) path
+    ws_full = kda.make_workspace(w.B, w.T, w.H, 128, 128)
+    out_f, s_f = _run(x, workspace=ws_full)
+    _compare("bf16", x, out_f, s_f)
+    bh, rec = w.B * w.H, kda.workspace_bytes(1, 64, 1, 128, 128)
+    ws_b = kda.make_workspace(w.B, w.T, w.H, 128, 128, nbytes=bh * rec * 2 + bh * 128 * 128 * 4)
+    out_b, s_b = _run(x, workspace=ws_b)
+    assert torch.equal(out_f, out_b) and torch.equal(s_f, s_b)
+
+
+def test_gdn_workspace_long_context_sampled_heads():
+    w = I.PREFILL_H32_T64K
+    x = _inputs(w)
+    ws = kda.make_workspace(w.B, w.T, w.H, 128, 128)
+    out, sT = _run(x, workspace=ws)
+    for h in (0, 19):
+        sub = {n: x[n][:, :, h:h + 1].contiguous() for n in ("q", "k", "v", "g", "beta")}
+        o_ref, s_ref = oracle.gdn_forward(sub["q"], sub["k"], sub["v"], sub["g"], sub["beta"], None)
+        assert oracle.parity_error(out[:, :, h:h + 1].cpu().numpy(), o_ref) <= TOL["bf16"]
+        assert oracle.parity_error(sT[:, h:h + 1].cpu().numpy(), s_ref) <= TOL["bf16"]
