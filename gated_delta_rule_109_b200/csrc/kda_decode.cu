@@ -27,15 +27,17 @@ namespace {
 constexpr int kDecodeThreads = 256;
 
 // PER_CHANNEL: log_alpha is [B, H, dk] (KDA); otherwise [B, H] or null (one
-// decay for all channels, or none).
-template <int DK, int DV, typename InT, bool PER_CHANNEL>
-__global__ void __launch_bounds__(kDecodeThreads, 2)
+// decay for all channels, or none).  NS CTAs share a head, each with DV / NS of its
+// value columns (columns of the state never mix, so they need no communication).
+template <int DK, int DV, typename InT, bool PER_CHANNEL, int NS>
+__global__ void __launch_bounds__(kDecodeThreads, NS == 1 ? 2 : 3)
 decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
                    const InT *__restrict__ v, const float *__restrict__ log_alpha,
                    const float *__restrict__ beta, float *__restrict__ state,
                    float *__restrict__ out, float scale)
 {
-    constexpr int CG = DV / 4;                 // float4 column groups per state row
+    constexpr int CGH = DV / 4;                // float4 column groups per state row
+    constexpr int CG = CGH / NS;               // ... handled by this CTA
     constexpr int RS = kDecodeThreads / CG;    // row stride between a thread's rows
     constexpr int RPT = DK / RS;               // state rows held per thread
     static_assert(RPT * RS == DK && CG * RS == kDecodeThreads, "shape");
@@ -44,15 +46,15 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
     __shared__ float4 red_r[RS][CG];
     __shared__ float s_kq;
 
-    const int bh = blockIdx.x;                 // b * H + h
+    const int bh = blockIdx.x / NS;            // b * H + h
     const int tid = threadIdx.x;
-    const int cg = tid % CG;
+    const int cg = (blockIdx.x % NS) * CG + tid % CG;   // column group within the head
     const int r0 = tid / CG;
 
-    float4 *S = reinterpret_cast<float4 *>(state) + (size_t)bh * DK * CG;
+    float4 *S = reinterpret_cast<float4 *>(state) + (size_t)bh * DK * CGH;
     float4 s[RPT];
 #pragma unroll
-    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(&S[(r0 + i * RS) * CG + cg]);
+    for (int i = 0; i < RPT; ++i) s[i] = __ldcs(&S[(r0 + i * RS) * CGH + cg]);
 
     const InT *qh = q + (size_t)bh * DK;
     const InT *kh = k + (size_t)bh * DK;
@@ -82,14 +84,14 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
         pp.x += kc * s[i].x; pp.y += kc * s[i].y; pp.z += kc * s[i].z; pp.w += kc * s[i].w;
         rr.x += qc * s[i].x; rr.y += qc * s[i].y; rr.z += qc * s[i].z; rr.w += qc * s[i].w;
     }
-    red_p[r0][cg] = pp;
-    red_r[r0][cg] = rr;
+    red_p[r0][tid % CG] = pp;
+    red_r[r0][tid % CG] = rr;
     __syncthreads();
 
     float4 p = make_float4(0.f, 0.f, 0.f, 0.f), r = p;
 #pragma unroll
     for (int j = 0; j < RS; ++j) {
-        const float4 a = red_p[j][cg], b = red_r[j][cg];
+        const float4 a = red_p[j][tid % CG], b = red_r[j][tid % CG];
         p.x += a.x; p.y += a.y; p.z += a.z; p.w += a.w;
         r.x += b.x; r.y += b.y; r.z += b.z; r.w += b.w;
     }
@@ -105,7 +107,7 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
     for (int i = 0; i < RPT; ++i) {
         const float kc = kr[i];
         s[i].x += kc * d.x; s[i].y += kc * d.y; s[i].z += kc * d.z; s[i].w += kc * d.w;
-        __stcs(&S[(r0 + i * RS) * CG + cg], s[i]);
+        __stcs(&S[(r0 + i * RS) * CGH + cg], s[i]);
     }
     if (r0 == 0) {
         const float kq = s_kq;
@@ -114,16 +116,23 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
         o.y = scale * (r.y + kq * d.y);
         o.z = scale * (r.z + kq * d.z);
         o.w = scale * (r.w + kq * d.w);
-        reinterpret_cast<float4 *>(out)[(size_t)bh * CG + cg] = o;
+        reinterpret_cast<float4 *>(out)[(size_t)bh * CGH + cg] = o;
     }
 }
+
+#ifndef KDA_DECODE_SPLIT
+#define KDA_DECODE_SPLIT 2
+#endif
 
 template <int DK, int DV, typename InT>
 cudaError_t launch_typed(const DecodeArgs &a, cudaStream_t stream)
 {
-    const unsigned grid = (unsigned)((size_t)a.B * a.H);
-    auto kernel = (a.gate == KDA_GATE_CHANNEL) ? decode_step_kernel<DK, DV, InT, true>
-                                               : decode_step_kernel<DK, DV, InT, false>;
+    // two CTAs per head when a head has 128 value columns (half the registers per
+    // thread, four CTAs per SM), else one
+    constexpr int NS = (DV == 128) ? KDA_DECODE_SPLIT : 1;
+    const unsigned grid = (unsigned)((size_t)a.B * a.H * NS);
+    auto kernel = (a.gate == KDA_GATE_CHANNEL) ? decode_step_kernel<DK, DV, InT, true, NS>
+                                               : decode_step_kernel<DK, DV, InT, false, NS>;
     kernel<<<grid, kDecodeThreads, 0, stream>>>(
         static_cast<const InT *>(a.q), static_cast<const InT *>(a.k),
         static_cast<const InT *>(a.v), a.log_alpha, a.beta, a.state, a.out, a.scale);
