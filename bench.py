@@ -235,7 +235,12 @@ def bench_prefill(w, K, W, device, gate="channel", workspace=None):
     barrier(device)
     per = [evs[i].elapsed_time(evs[i + 1]) for i in range(K)]
     kda.check_status(device)
-    return {"ms_total": sum(per), "ms_per_launch": per, "launches": launches, "x": x}
+    # per-head Frobenius norm of the final state (a health diagnostic of the recurrence)
+    norms = None
+    if sT is not None:
+        n = torch.linalg.vector_norm(sT, dim=(-2, -1)).flatten()
+        norms = {"max": float(n.max()), "mean": float(n.mean()), "min": float(n.min())}
+    return {"ms_total": sum(per), "ms_per_launch": per, "launches": launches, "x": x, "state_norm": norms}
 
 
 def bench_prefill_e2e(w, K, W, device, x, workspace=None):
@@ -743,7 +748,8 @@ def main(argv=None):
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
                     "steps": args.e2e_steps},
             "gpu_launches": pre["launches"],
-            "clocks": clk}
+            "clocks": clk,
+            "final_state_norm_per_head": pre.get("state_norm")}
 
     if not args.no_decode and args.only == "all":
         _add_decode(line, args, rank, world, device, hbm)
