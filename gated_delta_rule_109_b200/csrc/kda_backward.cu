@@ -64,6 +64,41 @@ __device__ __forceinline__ void cp_commit() { asm volatile("cp.async.commit_grou
 template <int N>
 __device__ __forceinline__ void cp_wait() { asm volatile("cp.async.wait_group %0;" :: "n"(N) : "memory"); }
 
+// R consecutive row values of one token as fp32 (one 8- or 16-byte shared load)
+template <int R>
+__device__ __forceinline__ void ld_rows(const float *p, float (&o)[R])
+{
+    if constexpr (R == 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(p);
+        o[0] = x.x; o[1] = x.y; o[2] = x.z; o[3] = x.w;
+    } else {
+        const float2 x = *reinterpret_cast<const float2 *>(p);
+        o[0] = x.x; o[1] = x.y;
+    }
+}
+template <int R>
+__device__ __forceinline__ void ld_rows(const __nv_bfloat16 *p, float (&o)[R])
+{
+    if constexpr (R == 4) {
+        const uint2 x = *reinterpret_cast<const uint2 *>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.x));
+        const float2 b = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x.y));
+        o[0] = a.x; o[1] = a.y; o[2] = b.x; o[3] = b.y;
+    } else {
+        const uint32_t x = *reinterpret_cast<const uint32_t *>(p);
+        const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162 *>(&x));
+        o[0] = a.x; o[1] = a.y;
+    }
+}
+template <int R>
+__device__ __forceinline__ void st_rows(float *p, const float (&x)[R])
+{
+    if constexpr (R == 4)
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    else
+        *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+}
+
 // One chunk's per-token inputs in shared memory (rows past the sequence end are
 // zero-filled): key rows (and query rows) in the input dtype, log_alpha rows,
 // beta, and the block's 8 value (and output-cotangent) columns.
@@ -162,13 +197,14 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
     using St = Stage<Tin, D, false>;
     St *st = reinterpret_cast<St *>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rb = R * lane;                   // this lane's rows: rb .. rb + R - 1
     const int nblk = D / kBW;
     const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
     const int b = bh / d.H, h = bh % d.H;
     const int col = blk * kBW + warp;
     float S[R];
 #pragma unroll
-    for (int i = 0; i < R; ++i) S[i] = s0 ? s0[((size_t)bh * D + lane + 32 * i) * D + col] : 0.f;
+    for (int i = 0; i < R; ++i) S[i] = s0 ? s0[((size_t)bh * D + rb + i) * D + col] : 0.f;
     auto stage = [&](int c) {
         stage_rows<Tin, D, false>(st[c & 1], k, nullptr, la, beta, b, h, c, d);
         stage_cols<Tin, D, false>(st[c & 1], v, nullptr, b, h, c, blk * kBW, d);
@@ -188,16 +224,14 @@ bwd_state_kernel(const Tin *__restrict__ k, const Tin *__restrict__ v, const flo
         __syncthreads();
         const int len = min(kBC, d.T - c * kBC);
         for (int t = 0; t < len; ++t) {
-            if (t % kSub == 0) {
-                float *dst = states + (((size_t)(c * kBC + t) / kSub * (gridDim.x / nblk) + bh) * D + col) * D;
-#pragma unroll
-                for (int i = 0; i < R; ++i) dst[lane + 32 * i] = S[i];
-            }
-            float part = 0.f, kk[R];
+            if (t % kSub == 0)
+                st_rows<R>(states + (((size_t)(c * kBC + t) / kSub * (gridDim.x / nblk) + bh) * D + col) * D + rb, S);
+            float part = 0.f, kk[R], aa[R];
+            ld_rows<R>(&s.k[t][rb], kk);
+            ld_rows<R>(&s.la[t][rb], aa);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                kk[i] = to_f32(s.k[t][lane + 32 * i]);
-                S[i] *= s.la[t][lane + 32 * i];
+                S[i] *= aa[i];
                 part += S[i] * kk[i];
             }
             const float p = warp_sum(part);
@@ -224,13 +258,14 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
     using St = Stage<Tin, D, true>;
     St *st = reinterpret_cast<St *>(smem);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int rb = R * lane;                   // this lane's rows: rb .. rb + R - 1
     const int nblk = D / kBW;
     const int blk = blockIdx.x % nblk, bh = blockIdx.x / nblk;
     const int b = bh / d.H, h = bh % d.H;
     const int col = blk * kBW + warp;
     float dS[R];
 #pragma unroll
-    for (int i = 0; i < R; ++i) dS[i] = d_final ? d_final[((size_t)bh * D + lane + 32 * i) * D + col] : 0.f;
+    for (int i = 0; i < R; ++i) dS[i] = d_final ? d_final[((size_t)bh * D + rb + i) * D + col] : 0.f;
     auto stage = [&](int c) {
         stage_rows<Tin, D, true>(st[c & 1], k, q, la, beta, b, h, c, d);
         stage_cols<Tin, D, true>(st[c & 1], v, dout, b, h, c, blk * kBW, d);
@@ -248,28 +283,28 @@ bwd_adjoint_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, const T
         __syncthreads();
         stage_exp(s);
         __syncthreads();
-        float *dst = dstates + (((size_t)c * (gridDim.x / nblk) + bh) * D + col) * D;
-#pragma unroll
-        for (int i = 0; i < R; ++i) dst[lane + 32 * i] = dS[i];
+        st_rows<R>(dstates + (((size_t)c * (gridDim.x / nblk) + bh) * D + col) * D + rb, dS);
         const int len = min(kBC, d.T - c * kBC);
         for (int t = len - 1; t >= 0; --t) {
             const float go = d.scale * s.dout[t][warp];
-            float part = 0.f, kk[R];
+            float part = 0.f, kk[R], qq[R], aa[R];
+            ld_rows<R>(&s.k[t][rb], kk);
+            ld_rows<R>(&s.q[t][rb], qq);
+            ld_rows<R>(&s.la[t][rb], aa);
 #pragma unroll
             for (int i = 0; i < R; ++i) {
-                kk[i] = to_f32(s.k[t][lane + 32 * i]);
-                dS[i] += to_f32(s.q[t][lane + 32 * i]) * go;
+                dS[i] += qq[i] * go;
                 part += dS[i] * kk[i];
             }
             const float dp = -s.beta[t] * warp_sum(part);
 #pragma unroll
-            for (int i = 0; i < R; ++i) dS[i] = s.la[t][lane + 32 * i] * (dS[i] + kk[i] * dp);
+            for (int i = 0; i < R; ++i) dS[i] = aa[i] * (dS[i] + kk[i] * dp);
         }
         __syncthreads();
     }
     if (d_s0) {
 #pragma unroll
-        for (int i = 0; i < R; ++i) d_s0[((size_t)bh * D + lane + 32 * i) * D + col] = dS[i];
+        for (int i = 0; i < R; ++i) d_s0[((size_t)bh * D + rb + i) * D + col] = dS[i];
     }
 }
 
@@ -294,6 +329,7 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
     GradSmem<Tin, D> &g = *reinterpret_cast<GradSmem<Tin, D> *>(smem);
     Stage<Tin, D, true> &s = g.s;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int rb = R * lane;                   // this lane's rows: rb .. rb + R - 1
     const int c = blockIdx.x % d.nc, bh = blockIdx.x / d.nc;
     const int b = bh / d.H, h = bh % d.H;
     const int t0 = c * kBC, len = min(kBC, d.T - t0);
@@ -316,13 +352,11 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
         // ---- backward sweep, one group of 8 tokens at a time (states recomputed from its checkpoint)
         float dS[R];
 #pragma unroll
-        for (int i = 0; i < R; ++i) dS[i] = dSe[(size_t)col * D + lane + 32 * i];
+        for (int i = 0; i < R; ++i) dS[i] = dSe[(size_t)col * D + rb + i];   // column-major: contiguous
         for (int j = (len - 1) / kSub; j >= 0; --j) {
             float Sb[kSub][R], pb[kSub], eb[kSub];
             float X[R];
-            const float *ck = states + (((size_t)(t0 / kSub + j) * BH + bh) * D + col) * D;
-#pragma unroll
-            for (int i = 0; i < R; ++i) X[i] = ck[lane + 32 * i];
+            ld_rows<R>(states + (((size_t)(t0 / kSub + j) * BH + bh) * D + col) * D + rb, X);
 #pragma unroll
             for (int u = 0; u < kSub; ++u) {
                 const int t = j * kSub + u;
@@ -330,23 +364,25 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
                 for (int i = 0; i < R; ++i) Sb[u][i] = X[i];
                 pb[u] = eb[u] = 0.f;
                 if (t < len) {
-                    float part = 0.f;
+                    float part = 0.f, kk[R], aa[R];
+                    ld_rows<R>(&s.k[t][rb], kk);
+                    ld_rows<R>(&s.la[t][rb], aa);
 #pragma unroll
                     for (int i = 0; i < R; ++i) {
-                        X[i] *= s.la[t][lane + 32 * i];
-                        part += X[i] * to_f32(s.k[t][lane + 32 * i]);
+                        X[i] *= aa[i];
+                        part += X[i] * kk[i];
                     }
                     pb[u] = warp_sum(part);
                     eb[u] = s.beta[t] * (to_f32(s.v[t][warp]) - pb[u]);
 #pragma unroll
-                    for (int i = 0; i < R; ++i) X[i] += to_f32(s.k[t][lane + 32 * i]) * eb[u];
+                    for (int i = 0; i < R; ++i) X[i] += kk[i] * eb[u];
                 }
             }
 #pragma unroll
             for (int u = kSub - 1; u >= 0; --u) {
                 const int t = j * kSub + u;
                 if (t >= len) continue;
-                const int rb = t & 1;                       // partials buffer of this token
+                const int buf = t & 1;                      // partials buffer of this token
                 const size_t row = ((size_t)b * d.T + t0 + t) * d.H + h;
                 // the accumulated sums of the previous column blocks, fetched early
                 float prev[(3 * D + 1 + kBThreads - 1) / kBThreads];
@@ -359,33 +395,34 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
                                               : dbeta[row];
                 }
                 const float bt = s.beta[t], go = d.scale * s.dout[t][warp];
-                float a[R], kk[R], St[R], part = 0.f;
+                float a[R], kk[R], qq[R], St[R], w0[R], w1[R], w2[R], part = 0.f;
+                ld_rows<R>(&s.la[t][rb], a);
+                ld_rows<R>(&s.k[t][rb], kk);
+                ld_rows<R>(&s.q[t][rb], qq);
 #pragma unroll
                 for (int i = 0; i < R; ++i) {
-                    const int r = lane + 32 * i;
-                    a[i] = s.la[t][r];
-                    kk[i] = to_f32(s.k[t][r]);
                     St[i] = a[i] * Sb[u][i];                       // S~
-                    const float Sn = St[i] + kk[i] * eb[u];        // S' (after the write)
-                    dS[i] += to_f32(s.q[t][r]) * go;
-                    g.red[rb][warp][0][r] = Sn * go;               // dq (this column's share)
+                    w0[i] = (St[i] + kk[i] * eb[u]) * go;          // dq share: S' (after the write) dO
+                    dS[i] += qq[i] * go;
                     part += dS[i] * kk[i];
                 }
+                st_rows<R>(&g.red[buf][warp][0][rb], w0);
                 const float de = warp_sum(part);
                 const float dp = -bt * de;
 #pragma unroll
                 for (int i = 0; i < R; ++i) {
-                    const int r = lane + 32 * i;
-                    g.red[rb][warp][1][r] = dS[i] * eb[u] + St[i] * dp;   // dk
-                    const float dSt = dS[i] + kk[i] * dp;                 // dS~
-                    g.red[rb][warp][2][r] = dSt * St[i];                  // dlog_alpha
+                    w1[i] = dS[i] * eb[u] + St[i] * dp;            // dk share
+                    const float dSt = dS[i] + kk[i] * dp;          // dS~
+                    w2[i] = dSt * St[i];                           // dlog_alpha share
                     dS[i] = a[i] * dSt;
                 }
+                st_rows<R>(&g.red[buf][warp][1][rb], w1);
+                st_rows<R>(&g.red[buf][warp][2][rb], w2);
                 if (lane == 0) {
-                    g.redb[rb][warp] = de * (to_f32(s.v[t][warp]) - pb[u]);
+                    g.redb[buf][warp] = de * (to_f32(s.v[t][warp]) - pb[u]);
                     dv[row * D + col] = bt * de;
                 }
-                // one barrier per token: buffer rb is written again two tokens later,
+                // one barrier per token: buffer buf is written again two tokens later,
                 // after the next token's barrier, by which time every thread has read it
                 __syncthreads();
 #pragma unroll
@@ -395,12 +432,12 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
                         const int qn = idx / D, r = idx % D;
                         float sum = prev[m];
 #pragma unroll
-                        for (int w = 0; w < kBW; ++w) sum += g.red[rb][w][qn][r];
+                        for (int w = 0; w < kBW; ++w) sum += g.red[buf][w][qn][r];
                         (qn == 0 ? dq : qn == 1 ? dk : dla)[row * D + r] = sum;
                     } else if (idx == 3 * D) {
                         float sum = prev[m];
 #pragma unroll
-                        for (int w = 0; w < kBW; ++w) sum += g.redb[rb][w];
+                        for (int w = 0; w < kBW; ++w) sum += g.redb[buf][w];
                         dbeta[row] = sum;
                     }
                 }
