@@ -69,16 +69,16 @@ def decode_bytes_per_head(dk, dv, in_bytes):
 # keyed by (kernel source, workload) -> (source digest at capture, bytes).
 # Reported only while the kernel source is unchanged (profiles/ holds the captures).
 MEASURED_TRAFFIC = {
-    ("kda_decode.cu", "decode_bf16_b256_h32_d128_1024steps"): ("a2103952ead4a8e9", 1.0332e9),
+    ("kda_decode.cu", "decode_bf16_b256_h32_d128_1024steps"): ("ea0a7f230dd3ccec", 1.0301e9),
     # captured on B4 H32 T4096 (938.4 MB = 0.979 of its algorithmic bytes) and scaled to
     # the long-context launch by token-heads processed (the kernel streams its inputs once)
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
     ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
     # two-kernel prefill, one kda_forward_ws call (prep + chain), captured on B1 H32 T8192
-    # (prep 339.7 + 577.3 MB, chain 610.3 + 118.8 MB) and scaled by 8 to T = 65536: every
+    # (prep 339.7 + 577.2 MB, chain 610.3 + 120.4 MB) and scaled by 8 to T = 65536: every
     # term (inputs, chunk records, outputs) grows with the token count
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("56dce53a347229e1", 8 * 1646.1e6),
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("56dce53a347229e1", 1646.1e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("8034c0593349183b", 8 * 1647.5e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("8034c0593349183b", 1647.5e6),
 }
 
 
