@@ -257,3 +257,15 @@ def test_backward_validates_before_launch(lib):
     assert wb(1, 65, 2, 128, 128) == (9 + 2) * 2 * 128 * 128 * 4
     assert wb(3, 64, 5, 64, 64) == (8 + 1) * 15 * 64 * 64 * 4
     assert wb(1, 0, 2, 128, 128) == 0 and wb(1, 64, 2, 96, 96) == 0 and wb(1, 64, 2, 64, 128) == 0
+
+
+def test_gdn_forward_ws_validates_like_gdn_forward(lib):
+    def g(ws=FAKE * 16, nbytes=1 << 30, la=FAKE, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, beta=FAKE, s0=None, out=FAKE, sT=None)
+        a.update(kw)
+        return lib.kda_gdn_forward_ws(a["q"], a["k"], a["v"], la, a["beta"], a["s0"], a["out"], a["sT"],
+                                      1, 8, 2, 128, 128, kda.KDA_BF16, ctypes.c_float(0.0), ws, nbytes, None)
+    assert g(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert g(ws=FAKE + 16) == kda.KDA_ERR_MISALIGNED      # workspace must be 256-byte aligned
+    assert g(la=FAKE + 2) == kda.KDA_ERR_MISALIGNED       # the scalar gate needs 4-byte alignment
+    assert g(v=FAKE + 8) == kda.KDA_ERR_MISALIGNED
