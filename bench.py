@@ -243,32 +243,46 @@ def bench_prefill(w, K, W, device, gate="channel", workspace=None):
     return {"ms_total": sum(per), "ms_per_launch": per, "launches": launches, "x": x, "state_norm": norms}
 
 
-def bench_prefill_e2e(w, K, W, device, x, workspace=None):
-    """Same metric through the public API with pinned host inputs, copies inside the timed region."""
+def bench_prefill_e2e(w, K, W, device, x, workspace=None, block_tokens=8192):
+    """Same metric through the public API with pinned host inputs, copies inside the
+    timed region.  With a workspace: kda_forward_host, which overlaps the copies of
+    one block of tokens with the kernels of the next; else device copies around
+    kda_forward."""
     import torch
     import gated_delta_rule_109_b200 as kda
     names = ("q", "k", "v", "log_alpha", "beta")
     host = {n: x[n].cpu().pin_memory() for n in names}
     s0h = x["initial_state"].cpu().pin_memory() if x["initial_state"] is not None else None
-    dev = {n: torch.empty_like(x[n]) for n in names}
-    s0d = torch.empty_like(x["initial_state"]) if s0h is not None else None
-    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
-    sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device) if w.final_state else None
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-    sT_h = torch.empty(sT.shape, dtype=sT.dtype).pin_memory() if sT is not None else None
+    out_h = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32).pin_memory()
+    sT_h = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32).pin_memory() if w.final_state else None
     h2d = sum(t.numel() * t.element_size() for t in host.values()) + (s0h.numel() * 4 if s0h is not None else 0)
-    d2h = out.numel() * 4 + (sT.numel() * 4 if sT is not None else 0)
+    d2h = out_h.numel() * 4 + (sT_h.numel() * 4 if sT_h is not None else 0)
+    host_path = workspace is not None
+    if host_path:
+        # the host path sizes its own workspace (one block of records)
+        hws = torch.empty(kda.forward_host_workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype, block_tokens),
+                          dtype=torch.uint8, device=device)
 
-    def step():
-        for n in names:
-            dev[n].copy_(host[n], non_blocking=True)
-        if s0h is not None:
-            s0d.copy_(s0h, non_blocking=True)
-        kda.forward(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], s0d,
-                    out=out, final_state=sT, return_final_state=sT is not None, workspace=workspace)
-        out_h.copy_(out, non_blocking=True)
-        if sT is not None:
-            sT_h.copy_(sT, non_blocking=True)
+        def step():
+            kda.forward_host(*(host[n] for n in names), s0h, out=out_h, final_state=sT_h,
+                             return_final_state=sT_h is not None, block_tokens=block_tokens, workspace=hws,
+                             device=device, synchronize=False)
+    else:
+        dev = {n: torch.empty_like(x[n]) for n in names}
+        s0d = torch.empty_like(x["initial_state"]) if s0h is not None else None
+        out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+        sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device) if w.final_state else None
+
+        def step():
+            for n in names:
+                dev[n].copy_(host[n], non_blocking=True)
+            if s0h is not None:
+                s0d.copy_(s0h, non_blocking=True)
+            kda.forward(dev["q"], dev["k"], dev["v"], dev["log_alpha"], dev["beta"], s0d,
+                        out=out, final_state=sT, return_final_state=sT is not None)
+            out_h.copy_(out, non_blocking=True)
+            if sT is not None:
+                sT_h.copy_(sT, non_blocking=True)
 
     for _ in range(W):
         step()
@@ -284,7 +298,9 @@ def bench_prefill_e2e(w, K, W, device, x, workspace=None):
     torch.cuda.synchronize(device)
     barrier(device)
     assert torch.isfinite(out_h[0, -1]).all()
-    return {"ms_total": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h}
+    return {"ms_total": e0.elapsed_time(e1), "h2d": h2d, "d2h": d2h,
+            "path": "kda_forward_host (copies and kernels overlapped per %d-token block)" % block_tokens
+            if host_path else "device copies around kda_forward"}
 
 
 # ---------------------------------------------------------------- decode
@@ -746,7 +762,7 @@ def main(argv=None):
             "roofline": roofline,
             "e2e": {"value": tokens_per_step * args.e2e_steps * world / (e2e_ms / 1e3), "unit": "tokens/s",
                     "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"],
-                    "steps": args.e2e_steps},
+                    "steps": args.e2e_steps, "path": e2e["path"]},
             "gpu_launches": pre["launches"],
             "clocks": clk,
             "final_state_norm_per_head": pre.get("state_norm")}

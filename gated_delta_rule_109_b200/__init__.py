@@ -30,7 +30,8 @@ KDA_PREP_LOGSIGMOID_GATE, KDA_PREP_L2NORM_QK = 1, 2
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
            "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_segment_local",
            "kda_segment_start_state", "kda_segment_correct", "kda_forward_noalloc",
-           "kda_forward_noalloc_scratch_bytes", "kda_backward", "kda_backward_workspace_bytes",
+           "kda_forward_noalloc_scratch_bytes", "kda_forward_host", "kda_forward_host_workspace_bytes",
+           "kda_backward", "kda_backward_workspace_bytes",
            "kda_decode_step", "kda_gdn_forward", "kda_gdn_forward_ws", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
            "kda_launch_count",
@@ -80,6 +81,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_forward_noalloc.restype = i
     lib.kda_forward_noalloc.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_forward_noalloc_scratch_bytes.restype = ctypes.c_size_t
+    lib.kda_forward_host.restype = i
+    lib.kda_forward_host.argtypes = [vp] * 8 + [i] * 6 + [f, i, vp, ctypes.c_size_t, vp]
+    lib.kda_forward_host_workspace_bytes.restype = ctypes.c_size_t
+    lib.kda_forward_host_workspace_bytes.argtypes = [i] * 7
     lib.kda_backward.restype = i
     lib.kda_backward.argtypes = [vp] * 14 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
     lib.kda_backward_workspace_bytes.restype = ctypes.c_size_t
@@ -312,6 +317,53 @@ def segment_correct(start, local_final, out, *, workspace, final_state=None):
                                     _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(dev))
     _check(st, "kda_segment_correct")
     return final_state
+
+
+def forward_host_workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, block_tokens: int = 0) -> int:
+    """Bytes of the device workspace ``kda_forward_host`` needs."""
+    code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
+    return int(load().kda_forward_host_workspace_bytes(B, T, H, dk, dv, code, int(block_tokens)))
+
+
+def forward_host(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
+                 return_final_state=True, block_tokens: int = 0, workspace=None, device=None,
+                 scale: float = 0.0, synchronize: bool = True):
+    """Prefill with host tensors in and out (``kda_forward_host``): copies and
+    kernels overlap block by block.  ``q, k, v, log_alpha, beta`` (and
+    ``initial_state``) are CPU tensors in the usual layouts (pinned memory for
+    asynchronous copies); ``out`` / ``final_state`` (CPU, fp32) are allocated
+    pinned when None.  ``workspace``: a uint8 tensor on ``device`` of at least
+    :func:`forward_host_workspace_bytes` bytes (allocated when None).  With
+    ``synchronize`` the call waits for the device stream before returning."""
+    lib = load()
+    dev = torch.device("cuda") if device is None else torch.device(device)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    cpu = torch.device("cpu")
+    for t, n, shp, dt in ((q, "q", (B, T, H, dk), q.dtype), (k, "k", (B, T, H, dk), q.dtype),
+                          (v, "v", (B, T, H, dv), q.dtype), (log_alpha, "log_alpha", (B, T, H, dk), torch.float32),
+                          (beta, "beta", (B, T, H), torch.float32)):
+        _need(t, n, shp, dt, cpu)
+    if initial_state is not None:
+        _need(initial_state, "initial_state", (B, H, dk, dv), torch.float32, cpu)
+    if out is None:
+        out = torch.empty((B, T, H, dv), dtype=torch.float32, pin_memory=True)
+    _need(out, "out", (B, T, H, dv), torch.float32, cpu)
+    if final_state is None and return_final_state:
+        final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
+    if final_state is not None:
+        _need(final_state, "final_state", (B, H, dk, dv), torch.float32, cpu)
+    nbytes = forward_host_workspace_bytes(B, T, H, dk, dv, q.dtype, block_tokens)
+    if workspace is None:
+        workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    st = lib.kda_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
+                              _ptr(out), _ptr(final_state), B, T, H, dk, dv, _dtype_code(q), float(scale),
+                              int(block_tokens), _ptr(workspace), workspace.numel() * workspace.element_size(),
+                              _stream(dev))
+    _check(st, "kda_forward_host")
+    if synchronize:
+        torch.cuda.current_stream(dev).synchronize()
+    return out, final_state
 
 
 def backward_workspace_bytes(B: int, T: int, H: int, dk: int, dv: int) -> int:

@@ -1,5 +1,6 @@
 // libkda C ABI: argument validation, dispatch to the kernels, status codes.
 // The contract of every entry point is documented in include/kda.h.
+#include <algorithm>
 #include <atomic>
 #include <math.h>
 #include <mutex>
@@ -161,6 +162,44 @@ kda_status decode_impl(const void *q, const void *k, const void *v, const float 
     a.gate = gate;
     cudaError_t e = kda::launch_decode(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
+// kda_forward_host: per-device copy streams and the events that order the slots
+struct HostPipe {
+    bool ready = false;
+    cudaStream_t h2d = nullptr, d2h = nullptr;
+    cudaEvent_t in_ready[2], comp_done[2], out_done[2], start, fin;
+};
+HostPipe g_pipe[kMaxDevices];
+std::mutex g_pipe_mu;
+
+size_t up256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Workspace of kda_forward_host: two input slots and two output slots of one block
+// of tokens each, the carried state, and the two-kernel records of one block.
+struct HostLayout {
+    int Tb;
+    size_t q, k, v, la, beta, slot_in, slot_out, state, recs, recs_bytes, total;
+};
+HostLayout host_layout(int B, int T, int H, int dk, int dv, kda_dtype dtype, int block_tokens)
+{
+    HostLayout L;
+    const int want = block_tokens > 0 ? ((block_tokens + 63) / 64) * 64 : 8192;
+    L.Tb = (int)std::min<long long>(want, ((long long)T + 63) / 64 * 64);
+    if (L.Tb <= 0) L.Tb = 64;
+    const size_t esz = dtype == KDA_BF16 ? 2 : 4, rows = (size_t)B * L.Tb * H;
+    L.q = 0;
+    L.k = L.q + up256(rows * dk * esz);
+    L.v = L.k + up256(rows * dk * esz);
+    L.la = L.v + up256(rows * dv * esz);
+    L.beta = L.la + up256(rows * dk * 4);
+    L.slot_in = L.beta + up256(rows * 4);
+    L.slot_out = up256(rows * dv * 4);
+    L.state = 2 * L.slot_in + 2 * L.slot_out;
+    L.recs = L.state + up256((size_t)B * H * dk * dv * 4);
+    L.recs_bytes = (dtype == KDA_BF16 && dk == 128 && dv == 128) ? kda::prefill_split_workspace_full(B, L.Tb, H) : 0;
+    L.total = L.recs + L.recs_bytes;
+    return L;
 }
 
 }  // namespace
@@ -357,6 +396,116 @@ kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
 {
     return decode_impl(q, k, v, log_alpha, beta, state_inout, out, B, H, dk, dv, dtype, scale, stream,
                        log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
+}
+
+size_t kda_forward_host_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype, int block_tokens)
+{
+    if (B <= 0 || H <= 0 || T < 0 || !head_dim_ok(dk) || !head_dim_ok(dv) || block_tokens < 0 ||
+        (dtype != KDA_BF16 && dtype != KDA_F32))
+        return 0;
+    return host_layout(B, T, H, dk, dv, dtype, block_tokens).total;
+}
+
+kda_status kda_forward_host(const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta,
+                            const float *initial_state, float *out, float *final_state,
+                            int B, int T, int H, int dk, int dv,
+                            kda_dtype dtype, float scale, int block_tokens,
+                            void *workspace, size_t workspace_bytes, void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    if (B <= 0 || H <= 0 || T < 0 || dk <= 0 || dv <= 0 || block_tokens < 0) return KDA_ERR_INVALID_ARG;
+    if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
+    if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
+    if (!head_dim_ok(dk) || !head_dim_ok(dv)) return KDA_ERR_UNSUPPORTED;
+    if ((int64_t)B * T * H > (int64_t)INT32_MAX / 4) return KDA_ERR_INVALID_ARG;
+    const size_t esz = dtype == KDA_BF16 ? 2 : 4;
+    const size_t state_bytes = sizeof(float) * (size_t)B * H * dk * dv;
+    if (T == 0) {
+        // no tokens: the final state is the initial state (or zeros), copied on the host
+        if (final_state && final_state != initial_state) {
+            if (initial_state) memcpy(final_state, initial_state, state_bytes);
+            else memset(final_state, 0, state_bytes);
+        }
+        return KDA_OK;
+    }
+    if (!q || !k || !v || !log_alpha || !beta || !out || !workspace) return KDA_ERR_INVALID_ARG;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return KDA_ERR_MISALIGNED;
+    const HostLayout L = host_layout(B, T, H, dk, dv, dtype, block_tokens);
+    if (workspace_bytes < L.total) return KDA_ERR_INVALID_ARG;
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (dev < 0 || dev >= kMaxDevices) return KDA_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_pipe_mu);
+    HostPipe &P = g_pipe[dev];
+    if (!P.ready) {
+        if ((e = cudaStreamCreateWithFlags(&P.h2d, cudaStreamNonBlocking)) != cudaSuccess ||
+            (e = cudaStreamCreateWithFlags(&P.d2h, cudaStreamNonBlocking)) != cudaSuccess)
+            return cuda_fail(e);
+        for (cudaEvent_t *ev : {&P.in_ready[0], &P.in_ready[1], &P.comp_done[0], &P.comp_done[1],
+                                &P.out_done[0], &P.out_done[1], &P.start, &P.fin})
+            if ((e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return cuda_fail(e);
+        P.ready = true;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    float *carry = reinterpret_cast<float *>(ws + L.state);
+    // the copies wait for the work already on the caller's stream (earlier users of the workspace)
+    if ((e = cudaEventRecord(P.start, st)) != cudaSuccess || (e = cudaStreamWaitEvent(P.h2d, P.start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(P.d2h, P.start, 0)) != cudaSuccess)
+        return cuda_fail(e);
+    if (initial_state &&
+        (e = cudaMemcpyAsync(carry, initial_state, state_bytes, cudaMemcpyHostToDevice, P.h2d)) != cudaSuccess)
+        return cuda_fail(e);
+    const int nblk = (T + L.Tb - 1) / L.Tb;
+    const size_t HK = (size_t)H * dk, HV = (size_t)H * dv;
+    for (int i = 0; i < nblk; ++i) {
+        const int t0 = i * L.Tb, Ti = min(L.Tb, T - t0), sl = i & 1;
+        uint8_t *in = ws + sl * L.slot_in;
+        uint8_t *dq = in + L.q, *dk_ = in + L.k, *dvv = in + L.v;
+        float *dla = reinterpret_cast<float *>(in + L.la), *dbt = reinterpret_cast<float *>(in + L.beta);
+        float *dout = reinterpret_cast<float *>(ws + 2 * L.slot_in + sl * L.slot_out);
+        // block i's inputs: the slot was last read by block i - 2's kernels
+        if (i >= 2 && (e = cudaStreamWaitEvent(P.h2d, P.comp_done[sl], 0)) != cudaSuccess) return cuda_fail(e);
+        for (int b = 0; b < B; ++b) {
+            const size_t src_row = (size_t)b * T + t0, dst_row = (size_t)b * Ti;
+            struct { void *dst; const void *src; size_t bytes; } cps[5] = {
+                {dq + dst_row * HK * esz, static_cast<const uint8_t *>(q) + src_row * HK * esz, Ti * HK * esz},
+                {dk_ + dst_row * HK * esz, static_cast<const uint8_t *>(k) + src_row * HK * esz, Ti * HK * esz},
+                {dvv + dst_row * HV * esz, static_cast<const uint8_t *>(v) + src_row * HV * esz, Ti * HV * esz},
+                {dla + dst_row * HK, log_alpha + src_row * HK, Ti * HK * sizeof(float)},
+                {dbt + dst_row * H, beta + src_row * H, (size_t)Ti * H * sizeof(float)}};
+            for (const auto &c : cps)
+                if ((e = cudaMemcpyAsync(c.dst, c.src, c.bytes, cudaMemcpyHostToDevice, P.h2d)) != cudaSuccess)
+                    return cuda_fail(e);
+        }
+        if ((e = cudaEventRecord(P.in_ready[sl], P.h2d)) != cudaSuccess) return cuda_fail(e);
+        // block i on the caller's stream; its output slot was last copied out for block i - 2
+        if ((e = cudaStreamWaitEvent(st, P.in_ready[sl], 0)) != cudaSuccess) return cuda_fail(e);
+        if (i >= 2 && (e = cudaStreamWaitEvent(st, P.out_done[sl], 0)) != cudaSuccess) return cuda_fail(e);
+        const kda_status fs = forward_impl(dq, dk_, dvv, dla, dbt, (i == 0 && !initial_state) ? nullptr : carry,
+                                           dout, carry, B, Ti, H, dk, dv, dtype, scale, stream,
+                                           kda::KDA_GATE_CHANNEL, L.recs_bytes ? ws + L.recs : nullptr,
+                                           L.recs_bytes);
+        if (fs != KDA_OK) return fs;
+        if ((e = cudaEventRecord(P.comp_done[sl], st)) != cudaSuccess) return cuda_fail(e);
+        // block i's outputs back to the host
+        if ((e = cudaStreamWaitEvent(P.d2h, P.comp_done[sl], 0)) != cudaSuccess) return cuda_fail(e);
+        for (int b = 0; b < B; ++b)
+            if ((e = cudaMemcpyAsync(out + ((size_t)b * T + t0) * HV, dout + (size_t)b * Ti * HV,
+                                     Ti * HV * sizeof(float), cudaMemcpyDeviceToHost, P.d2h)) != cudaSuccess)
+                return cuda_fail(e);
+        if ((e = cudaEventRecord(P.out_done[sl], P.d2h)) != cudaSuccess) return cuda_fail(e);
+    }
+    if (final_state &&
+        (e = cudaMemcpyAsync(final_state, carry, state_bytes, cudaMemcpyDeviceToHost, P.d2h)) != cudaSuccess)
+        return cuda_fail(e);
+    // the caller's stream completes after the last copy
+    if ((e = cudaEventRecord(P.fin, P.d2h)) != cudaSuccess || (e = cudaStreamWaitEvent(st, P.fin, 0)) != cudaSuccess)
+        return cuda_fail(e);
+    return KDA_OK;
 }
 
 size_t kda_backward_workspace_bytes(int B, int T, int H, int dk, int dv)

@@ -328,6 +328,39 @@ kda_status kda_gdn_decode_step(const void *q, const void *k, const void *v,
                                kda_dtype dtype, float scale, void *stream);
 
 /*
+ * kda_forward_host -- kda_forward with every tensor argument in HOST memory.
+ *
+ * For a prefill whose activations live on the host (no counterpart on the
+ * pages): the sequence is cut into blocks of block_tokens tokens (a multiple of
+ * 64; 0 = 8192) that carry the state, and the library overlaps the host-to-device
+ * copy of block i + 1, the kernels of block i and the device-to-host copy of
+ * block i - 1, with two internal copy streams.  The chunk boundaries are those of
+ * the whole sequence, so the results equal kda_forward_ws's bit for bit.
+ *
+ *   q, k, v, log_alpha, beta, initial_state (NULL = zero), out, final_state (NULL
+ *                 = not wanted): host buffers in kda_forward's layouts (page-locked
+ *                 memory lets the copies run asynchronously)
+ *   workspace     device buffer of kda_forward_host_workspace_bytes(...) bytes
+ *                 (256-byte aligned, caller-owned): two input slots and two output
+ *                 slots of one block, the carried state, one block's chunk records
+ *
+ * The kernels run on `stream`, which also waits for the last copy: synchronise it
+ * before reading out / final_state or reusing the host inputs.  Supported shapes,
+ * statuses and dispatch as for kda_forward_ws (per-channel gate).  T = 0 copies
+ * (or zeroes) the final state on the host and returns.
+ */
+kda_status kda_forward_host(const void *q, const void *k, const void *v,
+                            const float *log_alpha, const float *beta,
+                            const float *initial_state, float *out, float *final_state,
+                            int B, int T, int H, int dk, int dv,
+                            kda_dtype dtype, float scale, int block_tokens,
+                            void *workspace, size_t workspace_bytes, void *stream);
+
+/* Workspace bytes kda_forward_host needs for these sizes and block length (0 for
+ * invalid arguments). */
+size_t kda_forward_host_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype, int block_tokens);
+
+/*
  * kda_backward -- gradients of kda_forward with respect to every input.
  *
  * The pages give the forward's token step ("Kimi Delta Attention: The Linear

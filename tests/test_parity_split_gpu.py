@@ -231,3 +231,34 @@ def test_split_rejects_misaligned_workspace():
     with pytest.raises(kda.KDAError) as err:
         kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], workspace=ws[16:])
     assert err.value.status == kda.KDA_ERR_MISALIGNED
+
+
+# ------------------------------------------------------------ host buffers (kda_forward_host)
+@pytest.mark.parametrize("T,B,H,block,state", [(1000, 2, 3, 256, True), (300, 1, 2, 64, False),
+                                               (65, 2, 20, 0, True), (4096, 1, 4, 1024, True)])
+def test_forward_host_equals_device_path(T, B, H, block, state):
+    """Copies and kernels overlapped per block; chunk boundaries are the whole
+    sequence's, so the result is the workspace path's, bit for bit."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE if state else I.PREFILL_H16_T4K, B=B, H=H, T=T, seed=9600 + T)
+    x = I.make_inputs(w, "cuda")
+    out_d, s_d = _run(x, _ws(w))
+    host = {n: x[n].cpu().pin_memory() for n in NAMES}
+    s0 = x["initial_state"].cpu().pin_memory() if x["initial_state"] is not None else None
+    out_h, s_h = kda.forward_host(*(host[n] for n in NAMES), s0, block_tokens=block)
+    kda.check_status()
+    assert torch.equal(out_h, out_d.cpu()) and torch.equal(s_h, s_d.cpu())
+
+
+def test_forward_host_pageable_and_f32_and_empty():
+    w = I.scaled(I.TINY_F32, T=200, seed=9700)              # fp32 inputs: the SIMT path per block
+    x = I.make_inputs(w, "cuda")
+    out_d, s_d = _run(x, None)
+    host = {n: x[n].cpu() for n in NAMES}                   # pageable host memory
+    out_h, s_h = kda.forward_host(*(host[n] for n in NAMES), None, block_tokens=128)
+    kda.check_status()
+    o_ref, s_ref = oracle.forward(*(host[n] for n in NAMES), None)
+    assert oracle.parity_error(out_h.numpy(), o_ref) <= 1e-5 and oracle.parity_error(s_h.numpy(), s_ref) <= 1e-5
+    w0 = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=2, T=0, seed=9701)
+    x0 = I.make_inputs(w0, "cpu")
+    out0, s0 = kda.forward_host(*(x0[n] for n in NAMES), x0["initial_state"])
+    assert out0.numel() == 0 and torch.equal(s0, x0["initial_state"])
