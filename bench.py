@@ -243,7 +243,7 @@ def bench_prefill(w, K, W, device, gate="channel", workspace=None):
     return {"ms_total": sum(per), "ms_per_launch": per, "launches": launches, "x": x, "state_norm": norms}
 
 
-def bench_prefill_e2e(w, K, W, device, x, workspace=None, block_tokens=8192):
+def bench_prefill_e2e(w, K, W, device, x, workspace=None, block_tokens=4096):
     """Same metric through the public API with pinned host inputs, copies inside the
     timed region.  With a workspace: kda_forward_host, which overlaps the copies of
     one block of tokens with the kernels of the next; else device copies around

@@ -269,3 +269,27 @@ def test_gdn_forward_ws_validates_like_gdn_forward(lib):
     assert g(ws=FAKE + 16) == kda.KDA_ERR_MISALIGNED      # workspace must be 256-byte aligned
     assert g(la=FAKE + 2) == kda.KDA_ERR_MISALIGNED       # the scalar gate needs 4-byte alignment
     assert g(v=FAKE + 8) == kda.KDA_ERR_MISALIGNED
+
+
+def test_forward_host_validates_before_any_copy(lib):
+    WS = FAKE * 16
+
+    def fh(T=8, ws=WS, nbytes=1 << 40, block=0, dk=128, dtype=kda.KDA_BF16, **kw):
+        a = dict(q=FAKE, k=FAKE, v=FAKE, la=FAKE, beta=FAKE, s0=None, out=FAKE, sT=None)
+        a.update(kw)
+        return lib.kda_forward_host(a["q"], a["k"], a["v"], a["la"], a["beta"], a["s0"], a["out"], a["sT"],
+                                    1, T, 2, dk, 128, dtype, ctypes.c_float(0.0), block, ws, nbytes, None)
+    assert fh(q=None) == kda.KDA_ERR_INVALID_ARG
+    assert fh(out=None) == kda.KDA_ERR_INVALID_ARG
+    assert fh(ws=None) == kda.KDA_ERR_INVALID_ARG
+    assert fh(block=-1) == kda.KDA_ERR_INVALID_ARG
+    assert fh(T=-1) == kda.KDA_ERR_INVALID_ARG
+    assert fh(dtype=9) == kda.KDA_ERR_INVALID_ARG
+    assert fh(dk=96) == kda.KDA_ERR_UNSUPPORTED
+    assert fh(ws=WS + 16) == kda.KDA_ERR_MISALIGNED
+    need = lib.kda_forward_host_workspace_bytes(1, 8, 2, 128, 128, kda.KDA_BF16, 0)
+    assert need > 0 and fh(nbytes=need - 1) == kda.KDA_ERR_INVALID_ARG
+    # the workspace grows with the block length, not with T beyond one block
+    wb = lambda T, blk: lib.kda_forward_host_workspace_bytes(1, T, 32, 128, 128, kda.KDA_BF16, blk)
+    assert wb(65536, 4096) == wb(8192, 4096) < wb(65536, 8192)
+    assert wb(64, 0) == wb(64, 8192) and lib.kda_forward_host_workspace_bytes(1, 8, 2, 96, 96, kda.KDA_BF16, 0) == 0
