@@ -662,7 +662,7 @@ def main(argv=None):
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-tokens-per-step", type=int, default=1024)
     ap.add_argument("--no-decode", action="store_true")
-    ap.add_argument("--only", choices=["all", "prefill", "decode"], default="all",
+    ap.add_argument("--only", choices=["all", "prefill", "decode", "backward"], default="all",
                     help="time only one kernel (profiling runs); the default times both")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-workspace", action="store_true",
@@ -694,9 +694,12 @@ def main(argv=None):
     hbm, tf_burst, tf_sust, peak_src = load_peaks()
     in_bytes = 2 if w.dtype == "bf16" else 4
 
-    if args.only == "decode":
-        line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "impl": "kda", "only": "decode"}
-        _add_decode(line, args, rank, world, device, hbm)
+    if args.only in ("decode", "backward"):
+        line = {"metric": METRIC, "unit": "tokens/s", "n_gpus": world, "impl": "kda", "only": args.only}
+        if args.only == "decode":
+            _add_decode(line, args, rank, world, device, hbm)
+        else:
+            _add_backward(line, args, device, hbm, world)
         if rank == 0:
             print(json.dumps(line), flush=True)
         return 0
