@@ -293,3 +293,23 @@ def test_forward_host_validates_before_any_copy(lib):
     wb = lambda T, blk: lib.kda_forward_host_workspace_bytes(1, T, 32, 128, 128, kda.KDA_BF16, blk)
     assert wb(65536, 4096) == wb(8192, 4096) < wb(65536, 8192)
     assert wb(64, 0) == wb(64, 8192) and lib.kda_forward_host_workspace_bytes(1, 8, 2, 96, 96, kda.KDA_BF16, 0) == 0
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/kda.h compiles as pedantic C99, and a C program links libkda.so and
+    calls host-only entry points (no GPU needed)."""
+    src = tmp_path / "use_kda.c"
+    src.write_text('#include <stdio.h>\n#include <string.h>\n#include "kda.h"\n'
+                   'int main(void) {\n'
+                   '  if (kda_version() < 300) return 1;\n'
+                   '  if (strcmp(kda_status_string(KDA_ERR_TIMEOUT), "KDA_ERR_TIMEOUT") != 0) return 2;\n'
+                   '  if (kda_forward_workspace_bytes(1, 64, 1, 128, 128, KDA_BF16) == 0) return 3;\n'
+                   '  if (kda_forward(NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, 8, 1, 128, 128,\n'
+                   '                  KDA_BF16, 0.0f, NULL) != KDA_ERR_INVALID_ARG) return 4;\n'
+                   '  puts("ok");\n  return 0;\n}\n')
+    exe = tmp_path / "use_kda"
+    libdir = os.path.dirname(kbuild.LIB)
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-o", str(exe), "-L", libdir, "-lkda", "-Wl,-rpath," + libdir], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
