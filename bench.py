@@ -75,10 +75,10 @@ MEASURED_TRAFFIC = {
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
     ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
     # two-kernel prefill, one kda_forward_ws call (prep + chain), captured on B1 H32 T8192
-    # (prep 339.7 + 577.2 MB, chain 610.3 + 120.4 MB) and scaled by 8 to T = 65536: every
+    # (prep 342.6 + 576.9 MB, chain 610.4 + 117.2 MB) and scaled by 8 to T = 65536: every
     # term (inputs, chunk records, outputs) grows with the token count
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("8034c0593349183b", 8 * 1647.5e6),
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("8034c0593349183b", 1647.5e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("8af6b29bc6e2697e", 8 * 1647.1e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("8af6b29bc6e2697e", 1647.1e6),
 }
 
 
