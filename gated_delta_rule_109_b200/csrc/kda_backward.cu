@@ -50,6 +50,13 @@ __device__ __forceinline__ float warp_sum(float x)
     return x;
 }
 
+// L2 prefetch of a global range (16-byte aligned, a multiple of 16 bytes); a hint
+// that nothing waits for
+__device__ __forceinline__ void l2_prefetch(const void *src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(src), "r"(bytes) : "memory");
+}
+
 __device__ __forceinline__ void cp_async(void *dst, const void *src, int bytes, bool valid)
 {
     const uint32_t d = (uint32_t)__cvta_generic_to_shared(dst);
@@ -338,6 +345,19 @@ bwd_chunk_grad_kernel(const Tin *__restrict__ q, const Tin *__restrict__ k, cons
 
     for (int blk = 0; blk < D / kBW; ++blk) {
         const int col = blk * kBW + warp;
+        // warm L2 with the next column block's end adjoint and group checkpoints (the
+        // first block also with its own, while the chunk is staged): they come from
+        // DRAM, and this CTA is alone on its SM, so nothing else hides their latency
+        if (warp == 0) {
+            const int ng = (len - 1) / kSub + 1;
+            for (int pbk = (blk == 0 ? 0 : blk + 1); pbk <= blk + 1 && pbk < D / kBW; ++pbk) {
+                const size_t c0 = (size_t)pbk * kBW * D;
+                if (lane < ng)
+                    l2_prefetch(states + ((size_t)(t0 / kSub + lane) * BH + bh) * D * D + c0, kBW * D * 4);
+                else if (lane == 31)
+                    l2_prefetch(dSe + c0, kBW * D * 4);
+            }
+        }
         // the chunk's rows are staged once, the block's value and cotangent columns every block
         if (blk == 0) stage_rows<Tin, D, true>(s, k, q, la, beta, b, h, c, d);
         stage_cols<Tin, D, true>(s, v, dout, b, h, c, blk * kBW, d);
