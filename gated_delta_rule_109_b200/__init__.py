@@ -148,12 +148,31 @@ def _need(t: torch.Tensor, name: str, shape, dtype=None, device=None):
         raise ValueError("%s is on %s, expected %s" % (name, t.device, device))
 
 
+def _on_cuda(dev: torch.device, where: str):
+    """The kernels take device memory only: a host tensor is refused here, before
+    its address could reach a kernel."""
+    if dev.type != "cuda":
+        raise ValueError("%s takes CUDA tensors, got tensors on %s" % (where, dev))
+
+
+def _need_workspace(workspace, dev: torch.device, where: str):
+    """A caller's workspace: a contiguous CUDA tensor on the device the call runs on."""
+    if not isinstance(workspace, torch.Tensor):
+        raise TypeError("%s: workspace must be a torch.Tensor" % where)
+    if workspace.device.type != "cuda" or not workspace.is_contiguous():
+        raise ValueError("%s: workspace must be a contiguous CUDA tensor, got one on %s" % (where, workspace.device))
+    want = dev.index if dev.index is not None else torch.cuda.current_device()
+    if workspace.device.index != want:
+        raise ValueError("%s: workspace is on %s, the call runs on cuda:%d" % (where, workspace.device, want))
+
+
 def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, final_state,
              return_final_state, scale, workspace=None):
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
+    _on_cuda(dev, entry)
     code = _dtype_code(q)
     _need(q, "q", (B, T, H, dk), q.dtype, dev)
     _need(k, "k", (B, T, H, dk), q.dtype, dev)
@@ -171,8 +190,7 @@ def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, fi
     if final_state is not None:
         _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
     if workspace is not None:
-        if workspace.device != dev or not workspace.is_contiguous():
-            raise ValueError("workspace must be a contiguous tensor on %s" % dev)
+        _need_workspace(workspace, dev, entry)
         entry = entry + "_ws"
         st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                                  _ptr(initial_state), _ptr(out), _ptr(final_state),
@@ -192,6 +210,7 @@ def _decode(entry, gate_shape, q, k, v, log_alpha, beta, state, out, scale):
     B, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
+    _on_cuda(dev, entry)
     code = _dtype_code(q)
     _need(q, "q", (B, H, dk), q.dtype, dev)
     _need(k, "k", (B, H, dk), q.dtype, dev)
@@ -237,6 +256,7 @@ def forward_raw(q, k, v, gate, beta, initial_state=None, *, workspace, logsigmoi
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
+    _on_cuda(dev, "kda_forward_raw")
     code = _dtype_code(q)
     _need(q, "q", (B, T, H, dk), q.dtype, dev)
     _need(k, "k", (B, T, H, dk), q.dtype, dev)
@@ -252,8 +272,9 @@ def forward_raw(q, k, v, gate, beta, initial_state=None, *, workspace, logsigmoi
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     if final_state is not None:
         _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
-    if workspace is None or workspace.device != dev or not workspace.is_contiguous():
-        raise ValueError("workspace must be a contiguous tensor on %s" % dev)
+    if workspace is None:
+        raise ValueError("kda_forward_raw needs a workspace")
+    _need_workspace(workspace, dev, "kda_forward_raw")
     prep = (KDA_PREP_LOGSIGMOID_GATE if logsigmoid_gate else 0) | (KDA_PREP_L2NORM_QK if normalize_qk else 0)
     st = lib.kda_forward_raw(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(beta), _ptr(initial_state), _ptr(out),
                              _ptr(final_state), B, T, H, dk, dv, code, float(scale), prep, _ptr(workspace),
@@ -269,6 +290,8 @@ def segment_local(q, k, v, log_alpha, beta, initial_state=None, *, workspace, sc
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
+    _on_cuda(dev, "kda_segment_local")
+    _need_workspace(workspace, dev, "kda_segment_local")
     code = _dtype_code(q)
     for t, n, shp in ((q, "q", (B, T, H, dk)), (k, "k", (B, T, H, dk)), (v, "v", (B, T, H, dv))):
         _need(t, n, shp, q.dtype, dev)
@@ -293,6 +316,7 @@ def segment_start_state(transfers, local_finals):
     R, B, H, dk, _ = transfers.shape
     dv = local_finals.shape[-1]
     dev = transfers.device
+    _on_cuda(dev, "kda_segment_start_state")
     _need(transfers, "transfers", (R, B, H, dk, dk), torch.float32, dev)
     _need(local_finals, "local_finals", (R, B, H, dk, dv), torch.float32, dev)
     start = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
@@ -308,6 +332,8 @@ def segment_correct(start, local_final, out, *, workspace, final_state=None):
     B, T, H, dv = out.shape
     dk = start.shape[-2]
     dev = out.device
+    _on_cuda(dev, "kda_segment_correct")
+    _need_workspace(workspace, dev, "kda_segment_correct")
     _need(start, "start", (B, H, dk, dv), torch.float32, dev)
     _need(local_final, "local_final", (B, H, dk, dv), torch.float32, dev)
     _need(out, "out", (B, T, H, dv), torch.float32, dev)
@@ -353,9 +379,11 @@ def forward_host(q, k, v, log_alpha, beta, initial_state=None, *, out=None, fina
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, pin_memory=True)
     if final_state is not None:
         _need(final_state, "final_state", (B, H, dk, dv), torch.float32, cpu)
+    _on_cuda(dev, "kda_forward_host")
     nbytes = forward_host_workspace_bytes(B, T, H, dk, dv, q.dtype, block_tokens)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    _need_workspace(workspace, dev, "kda_forward_host")
     st = lib.kda_forward_host(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta), _ptr(initial_state),
                               _ptr(out), _ptr(final_state), B, T, H, dk, dv, _dtype_code(q), float(scale),
                               int(block_tokens), _ptr(workspace), workspace.numel() * workspace.element_size(),
@@ -385,6 +413,7 @@ def backward(q, k, v, log_alpha, beta, grad_out, initial_state=None, grad_final_
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     dev = q.device
+    _on_cuda(dev, "kda_backward")
     for t, n, shp in ((q, "q", (B, T, H, dk)), (k, "k", (B, T, H, dk)), (v, "v", (B, T, H, dv))):
         _need(t, n, shp, q.dtype, dev)
     _need(log_alpha, "log_alpha", (B, T, H, dk), torch.float32, dev)
@@ -397,6 +426,7 @@ def backward(q, k, v, log_alpha, beta, grad_out, initial_state=None, grad_final_
     nbytes = backward_workspace_bytes(B, T, H, dk, dv)
     if workspace is None:
         workspace = torch.empty(max(nbytes, 1), dtype=torch.uint8, device=dev)
+    _need_workspace(workspace, dev, "kda_backward")
     f32 = dict(dtype=torch.float32, device=dev)
     g = dict(dq=torch.empty((B, T, H, dk), **f32), dk=torch.empty((B, T, H, dk), **f32),
              dv=torch.empty((B, T, H, dv), **f32), dlog_alpha=torch.empty((B, T, H, dk), **f32),

@@ -9,6 +9,7 @@ import re
 import subprocess
 
 import pytest
+import torch
 
 import gated_delta_rule_109_b200 as kda
 from gated_delta_rule_109_b200 import build as kbuild
@@ -313,3 +314,43 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
                     str(src), "-o", str(exe), "-L", libdir, "-lkda", "-Wl,-rpath," + libdir], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def _host_prefill(B=1, T=8, H=2, d=128):
+    q = torch.zeros((B, T, H, d), dtype=torch.bfloat16)
+    return dict(q=q, k=q.clone(), v=q.clone(), log_alpha=torch.zeros((B, T, H, d)), beta=torch.zeros((B, T, H)))
+
+
+def test_binding_refuses_host_tensors_before_any_device_work(lib):
+    # the kernels take device memory only: host tensors are refused in the binding
+    x = _host_prefill()
+    args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"])
+    for call in (lambda: kda.forward(*args), lambda: kda.gdn_forward(x["q"], x["k"], x["v"], None, x["beta"]),
+                 lambda: kda.forward_noalloc(*args),
+                 lambda: kda.backward(*args, torch.zeros((1, 8, 2, 128))),
+                 lambda: kda.segment_local(*args, workspace=torch.empty(16, dtype=torch.uint8)),
+                 lambda: kda.segment_start_state(torch.zeros((1, 1, 2, 128, 128)), torch.zeros((1, 1, 2, 128, 128))),
+                 lambda: kda.segment_correct(torch.zeros((1, 2, 128, 128)), torch.zeros((1, 2, 128, 128)),
+                                             torch.zeros((1, 8, 2, 128)), workspace=torch.empty(16, dtype=torch.uint8)),
+                 lambda: kda.forward_raw(*args, workspace=torch.empty(16, dtype=torch.uint8))):
+        with pytest.raises(ValueError, match="CUDA tensors"):
+            call()
+    q1 = torch.zeros((1, 2, 128), dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA tensors"):
+        kda.decode_step(q1, q1, q1, torch.zeros((1, 2, 128)), torch.zeros((1, 2)), torch.zeros((1, 2, 128, 128)))
+
+
+def test_binding_refuses_a_workspace_off_the_device(lib):
+    dev = torch.device("cuda", 0)
+    with pytest.raises(TypeError):
+        kda._need_workspace(object(), dev, "kda_forward_ws")
+    with pytest.raises(ValueError, match="contiguous CUDA tensor"):
+        kda._need_workspace(torch.empty(64, dtype=torch.uint8), dev, "kda_forward_ws")
+    with pytest.raises(ValueError, match="contiguous CUDA tensor"):
+        kda._need_workspace(torch.empty((8, 8), dtype=torch.uint8).t(), dev, "kda_forward_ws")
+    # the host-buffer prefill: host inputs, but its workspace must be device memory
+    x = _host_prefill()
+    with pytest.raises(ValueError, match="contiguous CUDA tensor"):
+        kda.forward_host(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], out=torch.empty((1, 8, 2, 128)),
+                         final_state=torch.empty((1, 2, 128, 128)), workspace=torch.empty(64, dtype=torch.uint8),
+                         device="cuda:0")
