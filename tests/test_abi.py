@@ -354,3 +354,17 @@ def test_binding_refuses_a_workspace_off_the_device(lib):
         kda.forward_host(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], out=torch.empty((1, 8, 2, 128)),
                          final_state=torch.empty((1, 2, 128, 128)), workspace=torch.empty(64, dtype=torch.uint8),
                          device="cuda:0")
+
+
+def test_forward_host_empty_sequence_copies_the_state_on_the_host(lib):
+    # T = 0 touches no device: the final state is the initial state (or zeros), in host memory
+    import numpy as np
+    s0 = np.arange(2 * 64 * 64, dtype=np.float32).reshape(1, 2, 64, 64)
+    fin = np.full_like(s0, 7.0)
+    p = lambda a: a.ctypes.data_as(ctypes.c_void_p)
+    call = lambda s_in, s_out: lib.kda_forward_host(None, None, None, None, None, s_in, None, s_out, 1, 0, 2, 64, 64,
+                                                   kda.KDA_F32, ctypes.c_float(0.0), 0, None, 0, None)
+    assert call(p(s0), p(fin)) == kda.KDA_OK and np.array_equal(fin, s0)
+    assert call(None, p(fin)) == kda.KDA_OK and not fin.any()
+    assert call(p(s0), p(s0)) == kda.KDA_OK and s0[0, 1, 63, 63] == 2 * 64 * 64 - 1
+    assert call(p(s0), None) == kda.KDA_OK
