@@ -1,4 +1,4 @@
-"""Host logic of the multi-GPU benchmark path, on CPU with gloo, world size 2.
+"""Host logic of the multi-GPU benchmark path, on CPU with gloo, world sizes 2 and 4.
 
 Every rank runs its own independent batch (weak scaling, no data-path
 collective); the only cross-rank steps are the barrier and the max over ranks
@@ -46,24 +46,26 @@ def _worker(rank, world, port, q):
         q.put((rank, "error", repr(e)))
 
 
-@pytest.mark.timeout(180)
-def test_two_rank_weak_scaling_host_logic():
+@pytest.mark.timeout(240)
+@pytest.mark.parametrize("world", [2, 4])
+def test_weak_scaling_host_logic(world):
     ctx = mp.get_context("spawn")
     q = ctx.Queue()
     port = _free_port()
-    procs = [ctx.Process(target=_worker, args=(r, 2, port, q)) for r in range(2)]
+    procs = [ctx.Process(target=_worker, args=(r, world, port, q)) for r in range(world)]
     for p in procs:
         p.start()
-    res = [q.get(timeout=150) for _ in procs]
+    res = [q.get(timeout=200) for _ in procs]
     for p in procs:
         p.join(timeout=30)
     assert all(len(x) == 6 for x in res), res
     res.sort()
-    (r0, ws0, seed0, T0, mx0, _), (r1, ws1, seed1, T1, mx1, rc1) = res
-    assert ws0 == ws1 == 2
-    assert seed0 != seed1 and T0 == T1 == 65536      # independent batches of the same size
-    assert mx0 == mx1 == 15.0                          # max over ranks
-    assert rc1 == 0                                    # reference arm: rank 1 does no work
+    assert [x[0] for x in res] == list(range(world))
+    assert all(x[1] == world for x in res)
+    assert len({x[2] for x in res}) == world                 # independent batches ...
+    assert all(x[3] == 65536 for x in res)                   # ... of the same size
+    assert all(x[4] == 10.0 + 5.0 * (world - 1) for x in res)   # max over ranks, seen by every rank
+    assert all(x[5] == 0 for x in res[1:])                   # reference arm: ranks > 0 do no work
 
 
 def test_single_process_helpers_are_identities():
