@@ -46,9 +46,22 @@ def test_every_declared_symbol_is_exported(lib):
     assert set(kda.EXPORTS) == set(names)
 
 
-def test_library_is_built_for_sm100a():
-    out = subprocess.run(["strings", kbuild.LIB], capture_output=True, text=True).stdout
-    assert "sm_100a" in out
+def test_every_compile_and_the_link_target_sm100a_only(monkeypatch, tmp_path):
+    # the build's own command lines, recorded instead of run: one target, sm_100a
+    cmds = []
+
+    class Done:
+        returncode, stdout, stderr = 0, "", ""
+
+    monkeypatch.setattr(kbuild.subprocess, "run", lambda cmd, **kw: (cmds.append(cmd), Done())[1])
+    monkeypatch.setattr(kbuild.os, "replace", lambda a, b: None)
+    monkeypatch.setattr(kbuild, "BUILD", str(tmp_path))
+    kbuild.build(force=True)
+    assert len(cmds) == len(kbuild._sources()) + 1            # every kernel source, then the link
+    for c in cmds:
+        assert c.count("-gencode") == 1
+        assert c[c.index("-gencode") + 1] == "arch=compute_100a,code=sm_100a"
+    assert all("-c" in c for c in cmds[:-1]) and "-shared" in cmds[-1]
 
 
 def test_status_strings(lib):
