@@ -143,7 +143,9 @@ kda_status decode_impl(const void *q, const void *k, const void *v, const float 
     if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
     if (dtype != KDA_BF16 && dtype != KDA_F32) return KDA_ERR_INVALID_ARG;
     if (!isfinite(scale)) return KDA_ERR_INVALID_ARG;
-    if ((int64_t)B * H > (int64_t)INT32_MAX) return KDA_ERR_INVALID_ARG;
+    // the decode grid has up to 4 CTAs per head (two per 128 value columns, with
+    // room for one more split); keep B * H * 4 within a grid dimension
+    if ((int64_t)B * H > (int64_t)INT32_MAX / 4) return KDA_ERR_INVALID_ARG;
     const bool need_gate = gate != kda::KDA_GATE_NONE;
     if (!q || !k || !v || (need_gate && !log_alpha) || !beta || !state_inout || !out)
         return KDA_ERR_INVALID_ARG;

@@ -707,6 +707,9 @@ __device__ __forceinline__ void emit_out(float4 *dst, const float (&qs)[16], con
 //                        update does not wait for it, it runs beside the next S');
 //                        also: Kb and M of chunk kk are no longer read
 //   wq_free[s] (commit)  the first product has read the [Wr; Qr] in slot s
+// s_in and s_out may be one buffer (the state carried between blocks, or a final
+// state written over the initial one): every thread reads its own state elements
+// before it writes them, and neither pointer is declared __restrict__.
 constexpr int kChainThreads = 320;
 constexpr uint32_t CH_WQ = 0;                        // two slots of [Wr; Qr] (hi, lo) and e^m
 constexpr uint32_t CH_KTM = 2 * kWqBytes;            // Kb hi, Kb lo, M hi, M lo (48 KB)
@@ -728,8 +731,8 @@ static_assert(R_GAM + 512 == R_EL, "e^{G_last} and e^{G_last - m} are one contig
 constexpr uint32_t TMC_D1 = 0, TMC_D2 = 32, TMC_D3 = 64, TMC_COLS = 128;
 
 __global__ void __launch_bounds__(kChainThreads, 1)
-prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
-                     float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb,
+prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *s_in,
+                     float *s_out, float *__restrict__ out, int T, int H, int n0, int nb,
                      int mode, const float *__restrict__ s_add)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
@@ -1003,8 +1006,8 @@ constexpr uint32_t HS_SO = 2048, HS_SI = 128;                  // N = 128 B-oper
 constexpr uint32_t TMH_D1 = 0, TMH_D2 = 128, TMH_D3 = 256, TMH_S = 384, TMH_COLS = 512;
 
 __global__ void __launch_bounds__(kHeadThreads, 1)
-prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *__restrict__ s_in,
-                          float *__restrict__ s_out, float *__restrict__ out, int T, int H, int n0, int nb,
+prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *s_in,
+                          float *s_out, float *__restrict__ out, int T, int H, int n0, int nb,
                           int mode, const float *__restrict__ s_add)
 {
     extern __shared__ __align__(1024) uint8_t smem[];

@@ -10,9 +10,11 @@
  * decayed state holds for k_t, write beta_t times the prediction error along
  * k_t, and read the updated state with the query scaled by 1/sqrt(d_k).
  * Source: "Kimi Delta Attention: The Linear Attention Behind Kimi K2 and
- * Qwen3", §How Kimi Delta Attention works step by step (prose, `kda_step`
- * code and flowchart); "KDA Technical Deep Dive", §From attention to
- * recurrent state (delta rule) and §How the Kimi gate changes memory (gate).
+ * Qwen3", §TL;DR (per-channel decay Diag(alpha_t), delta rule scaled by
+ * beta_t) and §How Kimi Delta Attention works step by step (the order of the
+ * operations, in prose); "KDA Technical Deep Dive", §From attention to
+ * recurrent state (delta rule, forgetting form) and §How the Kimi gate
+ * changes memory (gate).
  *
  * Conventions shared by every call
  * --------------------------------

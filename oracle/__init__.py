@@ -5,10 +5,18 @@ CPU-baseline / reference leg may import this package.  The library's product
 path never calls it, and it shares no code with the CUDA path.
 
 Two implementations of the same definition, both fp64 on the exact input
-values, both following "Kimi Delta Attention: The Linear Attention Behind Kimi
-K2 and Qwen3", §How Kimi Delta Attention works step by step (the order:
-decay per channel, predict from the decayed state, error scaled by beta,
-delta-rule write, read with the query scaled by 1/sqrt(d_k)):
+values: the KDA recurrence per head and token t,
+
+    S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+    o_t = scale * S_t^T q_t,
+
+the per-channel decay and beta-scaled delta rule of "Kimi Delta Attention: The
+Linear Attention Behind Kimi K2 and Qwen3" (§TL;DR; the order of the operations
+is stated in prose in §How Kimi Delta Attention works step by step) with the
+forgetting factor (I - beta k k^T) of "KDA Technical Deep Dive", §From attention
+to recurrent state.  Both evaluate the product in its expanded form, decay,
+then the delta-rule error beta_t (v_t - S~^T k_t), then S_t = S~ + k_t e^T,
+then the read with the 1/sqrt(d_k)-scaled query:
 
 * ``forward``     -- plain C (``kda_oracle.c``), threaded over heads; used for
                      parity at realistic sizes and for the timed CPU baseline.
@@ -22,9 +30,9 @@ delta-rule write, read with the query scaled by 1/sqrt(d_k)):
                      reverse-mode automatic differentiation (torch.autograd, CPU,
                      fp64) of the same token recurrence.
 
-Both store the state as ``[B, H, dk, dv]`` (the transpose of the page's
-(d_v, d_k) matrix), so the per-channel decay scales rows and the page's
-``S @ k`` is ``S^T k`` here.
+Both store the state as ``[B, H, dk, dv]`` (the transpose of the pages'
+(d_v, d_k) key-to-value map), so the per-channel decay scales rows and the
+prediction for a key k is ``S^T k`` here.
 """
 from __future__ import annotations
 

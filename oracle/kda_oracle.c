@@ -5,23 +5,31 @@
  * loads or calls this file; only the tests, the smoke check and the
  * benchmark's CPU-baseline leg do.  It shares no code with the CUDA path.
  *
- * What it computes: the token-by-token recurrence exactly as written in
- * "Kimi Delta Attention: The Linear Attention Behind Kimi K2 and Qwen3",
- * §How Kimi Delta Attention works step by step (the prose order of the five
- * operations, the `kda_step` code and the flowchart), in fp64, on the exact
- * input values (bf16 and fp32 inputs arrive as fp32, which holds both
- * exactly).  For every head, with S the dk x dv state (rows = key channels):
+ * What it computes: the KDA recurrence, per head and token t,
  *
- *   1. decay per key channel:   S~ = Diag(alpha_t) S,  alpha_t = exp(log_alpha_t)
- *   2. predict:                 p  = S~^T k_t                      (length dv)
- *   3. error scaled by beta:    e  = beta_t (v_t - p)
- *   4. delta-rule write:        S  = S~ + k_t e^T
- *   5. read with scaled query:  o_t = scale * S^T q_t              (after the write)
+ *   S_t = (I - beta_t k_t k_t^T) Diag(alpha_t) S_{t-1} + beta_t k_t v_t^T,
+ *   o_t = scale * S_t^T q_t,
  *
- * The page stores the state as (d_v, d_k) and multiplies `S @ k`; this file
- * stores its transpose (dk x dv, value axis contiguous), so `S @ k` becomes
- * S^T k and the per-channel decay scales rows.  `scale` is the query scaling
- * 1/sqrt(d_k) of step 5 unless the caller passes another value.
+ * in fp64 on the exact input values (bf16 and fp32 inputs arrive as fp32,
+ * which holds both exactly).  The per-channel decay Diag(alpha_t) and the
+ * beta-scaled delta rule are the key equation of "Kimi Delta Attention: The
+ * Linear Attention Behind Kimi K2 and Qwen3" (§TL;DR, and the order of the
+ * operations stated in prose in §How Kimi Delta Attention works step by
+ * step); the factor (I - beta k k^T) is the forgetting form of the delta rule
+ * in "KDA Technical Deep Dive", §From attention to recurrent state.  The
+ * product is evaluated in its expanded form, which needs no dk x dk matrix:
+ * with S the dk x dv state (rows = key channels),
+ *
+ *   S~  = Diag(alpha_t) S,  alpha_t = exp(log_alpha_t)     (decay)
+ *   e   = beta_t (v_t - S~^T k_t)                           (delta-rule error)
+ *   S   = S~ + k_t e^T  = (I - beta_t k_t k_t^T) S~ + beta_t k_t v_t^T
+ *   o_t = scale * S^T q_t                                   (read after the write)
+ *
+ * The pages write the state as a (d_v, d_k) matrix that maps keys to values;
+ * this file stores its transpose (dk x dv, value axis contiguous), so the
+ * prediction is S~^T k and the per-channel decay scales rows.  `scale` is the
+ * 1/sqrt(d_k) query scaling of the KDA page's read unless the caller passes
+ * another value.
  *
  * Layouts (row-major, contiguous): q, k, log_alpha [B,T,H,dk] fp32;
  * v [B,T,H,dv] fp32; beta [B,T,H] fp32; s0 [B,H,dk,dv] fp64 or NULL (zeros);
@@ -63,28 +71,28 @@ static void run_one_head(const oracle_job *j, int bh, double *S, double *p, doub
         const double bt = (double)j->beta[tok * H + h];
         double *ot = j->out + (tok * H + h) * dv;
 
-        /* 1. decay each key channel (row) by alpha = exp(log_alpha) */
+        /* S~ = Diag(alpha_t) S: key channel c (row c) scaled by exp(log_alpha_t[c]) */
         for (int c = 0; c < dk; ++c) {
             const double a = exp((double)lat[c]);
             double *row = S + (size_t)c * dv;
             for (int x = 0; x < dv; ++x) row[x] *= a;
         }
-        /* 2. prediction p = S~^T k */
+        /* p = S~^T k_t: the value the decayed state maps k_t to */
         for (int x = 0; x < dv; ++x) p[x] = 0.0;
         for (int c = 0; c < dk; ++c) {
             const double kc = (double)kt[c];
             const double *row = S + (size_t)c * dv;
             for (int x = 0; x < dv; ++x) p[x] += row[x] * kc;
         }
-        /* 3. error e = beta (v - p) */
+        /* e = beta_t (v_t - p) */
         for (int x = 0; x < dv; ++x) e[x] = bt * ((double)vt[x] - p[x]);
-        /* 4. write S = S~ + k e^T */
+        /* S_t = S~ + k_t e^T = (I - beta_t k_t k_t^T) S~ + beta_t k_t v_t^T */
         for (int c = 0; c < dk; ++c) {
             const double kc = (double)kt[c];
             double *row = S + (size_t)c * dv;
             for (int x = 0; x < dv; ++x) row[x] += kc * e[x];
         }
-        /* 5. read o = scale * S^T q */
+        /* o_t = scale * S_t^T q_t (the state after this token's write) */
         for (int x = 0; x < dv; ++x) ot[x] = 0.0;
         for (int c = 0; c < dk; ++c) {
             const double qc = (double)qt[c];

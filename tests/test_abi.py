@@ -133,6 +133,9 @@ def test_forward_empty_sequence_without_state_is_a_no_op(lib):
     (dict(dk=32), kda.KDA_ERR_UNSUPPORTED),
     (dict(st=FAKE + 4), kda.KDA_ERR_MISALIGNED),
     (dict(k=FAKE + 2), kda.KDA_ERR_MISALIGNED),
+    # B * H beyond what the decode grid (several CTAs per head) can address
+    (dict(B=1 << 15, H=1 << 15), kda.KDA_ERR_INVALID_ARG),
+    (dict(B=(1 << 29) + 1, H=1), kda.KDA_ERR_INVALID_ARG),
 ])
 def test_decode_rejects_bad_arguments_before_launch(lib, kw, code):
     assert _dec(lib, **kw) == code
