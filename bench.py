@@ -95,6 +95,19 @@ def source_digest(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
+def cpu_model():
+    """The host CPU's model name (first processor in /proc/cpuinfo), or the platform string."""
+    try:
+        with open("/proc/cpuinfo") as f:
+            for ln in f:
+                if ln.lower().startswith("model name"):
+                    return ln.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    import platform
+    return platform.processor() or platform.machine()
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -423,10 +436,42 @@ def run_reference(args):
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "tokens_per_step": per_step},
             "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample, "cpu_model": cpu_model(),
+                             "host_cores_online": os.cpu_count()},
             "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
+
+
+def _add_other_prefills(line, args, world, device, hbm, rank=0):
+    """The two other bf16 prefill workloads (B1 H16 T4096; B4 H32 T16384 with a
+    carried state), each through kda_forward_ws with its whole-sequence workspace,
+    timed like the headline and reported with its own roofline."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    res = {}
+    for base in (I.PREFILL_H16_T4K, I.PREFILL_B4_T16K_STATE):
+        w = rank_workload(base, rank)
+        nb = kda.workspace_bytes(w.B, w.T, w.H, w.dk, w.dv, w.torch_dtype)
+        ws = torch.empty(nb, dtype=torch.uint8, device=device)
+        K = max(args.steps, 10)
+        pre = bench_prefill(w, K, args.warmup, device, workspace=ws)
+        ms_total = max_over_ranks(pre["ms_total"], device)
+        ms_launch = statistics.mean(pre["ms_per_launch"])
+        alg = (w.B * w.T * w.H * prefill_bytes_per_token_head(w.dk, w.dv, 2)
+               + (4 * w.B * w.H * w.dk * w.dv if w.final_state else 0)
+               + (4 * w.B * w.H * w.dk * w.dv if w.state_sd is not None else 0))
+        achieved = alg / (ms_launch / 1e3) / 1e9
+        res[w.name] = {"value": w.B * w.T * K * world / (ms_total / 1e3), "unit": "tokens/s",
+                       "ms_per_call": ms_total / K, "steps": K, "gpu_launches": pre["launches"],
+                       "path": "kda_forward_ws, whole-sequence workspace (%.2f GB)" % (nb / 1e9),
+                       "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                                    "frac": achieved / hbm, "traffic": None,
+                                    "algorithmic_bytes_per_launch": alg, "ms_per_launch": ms_launch}}
+        del pre, ws
+        torch.cuda.empty_cache()
+    line["other_prefills"] = res
 
 
 def _add_decode(line, args, rank, world, device, hbm):
@@ -773,6 +818,7 @@ def main(argv=None):
     if not args.no_decode and args.only == "all":
         _add_decode(line, args, rank, world, device, hbm)
     if not args.no_variants and args.only == "all":
+        _add_other_prefills(line, args, world, device, hbm, rank)
         _add_gdn(line, args, w, world, device, hbm)
         if ws_bytes:
             _add_raw(line, args, w, world, device, hbm)
@@ -782,7 +828,8 @@ def main(argv=None):
 
     if cb is not None:
         line["cpu_baseline"] = {"value": cb["value"], "unit": "tokens/s", "cores": cb["threads"],
-                                "kind": "oracle",
+                                "kind": "oracle", "cpu_model": cpu_model(),
+                                "host_cores_online": os.cpu_count(),
                                 "sample": "fp64 oracle on the first %d tokens of all %d heads of the %s "
                                           "workload (%.1f s)" % (cb["tokens"], w.H, w.name, cb["seconds"])}
     if rank == 0:
