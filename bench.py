@@ -592,7 +592,7 @@ def _add_time_split(line, args, w, device, segments=8):
     x = I.make_inputs(w, device)
     names = ("q", "k", "v", "log_alpha", "beta")
     segs = [{n: x[n][:, r * Ts:(r + 1) * Ts].contiguous() for n in names} for r in range(segments)]
-    ws = kda.make_workspace(w.B, Ts, w.H, w.dk, w.dv, w.torch_dtype, device=device)
+    ws = kda.make_workspace(w.B, Ts, w.H, w.dk, w.dv, w.torch_dtype, device=device, segment=True)
     outs, Ps, Fs, final = [], [], [], None
     for r in range(segments):
         o, lf, P = kda.segment_local(*(segs[r][n] for n in names), x["initial_state"] if r == 0 else None,

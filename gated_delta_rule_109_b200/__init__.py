@@ -28,7 +28,7 @@ KDA_PREP_LOGSIGMOID_GATE, KDA_PREP_L2NORM_QK = 1, 2
 
 # every symbol include/kda.h declares
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
-           "kda_forward_workspace_min_bytes", "kda_forward_raw", "kda_segment_local",
+           "kda_forward_workspace_min_bytes", "kda_segment_workspace_bytes", "kda_forward_raw", "kda_segment_local",
            "kda_segment_start_state", "kda_segment_correct", "kda_forward_noalloc",
            "kda_forward_noalloc_scratch_bytes", "kda_forward_host", "kda_forward_host_workspace_bytes",
            "kda_backward", "kda_backward_workspace_bytes",
@@ -67,7 +67,7 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_forward_ws.argtypes = [vp] * 8 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
     lib.kda_gdn_forward_ws.restype = i
     lib.kda_gdn_forward_ws.argtypes = [vp] * 8 + [i] * 6 + [f, vp, ctypes.c_size_t, vp]
-    for name in ("kda_forward_workspace_bytes", "kda_forward_workspace_min_bytes"):
+    for name in ("kda_forward_workspace_bytes", "kda_forward_workspace_min_bytes", "kda_segment_workspace_bytes"):
         getattr(lib, name).restype = ctypes.c_size_t
         getattr(lib, name).argtypes = [i] * 6
     lib.kda_forward_raw.restype = i
@@ -474,17 +474,21 @@ def noalloc_scratch_bytes() -> int:
     return int(load().kda_forward_noalloc_scratch_bytes())
 
 
-def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, minimum=False) -> int:
+def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, minimum=False, segment=False) -> int:
     """Workspace size for :func:`forward` (``kda_forward_workspace_bytes`` /
-    ``..._min_bytes``); 0 when the two-kernel prefill does not apply."""
+    ``..._min_bytes``), or with ``segment`` for :func:`segment_local` and
+    :func:`segment_correct` (``kda_segment_workspace_bytes``); 0 when the
+    two-kernel prefill does not apply."""
     code = KDA_BF16 if dtype == torch.bfloat16 else KDA_F32
-    fn = load().kda_forward_workspace_min_bytes if minimum else load().kda_forward_workspace_bytes
+    lib = load()
+    fn = (lib.kda_segment_workspace_bytes if segment else
+          lib.kda_forward_workspace_min_bytes if minimum else lib.kda_forward_workspace_bytes)
     return int(fn(int(B), int(T), int(H), int(dk), int(dv), code))
 
 
-def make_workspace(B, T, H, dk, dv, dtype=torch.bfloat16, device="cuda", nbytes=None):
+def make_workspace(B, T, H, dk, dv, dtype=torch.bfloat16, device="cuda", nbytes=None, segment=False):
     """A workspace tensor of ``workspace_bytes(...)`` bytes (or ``nbytes``), or None if not needed."""
-    n = workspace_bytes(B, T, H, dk, dv, dtype) if nbytes is None else int(nbytes)
+    n = workspace_bytes(B, T, H, dk, dv, dtype, segment=segment) if nbytes is None else int(nbytes)
     if n == 0:
         return None
     return torch.empty(n, dtype=torch.uint8, device=device)

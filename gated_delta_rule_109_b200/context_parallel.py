@@ -37,7 +37,7 @@ def forward_context_parallel(q, k, v, log_alpha, beta, initial_state=None, *, wo
 
     q, k, v, log_alpha, beta: this rank's segment ``[B, T_r, H, ·]``;
     initial_state: the sequence's initial state (used on rank 0 only);
-    workspace: ``kda.workspace_bytes(B, T_r, H, 128, 128)`` bytes.
+    workspace: ``kda.workspace_bytes(B, T_r, H, 128, 128, segment=True)`` bytes.
     Returns ``(out, final)``: this segment's outputs and the state after it (on
     the last rank: the sequence's final state).  Every rank takes the same
     collective steps (one all-gather).

@@ -99,7 +99,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
                         const float *beta, const float *initial_state, float *out, float *final_state,
                         int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
                         void *stream, kda::GateKind gate, void *workspace = nullptr,
-                        size_t workspace_bytes = 0, int prep_flags = 0)
+                        size_t workspace_bytes = 0, int prep_flags = 0, int T_whole = 0)
 {
     g_last_cuda_error[0] = '\0';
     const kda_status vs = validate_forward(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H,
@@ -128,7 +128,7 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
     cudaError_t e;
     if (workspace && kda::prefill_split_supported(a) &&
         workspace_bytes >= kda::prefill_split_workspace_min(B, T, H))
-        e = kda::launch_prefill_split(a, static_cast<uint8_t *>(workspace), workspace_bytes, st);
+        e = kda::launch_prefill_split(a, static_cast<uint8_t *>(workspace), workspace_bytes, st, T_whole);
     else if (!kda::prefill_tc_supported(a)) e = kda::launch_prefill_simt(a, st);
     else if (gate == kda::KDA_GATE_CHANNEL) e = kda::launch_prefill_tc(a, st);
     else e = kda::launch_prefill_gdn_tc(a, st);
@@ -302,6 +302,12 @@ kda_status kda_segment_correct(const float *start, const float *local_final, flo
 }
 
 size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype)
+{
+    if (B <= 0 || H <= 0 || T <= 0 || dtype != KDA_BF16 || dk != 128 || dv != 128) return 0;
+    return kda::prefill_split_workspace_best(B, T, H);
+}
+
+size_t kda_segment_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype)
 {
     if (B <= 0 || H <= 0 || T <= 0 || dtype != KDA_BF16 || dk != 128 || dv != 128) return 0;
     return kda::prefill_split_workspace_full(B, T, H);
@@ -490,7 +496,7 @@ kda_status kda_forward_host(const void *q, const void *k, const void *v,
         const kda_status fs = forward_impl(dq, dk_, dvv, dla, dbt, (i == 0 && !initial_state) ? nullptr : carry,
                                            dout, carry, B, Ti, H, dk, dv, dtype, scale, stream,
                                            kda::KDA_GATE_CHANNEL, L.recs_bytes ? ws + L.recs : nullptr,
-                                           L.recs_bytes);
+                                           L.recs_bytes, 0, T);
         if (fs != KDA_OK) return fs;
         if ((e = cudaEventRecord(P.comp_done[sl], st)) != cudaSuccess) return cuda_fail(e);
         // block i's outputs back to the host

@@ -58,10 +58,16 @@ cudaError_t take_gdn_device_status(unsigned int *status);
 // caller-provided workspace: bf16, dk = dv = 128, per-channel gate.
 bool prefill_split_supported(const ForwardArgs &a);
 size_t prefill_split_workspace_full(int B, int T, int H);   // whole sequence in one block
+size_t prefill_split_workspace_best(int B, int T, int H);   // the fastest schedule's workspace
 size_t prefill_split_workspace_min(int B, int T, int H);    // one chunk per block + state carry
-// The chain runs one CTA per (b, h, 32-column slice) while 4 B H CTAs fit on the
-// SMs, else one CTA per (b, h).
-cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream);
+// The chain runs one CTA per (b, h) when the heads fill the SMs, or when the sequence
+// is long and the heads few enough that the chunk-local kernel of the next block runs
+// beside it (pipelined over two workspace slots), else one CTA per (b, h, 32-column
+// slice).  T_whole: the length of the whole sequence when a is one block of it (the
+// host-memory path), so that the kernel choice is the whole sequence's.
+bool split_per_head(int B, int T_whole, int H);
+cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream,
+                                 int T_whole = 0);
 cudaError_t take_split_device_status(unsigned int *status);
 // Time-axis split (the chain is linear in (U, S_0)), one contiguous segment of the
 // sequence per call; the workspace holds the whole segment's records:

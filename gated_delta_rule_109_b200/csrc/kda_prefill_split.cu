@@ -39,6 +39,9 @@
 // brings them into shared memory with plain cp.async.bulk copies.  Every
 // mbarrier wait is bounded; a wait that runs out records KDA_ERR_TIMEOUT in a
 // device status word and the CTA stops after its copies in flight have landed.
+#include <algorithm>
+#include <mutex>
+
 #include "kda_tc_ptx.cuh"
 
 namespace kda {
@@ -208,21 +211,26 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     // ---- in-chunk inclusive sums over tokens, per channel, in shared memory: thread
     // (channel, token half) sums its 32 tokens in order, the second half then adds the
     // first half's total.
-    // Padded tokens add 0.  Per channel: G_last (the sum up to the chunk's last token)
-    // and the reference point m midway between the first and last G (the extremes when
-    // the decay is monotone; every token is checked against it in the split pass).
+    // Padded tokens add 0.  Per channel: G_last (the sum up to the chunk's last token),
+    // the reference point m midway between the first and last G (the extremes when the
+    // decay is monotone), and the chunk's minimum and maximum of G, which decide whether
+    // some split factor e^{|G - m|} could overflow (the same decision as testing every
+    // token: G - m rounds monotonically in G).
     float *sGm = reinterpret_cast<float *>(smem + PP_V);
     float *sGl = sGm + kDK;
     float *sTot = sGm + 2 * kDK;
+    float *sMin = sGm + 5 * kDK, *sMax = sGm + 7 * kDK;   // [2][128] each, after sInv
     {
         const int ch = tid & (kDK - 1), th = tid >> 7;
-        float run = 0.f;
+        float run = 0.f, lo = 3.0e38f, hi = -3.0e38f;
         if (gate_act) {
 #pragma unroll 8
             for (int i = 0; i < 32; ++i) {
                 float *gp = Gs + (32 * th + i) * kGP + ch;
                 run += (32 * th + i < c) ? log_sigmoid(*gp) : 0.f;
                 *gp = run;
+                lo = fminf(lo, run);
+                hi = fmaxf(hi, run);
             }
         } else {
             // separate loop: no log-sigmoid evaluated (and discarded) per element
@@ -231,11 +239,16 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                 float *gp = Gs + (32 * th + i) * kGP + ch;
                 run += *gp;
                 *gp = run;
+                lo = fminf(lo, run);
+                hi = fmaxf(hi, run);
             }
         }
         sTot[th * kDK + ch] = run;
+        sMin[th * kDK + ch] = lo;
+        sMax[th * kDK + ch] = hi;
     }
     __syncthreads();
+    bool wide = false;      // some |G - m| > 40 (or |m| > 80): the split exponentials could overflow
     {
         const int ch = tid & (kDK - 1), th = tid >> 7;
         const float tot0 = sTot[ch];
@@ -245,6 +258,9 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         } else {
             const float g_l = tot0 + sTot[kDK + ch];
             const float g_m = 0.5f * (Gs[ch] + g_l);
+            const float gmin = fminf(sMin[ch], sMin[kDK + ch] + tot0);
+            const float gmax = fmaxf(sMax[ch], sMax[kDK + ch] + tot0);
+            wide = !(gmax - g_m <= kGMaxTc && g_m - gmin <= kGMaxTc && fabsf(g_m) <= 2.f * kGMaxTc);
             sGm[ch] = g_m;
             sGl[ch] = g_l;
             reinterpret_cast<float *>(rec + R_EM)[ch] = __expf(g_m);
@@ -252,7 +268,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             reinterpret_cast<float *>(rec + R_EL)[ch] = __expf(g_l - g_m);
         }
     }
-    __syncthreads();
+    const bool wide_path = __syncthreads_or(wide) != 0;
     float G[2][16];
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
@@ -308,8 +324,9 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
     __syncthreads();        // the split pass writes over the scratch
 
-    bool wide = false;      // some |G - m| > 40 (or |m| > 80): the split exponentials could overflow
-    // ---- split operands: Kr (smem), Qr and Kb (smem and record)
+    // ---- split operands: Kr, Qr and Kb in shared memory (the Qr and Kb tiles, already in
+    // the record's byte order, reach the record by bulk copies once P1 is issued)
+    if (!wide_path) {
 #pragma unroll
     for (int hf = 0; hf < 2; ++hf) {
         const int t = lane + 32 * hf;
@@ -328,33 +345,29 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             }
             const uint32_t ok = core_off(t, ch0 + 8 * g, RW_SO, RW_SI);
             const uint32_t oq = core_off(64 + t, ch0 + 8 * g, RW_SO, RW_SI);
-            uint4 hv, lv;
+            float gm[8];
+            {
+                const float4 m0 = reinterpret_cast<const float4 *>(sGm + ch0 + 8 * g)[0];
+                const float4 m1 = reinterpret_cast<const float4 *>(sGm + ch0 + 8 * g)[1];
+                gm[0] = m0.x; gm[1] = m0.y; gm[2] = m0.z; gm[3] = m0.w;
+                gm[4] = m1.x; gm[5] = m1.y; gm[6] = m1.z; gm[7] = m1.w;
+            }
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-                const float g_m = sGm[ch0 + 8 * g + i];
-                const float x = G[hf][8 * g + i] - g_m;
-                wide |= !(fabsf(x) <= kGMaxTc && fabsf(g_m) <= 2.f * kGMaxTc);
-                up[i] = __expf(x);
+                up[i] = __expf(G[hf][8 * g + i] - gm[i]);
                 y[i] = kk[i] * up[i];
             }
             st_split8(smem, PP_P + ok, PP_P_LO + ok, y);                       // Kr
 #pragma unroll
             for (int i = 0; i < 8; ++i) y[i] = scale * qq[i] * up[i];
-            split8(y, hv, lv);                                                 // Qr
-            *reinterpret_cast<uint4 *>(smem + PP_P + oq) = hv;
-            *reinterpret_cast<uint4 *>(smem + PP_P_LO + oq) = lv;
-            *reinterpret_cast<uint4 *>(rec + R_WQ + oq) = hv;
-            *reinterpret_cast<uint4 *>(rec + R_WQ_LO + oq) = lv;
+            st_split8(smem, PP_P + oq, PP_P_LO + oq, y);                       // Qr
 #pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = kk[i] * __expf(sGm[ch0 + 8 * g + i] - G[hf][8 * g + i]);
-            split8(y, hv, lv);                                                 // Kb
-            *reinterpret_cast<uint4 *>(smem + PP_KB + ok) = hv;
-            *reinterpret_cast<uint4 *>(smem + PP_KB_LO + ok) = lv;
-            *reinterpret_cast<uint4 *>(rec + R_KT + ok) = hv;
-            *reinterpret_cast<uint4 *>(rec + R_KT_LO + ok) = lv;
+            for (int i = 0; i < 8; ++i) y[i] = kk[i] * __expf(gm[i] - G[hf][8 * g + i]);
+            st_split8(smem, PP_KB + ok, PP_KB_LO + ok, y);                     // Kb
         }
     }
-    const bool wide_path = __syncthreads_or(wide) != 0;
+    }
+    __syncthreads();        // the V region's scalars have been read
     // V (exact bf16; rows past the chunk's end zero-filled) into its operand tile; a
     // wide-range chunk first finishes with the per-token scalars kept in that region
     auto issue_v = [&]() {
@@ -443,8 +456,16 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                       sbase + PP_KB, sbase + PP_KB_LO, RW_SI, RW_SO, kDK / 16,
                       idesc_bf16(128, 64, 0, 0), false);
             umma_commit(mbar);
+            // Qr (rows 64..127 of [Kr; Qr]) and Kb to the record while P1 runs; both
+            // tiles are already in the record's byte order, Kb hi and lo contiguous
+            bulk_s2g(rec + R_WQ + 16384u, sbase + PP_P + 16384u, 16384u);
+            bulk_s2g(rec + R_WQ_LO + 16384u, sbase + PP_P_LO + 16384u, 16384u);
+            bulk_s2g(rec + R_KT, sbase + PP_KB, 32768u);
+            bulk_commit();
         }
-        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
+        const bool p1_done = mbar_wait(mbar, phase);
+        if (tid == 0) bulk_wait_read();      // the solve's scratch goes over Qr and Kb
+        failed = __syncthreads_or(!p1_done) != 0;
         phase ^= 1;
         if (!failed) {
             tc_fence_after();
@@ -474,12 +495,12 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                         const int j = 32 * half + 8 * g + e;
                         y[e] = (j <= i) ? x[8 * g + e] : 0.f;
                     }
-                    uint4 hv, lv;
-                    split8(y, hv, lv);
+                    // staged where R goes later (Qr lo, already copied out), then one
+                    // bulk copy to the record
                     const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
-                    *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
-                    *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
+                    st_split8(smem, PP_R + o, PP_R_LO + o, y);
                 }
+                proxy_fence();
             }
         }
     } else {
@@ -519,6 +540,10 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         for (int id = tid; id < 64 * 64; id += kNT) Am[(id >> 6) * kPitch + (id & 63)] = Aw[id];
     }
     __syncthreads();
+    if (!wide_path && !failed && tid == 0) {
+        bulk_s2g(rec + R_M, sbase + PP_R, 16384u);     // M hi and lo, contiguous in both
+        bulk_commit();
+    }
 
     if (!failed) {
         // ---- T = (I + A)^-1 by recursive doubling 16 -> 32 -> 64, fp32; R = T Diag(beta)
@@ -593,6 +618,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             *reinterpret_cast<float4 *>(Tm + (32 + i32) * kPitch + 4 * jq8) =
                 make_float4(-y.x, -y.y, -y.z, -y.w);
         }
+        if (tid == 0) bulk_wait_read();      // M has left the region R is written to
         __syncthreads();
         for (int id = tid; id < 512; id += kNT) {
             const int i = id >> 3, jg = id & 7;
@@ -636,11 +662,9 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                     float y[8];
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = x[8 * g + e];
-                    uint4 hv, lv;
-                    split8(y, hv, lv);
+                    // staged in the free [0, 32 KB): hi rows 0..63, then lo
                     const uint32_t o = core_off(lrow, c0 + 8 * g, RW_SO, RW_SI);
-                    *reinterpret_cast<uint4 *>(rec + R_WQ + o) = hv;
-                    *reinterpret_cast<uint4 *>(rec + R_WQ_LO + o) = lv;
+                    st_split8(smem, o, 16384u + o, y);
                 }
             }
         }
@@ -648,7 +672,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             // U: lane 64 + token, 64 value columns per thread = two slices
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
-                float *dst = reinterpret_cast<float *>(rec + R_U + (2 * half + s2) * 8192) + (lrow - 64) * kDVS;
+                // staged in the free [32 KB, 64 KB) in the record's [slice][token][32] order
+                float *dst = reinterpret_cast<float *>(smem + 32768 + (2 * half + s2) * 8192) + (lrow - 64) * kDVS;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float x[16];
@@ -663,12 +688,21 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
 
     if (failed && tid == 0) atomicOr(&g_split_device_status, 1u);
+    proxy_fence();
     tc_fence_before();
     __syncthreads();
+    if (!failed && tid == 0) {
+        // Wr (rows 0..63 of [Wr; Qr], hi then lo) and U to the record
+        bulk_s2g(rec + R_WQ, sbase, 16384u);
+        bulk_s2g(rec + R_WQ_LO, sbase + 16384u, 16384u);
+        bulk_s2g(rec + R_U, sbase + 32768u, 32768u);
+        bulk_commit();
+    }
     if (warp == 0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMP_COLS) : "memory");
     }
+    if (tid == 0) bulk_wait_read();          // shared memory stays until the copies have read it
 }
 
 // ---------------------------------------------------------------- chain kernels: modes
@@ -979,72 +1013,83 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *s_in,
     }
 }
 
-// ---------------------------------------------------------------- full-head chain kernel
-// The chain of one (b, h) with all 128 value columns in one CTA: each tensor-core
-// instruction is N = 128 wide (four times the columns per instruction of the
-// slice kernel), so a CTA per head walks a chunk in about the time a slice CTA
-// does.  Used when the heads alone fill the GPU.  The fp32 state lives in tensor
-// memory (columns 384..511, lane = key channel); warp w of warps 0..15 owns TMEM
-// lane quadrant w % 4 and value columns 32 (w / 4) .. +31 of it and of the
-// accumulators; warp 16 issues the products and the copies.  U rows are fetched
-// into registers (rows 0..63) while the first product runs; Qr S' rows 64..127
-// share those registers.
-constexpr int kHeadThreads = 17 * 32;
-constexpr uint32_t HC_WQ = 0;                                  // [Wr; Qr] hi, lo, e^m (one slot)
-constexpr uint32_t HC_KTM = kWqBytes;                          // Kb hi, Kb lo, M hi, M lo
-constexpr uint32_t HC_MA = HC_KTM + 24576, HC_MA_LO = HC_KTM + 32768;
-constexpr uint32_t HC_GAM = HC_KTM + 49152;                    // e^{G_last} [128], e^{G_last - m} [128]
-constexpr uint32_t HC_S = HC_GAM + 1024, HC_S_LO = HC_S + 32768;     // S': MN-major B, outer dk, inner column
-constexpr uint32_t HC_DL = HC_S + 65536, HC_DL_LO = HC_DL + 16384;   // Delta: MN-major B, outer token
-constexpr uint32_t HC_MBAR = HC_DL + 32768;                    // mma1, mma2, wq, ktm, bar_s, bar_d
-constexpr uint32_t HC_FAIL = HC_MBAR + 48;
-constexpr uint32_t HC_TMEMP = HC_MBAR + 64;
-constexpr uint32_t HC_MBAR3 = HC_MBAR + 72;                    // mma3: M Delta complete (output only)
-constexpr uint32_t HC_TOTAL = HC_TMEMP + 16;
-static_assert(HC_TOTAL <= 232448, "shared memory");
-constexpr uint32_t HS_SO = 2048, HS_SI = 128;                  // N = 128 B-operand strides
-constexpr uint32_t TMH_D1 = 0, TMH_D2 = 128, TMH_D3 = 256, TMH_S = 384, TMH_COLS = 512;
+// ---------------------------------------------------------------- per-head chain kernel
+// The chain of one (b, h) with all 128 value columns in one CTA, the state held
+// transposed: thread (warp w < 16, lane l) owns value column c = 32 (w % 4) + l (its
+// tensor-memory lane) and key channels 32 (w / 4) .. + 31 of S^T, in registers.  With
+// the value axis on the tensor-memory lanes, S'^T and Delta^T are A operands read from
+// tensor memory, and the records' tiles serve unchanged as B operands:
+//   D1^T = S'^T [Wr; Qr]^T        (M = 128 values, N = 128 rows, K = dk)
+//   Delta^T = U^T - D1^T[:, 0:64]
+//   D2^T = Delta^T Kb             (N = dk, K = tokens)
+//   D3^T = Delta^T M^T            (N = 64 output tokens)
+//   O^T = D1^T[:, 64:128] + D3^T,   S^T <- S^T Diag(e^{G_last}) + D2^T Diag(e^{G_last - m})
+// Every product is N = 64 or 128 wide, so one CTA per head walks a chunk in about the
+// time a 32-column slice CTA does, on a quarter of the SMs; and shared memory holds
+// only records: [Wr; Qr] in two slots (two chunks ahead), Kb, M, U and the decays in one.
+// Warp 16 issues the products, warp 17 the record copies and L2 prefetches.  Handoffs
+// are mbarriers (one arrival per compute warp):
+//   bar_s  S'^T of chunk kk is in tensor memory (and D1 of kk - 1 has been read back)
+//   bar_d  Delta^T of chunk kk is in tensor memory (and D3 of kk - 1 has been read back)
+//   bar_u  the state update of chunk kk has read its decays from the Kb/M slot
+//   mma1 / mma2 / mma3 (commit)  D1 / D2 / D3 of chunk kk complete
+//   wq_free[s] (commit)          D1 has read the [Wr; Qr] in slot s
+constexpr int kTThreads = 18 * 32;
+constexpr uint32_t TC_WQ = 0;                         // two slots of [Wr; Qr] hi, lo, e^m
+constexpr uint32_t TC_KTM = 2 * kWqBytes;             // Kb hi, Kb lo, M hi, M lo, then the decays
+constexpr uint32_t TC_DEC = TC_KTM + 49152;           // e^{G_last} [128], e^{G_last - m} [128]
+constexpr uint32_t TC_U = TC_DEC + 1024;              // U fp32 [value slice][token][32]
+constexpr uint32_t TC_MBAR = TC_U + 32768;            // mma1, mma2, mma3, wq[2], wq_free[2], ktm, bar_s, bar_d, bar_u
+constexpr uint32_t TC_FAIL = TC_MBAR + 88;
+constexpr uint32_t TC_TMEMP = TC_MBAR + 96;
+constexpr uint32_t TC_TOTAL = TC_MBAR + 112;
+static_assert(TC_TOTAL <= 232448, "shared memory");
+// tensor-memory columns (lane = value column)
+constexpr uint32_t TT_S = 0, TT_S_LO = 64;            // S'^T, bf16 pairs along dk: hi, lo
+constexpr uint32_t TT_DL = 128, TT_DL_LO = 160;       // Delta^T, bf16 pairs along tokens: hi, lo
+constexpr uint32_t TT_D3 = 192, TT_D1 = 256, TT_D2 = 384, TT_COLS = 512;
 
-__global__ void __launch_bounds__(kHeadThreads, 1)
-prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *s_in,
-                          float *s_out, float *__restrict__ out, int T, int H, int n0, int nb,
-                          int mode, const float *__restrict__ s_add)
+__global__ void __launch_bounds__(kTThreads, 1)
+prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float *s_out, float *__restrict__ out,
+                       int T, int H, int n0, int nb, int mode, const float *__restrict__ s_add)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
-    volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + HC_FAIL);
-    const float *sEm = reinterpret_cast<const float *>(smem + HC_WQ + 65536u);
-    const float *sGam = reinterpret_cast<const float *>(smem + HC_GAM);
-    const uint32_t mbar1 = sbase + HC_MBAR, mbar2 = mbar1 + 8, mbar_wq = mbar1 + 16, mbar_ktm = mbar1 + 24;
-    const uint32_t bar_s = mbar1 + 32, bar_d = mbar1 + 40, mbar3 = sbase + HC_MBAR3;
+    volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + TC_FAIL);
+    const uint32_t mbar1 = sbase + TC_MBAR, mbar2 = mbar1 + 8, mbar3 = mbar1 + 16, mbar_wq0 = mbar1 + 24;
+    const uint32_t wq_free0 = mbar1 + 40, mbar_ktm = mbar1 + 56, bar_s = mbar1 + 64, bar_d = mbar1 + 72;
+    const uint32_t bar_u = mbar1 + 80;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
     const int b = bh / H, h = bh % H;
-    const int r = 32 * (warp & 3) + lane;          // TMEM lane: key channel (S, D2) or row (D1, D3)
-    const int cg = (warp >> 2) & 3;                // value columns 32 cg .. 32 cg + 31
     const uint8_t *recs = ws + (size_t)bh * nb * kRec;
 
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     :: "r"(sbase + HC_TMEMP), "r"(TMH_COLS) : "memory");
+                     :: "r"(sbase + TC_TMEMP), "r"(TT_COLS) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     if (tid == 0) {
         mbar_init(mbar1, 1);
         mbar_init(mbar2, 1);
         mbar_init(mbar3, 1);
-        mbar_init(mbar_wq, 1);
+        mbar_init(mbar_wq0, 1);
+        mbar_init(mbar_wq0 + 8, 1);
+        mbar_init(wq_free0, 1);
+        mbar_init(wq_free0 + 8, 1);
         mbar_init(mbar_ktm, 1);
         mbar_init(bar_s, 16);
         mbar_init(bar_d, 16);
+        mbar_init(bar_u, 16);
         *sFail = 0u;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + HC_TMEMP);
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + TC_TMEMP);
+    // a wait that gives up marks the CTA failed; the others then stop at their next wait
     auto wait = [&](uint32_t bar, uint32_t parity) -> bool {
         if (mbar_try(bar, parity)) return true;        // fast path: no flag read, no clock
         if (*sFail) return false;
@@ -1054,187 +1099,195 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *s_in,
     };
 
     if (warp == 16) {
-        // ---------------- issuer (lane 0): products and record copies
+        // ---------------- issuer: the products (lane 0)
         if (lane == 0) {
-            bool wq_pending = false, ktm_pending = false;
-            uint32_t wq_par = 0u, ktm_par = 0u;
-            auto load_wq = [&](int kk) {
-                wq_pending = true;
-                wq_par = (uint32_t)kk & 1u;
-                mbar_expect_tx(mbar_wq, kWqBytes);
-                bulk_g2s(sbase + HC_WQ, recs + (size_t)kk * kRec + R_WQ, kWqBytes, mbar_wq);
-            };
-            auto load_ktm = [&](int kk) {
-                const uint8_t *rc = recs + (size_t)kk * kRec;
-                ktm_pending = true;
-                ktm_par = (uint32_t)kk & 1u;
-                mbar_expect_tx(mbar_ktm, 49152u + 1024u);
-                bulk_g2s(sbase + HC_KTM, rc + R_KT, 49152u, mbar_ktm);
-                bulk_g2s(sbase + HC_GAM, rc + R_GAM, 1024u, mbar_ktm);
-            };
-            load_wq(0);
-            load_ktm(0);
+            const uint32_t id1 = idesc_bf16(128, 2 * kC, 0, 0);    // B = [Wr; Qr], K-major (rows, dk)
+            const uint32_t id2 = idesc_bf16(128, kDK, 0, 1);       // B = Kb, MN-major (token, dk)
+            const uint32_t id3 = idesc_bf16(128, kC, 0, 0);        // B = M^T, K-major (output token, token)
             for (int kk = 0; kk < nb; ++kk) {
                 const uint32_t par = (uint32_t)kk & 1u;
-                if (!wait(bar_s, par)) break;          // S' written; [Wr; Qr] of kk seen by all
-                wq_pending = false;
+                if (!wait(bar_s, par)) break;
                 tc_fence_after();
-                mma_split(tmem + TMH_D1, sbase + HC_WQ, sbase + HC_WQ + 32768u, RW_SI, RW_SO,
-                          sbase + HC_S, sbase + HC_S_LO, HS_SO, HS_SI, kDK / 16, idesc_bf16(128, kDV, 0, 1), false);
+                const uint32_t wq = sbase + TC_WQ + kWqBytes * (kk & 1);
+                mma_split_ta(tmem + TT_D1, tmem + TT_S, tmem + TT_S_LO, wq, wq + 32768u, RW_SI, RW_SO, kDK / 16, id1);
                 umma_commit(mbar1);
-                if (!wait(mbar1, par)) break;
-                if (kk + 1 < nb) load_wq(kk + 1);
-                if (!wait(bar_d, par)) break;          // Delta written; Kb, M of kk seen by all
-                ktm_pending = false;
+                umma_commit(wq_free0 + 8u * (kk & 1));
+                if (!wait(bar_d, par)) break;
                 tc_fence_after();
-                mma_split(tmem + TMH_D2, sbase + HC_KTM, sbase + HC_KTM + 16384u, RW_SO, RW_SI,
-                          sbase + HC_DL, sbase + HC_DL_LO, HS_SO, HS_SI, kC / 16, idesc_bf16(128, kDV, 1, 1), false);
+                mma_split_ta(tmem + TT_D2, tmem + TT_DL, tmem + TT_DL_LO, sbase + TC_KTM, sbase + TC_KTM + 16384u,
+                             RW_SO, RW_SI, kC / 16, id2);
                 umma_commit(mbar2);
-                mma_split(tmem + TMH_D3, sbase + HC_MA, sbase + HC_MA_LO, H_SI, H_SO,
-                          sbase + HC_DL, sbase + HC_DL_LO, HS_SO, HS_SI, kC / 16, idesc_bf16(128, kDV, 0, 1), false);
+                mma_split_ta(tmem + TT_D3, tmem + TT_DL, tmem + TT_DL_LO, sbase + TC_KTM + 32768u,
+                             sbase + TC_KTM + 40960u, H_SI, H_SO, kC / 16, id3);
                 umma_commit(mbar3);
-                if (!wait(mbar3, par)) break;          // Kb and M read by both products
-                if (kk + 1 < nb) load_ktm(kk + 1);
+            }
+        }
+    } else if (warp == 17) {
+        // ---------------- copies (lane 0): [Wr; Qr] and e^m two chunks ahead (two slots,
+        // refilled once D1 has read them); Kb, M, U and the decays one chunk ahead (one slot,
+        // refilled once D2 and D3 have read it and the state update has read the decays);
+        // the whole record three chunks ahead prefetched into L2
+        if (lane == 0) {
+            uint32_t wq_pend = 0u, wq_par = 0u, ktm_par = 0u;
+            bool ktm_pending = false;
+            auto load_wq = [&](int kk) {
+                const uint32_t mb = mbar_wq0 + 8u * (kk & 1);
+                const uint32_t bit = 1u << (kk & 1);
+                wq_pend |= bit;
+                wq_par = ((kk >> 1) & 1) ? (wq_par | bit) : (wq_par & ~bit);
+                mbar_expect_tx(mb, kWqBytes);
+                bulk_g2s(sbase + TC_WQ + kWqBytes * (kk & 1), recs + (size_t)kk * kRec + R_WQ, kWqBytes, mb);
+            };
+            auto load_ktm = [&](int kk) {
+                const uint8_t *r = recs + (size_t)kk * kRec;
+                ktm_pending = true;
+                ktm_par = (uint32_t)kk & 1u;
+                mbar_expect_tx(mbar_ktm, 49152u + 1024u + 32768u);
+                bulk_g2s(sbase + TC_KTM, r + R_KT, 49152u, mbar_ktm);
+                bulk_g2s(sbase + TC_DEC, r + R_GAM, 1024u, mbar_ktm);
+                bulk_g2s(sbase + TC_U, r + R_U, 32768u, mbar_ktm);
+            };
+            auto prefetch = [&](int kk) {
+                const uint8_t *r = recs + (size_t)kk * kRec;
+                for (uint32_t o = 0; o < kRec; o += 32768u)
+                    l2_prefetch(r + o, (kRec - o) < 32768u ? (kRec - o) : 32768u);
+            };
+            for (int kk = 0; kk < 3 && kk < nb; ++kk) prefetch(kk);
+            load_wq(0);
+            if (nb > 1) load_wq(1);
+            load_ktm(0);
+            for (int kk = 0; kk < nb; ++kk) {
+                if (kk + 3 < nb) prefetch(kk + 3);
+                if (kk + 2 < nb) {
+                    if (!wait(wq_free0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u)) break;
+                    wq_pend &= ~(1u << (kk & 1));
+                    load_wq(kk + 2);
+                }
+                if (kk + 1 < nb) {
+                    if (!wait(mbar3, (uint32_t)kk & 1u) || !wait(bar_u, (uint32_t)kk & 1u)) break;
+                    load_ktm(kk + 1);
+                }
             }
             if (*sFail) {
-                if (wq_pending) mbar_wait(mbar_wq, wq_par);
+                // let the copies still in flight land before shared memory is released
+                for (int sl = 0; sl < 2; ++sl)
+                    if ((wq_pend >> sl) & 1u) mbar_wait(mbar_wq0 + 8u * sl, (wq_par >> sl) & 1u);
                 if (ktm_pending) mbar_wait(mbar_ktm, ktm_par);
             }
         }
     } else {
-        // ---------------- state: row r, columns 32 cg .. +31
-        const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
-        const uint32_t tS = tmem + tlane + TMH_S + 32 * cg;
+        // ---------------- state: value column c, key channels i0 .. i0 + 31
+        const int q4 = warp & 3, g = warp >> 2;
+        const int c = 32 * q4 + lane;
+        const int i0 = 32 * g;
+        const uint32_t tlane = (uint32_t)(32 * q4) << 16;
+        const float *sDec = reinterpret_cast<const float *>(smem + TC_DEC);
+        float S[32];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-            float x[16];
-#pragma unroll
-            for (int j = 0; j < 16; ++j)
-                x[j] = (mode & kChainIdentityS0) ? (r == 32 * cg + 16 * hh + j ? 1.f : 0.f)
-                       : s_in ? s_in[((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh + j] : 0.f;
-            tmem_st16(tS + 16 * hh, x);
-        }
-        tmem_wait_st();
-        float aux[32];            // rows 0..63: U of this chunk; rows 64..127: Qr S' of the last one
+        for (int j = 0; j < 32; ++j)
+            S[j] = (mode & kChainIdentityS0) ? (i0 + j == c ? 1.f : 0.f)
+                   : s_in ? s_in[((size_t)bh * kDK + i0 + j) * kDV + c] : 0.f;
+        float qs[16];             // Qr S' of this thread's 16 output tokens, kept until D3 is back
         auto store_out = [&](int kk) {
-            const int t = (n0 + kk) * kC + r - 64;
+            float o2[16];
+            tmem_ld16(tmem + tlane + TT_D3 + 16 * g, o2);
+            const int tb = (n0 + kk) * kC + 16 * g;
+            if (!(mode & kChainNoOut)) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float o2[16];
-                tmem_ld16(tmem + tlane + TMH_D3 + 32 * cg + 16 * hh, o2);
-                if (t < T && !(mode & kChainNoOut)) {
-                    float qv[16];
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) qv[e] = aux[16 * hh + e];
-                    emit_out(reinterpret_cast<float4 *>(out + (((size_t)b * T + t) * H + h) * kDV + 32 * cg + 16 * hh),
-                             qv, o2, (mode & kChainAccumOut) != 0);
+                for (int j = 0; j < 16; ++j) {
+                    const int t = tb + j;
+                    if (t < T) {
+                        float *p = out + (((size_t)b * T + t) * H + h) * kDV + c;
+                        const float v = qs[j] + o2[j];
+                        *p = (mode & kChainAccumOut) ? *p + v : v;
+                    }
                 }
             }
         };
         bool ok = true;
         for (int kk = 0; kk < nb && ok; ++kk) {
             const uint32_t par = (uint32_t)kk & 1u;
-            // ---- S' = Diag(e^m) S as a split B operand
-            if (!(ok = wait(mbar_wq, par))) break;
+            // ---- S'^T = S^T Diag(e^m) as the hi/lo A operand (pairs of key channels)
+            if (!(ok = wait(mbar_wq0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u))) break;
             {
-                const float em = sEm[r];
+                const float4 *em4 = reinterpret_cast<const float4 *>(smem + TC_WQ + kWqBytes * (kk & 1) + 65536u) + i0 / 4;
+                uint32_t hv[16], lv[16];
 #pragma unroll
-                for (int hh = 0; hh < 2; ++hh) {
-                    float x[16];
-                    tmem_ld16(tS + 16 * hh, x);
-#pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        float xv[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) xv[e] = em * x[8 * g + e];
-                        const uint32_t off = core_off(r, 32 * cg + 16 * hh + 8 * g, HS_SO, HS_SI);
-                        st_split8(smem, HC_S + off, HC_S_LO + off, xv);
-                    }
+                for (int e = 0; e < 8; ++e) {
+                    const float4 m = em4[e];
+                    split_pair(m.x * S[4 * e], m.y * S[4 * e + 1], hv[2 * e], lv[2 * e]);
+                    split_pair(m.z * S[4 * e + 2], m.w * S[4 * e + 3], hv[2 * e + 1], lv[2 * e + 1]);
                 }
+                tmem_st16u(tmem + tlane + TT_S + 16 * g, hv);
+                tmem_st16u(tmem + tlane + TT_S_LO + 16 * g, lv);
+                tmem_wait_st();
             }
-            proxy_fence();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_s);
 
-            // ---- the previous chunk's output while this chunk's first product runs
-            if (kk > 0 && r >= 64) {
+            // ---- the previous chunk's output while this chunk's D1 runs
+            if (kk > 0) {
                 if (!(ok = wait(mbar3, par ^ 1u))) break;
                 tc_fence_after();
                 store_out(kk - 1);
             }
-            // ---- this chunk's U rows (read while the first product runs)
-            if (r < 64 && (mode & kChainZeroU)) {
-#pragma unroll
-                for (int e = 0; e < 32; ++e) aux[e] = 0.f;
-            } else if (r < 64) {
-                const float4 *src = reinterpret_cast<const float4 *>(recs + (size_t)kk * kRec + R_U + cg * 8192u) + r * 8;
-#pragma unroll
-                for (int g = 0; g < 8; ++g) {
-                    const float4 u4 = src[g];
-                    aux[4 * g] = u4.x; aux[4 * g + 1] = u4.y; aux[4 * g + 2] = u4.z; aux[4 * g + 3] = u4.w;
-                }
-            }
 
-            // ---- Delta = U - Wr S' (rows 0..63); Qr S' kept for the output (rows 64..127)
+            // ---- Delta^T = U^T - D1^T[:, 0:64] for tokens 16 g .. 16 g + 15; Qr S' kept
             if (!(ok = wait(mbar1, par) && wait(mbar_ktm, par))) break;
             tc_fence_after();
-#pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
+            {
                 float x[16];
-                tmem_ld16(tmem + tlane + TMH_D1 + 32 * cg + 16 * hh, x);
-                if (r < 64) {
+                tmem_ld16(tmem + tlane + TT_D1 + 16 * g, x);
+                // U: value column c of tokens 16 g .. 16 g + 15 ([slice][token][32] in the slot)
+                const float *su = reinterpret_cast<const float *>(smem + TC_U) + q4 * 2048 + (16 * g) * kDVS + lane;
+                const bool zu = (mode & kChainZeroU) != 0;
+                uint32_t hv[8], lv[8];
 #pragma unroll
-                    for (int g = 0; g < 2; ++g) {
-                        float d[8];
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) d[e] = aux[16 * hh + 8 * g + e] - x[8 * g + e];
-                        const uint32_t o = core_off(r, 32 * cg + 16 * hh + 8 * g, HS_SO, HS_SI);
-                        st_split8(smem, HC_DL + o, HC_DL_LO + o, d);
-                    }
-                } else {
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) aux[16 * hh + e] = x[e];
+                for (int p = 0; p < 8; ++p) {
+                    const float u0 = zu ? 0.f : su[(2 * p) * kDVS], u1 = zu ? 0.f : su[(2 * p + 1) * kDVS];
+                    split_pair(u0 - x[2 * p], u1 - x[2 * p + 1], hv[p], lv[p]);
                 }
+                tmem_st8u(tmem + tlane + TT_DL + 8 * g, hv);
+                tmem_st8u(tmem + tlane + TT_DL_LO + 8 * g, lv);
+                tmem_ld16(tmem + tlane + TT_D1 + 64 + 16 * g, qs);
+                tmem_wait_st();
             }
-            const float gam = sGam[r], el = sGam[kDK + r];
-            proxy_fence();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_d);
 
-            // ---- S <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta
+            // ---- S^T <- S^T Diag(e^{G_last}) + D2^T Diag(e^{G_last - m})
             if (!(ok = wait(mbar2, par))) break;
             tc_fence_after();
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
-                float x[16], sv[16];
-                tmem_ld16(tmem + tlane + TMH_D2 + 32 * cg + 16 * hh, x);
-                tmem_ld16(tS + 16 * hh, sv);
+                float x[16];
+                tmem_ld16(tmem + tlane + TT_D2 + i0 + 16 * hh, x);
+                const float4 *gam4 = reinterpret_cast<const float4 *>(sDec + i0 + 16 * hh);
+                const float4 *el4 = reinterpret_cast<const float4 *>(sDec + kDK + i0 + 16 * hh);
 #pragma unroll
-                for (int j = 0; j < 16; ++j) sv[j] = gam * sv[j] + el * x[j];
-                tmem_st16(tS + 16 * hh, sv);
+                for (int e = 0; e < 4; ++e) {
+                    const float4 ga = gam4[e], el = el4[e];
+                    S[16 * hh + 4 * e] = ga.x * S[16 * hh + 4 * e] + el.x * x[4 * e];
+                    S[16 * hh + 4 * e + 1] = ga.y * S[16 * hh + 4 * e + 1] + el.y * x[4 * e + 1];
+                    S[16 * hh + 4 * e + 2] = ga.z * S[16 * hh + 4 * e + 2] + el.z * x[4 * e + 2];
+                    S[16 * hh + 4 * e + 3] = ga.w * S[16 * hh + 4 * e + 3] + el.w * x[4 * e + 3];
+                }
             }
-            tmem_wait_st();
             tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(bar_u);
         }
-        if (ok && nb > 0 && r >= 64 && (ok = wait(mbar3, (uint32_t)(nb - 1) & 1u))) {
+        if (ok && nb > 0 && (ok = wait(mbar3, (uint32_t)(nb - 1) & 1u))) {
             tc_fence_after();
             store_out(nb - 1);
         }
         if (ok && s_out) {
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float sv[16];
-                tmem_ld16(tS + 16 * hh, sv);
-                const size_t o = ((size_t)bh * kDK + r) * kDV + 32 * cg + 16 * hh;
-                if (s_add) {
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) sv[j] += s_add[o + j];
-                }
-                float4 *dst = reinterpret_cast<float4 *>(s_out + o);
-#pragma unroll
-                for (int g = 0; g < 4; ++g) dst[g] = make_float4(sv[4 * g], sv[4 * g + 1], sv[4 * g + 2], sv[4 * g + 3]);
+            for (int j = 0; j < 32; ++j) {
+                const size_t o = ((size_t)bh * kDK + i0 + j) * kDV + c;
+                s_out[o] = s_add ? S[j] + s_add[o] : S[j];
             }
         }
     }
@@ -1244,7 +1297,7 @@ prefill_chain_head_kernel(const uint8_t *__restrict__ ws, const float *s_in,
     if (tid == 0 && *sFail) atomicOr(&g_split_device_status, 1u);
     if (warp == 0) {
         tc_fence_after();
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMH_COLS) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TT_COLS) : "memory");
     }
 }
 
@@ -1280,6 +1333,52 @@ size_t prefill_split_workspace_full(int B, int T, int H)
     return (size_t)B * H * nchunks * kRec;
 }
 
+namespace {
+
+// The pipelined schedule: blocks of up to kPipeChunks chunks whose records alternate
+// between two workspace slots, so that the chunk-local kernel fills the next block
+// while the per-head chain walks the current one on its own SMs.
+constexpr int kPipeChunks = 64, kPipeMinChunks = 8;
+
+int device_sms()
+{
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                  cudaSuccess || sms <= 0) {
+        cudaGetLastError();         // no device here: size the schedule for a B200
+        return 148;
+    }
+    return sms;
+}
+
+// A shape that takes the pipelined schedule: the per-head chain leaves at least half
+// the SMs to the chunk-local kernel, and the sequence has two full blocks.
+bool pipelined_shape(size_t bh, size_t nch, int sms)
+{
+    return 2 * bh <= (size_t)sms && nch >= 2 * (size_t)kPipeChunks;
+}
+
+}  // namespace
+
+// Which chain kernel a problem runs, from the shape of its whole sequence, so that
+// every schedule of one problem (any workspace, the host-memory path) does the same
+// arithmetic: one CTA per (b, h) when the heads alone fill the SMs or the schedule is
+// pipelined, else one CTA per (b, h, 32-column slice).
+bool split_per_head(int B, int T_whole, int H)
+{
+    const size_t bh = (size_t)B * H, nch = ((size_t)T_whole + kC - 1) / kC;
+    const int sms = device_sms();
+    return bh * kNSL > (size_t)sms || pipelined_shape(bh, nch, sms);
+}
+
+size_t prefill_split_workspace_best(int B, int T, int H)
+{
+    const size_t bh = (size_t)B * H, nch = ((size_t)T + kC - 1) / kC;
+    if (pipelined_shape(bh, nch, device_sms()))
+        return 2 * (size_t)kPipeChunks * bh * kRec + bh * kDK * kDV * sizeof(float);
+    return prefill_split_workspace_full(B, T, H);
+}
+
 size_t prefill_split_workspace_min(int B, int T, int H)
 {
     const size_t bh = (size_t)B * H;
@@ -1290,7 +1389,7 @@ size_t prefill_split_workspace_min(int B, int T, int H)
 
 namespace {
 
-cudaError_t split_setup(size_t bh, bool &per_head)
+cudaError_t split_setup()
 {
     cudaError_t e = cudaFuncSetAttribute(prefill_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)PP_TOTAL);
@@ -1298,14 +1397,8 @@ cudaError_t split_setup(size_t bh, bool &per_head)
         e = cudaFuncSetAttribute(prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)CH_TOTAL);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_chain_head_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)HC_TOTAL);
-    int dev = 0, sms = 0;
-    if (e == cudaSuccess) e = cudaGetDevice(&dev);
-    if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    // value slices while they fit on the SMs in one wave, whole heads once the heads
-    // alone fill them (a head CTA walks a chunk in about the time a slice CTA does)
-    per_head = bh * kNSL > (size_t)sms;
+        e = cudaFuncSetAttribute(prefill_chain_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TC_TOTAL);
     return e;
 }
 
@@ -1332,8 +1425,8 @@ cudaError_t run_chain(const ForwardArgs &a, bool per_head, const uint8_t *ws, in
 {
     const size_t bh = (size_t)a.B * a.H;
     if (per_head)
-        prefill_chain_head_kernel<<<(unsigned)bh, kHeadThreads, HC_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T, a.H,
-                                                                                  n0, nb, mode, s_add);
+        prefill_chain_t_kernel<<<(unsigned)bh, kTThreads, TC_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T, a.H,
+                                                                            n0, nb, mode, s_add);
     else
         prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
                                                                                      a.H, n0, nb, mode, s_add);
@@ -1390,12 +1483,99 @@ affine_compose_kernel(const float *__restrict__ P, const float *__restrict__ F, 
 // allows: prep over the block's chunks of every head, then the chain over them.
 // When L < the number of chunks, the state between blocks is carried in the
 // workspace after the records.
-cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream)
+namespace {
+
+// Per-device streams and events of the pipelined schedule, created on first use: the
+// chain runs on a stream of the greatest priority, so that its CTAs take SMs as soon as
+// they free up, and the chunk-local kernel on one of the least.
+struct SplitStreams {
+    bool ready = false;
+    cudaStream_t chain = nullptr, prep = nullptr;
+    cudaEvent_t start = nullptr, prep_done[2] = {nullptr, nullptr}, chain_done[2] = {nullptr, nullptr};
+};
+constexpr int kMaxDevices = 64;
+SplitStreams g_split_streams[kMaxDevices];
+std::mutex g_split_streams_mu;
+
+cudaError_t split_streams(SplitStreams *&out)
+{
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    SplitStreams &S = g_split_streams[dev];
+    if (!S.ready) {
+        int least = 0, greatest = 0;
+        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
+        if (!S.chain && (e = cudaStreamCreateWithPriority(&S.chain, cudaStreamNonBlocking, greatest)) != cudaSuccess)
+            return e;
+        if (!S.prep && (e = cudaStreamCreateWithPriority(&S.prep, cudaStreamNonBlocking, least)) != cudaSuccess)
+            return e;
+        for (cudaEvent_t *ev : {&S.start, &S.prep_done[0], &S.prep_done[1], &S.chain_done[0], &S.chain_done[1]})
+            if (!*ev && (e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
+        S.ready = true;
+    }
+    out = &S;
+    return cudaSuccess;
+}
+
+// Blocks of L chunks: prep(i + 1) fills slot (i + 1) % 2 while chain(i) reads slot i % 2;
+// prep(i + 1) waits for chain(i - 1), the previous reader of its slot.  Only events order
+// the two kernels; neither waits on the other inside a kernel.
+cudaError_t run_pipelined(const ForwardArgs &a, uint8_t *ws, int L, cudaStream_t stream)
+{
+    const int nchunks = (a.T + kC - 1) / kC;
+    const size_t bh = (size_t)a.B * a.H;
+    const size_t slot = bh * (size_t)L * kRec;
+    float *carry = reinterpret_cast<float *>(ws + 2 * slot);
+    std::lock_guard<std::mutex> lock(g_split_streams_mu);
+    SplitStreams *S = nullptr;
+    cudaError_t e = split_streams(S);
+    if (e != cudaSuccess) return e;
+    // fork: both streams start after the work already on the caller's stream
+    if ((e = cudaEventRecord(S->start, stream)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(S->prep, S->start, 0)) != cudaSuccess ||
+        (e = cudaStreamWaitEvent(S->chain, S->start, 0)) != cudaSuccess)
+        return e;
+    const int nblk = (nchunks + L - 1) / L;
+    e = run_prep(a, ws, 0, min(L, nchunks), S->prep);
+    if (e == cudaSuccess) e = cudaEventRecord(S->prep_done[0], S->prep);
+    for (int i = 0; i < nblk && e == cudaSuccess; ++i) {
+        const int n0 = i * L, nb = min(L, nchunks - n0);
+        e = cudaStreamWaitEvent(S->chain, S->prep_done[i & 1], 0);
+        if (e == cudaSuccess)
+            e = run_chain(a, true, ws + (size_t)(i & 1) * slot, n0, nb, i == 0 ? a.s0 : carry,
+                          i == nblk - 1 ? a.sT : carry, 0, nullptr, S->chain);
+        if (e == cudaSuccess) e = cudaEventRecord(S->chain_done[i & 1], S->chain);
+        if (e == cudaSuccess && i + 1 < nblk) {
+            const int n1 = n0 + nb;
+            if (i >= 1) e = cudaStreamWaitEvent(S->prep, S->chain_done[(i - 1) & 1], 0);
+            if (e == cudaSuccess)
+                e = run_prep(a, ws + (size_t)((i + 1) & 1) * slot, n1, min(L, nchunks - n1), S->prep);
+            if (e == cudaSuccess) e = cudaEventRecord(S->prep_done[(i + 1) & 1], S->prep);
+        }
+    }
+    // join: the caller's stream waits for the last chain, which follows every prep
+    const cudaError_t j = cudaStreamWaitEvent(stream, S->chain_done[(nblk - 1) & 1], 0);
+    return e != cudaSuccess ? e : j;
+}
+
+}  // namespace
+
+cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_bytes, cudaStream_t stream, int T_whole)
 {
     const int nchunks = (a.T + kC - 1) / kC;
     const size_t bh = (size_t)a.B * a.H;
     const size_t per_chunk = bh * kRec;
     const size_t state_bytes = bh * kDK * kDV * sizeof(float);
+    const bool per_head = split_per_head(a.B, T_whole > 0 ? T_whole : a.T, a.H);
+    cudaError_t e = split_setup();
+    if (e != cudaSuccess) return e;
+    if (per_head && pipelined_shape(bh, (size_t)nchunks, device_sms()) &&
+        ws_bytes >= state_bytes + 2 * (size_t)kPipeMinChunks * per_chunk) {
+        const size_t fit = (ws_bytes - state_bytes) / (2 * per_chunk);
+        return run_pipelined(a, ws, (int)std::min<size_t>(fit, kPipeChunks), stream);
+    }
     int L;
     if (ws_bytes >= per_chunk * (size_t)nchunks) {
         L = nchunks;
@@ -1404,9 +1584,6 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
         L = (int)((ws_bytes - state_bytes) / per_chunk);
     }
     float *carry = (L < nchunks) ? reinterpret_cast<float *>(ws + per_chunk * (size_t)L) : nullptr;
-    bool per_head = false;
-    cudaError_t e = split_setup(bh, per_head);
-    if (e != cudaSuccess) return e;
     for (int n0 = 0; n0 < nchunks; n0 += L) {
         const int nb = min(L, nchunks - n0);
         e = run_prep(a, ws, n0, nb, stream);
@@ -1424,8 +1601,8 @@ cudaError_t launch_prefill_split(const ForwardArgs &a, uint8_t *ws, size_t ws_by
 cudaError_t launch_segment_local(const ForwardArgs &a, float *transfer, uint8_t *ws, cudaStream_t stream)
 {
     const int nchunks = (a.T + kC - 1) / kC;
-    bool per_head = false;
-    cudaError_t e = split_setup((size_t)a.B * a.H, per_head);
+    const bool per_head = (size_t)a.B * a.H * kNSL > (size_t)device_sms();
+    cudaError_t e = split_setup();
     if (e == cudaSuccess) e = run_prep(a, ws, 0, nchunks, stream);
     // outputs and final state of the segment from the given start (zero if none)
     if (e == cudaSuccess) e = run_chain(a, per_head, ws, 0, nchunks, a.s0, a.sT, 0, nullptr, stream);
@@ -1440,8 +1617,8 @@ cudaError_t launch_segment_correct(const ForwardArgs &a, const float *start, con
                                    const uint8_t *ws, cudaStream_t stream)
 {
     const int nchunks = (a.T + kC - 1) / kC;
-    bool per_head = false;
-    cudaError_t e = split_setup((size_t)a.B * a.H, per_head);
+    const bool per_head = (size_t)a.B * a.H * kNSL > (size_t)device_sms();
+    cudaError_t e = split_setup();
     // out += outputs of the start state propagated alone; final = local final + that state
     if (e == cudaSuccess)
         e = run_chain(a, per_head, ws, 0, nchunks, start, a.sT, kChainZeroU | kChainAccumOut, local_final, stream);

@@ -78,6 +78,33 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float (&v)[16])
 }
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
+// Stores of raw 32-bit words (packed bf16 pairs of an A operand held in tensor memory).
+__device__ __forceinline__ void tmem_st16u(uint32_t taddr, const uint32_t (&v)[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+                 "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                    "r"(v[7]), "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]),
+                    "r"(v[14]), "r"(v[15]) : "memory");
+}
+__device__ __forceinline__ void tmem_st8u(uint32_t taddr, const uint32_t (&v)[8])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "r"(taddr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]),
+                    "r"(v[7]) : "memory");
+}
+
+// Split two fp32 values into a packed bf16 pair (first value in the low half) and the
+// packed pair of their remainders: x = hi + lo to about 16 significant bits.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uint32_t &lo)
+{
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(hv);
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t *>(&hv);
+    lo = *reinterpret_cast<const uint32_t *>(&lv);
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(mbar), "r"(count) : "memory");
@@ -98,6 +125,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
     asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
                  :: "r"(dst), "l"(src), "r"(bytes), "r"(mbar) : "memory");
 }
+
+// shared -> global bulk copy through the async proxy (16-byte aligned addresses, a
+// multiple of 16 bytes), tracked in the issuing thread's bulk group.  The shared
+// source must have been written before a fence.proxy.async by its writers.
+__device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes)
+{
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;"
+                 :: "l"(dst), "r"(src), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// wait until every committed bulk copy of this thread has read its shared source
+__device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
 // 16-byte global -> shared copy (sm_80 cp.async); src_bytes = 0 zero-fills the
 // destination without reading the source.
@@ -164,6 +203,38 @@ __device__ __forceinline__ void st_split8(uint8_t *smem, uint32_t off_hi, uint32
     split8(x, hi, lo);
     *reinterpret_cast<uint4 *>(smem + off_hi) = hi;
     *reinterpret_cast<uint4 *>(smem + off_lo) = lo;
+}
+
+// tcgen05.mma with the A operand in tensor memory: lane = row of A, each 32-bit
+// column a pair of consecutive K elements (the first in the low half), a K step of
+// 16 taking 8 columns.
+__device__ __forceinline__ void umma_bf16_ta(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n"
+                 :: "r"(d_tmem), "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+
+// D = A B on hi/lo split operands with A (hi and lo) in tensor memory and B in shared
+// memory: hi*hi + lo*hi + hi*lo, K in `ksteps` steps of 16.
+__device__ __forceinline__ void mma_split_ta(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
+                                             uint32_t b_lo, uint32_t b_lbo, uint32_t b_sbo, int ksteps,
+                                             uint32_t idesc)
+{
+    const uint64_t db[2] = {smem_desc(b_hi, b_lbo, b_sbo), smem_desc(b_lo, b_lbo, b_sbo)};
+    const uint64_t sb = (2u * b_lbo) >> 4;
+    bool acc = false;
+#pragma unroll
+    for (int tt = 0; tt < 3; ++tt) {
+        const uint32_t a = tt == 1 ? a_lo : a_hi;
+        uint64_t bd = db[tt == 2 ? 1 : 0];
+#pragma unroll
+        for (int ks = 0; ks < ksteps; ++ks) {
+            umma_bf16_ta(d, a + 8u * (uint32_t)ks, bd, idesc, acc ? 1u : 0u);
+            acc = true;
+            bd += sb;
+        }
+    }
 }
 
 // One product D (+)= A B on bf16 hi/lo split operands: hi*hi, plus lo*hi when A has

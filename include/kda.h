@@ -104,10 +104,18 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
  * record per chunk into the workspace; the other walks the chunks of each
  * (b, h) in order, carrying the state through them ("KDA Technical Deep
  * Dive", §Systems and implementation tradeoffs, Training: chunk-local work in
- * parallel, the boundary state seeding the next chunk).  With
- * kda_forward_workspace_bytes() the whole sequence is one block; with less
- * (but at least the minimum) the sequence is processed in blocks of as many
- * chunks as fit, the state between blocks kept in the workspace.
+ * parallel, the boundary state seeding the next chunk).  Blocks of chunks
+ * carry the state between them in the workspace:
+ *   - few heads, long sequence (2 B H at most the SM count, at least 128 chunks),
+ *     and room for two blocks of 8 or more chunks: pipelined.  The chain of
+ *     block i (one CTA per (b, h)) runs beside the chunk-local kernel of block
+ *     i + 1 on the other SMs, their records in alternating halves of the
+ *     workspace, on two internal streams (created on first use) ordered by
+ *     events; the caller's stream waits for the last kernel.
+ *   - otherwise: the chunk-local kernel, then the chain, per block of as many
+ *     chunks as fit (the whole sequence with its full record size).
+ * Which chain kernel runs depends only on B, T and H, so every workspace size
+ * gives bit-identical results.
  *
  *   workspace        device memory, 256-byte aligned, owned by the caller; its
  *                    contents on entry do not matter and on return are
@@ -127,14 +135,25 @@ kda_status kda_forward_ws(const void *q, const void *k, const void *v,
                           void *stream);
 
 /*
- * Workspace sizes for kda_forward_ws: the size at which the whole sequence is
- * one block (the fastest), and the smallest size that still takes the
- * two-kernel path (one chunk per block plus the carried state).  Both are 0
- * when the two-kernel path does not apply (dtype, head dimensions, T = 0 or
- * bad sizes).  About 145 KB per chunk of 64 tokens per (b, h).
+ * Workspace sizes for kda_forward_ws: the size the fastest schedule uses, and the
+ * smallest size that still takes the two-kernel path (one chunk per block plus the
+ * carried state).  Both are 0 when the two-kernel path does not apply (dtype, head
+ * dimensions, T = 0 or bad sizes).  The records take about 145 KB per chunk of 64
+ * tokens per (b, h).  For few heads (2 B H at most the SM count) and sequences of
+ * at least 128 chunks, the fastest schedule is pipelined: blocks of 64 chunks whose
+ * records alternate between two slots while the chain of one block runs beside the
+ * chunk-local kernel of the next, so the size is two blocks' records plus the carried
+ * state (0.61 GB for B1 H32 T65536); otherwise it is the whole sequence's records.
  */
 size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 size_t kda_forward_workspace_min_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
+
+/*
+ * Workspace size for kda_segment_local / kda_segment_correct: every chunk record of
+ * the segment (they must all stay for the correction).  0 where the two-kernel path
+ * does not apply.
+ */
+size_t kda_segment_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 
 /* Steps before the path that kda_forward_raw can fuse into the prefill. */
 enum {
@@ -193,7 +212,7 @@ kda_status kda_forward_raw(const void *q, const void *k, const void *v,
  * kda_segment_local -- outputs `out` and `local_final` of the segment from
  *   `initial_state` (NULL = zero), and its `transfer` [B, H, dk, dk] fp32
  *   (16-byte aligned).  Other arguments as kda_forward_ws; the workspace must
- *   hold the whole segment (kda_forward_workspace_bytes) and must be passed
+ *   hold the whole segment (kda_segment_workspace_bytes) and must be passed
  *   unchanged to kda_segment_correct.  T >= 1.
  */
 kda_status kda_segment_local(const void *q, const void *k, const void *v,

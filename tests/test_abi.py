@@ -184,15 +184,24 @@ def test_workspace_sizes(lib):
     rec = full(1, 64, 1, 128, 128, kda.KDA_BF16)      # bytes of one chunk record (b, h, chunk)
     assert rec % 256 == 0 or rec % 16 == 0
     assert 140_000 < rec < 160_000
-    assert full(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec
-    assert full(4, 16384, 32, 128, 128, kda.KDA_BF16) == 128 * 256 * rec
+    assert full(4, 16384, 32, 128, 128, kda.KDA_BF16) == 128 * 256 * rec      # many heads: whole sequence
     assert full(2, 65, 3, 128, 128, kda.KDA_BF16) == 6 * 2 * rec             # ragged tail: 2 chunks
     assert mini(2, 65, 3, 128, 128, kda.KDA_BF16) == 6 * rec + 6 * 128 * 128 * 4
     assert mini(2, 64, 3, 128, 128, kda.KDA_BF16) == full(2, 64, 3, 128, 128, kda.KDA_BF16) == 6 * rec
     for args in [(1, 100, 2, 64, 64, kda.KDA_BF16), (1, 100, 2, 128, 128, kda.KDA_F32),
                  (1, 0, 2, 128, 128, kda.KDA_BF16), (0, 10, 2, 128, 128, kda.KDA_BF16)]:
         assert full(*args) == 0 and mini(*args) == 0
-    assert kda.workspace_bytes(1, 65536, 32, 128, 128) == 32 * 1024 * rec
+    # few heads and a long sequence: the pipelined schedule's two slots of 64 chunks
+    # and the carried state, far less than the whole sequence's records
+    state32 = 32 * 128 * 128 * 4
+    assert kda.workspace_bytes(1, 65536, 32, 128, 128) == 2 * 64 * 32 * rec + state32
+    assert kda.workspace_bytes(1, 8192, 32, 128, 128) == 2 * 64 * 32 * rec + state32
+    assert kda.workspace_bytes(1, 8128, 32, 128, 128) == 32 * 127 * rec            # under 128 chunks
+    # segments keep every record of the segment
+    seg = lambda *a: lib.kda_segment_workspace_bytes(*a)
+    assert seg(1, 65536, 32, 128, 128, kda.KDA_BF16) == 32 * 1024 * rec
+    assert kda.workspace_bytes(1, 8192, 32, 128, 128, segment=True) == 32 * 128 * rec
+    assert seg(1, 100, 2, 64, 64, kda.KDA_BF16) == 0
 
 
 def test_forward_ws_validates_like_forward(lib):

@@ -30,7 +30,7 @@ def test_three_rank_split_with_kernel_ops(monkeypatch):
     cuts = [0, 200, 450, 600]
     R = len(cuts) - 1
     segs = [{n: x[n][:, cuts[r]:cuts[r + 1]].contiguous() for n in NAMES} for r in range(R)]
-    wss = [kda.make_workspace(w.B, cuts[r + 1] - cuts[r], w.H, 128, 128) for r in range(R)]
+    wss = [kda.make_workspace(w.B, cuts[r + 1] - cuts[r], w.H, 128, 128, segment=True) for r in range(R)]
     pairs = []
     for r in range(R):
         _, lf, P = cp.KERNEL_OPS.segment_local(*(segs[r][n] for n in NAMES), x["initial_state"] if r == 0 else None,

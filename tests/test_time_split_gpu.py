@@ -31,7 +31,7 @@ def _split_run(x, cuts):
     for r in range(len(bounds) - 1):
         a, b = bounds[r], bounds[r + 1]
         seg = {n: x[n][:, a:b].contiguous() for n in NAMES}
-        ws = kda.make_workspace(B, b - a, H, 128, 128)
+        ws = kda.make_workspace(B, b - a, H, 128, 128, segment=True)
         o, lf, P = kda.segment_local(*(seg[n] for n in NAMES), x["initial_state"] if r == 0 else None, workspace=ws)
         outs.append(o); Ps.append(P); Fs.append(lf); wss.append(ws)
     final = Fs[0]
@@ -73,7 +73,7 @@ def test_transfer_is_the_state_map_with_zero_values():
     """P S0 = the final state of the segment run from S0 with zero values."""
     w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=2, T=200, seed=7200)
     x = I.make_inputs(w, "cuda")
-    ws = kda.make_workspace(w.B, w.T, w.H, 128, 128)
+    ws = kda.make_workspace(w.B, w.T, w.H, 128, 128, segment=True)
     _, _, P = kda.segment_local(*(x[n] for n in NAMES), None, workspace=ws)
     z = torch.zeros_like(x["v"])
     _, s_ref = oracle.forward(x["q"], x["k"], z, x["log_alpha"], x["beta"], x["initial_state"])
