@@ -46,6 +46,14 @@ decode_step_kernel(const InT *__restrict__ q, const InT *__restrict__ k,
     __shared__ float4 red_r[RS][CG];
     __shared__ float s_kq;
 
+    // Programmatic dependent launch: once every CTA of this step has started, the next
+    // step may be launched, so that its CTAs take the SM slots this step's last wave
+    // frees instead of waiting for the launch after it completes.  Nothing is read
+    // before the kernel ahead on the stream (the previous step, or whatever produced
+    // this step's inputs) has completed and its writes are visible.
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+
     const int bh = blockIdx.x / NS;            // b * H + h
     const int tid = threadIdx.x;
     const int cg = (blockIdx.x % NS) * CG + tid % CG;   // column group within the head
@@ -133,10 +141,20 @@ cudaError_t launch_typed(const DecodeArgs &a, cudaStream_t stream)
     const unsigned grid = (unsigned)((size_t)a.B * a.H * NS);
     auto kernel = (a.gate == KDA_GATE_CHANNEL) ? decode_step_kernel<DK, DV, InT, true, NS>
                                                : decode_step_kernel<DK, DV, InT, false, NS>;
-    kernel<<<grid, kDecodeThreads, 0, stream>>>(
-        static_cast<const InT *>(a.q), static_cast<const InT *>(a.k),
-        static_cast<const InT *>(a.v), a.log_alpha, a.beta, a.state, a.out, a.scale);
-    cudaError_t e2 = cudaGetLastError();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(kDecodeThreads);
+    cfg.dynamicSmemBytes = 0;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e2 = cudaLaunchKernelEx(&cfg, kernel, static_cast<const InT *>(a.q), static_cast<const InT *>(a.k),
+                                        static_cast<const InT *>(a.v), a.log_alpha, a.beta, a.state, a.out,
+                                        a.scale);
+    if (e2 == cudaSuccess) e2 = cudaGetLastError();
     if (e2 == cudaSuccess) note_launch();
     return e2;
 }

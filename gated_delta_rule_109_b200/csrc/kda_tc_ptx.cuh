@@ -9,6 +9,8 @@
 // and SBO the stride along M/N.
 #pragma once
 
+#include <cuda.h>
+
 #include "kda_internal.cuh"
 
 namespace kda {
@@ -137,6 +139,20 @@ __device__ __forceinline__ void bulk_s2g(void *dst, uint32_t src, uint32_t bytes
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // wait until every committed bulk copy of this thread has read its shared source
 __device__ __forceinline__ void bulk_wait_read() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+
+// TMA tensor store (and reduce-add) of one 4-D box from shared memory through a tensor
+// map passed as a __grid_constant__ kernel parameter; tracked in the issuing thread's
+// bulk group like bulk_s2g.  Coordinates are element indices, innermost first.
+__device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 :: "l"(tmap), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
+__device__ __forceinline__ void tma_reduce_add_4d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3)
+{
+    asm volatile("cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
+                 :: "l"(tmap), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
 
 // 16-byte global -> shared copy (sm_80 cp.async); src_bytes = 0 zero-fills the
 // destination without reading the source.
