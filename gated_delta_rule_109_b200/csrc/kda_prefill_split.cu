@@ -1030,9 +1030,10 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *s_in,
 // Every product is N = 64 or 128 wide, so one CTA per head walks a chunk in about the
 // time a 32-column slice CTA does, on a quarter of the SMs; and shared memory holds
 // only records: [Wr; Qr] in two slots (two chunks ahead), Kb, M, U and the decays in one.
-// A chunk's outputs are staged in its [Wr; Qr] slot once D1 has read it and leave by
-// one TMA tensor store: plain stores from 512 threads slowed the next chunk's D1 by a
-// third.  Warp 16 issues the products; warp 17 the record copies, the output stores
+// A chunk's outputs are staged in the hi half of its [Wr; Qr] slot once D1 has read it
+// and leave by one TMA tensor store (plain stores from 512 threads slowed the next
+// chunk's D1 by a third); the slot's lo half and e^m are refilled as soon as D1 is
+// done, the hi half once the store has read it.  Warp 16 issues the products; warp 17 the record copies, the output stores
 // and L2 prefetches.  Handoffs are mbarriers (one arrival per compute warp):
 //   bar_s  S'^T of chunk kk is in tensor memory (and D1 of kk - 1 has been read back)
 //   bar_d  Delta^T of chunk kk is in tensor memory (and D3 of kk - 1 has been read back)
@@ -1045,7 +1046,7 @@ constexpr uint32_t TC_WQ = 0;                         // two slots of [Wr; Qr] h
 constexpr uint32_t TC_KTM = 2 * kWqBytes;             // Kb hi, Kb lo, M hi, M lo, then the decays
 constexpr uint32_t TC_DEC = TC_KTM + 49152;           // e^{G_last} [128], e^{G_last - m} [128]
 constexpr uint32_t TC_U = TC_DEC + 1024;              // U fp32 [value slice][token][32]
-constexpr uint32_t TC_MBAR = TC_U + 32768;            // mma1, mma2, mma3, wq[2], (2 unused), ktm, bar_s, bar_d, bar_u
+constexpr uint32_t TC_MBAR = TC_U + 32768;            // mma1, mma2, mma3, wq_lo[2], wq_hi[2], ktm, bar_s, bar_d, bar_u
 constexpr uint32_t TC_FAIL = TC_MBAR + 88;
 constexpr uint32_t TC_TMEMP = TC_MBAR + 96;
 constexpr uint32_t TC_OUTST = TC_MBAR + 104;          // out_st
@@ -1064,8 +1065,10 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
     volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + TC_FAIL);
-    const uint32_t mbar1 = sbase + TC_MBAR, mbar2 = mbar1 + 8, mbar3 = mbar1 + 16, mbar_wq0 = mbar1 + 24;
-    const uint32_t wq_free0 = mbar1 + 40, mbar_ktm = mbar1 + 56, bar_s = mbar1 + 64, bar_d = mbar1 + 72;
+    // [Wr; Qr] slots arrive in two halves: lo with e^m (wq_lo), then hi (wq_hi), whose
+    // region also stages the outputs
+    const uint32_t mbar1 = sbase + TC_MBAR, mbar2 = mbar1 + 8, mbar3 = mbar1 + 16, wq_lo0 = mbar1 + 24;
+    const uint32_t wq_hi0 = mbar1 + 40, mbar_ktm = mbar1 + 56, bar_s = mbar1 + 64, bar_d = mbar1 + 72;
     const uint32_t bar_u = mbar1 + 80, out_st = sbase + TC_OUTST;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -1082,10 +1085,10 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
         mbar_init(mbar1, 1);
         mbar_init(mbar2, 1);
         mbar_init(mbar3, 1);
-        mbar_init(mbar_wq0, 1);
-        mbar_init(mbar_wq0 + 8, 1);
-        mbar_init(wq_free0, 1);
-        mbar_init(wq_free0 + 8, 1);
+        mbar_init(wq_lo0, 1);
+        mbar_init(wq_lo0 + 8, 1);
+        mbar_init(wq_hi0, 1);
+        mbar_init(wq_hi0 + 8, 1);
         mbar_init(mbar_ktm, 1);
         mbar_init(bar_s, 16);
         mbar_init(bar_d, 16);
@@ -1115,7 +1118,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
             const uint32_t id3 = idesc_bf16(128, kC, 0, 0);        // B = M^T, K-major (output token, token)
             for (int kk = 0; kk < nb; ++kk) {
                 const uint32_t par = (uint32_t)kk & 1u;
-                if (!wait(bar_s, par)) break;
+                if (!wait(bar_s, par) || !wait(wq_hi0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u)) break;
                 tc_fence_after();
                 const uint32_t wq = sbase + TC_WQ + kWqBytes * (kk & 1);
                 mma_split_ta(tmem + TT_D1, tmem + TT_S, tmem + TT_S_LO, wq, wq + 32768u, RW_SI, RW_SO, kDK / 16, id1);
@@ -1137,15 +1140,17 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
         // has read the decays); the outputs of each chunk by one tensor store (or
         // reduce-add); the whole record three chunks ahead prefetched into L2
         if (lane == 0) {
-            uint32_t wq_pend = 0u, wq_par = 0u, ktm_par = 0u;
+            uint32_t pend = 0u, par_bits = 0u, ktm_par = 0u;   // bit 2 s + h: slot s, half h (1 = hi) in flight
             bool ktm_pending = false;
-            auto load_wq = [&](int kk) {
-                const uint32_t mb = mbar_wq0 + 8u * (kk & 1);
-                const uint32_t bit = 1u << (kk & 1);
-                wq_pend |= bit;
-                wq_par = ((kk >> 1) & 1) ? (wq_par | bit) : (wq_par & ~bit);
-                mbar_expect_tx(mb, kWqBytes);
-                bulk_g2s(sbase + TC_WQ + kWqBytes * (kk & 1), recs + (size_t)kk * kRec + R_WQ, kWqBytes, mb);
+            auto load_half = [&](int kk, int hi) {
+                const int sl = kk & 1;
+                const uint32_t mb = (hi ? wq_hi0 : wq_lo0) + 8u * sl;
+                const uint32_t bit = 1u << (2 * sl + hi);
+                pend |= bit;
+                par_bits = ((kk >> 1) & 1) ? (par_bits | bit) : (par_bits & ~bit);
+                const uint32_t off = hi ? 0u : 32768u, bytes = hi ? 32768u : kWqBytes - 32768u;
+                mbar_expect_tx(mb, bytes);
+                bulk_g2s(sbase + TC_WQ + kWqBytes * sl + off, recs + (size_t)kk * kRec + R_WQ + off, bytes, mb);
             };
             auto load_ktm = [&](int kk) {
                 const uint8_t *r = recs + (size_t)kk * kRec;
@@ -1162,18 +1167,25 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                     l2_prefetch(r + o, (kRec - o) < 32768u ? (kRec - o) : 32768u);
             };
             for (int kk = 0; kk < 3 && kk < nb; ++kk) prefetch(kk);
-            load_wq(0);
-            if (nb > 1) load_wq(1);
+            for (int kk = 0; kk < 2 && kk < nb; ++kk) {
+                load_half(kk, 0);
+                load_half(kk, 1);
+            }
             load_ktm(0);
             for (int kk = 0; kk < nb; ++kk) {
                 if (kk + 3 < nb) prefetch(kk + 3);
+                // D3 done (so D2 and D1 too) and the decays read: the Kb/M slot refills first
+                // (the next Delta waits for it), then slot kk % 2's lo half and e^m
+                if (!wait(mbar3, (uint32_t)kk & 1u)) break;
+                pend &= ~(1u << (2 * (kk & 1)));
                 if (kk + 1 < nb) {
-                    if (!wait(mbar3, (uint32_t)kk & 1u) || !wait(bar_u, (uint32_t)kk & 1u)) break;
+                    if (!wait(bar_u, (uint32_t)kk & 1u)) break;
                     load_ktm(kk + 1);
                 }
-                // staged outputs imply D1 and D3 of kk are done
+                if (kk + 2 < nb) load_half(kk + 2, 0);
+                // the outputs of kk, staged in the slot's hi half, leave by one tensor store
                 if (!wait(out_st, (uint32_t)kk & 1u)) break;
-                wq_pend &= ~(1u << (kk & 1));
+                pend &= ~(1u << (2 * (kk & 1) + 1));
                 if (!(mode & kChainNoOut)) {
                     const uint32_t src = sbase + TC_WQ + kWqBytes * (kk & 1);
                     if (mode & kChainAccumOut) tma_reduce_add_4d(&out_map, src, 0, h, (n0 + kk) * kC, b);
@@ -1181,15 +1193,17 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                     bulk_commit();
                 }
                 if (kk + 2 < nb) {
-                    bulk_wait_read();                  // the outputs have left the slot
-                    load_wq(kk + 2);
+                    bulk_wait_read();                  // the outputs have left the hi half
+                    load_half(kk + 2, 1);
                 }
             }
             bulk_wait_read();
             if (*sFail) {
                 // let the copies still in flight land before shared memory is released
                 for (int sl = 0; sl < 2; ++sl)
-                    if ((wq_pend >> sl) & 1u) mbar_wait(mbar_wq0 + 8u * sl, (wq_par >> sl) & 1u);
+                    for (int hi = 0; hi < 2; ++hi)
+                        if ((pend >> (2 * sl + hi)) & 1u)
+                            mbar_wait((hi ? wq_hi0 : wq_lo0) + 8u * sl, (par_bits >> (2 * sl + hi)) & 1u);
                 if (ktm_pending) mbar_wait(mbar_ktm, ktm_par);
             }
         }
@@ -1207,7 +1221,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                    : s_in ? s_in[((size_t)bh * kDK + i0 + j) * kDV + c] : 0.f;
         // S'^T = S^T Diag(e^m) of chunk kk as the hi/lo A operand (pairs of key channels)
         auto put_s = [&](int kk) -> bool {
-            if (!wait(mbar_wq0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u)) return false;
+            if (!wait(wq_lo0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u)) return false;
             const float4 *em4 = reinterpret_cast<const float4 *>(smem + TC_WQ + kWqBytes * (kk & 1) + 65536u) + i0 / 4;
             uint32_t hv[16], lv[16];
 #pragma unroll
@@ -1260,7 +1274,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
             // the next chunk's S'^T = S^T Diag(e^m') (its e^m arrived two chunks ahead)
             if (!(ok = wait(mbar2, par))) break;
             const bool next = kk + 1 < nb;
-            if (next && !(ok = wait(mbar_wq0 + 8u * ((kk + 1) & 1), (uint32_t)((kk + 1) >> 1) & 1u))) break;
+            if (next && !(ok = wait(wq_lo0 + 8u * ((kk + 1) & 1), (uint32_t)((kk + 1) >> 1) & 1u))) break;
             tc_fence_after();
             {
                 const float4 *em4 =
