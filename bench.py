@@ -74,11 +74,12 @@ MEASURED_TRAFFIC = {
     # the long-context launch by token-heads processed (the kernel streams its inputs once)
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
     ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
-    # two-kernel prefill, one kda_forward_ws call (prep + chain), captured on B1 H32 T8192
-    # (prep 342.6 + 576.9 MB, chain 610.4 + 117.2 MB) and scaled by 8 to T = 65536: every
+    # two-kernel prefill, one kda_forward_ws call with the pipelined schedule (two blocks
+    # of 64 chunks: prep 169.4 + 247.6 and 169.5 + 244.8 MB, per-head chain 305.3 + 50.9
+    # and 307.3 + 50.6 MB), captured on B1 H32 T8192 and scaled by 8 to T = 65536: every
     # term (inputs, chunk records, outputs) grows with the token count
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("8af6b29bc6e2697e", 8 * 1647.1e6),
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("8af6b29bc6e2697e", 1647.1e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("b4492d60b8c3b70b", 8 * 1545.4e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("b4492d60b8c3b70b", 1545.4e6),
 }
 
 
@@ -770,8 +771,13 @@ def main(argv=None):
     achieved = alg_bytes / (ms_launch / 1e3) / 1e9
     tc = (w.dtype == "bf16" and w.dk == 128 and w.dv == 128)   # the library's dispatch rule
     kname, ksrc = ("prefill_tc_kernel", "kda_prefill_tc.cu") if tc else ("prefill_simt_kernel", "kda_prefill_simt.cu")
+    # the library's schedule rule: few heads (2 B H <= SMs) and >= 128 chunks pipeline the
+    # chunk-local kernel beside a per-head chain; else the chain runs after it
+    pipelined = split and 2 * w.B * w.H <= torch.cuda.get_device_properties(device).multi_processor_count \
+        and (w.T + 63) // 64 >= 128
     if split:
-        kname, ksrc = "prefill_prep_kernel + prefill_chain_kernel", "kda_prefill_split.cu"
+        kname, ksrc = ("prefill_prep_kernel + prefill_chain_t_kernel (pipelined)" if pipelined
+                       else "prefill_prep_kernel + prefill_chain_kernel"), "kda_prefill_split.cu"
     traffic = measured_traffic(ksrc, w.name)
     alg_flops = w.B * w.T * w.H * prefill_flops_per_token_head(w.dk)
     roofline = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
@@ -799,8 +805,11 @@ def main(argv=None):
             "dtype": "bf16" if tc else "f32", "data": "synthetic",
             "arithmetic": ("tcgen05 bf16 products of hi/lo-split operands (3 terms), fp32 accumulation "
                            "in tensor memory, fp32 CUDA-core solve and scans") if tc else "fp32 CUDA cores",
-            "path": ("two kernels per call (chunk-local records in a %.2f GB caller workspace, then the "
-                     "state chain)" % (ws_bytes / 1e9)) if split else "one fused kernel per call",
+            "path": (("two kernels per block of 64 chunks, pipelined: the per-head state chain of block i "
+                      "beside the chunk-local kernel of block i+1 (records in two slots of a %.2f GB caller "
+                      "workspace)" if pipelined else
+                      "two kernels per call (chunk-local records in a %.2f GB caller workspace, then the "
+                      "state chain)") % (ws_bytes / 1e9)) if split else "one fused kernel per call",
             "config": {"workload": w.name, "B": w.B, "T": w.T, "H": w.H, "dk": w.dk, "dv": w.dv,
                        "input_dtype": w.dtype, "chunk": 64, "final_state": w.final_state,
                        "l2": "no flush: inputs %.2f GB per step > 126 MB L2" % (alg_bytes / 1e9),
