@@ -497,6 +497,40 @@ def _add_decode(line, args, rank, world, device, hbm):
                 "steps": dec["e2e_steps"]}}
 
 
+def _add_noalloc(line, args, w, world, device, hbm):
+    """The long-context prefill without a caller workspace: kda_forward (the one-kernel
+    fused prefill) and kda_forward_noalloc (the two-kernel prefill on the library's
+    static scratch), each timed like the headline."""
+    import torch
+    import gated_delta_rule_109_b200 as kda
+    from gated_delta_rule_109_b200 import inputs as I
+    x = I.make_inputs(w, device)
+    args_ = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+    out = torch.empty((w.B, w.T, w.H, w.dv), dtype=torch.float32, device=device)
+    sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
+    res = {}
+    alg = (w.B * w.T * w.H * prefill_bytes_per_token_head(w.dk, w.dv, 2) + 4 * w.B * w.H * w.dk * w.dv)
+    for name, fn in (("kda_forward", kda.forward), ("kda_forward_noalloc", kda.forward_noalloc)):
+        for _ in range(args.warmup):
+            fn(*args_, out=out, final_state=sT)
+        torch.cuda.synchronize(device)
+        kda.check_status(device)
+        stream = torch.cuda.current_stream(device)
+        K = max(3, min(args.steps, 5))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(device)
+        e0.record(stream)
+        for _ in range(K):
+            fn(*args_, out=out, final_state=sT)
+        e1.record(stream)
+        torch.cuda.synchronize(device)
+        ms = max_over_ranks(e0.elapsed_time(e1), device) / K
+        res[name] = {"ms_per_call": ms, "value": w.B * w.T * world / (ms / 1e3), "unit": "tokens/s",
+                     "roofline_frac": alg / (ms / 1e3) / 1e9 / hbm}
+    res["scratch_bytes"] = kda.noalloc_scratch_bytes()
+    line["noalloc_prefill"] = res
+
+
 def _add_gdn(line, args, w, world, device, hbm, use_workspace=True):
     """The Gated DeltaNet specialisation timed on the same workload shape (the
     two-kernel path with a workspace when the shape has one)."""
@@ -828,6 +862,8 @@ def main(argv=None):
         _add_decode(line, args, rank, world, device, hbm)
     if not args.no_variants and args.only == "all":
         _add_other_prefills(line, args, world, device, hbm, rank)
+        if ws_bytes:
+            _add_noalloc(line, args, w, world, device, hbm)
         _add_gdn(line, args, w, world, device, hbm)
         if ws_bytes:
             _add_raw(line, args, w, world, device, hbm)
