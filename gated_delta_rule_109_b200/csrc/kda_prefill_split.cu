@@ -1035,7 +1035,10 @@ prefill_chain_kernel(const uint8_t *__restrict__ ws, const float *s_in,
 // chunk's D1 by a third); the slot's lo half and e^m are refilled as soon as D1 is
 // done, the hi half once the store has read it.  Warp 16 issues the products; warp 17 the record copies, the output stores
 // and L2 prefetches.  Handoffs are mbarriers (one arrival per compute warp):
-//   bar_s  S'^T of chunk kk is in tensor memory (and D1 of kk - 1 has been read back)
+//   bar_s  S'^T of chunk kk is in tensor memory (and D1 of kk - 1 has been read back):
+//          two barriers, the K steps of key channels 32 j + 0..15 (even) first, then
+//          32 j + 16..31 (odd), so that D1 starts on the first half while the second
+//          is still being split
 //   bar_d  Delta^T of chunk kk is in tensor memory (and D3 of kk - 1 has been read back)
 //   bar_u  the state update of chunk kk has read its decays from the Kb/M slot
 //   out_st the outputs of chunk kk are staged in its [Wr; Qr] slot (so D1 and D3 of kk
@@ -1050,7 +1053,8 @@ constexpr uint32_t TC_MBAR = TC_U + 32768;            // mma1, mma2, mma3, wq_lo
 constexpr uint32_t TC_FAIL = TC_MBAR + 88;
 constexpr uint32_t TC_TMEMP = TC_MBAR + 96;
 constexpr uint32_t TC_OUTST = TC_MBAR + 104;          // out_st
-constexpr uint32_t TC_TOTAL = TC_MBAR + 112;
+constexpr uint32_t TC_BARS1 = TC_MBAR + 112;          // bar_s1 (S'^T odd K steps)
+constexpr uint32_t TC_TOTAL = TC_MBAR + 120;
 static_assert(TC_TOTAL <= 232448, "shared memory");
 // tensor-memory columns (lane = value column)
 constexpr uint32_t TT_S = 0, TT_S_LO = 64;            // S'^T, bf16 pairs along dk: hi, lo
@@ -1069,7 +1073,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
     // region also stages the outputs
     const uint32_t mbar1 = sbase + TC_MBAR, mbar2 = mbar1 + 8, mbar3 = mbar1 + 16, wq_lo0 = mbar1 + 24;
     const uint32_t wq_hi0 = mbar1 + 40, mbar_ktm = mbar1 + 56, bar_s = mbar1 + 64, bar_d = mbar1 + 72;
-    const uint32_t bar_u = mbar1 + 80, out_st = sbase + TC_OUTST;
+    const uint32_t bar_u = mbar1 + 80, out_st = sbase + TC_OUTST, bar_s1 = sbase + TC_BARS1;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x;
@@ -1091,6 +1095,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
         mbar_init(wq_hi0 + 8, 1);
         mbar_init(mbar_ktm, 1);
         mbar_init(bar_s, 16);
+        mbar_init(bar_s1, 16);
         mbar_init(bar_d, 16);
         mbar_init(bar_u, 16);
         mbar_init(out_st, 16);
@@ -1121,7 +1126,13 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                 if (!wait(bar_s, par) || !wait(wq_hi0 + 8u * (kk & 1), (uint32_t)(kk >> 1) & 1u)) break;
                 tc_fence_after();
                 const uint32_t wq = sbase + TC_WQ + kWqBytes * (kk & 1);
-                mma_split_ta(tmem + TT_D1, tmem + TT_S, tmem + TT_S_LO, wq, wq + 32768u, RW_SI, RW_SO, kDK / 16, id1);
+                // the even K steps (key channels 32 j .. + 15) while the odd ones are split
+                mma_split_ta_steps(tmem + TT_D1, tmem + TT_S, tmem + TT_S_LO, wq, wq + 32768u, RW_SI, RW_SO, 0, 2,
+                                   kDK / 32, id1, false);
+                if (!wait(bar_s1, par)) break;
+                tc_fence_after();
+                mma_split_ta_steps(tmem + TT_D1, tmem + TT_S, tmem + TT_S_LO, wq, wq + 32768u, RW_SI, RW_SO, 1, 2,
+                                   kDK / 32, id1, true);
                 umma_commit(mbar1);
                 if (!wait(bar_d, par)) break;
                 tc_fence_after();
@@ -1235,7 +1246,10 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(bar_s);
+            if (lane == 0) {
+                mbar_arrive(bar_s);
+                mbar_arrive(bar_s1);
+            }
             return true;
         };
         // this thread's 16 outputs of chunk kk (value column c, tokens 16 g .. + 15): Qr S'
@@ -1263,12 +1277,14 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                 }
                 tmem_st8u(tmem + tlane + TT_DL + 8 * g, hv);
                 tmem_st8u(tmem + tlane + TT_DL_LO + 8 * g, lv);
-                tmem_ld16(tmem + tlane + TT_D1 + 64 + 16 * g, o);
                 tmem_wait_st();
             }
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(bar_d);
+            // Qr S' of this thread's outputs, read while D2 runs (D1's columns stay until the
+            // next chunk's D1, which waits for this chunk's S'^T handoff)
+            tmem_ld16(tmem + tlane + TT_D1 + 64 + 16 * g, o);
 
             // ---- S^T <- S^T Diag(e^{G_last}) + D2^T Diag(e^{G_last - m}), and in the same pass
             // the next chunk's S'^T = S^T Diag(e^m') (its e^m arrived two chunks ahead)
@@ -1303,16 +1319,14 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                     if (next) {
                         tmem_st8u(tmem + tlane + TT_S + 16 * g + 8 * hh, hv);
                         tmem_st8u(tmem + tlane + TT_S_LO + 16 * g + 8 * hh, lv);
+                        tmem_wait_st();
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(hh == 0 ? bar_s : bar_s1);
                     }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar_u);      // the decays are read: the Kb/M slot may refill
-                if (next) {
-                    tmem_wait_st();
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) mbar_arrive(bar_s);
-                }
             }
 
             // ---- O = Qr S' + M Delta of this chunk, staged row-major [token][value] in its

@@ -253,6 +253,28 @@ __device__ __forceinline__ void mma_split_ta(uint32_t d, uint32_t a_hi, uint32_t
     }
 }
 
+// The K steps ks0, ks0 + kstride, ... (kcount of them) of mma_split_ta, all three
+// terms; `accumulate` false starts D afresh with the first instruction.
+__device__ __forceinline__ void mma_split_ta_steps(uint32_t d, uint32_t a_hi, uint32_t a_lo, uint32_t b_hi,
+                                                   uint32_t b_lo, uint32_t b_lbo, uint32_t b_sbo, int ks0,
+                                                   int kstride, int kcount, uint32_t idesc, bool accumulate)
+{
+    const uint64_t db[2] = {smem_desc(b_hi, b_lbo, b_sbo), smem_desc(b_lo, b_lbo, b_sbo)};
+    const uint64_t sb = (2u * b_lbo) >> 4;
+    bool acc = accumulate;
+#pragma unroll
+    for (int tt = 0; tt < 3; ++tt) {
+        const uint32_t a = tt == 1 ? a_lo : a_hi;
+        const uint64_t b0 = db[tt == 2 ? 1 : 0];
+#pragma unroll
+        for (int i = 0; i < kcount; ++i) {
+            const int ks = ks0 + i * kstride;
+            umma_bf16_ta(d, a + 8u * (uint32_t)ks, b0 + sb * (uint64_t)ks, idesc, acc ? 1u : 0u);
+            acc = true;
+        }
+    }
+}
+
 // One product D (+)= A B on bf16 hi/lo split operands: hi*hi, plus lo*hi when A has
 // a lo part and hi*lo when B has one (an operand without a lo part is an exact
 // bf16 input).  Each term walks K in `ksteps` steps of 16 (two core matrices,
