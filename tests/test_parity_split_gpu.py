@@ -262,3 +262,37 @@ def test_forward_host_pageable_and_f32_and_empty():
     x0 = I.make_inputs(w0, "cpu")
     out0, s0 = kda.forward_host(*(x0[n] for n in NAMES), x0["initial_state"])
     assert out0.numel() == 0 and torch.equal(s0, x0["initial_state"])
+
+
+# ------------------------------------------------------------ the pipelined schedule
+def test_pipelined_schedule_every_workspace_size_bit_identical():
+    """Few heads and at least 128 chunks: blocks of 64 chunks with the per-head chain
+    beside the chunk-local kernel of the next block.  Batch > 1, a ragged tail and a
+    carried state; the pipelined workspace, the smallest one that still pipelines
+    (two blocks of 8 chunks), one below that (sequential blocks, same chain kernel)
+    and the whole sequence's records all give the same bits, within the bar of the
+    oracle."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE, B=2, H=3, T=8192 + 61, seed=3131)     # 130 chunks
+    x = I.make_inputs(w, "cuda")
+    bh, rec = w.B * w.H, kda.workspace_bytes(1, 64, 1, 128, 128)
+    state = bh * 128 * 128 * 4
+    best = kda.workspace_bytes(w.B, w.T, w.H, 128, 128)
+    assert best == 2 * 64 * bh * rec + state
+    out_p, s_p = _run(x, _ws(w))
+    _compare(x, out_p, s_p)
+    for nbytes in (2 * 8 * bh * rec + state, 2 * 8 * bh * rec + state - 256, 130 * bh * rec):
+        out_b, s_b = _run(x, _ws(w, nbytes))
+        assert torch.equal(out_p, out_b) and torch.equal(s_p, s_b), nbytes
+
+
+def test_pipelined_schedule_host_memory_path_bit_identical():
+    """kda_forward_host on a pipelined shape picks the same chain kernel as the device
+    call (the whole sequence's length decides), so the bits agree."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=2, T=8192 + 5, seed=3132)
+    x = I.make_inputs(w, "cuda")
+    out_d, s_d = _run(x, _ws(w))
+    host = {n: x[n].cpu().pin_memory() for n in NAMES}
+    out_h, s_h = kda.forward_host(*(host[n] for n in NAMES), x["initial_state"].cpu().pin_memory(),
+                                  block_tokens=2048)
+    kda.check_status()
+    assert torch.equal(out_h, out_d.cpu()) and torch.equal(s_h, s_d.cpu())
