@@ -498,9 +498,11 @@ def _add_decode(line, args, rank, world, device, hbm):
 
 
 def _add_noalloc(line, args, w, world, device, hbm):
-    """The long-context prefill without a caller workspace: kda_forward (the one-kernel
-    fused prefill) and kda_forward_noalloc (the two-kernel prefill on the library's
-    static scratch), each timed like the headline."""
+    """The long-context prefill without a caller workspace, each call timed like the
+    headline: kda_forward (the two-kernel prefill on a workspace from the library's
+    pool), kda_forward_ws with no workspace (the one-kernel prefill) and
+    kda_forward_noalloc (the two-kernel prefill on the library's static scratch)."""
+    import functools
     import torch
     import gated_delta_rule_109_b200 as kda
     from gated_delta_rule_109_b200 import inputs as I
@@ -510,7 +512,10 @@ def _add_noalloc(line, args, w, world, device, hbm):
     sT = torch.empty((w.B, w.H, w.dk, w.dv), dtype=torch.float32, device=device)
     res = {}
     alg = (w.B * w.T * w.H * prefill_bytes_per_token_head(w.dk, w.dv, 2) + 4 * w.B * w.H * w.dk * w.dv)
-    for name, fn in (("kda_forward", kda.forward), ("kda_forward_noalloc", kda.forward_noalloc)):
+    calls = (("kda_forward", kda.forward),
+             ("kda_forward_ws (no workspace: one kernel)", functools.partial(kda.forward, one_kernel=True)),
+             ("kda_forward_noalloc", kda.forward_noalloc))
+    for name, fn in calls:
         for _ in range(args.warmup):
             fn(*args_, out=out, final_state=sT)
         torch.cuda.synchronize(device)
@@ -528,6 +533,7 @@ def _add_noalloc(line, args, w, world, device, hbm):
         res[name] = {"ms_per_call": ms, "value": w.B * w.T * world / (ms / 1e3), "unit": "tokens/s",
                      "roofline_frac": alg / (ms / 1e3) / 1e9 / hbm}
     res["scratch_bytes"] = kda.noalloc_scratch_bytes()
+    res["pool_bytes"] = kda.workspace_pool_bytes(device)
     line["noalloc_prefill"] = res
 
 

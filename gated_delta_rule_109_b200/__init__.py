@@ -30,7 +30,8 @@ KDA_PREP_LOGSIGMOID_GATE, KDA_PREP_L2NORM_QK = 1, 2
 EXPORTS = ("kda_forward", "kda_forward_ws", "kda_forward_workspace_bytes",
            "kda_forward_workspace_min_bytes", "kda_segment_workspace_bytes", "kda_forward_raw", "kda_segment_local",
            "kda_segment_start_state", "kda_segment_correct", "kda_forward_noalloc",
-           "kda_forward_noalloc_scratch_bytes", "kda_forward_host", "kda_forward_host_workspace_bytes",
+           "kda_forward_noalloc_scratch_bytes", "kda_workspace_pool_bytes", "kda_workspace_pool_trim",
+           "kda_forward_host", "kda_forward_host_workspace_bytes",
            "kda_backward", "kda_backward_workspace_bytes",
            "kda_decode_step", "kda_gdn_forward", "kda_gdn_forward_ws", "kda_gdn_decode_step",
            "kda_status_string", "kda_check_status", "kda_selftest_timeout", "kda_last_cuda_error",
@@ -90,6 +91,10 @@ def load(path: Optional[str] = None) -> ctypes.CDLL:
     lib.kda_backward_workspace_bytes.restype = ctypes.c_size_t
     lib.kda_backward_workspace_bytes.argtypes = [i] * 5
     lib.kda_forward_noalloc_scratch_bytes.argtypes = []
+    lib.kda_workspace_pool_bytes.restype = ctypes.c_size_t
+    lib.kda_workspace_pool_bytes.argtypes = []
+    lib.kda_workspace_pool_trim.restype = i
+    lib.kda_workspace_pool_trim.argtypes = [vp]
     lib.kda_gdn_forward.restype = i
     lib.kda_gdn_forward.argtypes = [vp] * 8 + [i] * 6 + [f, vp]
     lib.kda_gdn_decode_step.restype = i
@@ -167,7 +172,7 @@ def _need_workspace(workspace, dev: torch.device, where: str):
 
 
 def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, final_state,
-             return_final_state, scale, workspace=None):
+             return_final_state, scale, workspace=None, one_kernel=False):
     lib = load()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -189,13 +194,17 @@ def _forward(entry, gate_shape, q, k, v, log_alpha, beta, initial_state, out, fi
         final_state = torch.empty((B, H, dk, dv), dtype=torch.float32, device=dev)
     if final_state is not None:
         _need(final_state, "final_state", (B, H, dk, dv), torch.float32, dev)
-    if workspace is not None:
-        _need_workspace(workspace, dev, entry)
+    if workspace is not None and one_kernel:
+        raise ValueError("%s: one_kernel takes no workspace" % entry)
+    if workspace is not None or one_kernel:
+        if workspace is not None:
+            _need_workspace(workspace, dev, entry)
         entry = entry + "_ws"
         st = getattr(lib, entry)(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
                                  _ptr(initial_state), _ptr(out), _ptr(final_state),
                                  B, T, H, dk, dv, code, float(scale), _ptr(workspace),
-                                 workspace.numel() * workspace.element_size(), _stream(dev))
+                                 0 if workspace is None else workspace.numel() * workspace.element_size(),
+                                 _stream(dev))
     else:
         fn = getattr(lib, entry)
         st = fn(_ptr(q), _ptr(k), _ptr(v), _ptr(log_alpha), _ptr(beta),
@@ -230,7 +239,7 @@ def _decode(entry, gate_shape, q, k, v, log_alpha, beta, state, out, scale):
 
 
 def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
-            return_final_state=True, scale: float = 0.0, workspace=None):
+            return_final_state=True, scale: float = 0.0, workspace=None, one_kernel=False):
     """Chunked KDA prefill (``kda_forward``, or ``kda_forward_ws`` with a workspace).
 
     q, k ``[B,T,H,dk]`` and v ``[B,T,H,dv]`` (bf16 or fp32, one dtype);
@@ -239,11 +248,13 @@ def forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_sta
     final_state [B,H,dk,dv] fp32 or None)``.  ``final_state`` may be passed as
     the same tensor as ``initial_state`` to carry the state in place.
     ``scale`` 0 means 1/sqrt(dk).  ``workspace``: a contiguous device tensor
-    (see :func:`workspace_bytes` / :func:`make_workspace`) enabling the
-    two-kernel prefill for bf16 inputs with dk = dv = 128.
+    (see :func:`workspace_bytes` / :func:`make_workspace`) for the two-kernel
+    prefill (bf16 inputs, dk = dv = 128); without one, ``kda_forward`` takes it
+    from the library's pool.  ``one_kernel``: ``kda_forward_ws`` with no
+    workspace, the one-kernel prefill that needs no memory beyond its arguments.
     """
     return _forward("kda_forward", lambda B, T, H, dk: (B, T, H, dk), q, k, v, log_alpha, beta,
-                    initial_state, out, final_state, return_final_state, scale, workspace)
+                    initial_state, out, final_state, return_final_state, scale, workspace, one_kernel)
 
 
 def forward_raw(q, k, v, gate, beta, initial_state=None, *, workspace, logsigmoid_gate=True,
@@ -474,6 +485,24 @@ def noalloc_scratch_bytes() -> int:
     return int(load().kda_forward_noalloc_scratch_bytes())
 
 
+def workspace_pool_bytes(device=None) -> int:
+    """Device memory held by the workspace pool of ``kda_forward`` on ``device``
+    (``kda_workspace_pool_bytes``)."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _on_cuda(dev, "kda_workspace_pool_bytes")
+    with torch.cuda.device(dev):
+        return int(load().kda_workspace_pool_bytes())
+
+
+def workspace_pool_trim(device=None):
+    """Return the pool's unused memory to the device (``kda_workspace_pool_trim``),
+    after the work enqueued on the current stream."""
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+    _on_cuda(dev, "kda_workspace_pool_trim")
+    with torch.cuda.device(dev):
+        _check(load().kda_workspace_pool_trim(_stream(dev)), "kda_workspace_pool_trim")
+
+
 def workspace_bytes(B, T, H, dk, dv, dtype=torch.bfloat16, minimum=False, segment=False) -> int:
     """Workspace size for :func:`forward` (``kda_forward_workspace_bytes`` /
     ``..._min_bytes``), or with ``segment`` for :func:`segment_local` and
@@ -506,7 +535,7 @@ def decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0
 
 
 def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final_state=None,
-                return_final_state=True, scale: float = 0.0, workspace=None):
+                return_final_state=True, scale: float = 0.0, workspace=None, one_kernel=False):
     """Chunked prefill of Gated DeltaNet / DeltaNet (``kda_gdn_forward``, or
     ``kda_gdn_forward_ws`` with a workspace).
 
@@ -515,7 +544,7 @@ def gdn_forward(q, k, v, log_alpha, beta, initial_state=None, *, out=None, final
     """
     shape = None if log_alpha is None else (lambda B, T, H, dk: (B, T, H))
     return _forward("kda_gdn_forward", shape, q, k, v, log_alpha, beta, initial_state, out,
-                    final_state, return_final_state, scale, workspace)
+                    final_state, return_final_state, scale, workspace, one_kernel)
 
 
 def gdn_decode_step(q, k, v, log_alpha, beta, state, *, out=None, scale: float = 0.0):

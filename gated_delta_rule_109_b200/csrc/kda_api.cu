@@ -39,6 +39,44 @@ struct ScratchSlot {
 ScratchSlot g_scratch[kMaxDevices];
 std::mutex g_scratch_mu;
 
+// Workspace of kda_forward and kda_gdn_forward: one stream-ordered memory pool per
+// device, owned by the library.  A call takes its workspace from the pool on its
+// stream and gives it back on the same stream once its kernels are enqueued; the
+// pool keeps up to kPoolKeep bytes between calls, so that after the first call of
+// a shape the allocation is a lookup.  A call asks for at most kPoolKeep bytes
+// unless the smallest workspace of its shape is larger.
+constexpr size_t kPoolKeep = size_t(1) << 30;
+cudaMemPool_t g_pool[kMaxDevices] = {};
+std::mutex g_pool_mu;
+
+cudaError_t device_pool(bool create, cudaMemPool_t *out)
+{
+    *out = nullptr;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lock(g_pool_mu);
+    if (!g_pool[dev] && create) {
+        cudaMemPoolProps props;
+        memset(&props, 0, sizeof(props));
+        props.allocType = cudaMemAllocationTypePinned;
+        props.handleTypes = cudaMemHandleTypeNone;
+        props.location.type = cudaMemLocationTypeDevice;
+        props.location.id = dev;
+        cudaMemPool_t pool = nullptr;
+        if ((e = cudaMemPoolCreate(&pool, &props)) != cudaSuccess) return e;
+        uint64_t keep = kPoolKeep;
+        if ((e = cudaMemPoolSetAttribute(pool, cudaMemPoolAttrReleaseThreshold, &keep)) != cudaSuccess) {
+            cudaMemPoolDestroy(pool);
+            return e;
+        }
+        g_pool[dev] = pool;
+    }
+    *out = g_pool[dev];
+    return cudaSuccess;
+}
+
 }  // namespace
 
 void kda::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
@@ -135,6 +173,41 @@ kda_status forward_impl(const void *q, const void *k, const void *v, const float
     return e == cudaSuccess ? KDA_OK : cuda_fail(e);
 }
 
+// kda_forward / kda_gdn_forward: the two-kernel prefill on a workspace from the
+// library's pool where it applies (bf16, dk = dv = 128); the one-kernel prefill,
+// which needs no memory beyond its arguments, for other shapes or when the pool
+// cannot supply the workspace.
+kda_status forward_pooled(const void *q, const void *k, const void *v, const float *log_alpha,
+                          const float *beta, const float *initial_state, float *out, float *final_state,
+                          int B, int T, int H, int dk, int dv, kda_dtype dtype, float scale,
+                          void *stream, kda::GateKind gate)
+{
+    g_last_cuda_error[0] = '\0';
+    const kda_status vs = validate_forward(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H,
+                                           dk, dv, dtype, scale, gate, nullptr);
+    if (vs != KDA_OK) return vs;
+    if (T == 0 || dtype != KDA_BF16 || dk != 128 || dv != 128)
+        return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv, dtype,
+                            scale, stream, gate);
+    const size_t want = std::max(std::min(kda::prefill_split_workspace_best(B, T, H), kPoolKeep),
+                                 kda::prefill_split_workspace_min(B, T, H));
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = device_pool(true, &pool);
+    if (e != cudaSuccess) return cuda_fail(e);
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    void *ws = nullptr;
+    if (cudaMallocFromPoolAsync(&ws, want, pool, st) != cudaSuccess) {
+        cudaGetLastError();             // no room for the workspace: the one-kernel prefill
+        return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv, dtype,
+                            scale, stream, gate);
+    }
+    const kda_status rs = forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk,
+                                       dv, dtype, scale, stream, gate, ws, want);
+    e = cudaFreeAsync(ws, st);          // after every kernel of the call (they join the caller's stream)
+    if (rs != KDA_OK) return rs;
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
 kda_status decode_impl(const void *q, const void *k, const void *v, const float *log_alpha,
                        const float *beta, float *state_inout, float *out, int B, int H, int dk, int dv,
                        kda_dtype dtype, float scale, void *stream, kda::GateKind gate)
@@ -214,8 +287,8 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
                        int B, int T, int H, int dk, int dv,
                        kda_dtype dtype, float scale, void *stream)
 {
-    return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
-                        dtype, scale, stream, kda::KDA_GATE_CHANNEL);
+    return forward_pooled(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                          dtype, scale, stream, kda::KDA_GATE_CHANNEL);
 }
 
 kda_status kda_forward_raw(const void *q, const void *k, const void *v,
@@ -365,6 +438,34 @@ kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
 
 size_t kda_forward_noalloc_scratch_bytes(void) { return kScratchBytes; }
 
+size_t kda_workspace_pool_bytes(void)
+{
+    cudaMemPool_t pool = nullptr;
+    if (device_pool(false, &pool) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    uint64_t held = 0;
+    if (!pool || cudaMemPoolGetAttribute(pool, cudaMemPoolAttrReservedMemCurrent, &held) != cudaSuccess) {
+        cudaGetLastError();
+        return 0;
+    }
+    return (size_t)held;
+}
+
+kda_status kda_workspace_pool_trim(void *stream)
+{
+    g_last_cuda_error[0] = '\0';
+    cudaMemPool_t pool = nullptr;
+    cudaError_t e = device_pool(false, &pool);
+    if (e != cudaSuccess) return cuda_fail(e);
+    if (!pool) return KDA_OK;
+    // the calls already enqueued on the stream give their workspaces back first
+    if ((e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream))) != cudaSuccess) return cuda_fail(e);
+    e = cudaMemPoolTrimTo(pool, 0);
+    return e == cudaSuccess ? KDA_OK : cuda_fail(e);
+}
+
 kda_status kda_decode_step(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,
                            float *state_inout, float *out,
@@ -381,8 +482,8 @@ kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
                            int B, int T, int H, int dk, int dv,
                            kda_dtype dtype, float scale, void *stream)
 {
-    return forward_impl(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
-                        dtype, scale, stream, log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
+    return forward_pooled(q, k, v, log_alpha, beta, initial_state, out, final_state, B, T, H, dk, dv,
+                          dtype, scale, stream, log_alpha ? kda::KDA_GATE_SCALAR : kda::KDA_GATE_NONE);
 }
 
 kda_status kda_gdn_forward_ws(const void *q, const void *k, const void *v,

@@ -20,7 +20,9 @@
  * --------------------------------
  * - All tensor arguments are DEVICE pointers to dense, contiguous, row-major
  *   arrays on the current CUDA device.  The caller owns and allocates every
- *   buffer; the library allocates no device memory.
+ *   buffer.  The library's own device memory is the workspace pool of
+ *   kda_forward and kda_gdn_forward (see kda_forward) and the fixed scratch of
+ *   kda_forward_noalloc; every other call uses only what it is given.
  * - The state is stored as [dk, dv] per head (key channels are rows, the value
  *   axis is contiguous).  The pages write the same matrix as (d_v, d_k); this
  *   is its transpose, so the per-channel decay scales rows.
@@ -86,6 +88,17 @@ typedef enum kda_dtype {
  * Supported head dimensions: dk, dv in {64, 128} for both dtypes.  T = 0
  * writes no output and sets final_state to initial_state (or zeros).
  * q, k, v, log_alpha, beta and out may be NULL only when T = 0.
+ *
+ * Schedule: with bf16 inputs and dk = dv = 128 the call is kda_forward_ws on a
+ * workspace the library takes from its own stream-ordered memory pool (one
+ * per device, created on first use) and gives back on `stream` once the
+ * call's kernels are enqueued, so results are bit-identical to kda_forward_ws.
+ * The workspace is kda_forward_workspace_bytes() capped at 1 GiB (never below
+ * kda_forward_workspace_min_bytes()); the pool keeps up to 1 GiB between
+ * calls (kda_workspace_pool_bytes, kda_workspace_pool_trim).  If the pool
+ * cannot supply it, and for other dtypes or head dimensions, the call runs the
+ * one-kernel prefill, which needs no device memory beyond its arguments (what
+ * kda_forward_ws does with no workspace).
  */
 kda_status kda_forward(const void *q, const void *k, const void *v,
                        const float *log_alpha, const float *beta,
@@ -124,8 +137,10 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
  *   workspace_bytes  its size in bytes.
  *
  * With a NULL or too small workspace, or for other dtypes and head dimensions,
- * the call is exactly kda_forward.  A workspace not 256-byte aligned is
- * KDA_ERR_MISALIGNED.
+ * the call runs the one-kernel prefill: each (b, h) walks its chunks in one CTA
+ * that computes the chunk-local quantities and carries the state, using no
+ * device memory beyond the call's arguments.  A workspace not 256-byte aligned
+ * is KDA_ERR_MISALIGNED.
  */
 kda_status kda_forward_ws(const void *q, const void *k, const void *v,
                           const float *log_alpha, const float *beta,
@@ -254,7 +269,8 @@ kda_status kda_segment_correct(const float *start, const float *local_final, flo
  * so the sequence runs in blocks of as many 64-token chunks as fit it (results
  * are bit-identical to kda_forward_ws with a workspace of that size).  When a
  * single chunk of every (b, h) plus the carried state does not fit, and for
- * other dtypes or head dimensions, the call is kda_forward.  Calls that use the
+ * other dtypes or head dimensions, the call runs the one-kernel prefill
+ * (kda_forward_ws with no workspace).  Calls that use the
  * scratch on one device are ordered by the library (an event per device), on
  * any streams; they run one after another.
  */
@@ -266,6 +282,19 @@ kda_status kda_forward_noalloc(const void *q, const void *k, const void *v,
 
 /* Size in bytes of the scratch kda_forward_noalloc uses on each device. */
 size_t kda_forward_noalloc_scratch_bytes(void);
+
+/*
+ * The workspace pool of kda_forward and kda_gdn_forward on the current device.
+ *
+ * kda_workspace_pool_bytes -- device memory the pool holds now (in use by
+ *   calls in flight or kept for the next ones); 0 before the first call.
+ * kda_workspace_pool_trim -- waits for the work enqueued on `stream`, then
+ *   returns to the device every byte of the pool that no call still uses
+ *   (workspaces of calls in flight on other streams stay).  A later call
+ *   takes memory again.  KDA_OK when there is no pool yet.
+ */
+size_t kda_workspace_pool_bytes(void);
+kda_status kda_workspace_pool_trim(void *stream);
 
 /*
  * kda_decode_step -- one token per sequence, state updated in place.
@@ -310,7 +339,8 @@ kda_status kda_decode_step(const void *q, const void *k, const void *v,
  *   initial_state, out, final_state: as for kda_forward.
  *
  * log_alpha must be finite and <= 0 (alpha in (0, 1]).  Everything else --
- * sizes, head dimensions, aliasing, T = 0, statuses -- is as for kda_forward.
+ * sizes, head dimensions, aliasing, T = 0, statuses, the pooled workspace and
+ * the one-kernel fallback -- is as for kda_forward.
  */
 kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
                            const float *log_alpha, const float *beta,
@@ -323,7 +353,8 @@ kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
  * as kda_forward_ws is to kda_forward: bf16 with dk = dv = 128 and a workspace of
  * at least kda_forward_workspace_min_bytes(B, T, H, dk, dv, dtype) bytes (256-byte
  * aligned) take the two-kernel prefill, with each token's scalar decay (or none)
- * staged in every key channel; anything else is kda_gdn_forward.  Same arguments,
+ * staged in every key channel; anything else runs the one-kernel scalar-gate
+ * prefill, which needs no device memory beyond its arguments.  Same arguments,
  * statuses and results as kda_gdn_forward.
  */
 kda_status kda_gdn_forward_ws(const void *q, const void *k, const void *v,

@@ -6,9 +6,10 @@ of B256 H32.  Here the same calls, on the same seeded inputs, are compared
 with the fp64 oracle on ALL of their outputs and final states:
 
 * prefill: every (b, h) of every token, through each prefill entry point of
-  the C ABI (``kda_forward_ws`` with the whole-sequence workspace, which the
-  benchmark times; ``kda_forward``; ``kda_forward_noalloc``), against one
-  oracle run per workload;
+  the C ABI (``kda_forward_ws`` with the fastest workspace, which the
+  benchmark times; ``kda_forward`` on its pooled workspace; ``kda_forward_ws``
+  with no workspace, the one-kernel prefill; ``kda_forward_noalloc``),
+  against one oracle run per workload;
 * decode: the output of every one of the 1024 steps for every sequence and
   head, and the state after the last step.  A decode step is one token of the
   recurrence, so the oracle runs each group of sequences through all 1024
@@ -79,6 +80,8 @@ def _prefill_paths(w, x):
     del ws
     torch.cuda.empty_cache()
     res["kda_forward"] = kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+    res["kda_forward_ws (no workspace: one kernel)"] = kda.forward(
+        x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"], one_kernel=True)
     res["kda_forward_noalloc"] = kda.forward_noalloc(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"],
                                                      x["initial_state"])
     torch.cuda.synchronize()

@@ -63,12 +63,18 @@ for gate in ("scalar", "none"):
 SWEEP += [("scalar", "bf16", 128, 64, 100, 2, 3, True), ("scalar", "f32", 64, 128, 100, 2, 3, True)]
 
 
-@pytest.mark.parametrize("gate,dt,dk,dv,T,B,H,state", SWEEP)
-def test_gdn_shape_sweep(gate, dt, dk, dv, T, B, H, state):
+# kda_gdn_forward takes the two-kernel prefill on a pooled workspace for bf16 with
+# dk = dv = 128; the one-kernel scalar-gate prefill is swept on those shapes too
+PATHS = [(case, False) for case in SWEEP]
+PATHS += [(case, True) for case in SWEEP if case[1:4] == ("bf16", 128, 128)]
+
+
+@pytest.mark.parametrize("gate,dt,dk,dv,T,B,H,state,one_kernel", [c + (o,) for c, o in PATHS])
+def test_gdn_shape_sweep(gate, dt, dk, dv, T, B, H, state, one_kernel):
     w = I.scaled(I.PREFILL_B4_T16K_STATE if state else I.PREFILL_H16_T4K,
                  B=B, H=H, T=T, dk=dk, dv=dv, dtype=dt, seed=2000 + T + dk)
     x = _inputs(w, gate)
-    out, sT = _run(x)
+    out, sT = _run(x, one_kernel=one_kernel)
     _compare(dt, x, out, sT)
 
 
@@ -104,10 +110,10 @@ def test_gdn_matches_kda_with_broadcast_gate():
 
 
 # ------------------------------------------------------------ edge values
-@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("dt,one_kernel", [("bf16", False), ("bf16", True), ("f32", False)])
 @pytest.mark.parametrize("case", ["decay_minus5", "forget_all_minus100", "tiny_decay", "beta0", "beta1",
                                   "mixed_extreme"])
-def test_gdn_extreme_gates(dt, case):
+def test_gdn_extreme_gates(dt, one_kernel, case):
     w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=2, T=200, dtype=dt, seed=32)
     x = _inputs(w)
     if case == "decay_minus5":
@@ -123,7 +129,7 @@ def test_gdn_extreme_gates(dt, case):
     elif case == "mixed_extreme":
         x["g"][:, 64:128] = -3.0
         x["g"][:, 130:133] = -60.0
-    out, sT = _run(x)
+    out, sT = _run(x, one_kernel=one_kernel)
     assert torch.isfinite(out).all() and torch.isfinite(sT).all()
     _compare(dt, x, out, sT)
 

@@ -26,10 +26,10 @@ def _built():
     build.build()
 
 
-def _run_gpu(x, with_state_out=True, initial_state="input"):
+def _run_gpu(x, with_state_out=True, initial_state="input", one_kernel=False):
     s0 = x["initial_state"] if initial_state == "input" else initial_state
     out, sT = kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], s0,
-                          return_final_state=with_state_out)
+                          return_final_state=with_state_out, one_kernel=one_kernel)
     torch.cuda.synchronize()
     kda.check_status()
     return out, sT
@@ -114,12 +114,18 @@ for dt in ("bf16", "f32"):
 SWEEP += [("bf16", 128, 64, 100, 2, 3, True), ("f32", 64, 128, 100, 2, 3, True)]
 
 
-@pytest.mark.parametrize("dt,dk,dv,T,B,H,state", SWEEP)
-def test_shape_sweep(dt, dk, dv, T, B, H, state):
+# kda_forward takes the two-kernel prefill on a pooled workspace for bf16 with
+# dk = dv = 128; the one-kernel prefill (no workspace) is swept on those shapes too
+PATHS = [(case, False) for case in SWEEP]
+PATHS += [(case, True) for case in SWEEP if case[:3] == ("bf16", 128, 128)]
+
+
+@pytest.mark.parametrize("dt,dk,dv,T,B,H,state,one_kernel", [c + (o,) for c, o in PATHS])
+def test_shape_sweep(dt, dk, dv, T, B, H, state, one_kernel):
     w = I.scaled(I.PREFILL_B4_T16K_STATE if state else I.PREFILL_H16_T4K,
                  B=B, H=H, T=T, dk=dk, dv=dv, dtype=dt, seed=1000 + T + dk)
     x = I.make_inputs(w, "cuda")
-    out, sT = _run_gpu(x)
+    out, sT = _run_gpu(x, one_kernel=one_kernel)
     _compare(w, x, out, sT)
 
 
@@ -166,10 +172,10 @@ def test_split_sequence_carry_matches_single_pass():
 
 
 # ------------------------------------------------------------ edge values
-@pytest.mark.parametrize("dt", ["bf16", "f32"])
+@pytest.mark.parametrize("dt,one_kernel", [("bf16", False), ("bf16", True), ("f32", False)])
 @pytest.mark.parametrize("case", ["decay_minus5", "near_threshold", "no_decay", "beta0", "beta1",
                                   "mixed_extreme"])
-def test_extreme_gates(dt, case):
+def test_extreme_gates(dt, one_kernel, case):
     w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=2, T=200, dtype=dt, seed=31)
     x = I.make_inputs(w, "cuda")
     if case == "decay_minus5":
@@ -187,7 +193,7 @@ def test_extreme_gates(dt, case):
         # one chunk of very strong forgetting in the middle of mild ones
         x["log_alpha"][:, 64:128] = -3.0
         x["log_alpha"][:, 128:140, :, :7] = -20.0
-    out, sT = _run_gpu(x)
+    out, sT = _run_gpu(x, one_kernel=one_kernel)
     assert torch.isfinite(out).all() and torch.isfinite(sT).all()
     _compare(w, x, out, sT)
 
@@ -248,19 +254,60 @@ def test_deterministic():
 
 
 def test_no_device_memory_grows_with_sequence_length():
-    """The library allocates nothing: free device memory is unchanged by a call,
-    whatever T (the fixed-state property measured on the first page's demo)."""
+    """Device memory does not grow with T (the fixed-state property measured on the
+    first page's demo): the one-kernel prefill takes nothing, and kda_forward's
+    pooled workspace is two blocks of 64 chunks once the sequence is long enough,
+    whatever T; a repeated call of a shape takes no new memory."""
+    kda.workspace_pool_trim()
+    assert kda.workspace_pool_bytes() == 0
     for T in (4096, 16384, 65536):
         w = I.scaled(I.PREFILL_H16_T4K, H=4, T=T, seed=3)
         x = I.make_inputs(w, "cuda")
         out = torch.empty((1, T, 4, 128), device="cuda")
         sT = torch.empty((1, 4, 128, 128), device="cuda")
-        kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, out=out, final_state=sT)
-        torch.cuda.synchronize()
-        free0 = torch.cuda.mem_get_info()[0]
-        kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, out=out, final_state=sT)
-        torch.cuda.synchronize()
-        assert torch.cuda.mem_get_info()[0] == free0
+        for one_kernel in (True, False):
+            kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, out=out, final_state=sT,
+                        one_kernel=one_kernel)
+            torch.cuda.synchronize()
+            free0 = torch.cuda.mem_get_info()[0]
+            kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None, out=out, final_state=sT,
+                        one_kernel=one_kernel)
+            torch.cuda.synchronize()
+            assert torch.cuda.mem_get_info()[0] == free0, (T, one_kernel)
+    # pipelined sizes do not depend on T; the pool holds the two shapes' workspaces
+    ws_long = kda.workspace_bytes(1, 65536, 4, 128, 128)
+    assert ws_long == kda.workspace_bytes(1, 16384, 4, 128, 128)
+    held = kda.workspace_pool_bytes()
+    assert ws_long <= held <= kda.workspace_bytes(1, 4096, 4, 128, 128) + ws_long + (64 << 20)
+    free_before = torch.cuda.mem_get_info()[0]
+    kda.workspace_pool_trim()
+    assert kda.workspace_pool_bytes() == 0
+    assert torch.cuda.mem_get_info()[0] >= free_before + held // 2
+
+
+def test_pooled_workspace_is_capped_and_shared_by_streams():
+    """A shape whose fastest workspace is above 1 GiB runs in blocks within 1 GiB
+    (bit-identical to the full workspace); calls on two streams take their own
+    workspaces from the pool."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE, B=4, H=32, T=8192, seed=13)
+    assert kda.workspace_bytes(w.B, w.T, w.H, 128, 128) > (1 << 30)
+    x = I.make_inputs(w, "cuda")
+    ws = kda.make_workspace(w.B, w.T, w.H, 128, 128)
+    o_ws, s_ws = kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"], workspace=ws)
+    del ws
+    kda.workspace_pool_trim()
+    o_p, s_p = _run_gpu(x)
+    assert torch.equal(o_p, o_ws) and torch.equal(s_p, s_ws)
+    assert kda.workspace_pool_bytes() <= (1 << 30) + (64 << 20)
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    res = [None, None]
+    for i, st in enumerate(streams):
+        with torch.cuda.stream(st):
+            res[i] = kda.forward(x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], x["initial_state"])
+    torch.cuda.synchronize()
+    kda.check_status()
+    for o, s in res:
+        assert torch.equal(o, o_ws) and torch.equal(s, s_ws)
 
 
 def test_binding_rejects_mismatched_tensors():

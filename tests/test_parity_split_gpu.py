@@ -109,7 +109,7 @@ def test_too_small_workspace_takes_the_fused_kernel():
     x = I.make_inputs(w, "cuda")
     small = kda.workspace_bytes(w.B, w.T, w.H, 128, 128, minimum=True) - 256
     out, sT = _run(x, _ws(w, small))
-    ref_o, ref_s = _run(x, None)
+    ref_o, ref_s = _run(x, None, one_kernel=True)
     assert torch.equal(out, ref_o) and torch.equal(sT, ref_s)
 
 
@@ -151,7 +151,7 @@ def test_split_agrees_with_fused_kernel():
     w = I.scaled(I.PREFILL_B4_T16K_STATE, B=2, H=4, T=1000, seed=79)
     x = I.make_inputs(w, "cuda")
     out_s, s_s = _run(x, _ws(w))
-    out_f, s_f = _run(x, None)
+    out_f, s_f = _run(x, None, one_kernel=True)
     assert oracle.parity_error(out_s.cpu().numpy(), out_f.cpu().double().numpy()) <= 2 * TOL
     assert oracle.parity_error(s_s.cpu().numpy(), s_f.cpu().double().numpy()) <= 2 * TOL
 
@@ -262,6 +262,18 @@ def test_forward_host_pageable_and_f32_and_empty():
     x0 = I.make_inputs(w0, "cpu")
     out0, s0 = kda.forward_host(*(x0[n] for n in NAMES), x0["initial_state"])
     assert out0.numel() == 0 and torch.equal(s0, x0["initial_state"])
+
+
+# ------------------------------------------------------------ kda_forward without a workspace
+@pytest.mark.parametrize("B,H,T,state", [(1, 2, 8197, True), (2, 3, 200, True), (3, 4, 130, False)])
+def test_kda_forward_pooled_workspace_is_the_workspace_path(B, H, T, state):
+    """kda_forward takes the same schedule on a workspace from the library's pool:
+    bit-identical to kda_forward_ws with the fastest workspace."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE if state else I.PREFILL_H16_T4K, B=B, H=H, T=T, seed=9900 + T)
+    x = I.make_inputs(w, "cuda")
+    out_w, s_w = _run(x, _ws(w))
+    out_p, s_p = _run(x, None)
+    assert torch.equal(out_p, out_w) and torch.equal(s_p, s_w)
 
 
 # ------------------------------------------------------------ the pipelined schedule
