@@ -71,6 +71,14 @@ constexpr uint32_t R_M = R_KT + 32768, R_M_LO = R_M + 8192;
 constexpr uint32_t R_U = R_M + 16384, R_GAM = R_U + 32768, R_EL = R_GAM + 512;
 constexpr uint32_t kRec = R_EL + 512;
 static_assert(kRec % 16 == 0 && R_KT % 16 == 0, "bulk-copy alignment");
+// The chunk-local kernels stage U as the 256 rows (slice, token) of 128 bytes of one
+// TMA box with the 128-byte swizzle (16-byte piece j of row r at piece j ^ (r % 8)), so
+// that the 32 tokens a warp writes at once fall on distinct banks; the tensor store
+// writes the record's plain [slice][token][32] order.
+__device__ __forceinline__ uint32_t u_stage_off(int r, int j)
+{
+    return (uint32_t)r * 128u + ((uint32_t)(j ^ (r & 7)) << 4);
+}
 
 constexpr uint32_t RW_SO = 2048, RW_SI = 128;   // outer row or token (8 per group), inner dk (128)
 constexpr uint32_t H_SO = 1024, H_SI = 128;     // outer row, inner token (64)
@@ -107,11 +115,91 @@ static_assert(PP_GS + 64 * kGP * 4 <= PP_P_LO, "scan scratch");
 
 constexpr uint32_t TMP_AM = 0, TMP_W = 0, TMP_U = 128, TMP_COLS = 256;
 
+// T = (I + A)^-1 for a strictly lower triangular 64 x 64 fp32 A (row pitch kPitch),
+// by forward substitution on the four 16 x 16 diagonal blocks and recursive doubling
+// 16 -> 32 -> 64 (T21 = -T22 A21 T11 at each level), all in fp32.  Called by every
+// thread of a 256-thread CTA; A is overwritten with intermediate products, and T is
+// complete (every thread may read it) after the caller's next __syncthreads().
+__device__ __forceinline__ void unit_lower_inverse(float *__restrict__ Am, float *__restrict__ Tm, int tid)
+{
+    if (tid < 64) {
+        const int blk = tid >> 4, j = tid & 15, o = 16 * blk;
+        float xs[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            float s = (i == j) ? 1.f : 0.f;
+#pragma unroll
+            for (int l = 0; l < i; ++l) s -= Am[(o + i) * kPitch + o + l] * xs[l];
+            xs[i] = s;
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) Tm[(o + i) * kPitch + o + j] = xs[i];
+    } else {
+        for (int e = tid - 64; e < 6 * 256; e += kNT - 64) {
+            const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
+            const int rb = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
+            const int cb = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
+            Tm[(16 * rb + i) * kPitch + 16 * cb + j] = 0.f;
+        }
+    }
+    __syncthreads();
+    const int p = tid >> 6, i16 = (tid >> 2) & 15, jq = tid & 3;
+    if (tid < 128) {
+        const int a = 2 * p + 1, bb = 2 * p;
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {
+            const float av = Am[(16 * a + i16) * kPitch + 16 * bb + l];
+            const float4 tv = *reinterpret_cast<const float4 *>(Tm + (16 * bb + l) * kPitch + 16 * bb + 4 * jq);
+            y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
+        }
+        *reinterpret_cast<float4 *>(Am + (16 * bb + i16) * kPitch + 16 * a + 4 * jq) = y;
+    }
+    __syncthreads();
+    if (tid < 128) {
+        const int a = 2 * p + 1, bb = 2 * p;
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+        for (int l = 0; l < 16; ++l) {
+            const float tv = Tm[(16 * a + i16) * kPitch + 16 * a + l];
+            const float4 yv = *reinterpret_cast<const float4 *>(Am + (16 * bb + l) * kPitch + 16 * a + 4 * jq);
+            y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
+        }
+        *reinterpret_cast<float4 *>(Tm + (16 * a + i16) * kPitch + 16 * bb + 4 * jq) =
+            make_float4(-y.x, -y.y, -y.z, -y.w);
+    }
+    __syncthreads();
+    const int i32 = tid >> 3, jq8 = tid & 7;
+    {
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) {
+            const float av = Am[(32 + i32) * kPitch + l];
+            const float4 tv = *reinterpret_cast<const float4 *>(Tm + l * kPitch + 4 * jq8);
+            y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
+        }
+        *reinterpret_cast<float4 *>(Am + i32 * kPitch + 32 + 4 * jq8) = y;
+    }
+    __syncthreads();
+    {
+        float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 8
+        for (int l = 0; l < 32; ++l) {
+            const float tv = Tm[(32 + i32) * kPitch + 32 + l];
+            const float4 yv = *reinterpret_cast<const float4 *>(Am + l * kPitch + 32 + 4 * jq8);
+            y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
+        }
+        *reinterpret_cast<float4 *>(Tm + (32 + i32) * kPitch + 4 * jq8) =
+            make_float4(-y.x, -y.y, -y.z, -y.w);
+    }
+}
+
 __global__ void __launch_bounds__(kNT, 2)
 prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                     const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                     const float *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H,
-                    int n0, int nb, float scale, int prep_flags, int gate, int pf_dist)
+                    int n0, int nb, float scale, int prep_flags, int gate, int pf_dist,
+                    const __grid_constant__ CUtensorMap u_map)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -376,7 +464,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     auto issue_v = [&]() {
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-            const int id = tid + kNT * r, t = id >> 4, g = id & 15;
+            // eight consecutive threads fill the eight rows of one core matrix (no bank conflicts)
+            const int id = tid + kNT * r, t = (id & 7) | ((id >> 7) << 3), g = (id >> 3) & 15;
             const bool okt = t < c;
             cp_async16(sbase + PP_V + core_off(t, 8 * g, RW_SO, RW_SI), v + row(okt ? t : 0) * kDV + 8 * g,
                        okt ? 16u : 0u);
@@ -551,76 +640,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     if (!failed) {
         // ---- T = (I + A)^-1 by recursive doubling 16 -> 32 -> 64, fp32; R = T Diag(beta)
         float *Tm = reinterpret_cast<float *>(smem + PP_TMAT);
-        if (tid < 64) {
-            const int blk = tid >> 4, j = tid & 15, o = 16 * blk;
-            float xs[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-                float s = (i == j) ? 1.f : 0.f;
-#pragma unroll
-                for (int l = 0; l < i; ++l) s -= Am[(o + i) * kPitch + o + l] * xs[l];
-                xs[i] = s;
-            }
-#pragma unroll
-            for (int i = 0; i < 16; ++i) Tm[(o + i) * kPitch + o + j] = xs[i];
-        } else {
-            for (int e = tid - 64; e < 6 * 256; e += kNT - 64) {
-                const int blk = e >> 8, i = (e >> 4) & 15, j = e & 15;
-                const int rb = (blk < 3) ? 0 : (blk < 5 ? 1 : 2);
-                const int cb = (blk < 3) ? blk + 1 : (blk < 5 ? blk - 1 : 3);
-                Tm[(16 * rb + i) * kPitch + 16 * cb + j] = 0.f;
-            }
-        }
-        __syncthreads();
-        const int p = tid >> 6, i16 = (tid >> 2) & 15, jq = tid & 3;
-        if (tid < 128) {
-            const int a = 2 * p + 1, bb = 2 * p;
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int l = 0; l < 16; ++l) {
-                const float av = Am[(16 * a + i16) * kPitch + 16 * bb + l];
-                const float4 tv = *reinterpret_cast<const float4 *>(Tm + (16 * bb + l) * kPitch + 16 * bb + 4 * jq);
-                y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
-            }
-            *reinterpret_cast<float4 *>(Am + (16 * bb + i16) * kPitch + 16 * a + 4 * jq) = y;
-        }
-        __syncthreads();
-        if (tid < 128) {
-            const int a = 2 * p + 1, bb = 2 * p;
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-            for (int l = 0; l < 16; ++l) {
-                const float tv = Tm[(16 * a + i16) * kPitch + 16 * a + l];
-                const float4 yv = *reinterpret_cast<const float4 *>(Am + (16 * bb + l) * kPitch + 16 * a + 4 * jq);
-                y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
-            }
-            *reinterpret_cast<float4 *>(Tm + (16 * a + i16) * kPitch + 16 * bb + 4 * jq) =
-                make_float4(-y.x, -y.y, -y.z, -y.w);
-        }
-        __syncthreads();
-        const int i32 = tid >> 3, jq8 = tid & 7;
-        {
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-            for (int l = 0; l < 32; ++l) {
-                const float av = Am[(32 + i32) * kPitch + l];
-                const float4 tv = *reinterpret_cast<const float4 *>(Tm + l * kPitch + 4 * jq8);
-                y.x += av * tv.x; y.y += av * tv.y; y.z += av * tv.z; y.w += av * tv.w;
-            }
-            *reinterpret_cast<float4 *>(Am + i32 * kPitch + 32 + 4 * jq8) = y;
-        }
-        __syncthreads();
-        {
-            float4 y = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 8
-            for (int l = 0; l < 32; ++l) {
-                const float tv = Tm[(32 + i32) * kPitch + 32 + l];
-                const float4 yv = *reinterpret_cast<const float4 *>(Am + l * kPitch + 32 + 4 * jq8);
-                y.x += tv * yv.x; y.y += tv * yv.y; y.z += tv * yv.z; y.w += tv * yv.w;
-            }
-            *reinterpret_cast<float4 *>(Tm + (32 + i32) * kPitch + 4 * jq8) =
-                make_float4(-y.x, -y.y, -y.z, -y.w);
-        }
+        unit_lower_inverse(Am, Tm, tid);
         if (tid == 0) bulk_wait_read();      // M has left the region R is written to
         __syncthreads();
         for (int id = tid; id < 512; id += kNT) {
@@ -672,18 +692,18 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
             }
         }
         if (!failed && lrow >= 64) {
-            // U: lane 64 + token, 64 value columns per thread = two slices
+            // U: lane 64 + token, 64 value columns per thread = two slices, staged in the
+            // free [32 KB, 64 KB) as the swizzled rows of the tensor store's box
 #pragma unroll
             for (int s2 = 0; s2 < 2; ++s2) {
-                // staged in the free [32 KB, 64 KB) in the record's [slice][token][32] order
-                float *dst = reinterpret_cast<float *>(smem + 32768 + (2 * half + s2) * 8192) + (lrow - 64) * kDVS;
+                const int r = (2 * half + s2) * kC + lrow - 64;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float x[16];
                     tmem_ld16(tmem + tlane + TMP_U + 64 * half + 32 * s2 + 16 * hh, x);
 #pragma unroll
                     for (int g = 0; g < 4; ++g)
-                        reinterpret_cast<float4 *>(dst + 16 * hh)[g] =
+                        *reinterpret_cast<float4 *>(smem + 32768 + u_stage_off(r, 4 * hh + g)) =
                             make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
                 }
             }
@@ -698,7 +718,7 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         // Wr (rows 0..63 of [Wr; Qr], hi then lo) and U to the record
         bulk_s2g(rec + R_WQ, sbase, 16384u);
         bulk_s2g(rec + R_WQ_LO, sbase + 16384u, 16384u);
-        bulk_s2g(rec + R_U, sbase + 32768u, 32768u);
+        tma_store_3d(&u_map, sbase + 32768u, 0, 0, bh * nb + nloc);
         bulk_commit();
     }
     if (warp == 0) {
@@ -707,6 +727,9 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     }
     if (tid == 0) bulk_wait_read();          // shared memory stays until the copies have read it
 }
+
+// ---------------------------------------------------------------- scalar-gate chunk-local kernel
+#include "kda_prep_scalar.cuh"
 
 // ---------------------------------------------------------------- chain kernels: modes
 // The chain is linear in (U, S_0), which lets one segment of a sequence be run from
@@ -1061,6 +1084,10 @@ constexpr uint32_t TT_S = 0, TT_S_LO = 64;            // S'^T, bf16 pairs along 
 constexpr uint32_t TT_DL = 128, TT_DL_LO = 160;       // Delta^T, bf16 pairs along tokens: hi, lo
 constexpr uint32_t TT_D3 = 192, TT_D1 = 256, TT_D2 = 384, TT_COLS = 512;
 
+// kScalar: records of the scalar-gate chunk-local kernel (e^m = e^{G_last - m} = 1 and
+// one e^{G_last} in every channel), so the state update is one multiply-add per value
+// and S'^T = S^T.
+template <bool kScalar>
 __global__ void __launch_bounds__(kTThreads, 1)
 prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float *s_out,
                        const __grid_constant__ CUtensorMap out_map, int T, int H, int n0, int nb, int mode,
@@ -1237,9 +1264,15 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
             uint32_t hv[16], lv[16];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-                const float4 m = em4[e];
-                split_pair(m.x * S[4 * e], m.y * S[4 * e + 1], hv[2 * e], lv[2 * e]);
-                split_pair(m.z * S[4 * e + 2], m.w * S[4 * e + 3], hv[2 * e + 1], lv[2 * e + 1]);
+                const float2 s01 = make_float2(S[4 * e], S[4 * e + 1]), s23 = make_float2(S[4 * e + 2], S[4 * e + 3]);
+                if (kScalar) {
+                    split_pair2(s01, hv[2 * e], lv[2 * e]);
+                    split_pair2(s23, hv[2 * e + 1], lv[2 * e + 1]);
+                } else {
+                    const float4 m = em4[e];
+                    split_pair2(mul2(make_float2(m.x, m.y), s01), hv[2 * e], lv[2 * e]);
+                    split_pair2(mul2(make_float2(m.z, m.w), s23), hv[2 * e + 1], lv[2 * e + 1]);
+                }
             }
             tmem_st16u(tmem + tlane + TT_S + 16 * g, hv);
             tmem_st16u(tmem + tlane + TT_S_LO + 16 * g, lv);
@@ -1273,7 +1306,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
 #pragma unroll
                 for (int p = 0; p < 8; ++p) {
                     const float u0 = zu ? 0.f : su[(2 * p) * kDVS], u1 = zu ? 0.f : su[(2 * p + 1) * kDVS];
-                    split_pair(u0 - x[2 * p], u1 - x[2 * p + 1], hv[p], lv[p]);
+                    split_pair2(sub2(make_float2(u0, u1), make_float2(x[2 * p], x[2 * p + 1])), hv[p], lv[p]);
                 }
                 tmem_st8u(tmem + tlane + TT_DL + 8 * g, hv);
                 tmem_st8u(tmem + tlane + TT_DL_LO + 8 * g, lv);
@@ -1295,6 +1328,7 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
             {
                 const float4 *em4 =
                     reinterpret_cast<const float4 *>(smem + TC_WQ + kWqBytes * ((kk + 1) & 1) + 65536u) + i0 / 4;
+                const float gam_s = sDec[0];
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
                     float x[16];
@@ -1304,17 +1338,28 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                     uint32_t hv[8], lv[8];
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const float4 ga = gam4[e], el = el4[e];
                         float *sv = S + 16 * hh + 4 * e;
-                        sv[0] = ga.x * sv[0] + el.x * x[4 * e];
-                        sv[1] = ga.y * sv[1] + el.y * x[4 * e + 1];
-                        sv[2] = ga.z * sv[2] + el.z * x[4 * e + 2];
-                        sv[3] = ga.w * sv[3] + el.w * x[4 * e + 3];
-                        if (next) {
-                            const float4 m = em4[4 * hh + e];
-                            split_pair(m.x * sv[0], m.y * sv[1], hv[2 * e], lv[2 * e]);
-                            split_pair(m.z * sv[2], m.w * sv[3], hv[2 * e + 1], lv[2 * e + 1]);
+                        const float2 x01 = make_float2(x[4 * e], x[4 * e + 1]), x23 = make_float2(x[4 * e + 2], x[4 * e + 3]);
+                        float2 s01 = make_float2(sv[0], sv[1]), s23 = make_float2(sv[2], sv[3]);
+                        if (kScalar) {
+                            const float2 gg = make_float2(gam_s, gam_s);
+                            s01 = fma2(gg, s01, x01);
+                            s23 = fma2(gg, s23, x23);
+                            if (next) {
+                                split_pair2(s01, hv[2 * e], lv[2 * e]);
+                                split_pair2(s23, hv[2 * e + 1], lv[2 * e + 1]);
+                            }
+                        } else {
+                            const float4 ga = gam4[e], el = el4[e];
+                            s01 = fma2(make_float2(ga.x, ga.y), s01, mul2(make_float2(el.x, el.y), x01));
+                            s23 = fma2(make_float2(ga.z, ga.w), s23, mul2(make_float2(el.z, el.w), x23));
+                            if (next) {
+                                const float4 m = em4[4 * hh + e];
+                                split_pair2(mul2(make_float2(m.x, m.y), s01), hv[2 * e], lv[2 * e]);
+                                split_pair2(mul2(make_float2(m.z, m.w), s23), hv[2 * e + 1], lv[2 * e + 1]);
+                            }
                         }
+                        sv[0] = s01.x; sv[1] = s01.y; sv[2] = s23.x; sv[3] = s23.y;
                     }
                     if (next) {
                         tmem_st8u(tmem + tlane + TT_S + 16 * g + 8 * hh, hv);
@@ -1460,24 +1505,46 @@ cudaError_t split_setup()
         e = cudaFuncSetAttribute(prefill_chain_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)CH_TOTAL);
     if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(prefill_chain_t_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        e = cudaFuncSetAttribute(prefill_chain_t_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)TC_TOTAL);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_chain_t_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)TC_TOTAL);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(prefill_prep_scalar_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)PS_TOTAL);
     return e;
 }
+
+// A scalar gate (or none) with no fused steps before the path: the records come from
+// prefill_prep_scalar_kernel, with the decays the per-head chain's kScalar form assumes.
+bool scalar_records(const ForwardArgs &a) { return a.gate != KDA_GATE_CHANNEL && a.prep_flags == 0; }
+
+cudaError_t rec_u_tensor_map(uint8_t *ws, size_t nrec, CUtensorMap *m);
 
 cudaError_t run_prep(const ForwardArgs &a, uint8_t *ws, int n0, int nb, cudaStream_t stream)
 {
     const size_t bh = (size_t)a.B * a.H;
+    CUtensorMap u_map;
+    memset(&u_map, 0, sizeof(u_map));
+    cudaError_t em = rec_u_tensor_map(ws, bh * (size_t)nb, &u_map);
+    if (em != cudaSuccess) return em;
     // prefetch distance: half the SM count (measured best among an eighth, a quarter,
     // three eighths, a half, one and two SM counts on the long-context shapes)
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
+    if (scalar_records(a))
+        prefill_prep_scalar_kernel<<<(unsigned)(bh * nb), kNT, PS_TOTAL, stream>>>(
+            static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
+            static_cast<const __nv_bfloat16 *>(a.v), a.gate == KDA_GATE_SCALAR ? a.log_alpha : nullptr, a.beta,
+            ws, a.T, a.H, n0, nb, a.scale, sms / 2, u_map);
+    else
+        prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
         static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
         static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale,
-        a.prep_flags, a.gate, sms / 2);
+        a.prep_flags, a.gate, sms / 2, u_map);
     e = cudaGetLastError();
     if (e == cudaSuccess) note_launch();
     return e;
@@ -1518,6 +1585,22 @@ cudaError_t out_tensor_map(const ForwardArgs &a, CUtensorMap *m)
     return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
 }
 
+// The U rows of nrec consecutive records from ws as a 3-D tensor (32 floats, 256 rows of
+// (slice, token), record), one box per record, 128-byte swizzle in shared memory.
+cudaError_t rec_u_tensor_map(uint8_t *ws, size_t nrec, CUtensorMap *m)
+{
+    const PFN_cuTensorMapEncodeTiled_v12000 enc = tensor_map_encoder();
+    if (!enc) return cudaErrorNotSupported;
+    const cuuint64_t dims[3] = {(cuuint64_t)kDVS, (cuuint64_t)(kNSL * kC), (cuuint64_t)nrec};
+    const cuuint64_t strides[2] = {(cuuint64_t)kDVS * 4u, (cuuint64_t)kRec};
+    const cuuint32_t box[3] = {(cuuint32_t)kDVS, (cuuint32_t)(kNSL * kC), 1u};
+    const cuuint32_t estr[3] = {1u, 1u, 1u};
+    const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ws + R_U, dims, strides, box, estr,
+                           CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 cudaError_t run_chain(const ForwardArgs &a, bool per_head, const uint8_t *ws, int n0, int nb, const float *s_in,
                       float *s_out, int mode, const float *s_add, cudaStream_t stream)
 {
@@ -1529,8 +1612,12 @@ cudaError_t run_chain(const ForwardArgs &a, bool per_head, const uint8_t *ws, in
             const cudaError_t e = out_tensor_map(a, &out_map);
             if (e != cudaSuccess) return e;
         }
-        prefill_chain_t_kernel<<<(unsigned)bh, kTThreads, TC_TOTAL, stream>>>(ws, s_in, s_out, out_map, a.T, a.H,
-                                                                            n0, nb, mode, s_add);
+        if (scalar_records(a))
+            prefill_chain_t_kernel<true><<<(unsigned)bh, kTThreads, TC_TOTAL, stream>>>(ws, s_in, s_out, out_map, a.T,
+                                                                                     a.H, n0, nb, mode, s_add);
+        else
+            prefill_chain_t_kernel<false><<<(unsigned)bh, kTThreads, TC_TOTAL, stream>>>(ws, s_in, s_out, out_map,
+                                                                                      a.T, a.H, n0, nb, mode, s_add);
     } else
         prefill_chain_kernel<<<(unsigned)(bh * kNSL), kChainThreads, CH_TOTAL, stream>>>(ws, s_in, s_out, a.out, a.T,
                                                                                      a.H, n0, nb, mode, s_add);

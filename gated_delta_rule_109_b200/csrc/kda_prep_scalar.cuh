@@ -1,0 +1,311 @@
+// Chunk-local kernel of the two-kernel prefill for the scalar-gate members of the
+// family (Gated DeltaNet: one decay per token and head; DeltaNet: none), bf16 inputs,
+// dk = dv = 128.  Included by kda_prefill_split.cu inside its namespace: it writes the
+// same chunk record as prefill_prep_kernel, read by the same chain kernels.
+//
+// With one decay per token every factor of the chunk algebra is a per-token scalar
+// ("Kimi Delta Attention: The Linear Attention Behind Kimi K2 and Qwen3", §DeltaNet,
+// Gated DeltaNet, and KDA, comparison table: a scalar alpha_t instead of Diag(alpha_t)),
+// so the decay factors out of the contractions.  With G_t the in-chunk inclusive sum of
+// log alpha (G non-increasing, G <= 0):
+//
+//   [K; Q] K^T            exact bf16 inputs: one tensor-core term
+//   A_ij = beta_i e^{G_i - G_j} (k_i . k_j)         (j < i),  every factor <= 1
+//   M_ij = scale e^{G_i - G_j} (q_i . k_j)          (j <= i)
+//   R = (I + A)^-1 Diag(beta)
+//   Wr = (R Diag(e^G)) K,  U = R V                   K and V exact: two terms each
+//   Qr = scale Diag(e^G) Q,  Kb = Diag(e^{G_last - G}) K
+//
+// which is the record of the per-channel kernel with the reference point m = 0:
+// e^m = e^{G_last - m} = 1 and e^{G_last} in every channel.  No factor exceeds 1, so
+// no chunk needs the per-channel kernel's wide-range path.
+
+// shared memory (bytes); tiles in the no-swizzle canonical layout of kda_tc_ptx.cuh
+constexpr uint32_t PS_K = 0;              // K rows: K-major (outer token, inner dk); the B of P1, MN-major B of Wr
+constexpr uint32_t PS_Q = 16384;          // Q rows: rows 64..127 of the [K; Q] A tile of P1
+constexpr uint32_t PS_QR = 32768;         // Qr hi, lo staged in the record's byte order
+constexpr uint32_t PS_KB = 65536;         // Kb hi, lo staged in the record's byte order
+constexpr uint32_t PS_V = 98304;          // V: MN-major B of U
+constexpr uint32_t PS_BETA = 114688;      // fp32 [64]
+constexpr uint32_t PS_G = PS_BETA + 256;  // fp32 [64]: log alpha, then G
+constexpr uint32_t PS_MBAR = PS_G + 256;
+constexpr uint32_t PS_TMEMP = PS_MBAR + 8;
+constexpr uint32_t PS_TOTAL = PS_TMEMP + 8;
+static_assert(PS_TOTAL <= 115712, "two CTAs per SM");
+// after P1 (the [K; Q] tile's Q rows and both staging areas are free): the solve's A and
+// T (fp32, row pitch kPitch), M staged for its bulk copy, then R over M:
+// [R Diag(e^G) hi | lo | R hi | lo], 8 KB each (K-major, outer row, inner token)
+constexpr uint32_t PS_AMAT = 16384, PS_TMAT = PS_AMAT + 64 * kPitch * 4;
+constexpr uint32_t PS_M = PS_TMAT + 64 * kPitch * 4, PS_R = PS_M;
+static_assert(PS_R + 32768 <= PS_V, "R tiles below V");
+// after P2: Wr hi, lo and U staged for their bulk copies
+constexpr uint32_t PS_WR = 16384, PS_U = 49152;
+static_assert(PS_U + 32768 <= PS_V, "U below V");
+
+__global__ void __launch_bounds__(kNT, 2)
+prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
+                           const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
+                           const float *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H, int n0, int nb,
+                           float scale, int pf_dist, const __grid_constant__ CUtensorMap u_map)
+{
+    extern __shared__ __align__(1024) uint8_t smem[];
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
+    float *sBeta = reinterpret_cast<float *>(smem + PS_BETA);
+    float *sG = reinterpret_cast<float *>(smem + PS_G);
+    const uint32_t mbar = sbase + PS_MBAR;
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int nloc = blockIdx.x % nb;
+    const int bh = blockIdx.x / nb;
+    const int b = bh / H, h = bh % H;
+    const int t0 = (n0 + nloc) * kC;
+    const int c = min(kC, T - t0);
+    const int lrow = 32 * (warp & 3) + lane;          // tensor-memory lane of the readouts
+    const int half = warp >> 2;
+    uint8_t *rec = ws + ((size_t)bh * nb + nloc) * kRec;
+    auto row = [&](int t) { return ((size_t)b * T + t0 + t) * H + h; };
+
+    // ---- loads, all at once: k, q, v rows into their operand tiles (rows past the
+    // chunk's end zero-filled), the decays and beta (zero past the end)
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        // eight consecutive threads take the eight rows of one core matrix: a warp's
+        // 16-byte pieces then fill 512 contiguous bytes of the tile (no bank conflicts)
+        const int id = tid + kNT * r, t = (id & 7) | ((id >> 7) << 3), g = (id >> 3) & 15;
+        const bool okt = t < c;
+        const size_t o = row(okt ? t : 0);
+        const uint32_t so = core_off(t, 8 * g, RW_SO, RW_SI);
+        cp_async16(sbase + PS_K + so, k + o * kDK + 8 * g, okt ? 16u : 0u);
+        cp_async16(sbase + PS_Q + so, q + o * kDK + 8 * g, okt ? 16u : 0u);
+        cp_async16(sbase + PS_V + so, v + o * kDV + 8 * g, okt ? 16u : 0u);
+    }
+    cp_async_commit();
+    if (tid < kC) {
+        const bool okt = tid < c;
+        sG[tid] = (okt && log_alpha) ? log_alpha[row(tid)] : 0.f;
+        sBeta[tid] = okt ? beta[row(tid)] : 0.f;
+    }
+    // warm L2 with the inputs of the CTA pf_dist places further on
+    if (pf_dist > 0 && blockIdx.x + (unsigned)pf_dist < gridDim.x) {
+        const int xb = (int)blockIdx.x + pf_dist;
+        const int pbh = xb / nb, pb = pbh / H, ph = pbh % H;
+        const int pt0 = (n0 + xb % nb) * kC, pc = min(kC, T - pt0);
+        const int t = tid >> 2, which = tid & 3;
+        if (t < pc) {
+            const size_t r = ((size_t)pb * T + pt0 + t) * H + ph;
+            if (which == 0) l2_prefetch(q + r * kDK, kDK * 2);
+            else if (which == 1) l2_prefetch(k + r * kDK, kDK * 2);
+            else if (which == 2) l2_prefetch(v + r * kDV, kDV * 2);
+            else {
+                asm volatile("prefetch.global.L2 [%0];" :: "l"(beta + r) : "memory");
+                if (log_alpha) asm volatile("prefetch.global.L2 [%0];" :: "l"(log_alpha + r) : "memory");
+            }
+        }
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     :: "r"(sbase + PS_TMEMP), "r"(TMP_COLS) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    if (tid == 0) {
+        mbar_init(mbar, 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    cp_async_wait_all();
+    proxy_fence();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + PS_TMEMP);
+    const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
+
+    // ---- P1: [K; Q] K^T on the exact inputs; rows 0..63 -> A, rows 64..127 -> M
+    if (tid == 0) {
+        mma_split(tmem + TMP_AM, sbase + PS_K, 0u, RW_SI, RW_SO, sbase + PS_K, 0u, RW_SI, RW_SO, kDK / 16,
+                  idesc_bf16(128, 64, 0, 0), false, false, false);
+        umma_commit(mbar);
+    }
+    // ---- in-chunk inclusive sums of the decay (warp 0; padded tokens add 0)
+    if (warp == 0) {
+        float a0 = sG[lane], a1 = sG[lane + 32];
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const float u0 = __shfl_up_sync(0xffffffffu, a0, o);
+            const float u1 = __shfl_up_sync(0xffffffffu, a1, o);
+            if (lane >= o) { a0 += u0; a1 += u1; }
+        }
+        a1 += __shfl_sync(0xffffffffu, a0, 31);
+        sG[lane] = a0;
+        sG[lane + 32] = a1;
+    }
+    __syncthreads();
+    const float g_last = sG[kC - 1];
+    // the record's per-channel decays with m = 0: e^m = 1, e^{G_last}, e^{G_last - m} = 1
+    if (tid < kDK) {
+        reinterpret_cast<float *>(rec + R_EM)[tid] = 1.f;
+        reinterpret_cast<float *>(rec + R_GAM)[tid] = __expf(g_last);
+        reinterpret_cast<float *>(rec + R_EL)[tid] = 1.f;
+    }
+    // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, staged in the record's order
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int id = tid + kNT * r, t = (id & 7) | ((id >> 7) << 3), g = (id >> 3) & 15;
+        const uint32_t o = core_off(t, 8 * g, RW_SO, RW_SI);
+        const uint4 qv = *reinterpret_cast<const uint4 *>(smem + PS_Q + o);
+        const uint4 kv = *reinterpret_cast<const uint4 *>(smem + PS_K + o);
+        const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
+        const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv);
+        const float gt = sG[t];
+        const float fq = scale * __expf(gt), fk = __expf(g_last - gt);
+        float y[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = fq * __bfloat162float(qb[i]);
+        st_split8(smem, PS_QR + o, PS_QR + 16384u + o, y);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) y[i] = fk * __bfloat162float(kb[i]);
+        st_split8(smem, PS_KB + o, PS_KB + 16384u + o, y);
+    }
+    proxy_fence();
+    __syncthreads();
+    if (tid == 0) {
+        bulk_s2g(rec + R_WQ + 16384u, sbase + PS_QR, 16384u);
+        bulk_s2g(rec + R_WQ_LO + 16384u, sbase + PS_QR + 16384u, 16384u);
+        bulk_s2g(rec + R_KT, sbase + PS_KB, 32768u);
+        bulk_commit();
+    }
+    uint32_t phase = 0;
+    const bool p1_done = mbar_wait(mbar, phase);
+    if (tid == 0) bulk_wait_read();          // the solve's scratch goes over the staging
+    bool failed = __syncthreads_or(!p1_done) != 0;
+    phase ^= 1;
+
+    float *Am = reinterpret_cast<float *>(smem + PS_AMAT);
+    float *Tm = reinterpret_cast<float *>(smem + PS_TMAT);
+    if (!failed) {
+        tc_fence_after();
+        float x[32];
+        tmem_ld16(tmem + tlane + TMP_AM + 32 * half, *reinterpret_cast<float (*)[16]>(x));
+        tmem_ld16(tmem + tlane + TMP_AM + 32 * half + 16, *reinterpret_cast<float (*)[16]>(x + 16));
+        if (lrow < 64) {
+            const int i = lrow;
+            const float bi = sBeta[i], gi = sG[i];
+#pragma unroll
+            for (int e4 = 0; e4 < 8; ++e4) {
+                float y[4];
+#pragma unroll
+                for (int e = 0; e < 4; ++e) {
+                    const int j = 32 * half + 4 * e4 + e;
+                    y[e] = (j < i) ? bi * __expf(gi - sG[j]) * x[4 * e4 + e] : 0.f;
+                }
+                *reinterpret_cast<float4 *>(Am + i * kPitch + 32 * half + 4 * e4) = make_float4(y[0], y[1], y[2], y[3]);
+            }
+        } else {
+            const int i = lrow - 64;
+            const float gi = sG[i];
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                    const int j = 32 * half + 8 * g + e;
+                    y[e] = (j <= i) ? scale * __expf(gi - sG[j]) * x[8 * g + e] : 0.f;
+                }
+                const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
+                st_split8(smem, PS_M + o, PS_M + 8192u + o, y);
+            }
+            proxy_fence();
+        }
+    }
+    __syncthreads();
+    if (!failed && tid == 0) {
+        bulk_s2g(rec + R_M, sbase + PS_M, 16384u);        // M hi and lo, contiguous in both
+        bulk_commit();
+    }
+
+    if (!failed) {
+        // ---- T = (I + A)^-1; R = T Diag(beta) and R Diag(e^G), split, as the A of P2
+        unit_lower_inverse(Am, Tm, tid);
+        if (tid == 0) bulk_wait_read();      // M has left the region R is written to
+        __syncthreads();
+        for (int id = tid; id < 512; id += kNT) {
+            const int i = id >> 3, jg = id & 7;
+            const float4 t0v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg);
+            const float4 t1v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg + 4);
+            const float *bj = sBeta + 8 * jg;
+            const float *gj = sG + 8 * jg;
+            float y[8] = {t0v.x * bj[0], t0v.y * bj[1], t0v.z * bj[2], t0v.w * bj[3],
+                          t1v.x * bj[4], t1v.y * bj[5], t1v.z * bj[6], t1v.w * bj[7]};
+            const uint32_t o = core_off(i, 8 * jg, H_SO, H_SI);
+            st_split8(smem, PS_R + 16384u + o, PS_R + 24576u + o, y);              // R
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] *= __expf(gj[e]);
+            st_split8(smem, PS_R + o, PS_R + 8192u + o, y);                        // R Diag(e^G)
+        }
+        proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tc_fence_after();
+            // [R e^G; .] K (K rows read MN-major as B): rows 0..63 are Wr;
+            // [. ; R] V (the tile viewed from R e^G lo, so rows 64..127 are R): rows 64..127
+            // are U.  K and V are exact bf16: two terms each
+            mma_split(tmem + TMP_W, sbase + PS_R, sbase + PS_R + 8192u, H_SI, H_SO,
+                      sbase + PS_K, 0u, RW_SO, RW_SI, kC / 16, idesc_bf16(128, kDK, 0, 1), false, true, false);
+            mma_split(tmem + TMP_U, sbase + PS_R + 8192u, sbase + PS_R + 16384u, H_SI, H_SO,
+                      sbase + PS_V, 0u, RW_SO, RW_SI, kC / 16, idesc_bf16(128, kDV, 0, 1), false, true, false);
+            umma_commit(mbar);
+        }
+        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
+        if (!failed) tc_fence_after();
+        if (!failed && lrow < 64) {
+            // Wr: lane = row i, 64 key channels per thread, staged hi then lo
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                float x[16];
+                const int c0 = 64 * half + 16 * r;
+                tmem_ld16(tmem + tlane + TMP_W + c0, x);
+#pragma unroll
+                for (int g = 0; g < 2; ++g) {
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) y[e] = x[8 * g + e];
+                    const uint32_t o = core_off(lrow, c0 + 8 * g, RW_SO, RW_SI);
+                    st_split8(smem, PS_WR + o, PS_WR + 16384u + o, y);
+                }
+            }
+        }
+        if (!failed && lrow >= 64) {
+            // U: lane 64 + token, 64 value columns per thread = two slices, staged as the
+            // swizzled rows of the tensor store's box
+#pragma unroll
+            for (int s2 = 0; s2 < 2; ++s2) {
+                const int r = (2 * half + s2) * kC + lrow - 64;
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    float x[16];
+                    tmem_ld16(tmem + tlane + TMP_U + 64 * half + 32 * s2 + 16 * hh, x);
+#pragma unroll
+                    for (int g = 0; g < 4; ++g)
+                        *reinterpret_cast<float4 *>(smem + PS_U + u_stage_off(r, 4 * hh + g)) =
+                            make_float4(x[4 * g], x[4 * g + 1], x[4 * g + 2], x[4 * g + 3]);
+                }
+            }
+        }
+    }
+
+    if (failed && tid == 0) atomicOr(&g_split_device_status, 1u);
+    proxy_fence();
+    tc_fence_before();
+    __syncthreads();
+    if (!failed && tid == 0) {
+        bulk_s2g(rec + R_WQ, sbase + PS_WR, 16384u);
+        bulk_s2g(rec + R_WQ_LO, sbase + PS_WR + 16384u, 16384u);
+        tma_store_3d(&u_map, sbase + PS_U, 0, 0, bh * nb + nloc);
+        bulk_commit();
+    }
+    if (warp == 0) {
+        tc_fence_after();
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMP_COLS) : "memory");
+    }
+    if (tid == 0) bulk_wait_read();          // shared memory stays until the copies have read it
+}

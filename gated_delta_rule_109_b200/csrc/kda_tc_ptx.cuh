@@ -107,6 +107,49 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t &hi, uin
     lo = *reinterpret_cast<const uint32_t *>(&lv);
 }
 
+// Packed fp32 pair arithmetic (the f32x2 forms of sm_100): one instruction does the
+// operation on both lanes of a pair, each lane rounded as its scalar form.
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+        "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+    return d;
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b)
+{
+    float2 d;
+    asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+        "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+        "sub.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+        : "=f"(d.x), "=f"(d.y) : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+    return d;
+}
+
+// split_pair on a packed pair: the bf16 pair widened back by shifts and the two
+// remainders taken by one packed subtraction (exact: x - hi has at most 16
+// significant bits), so the bits are those of split_pair.
+__device__ __forceinline__ void split_pair2(float2 x, uint32_t &hi, uint32_t &lo)
+{
+    const __nv_bfloat162 hv = __floats2bfloat162_rn(x.x, x.y);
+    const uint32_t hb = *reinterpret_cast<const uint32_t *>(&hv);
+    const float2 r = sub2(x, make_float2(__uint_as_float(hb << 16), __uint_as_float(hb & 0xffff0000u)));
+    const __nv_bfloat162 lv = __floats2bfloat162_rn(r.x, r.y);
+    hi = hb;
+    lo = *reinterpret_cast<const uint32_t *>(&lv);
+}
+
 __device__ __forceinline__ void mbar_init(uint32_t mbar, uint32_t count)
 {
     asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" :: "r"(mbar), "r"(count) : "memory");
@@ -147,6 +190,11 @@ __device__ __forceinline__ void tma_store_4d(const void *tmap, uint32_t src, int
 {
     asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];"
                  :: "l"(tmap), "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3) : "memory");
+}
+__device__ __forceinline__ void tma_store_3d(const void *tmap, uint32_t src, int c0, int c1, int c2)
+{
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];"
+                 :: "l"(tmap), "r"(src), "r"(c0), "r"(c1), "r"(c2) : "memory");
 }
 __device__ __forceinline__ void tma_reduce_add_4d(const void *tmap, uint32_t src, int c0, int c1, int c2, int c3)
 {
