@@ -17,8 +17,11 @@
 //   Qr = scale Diag(e^G) Q,  Kb = Diag(e^{G_last - G}) K
 //
 // which is the record of the per-channel kernel with the reference point m = 0:
-// e^m = e^{G_last - m} = 1 and e^{G_last} in every channel.  No factor exceeds 1, so
-// no chunk needs the per-channel kernel's wide-range path.
+// e^m = e^{G_last - m} = 1 and e^{G_last} in every channel.  No factor exceeds 1.
+// Exponentials are per token, not per pair: e^{G_i - G_j} = a_i b_j with
+// a = e^{G - G_ref}, b = e^{G_ref - G} and G_ref midway between the chunk's extremes of
+// G; a chunk whose range of G exceeds 2 kScalarGMax (a factor could overflow) takes
+// e^{G_i - G_j} pair by pair instead.
 
 // shared memory (bytes); tiles in the no-swizzle canonical layout of kda_tc_ptx.cuh
 constexpr uint32_t PS_K = 0;              // K rows: K-major (outer token, inner dk); the B of P1, MN-major B of Wr
@@ -27,8 +30,10 @@ constexpr uint32_t PS_QR = 32768;         // Qr hi, lo staged in the record's by
 constexpr uint32_t PS_KB = 65536;         // Kb hi, lo staged in the record's byte order
 constexpr uint32_t PS_V = 98304;          // V: MN-major B of U
 constexpr uint32_t PS_BETA = 114688;      // fp32 [64]
-constexpr uint32_t PS_G = PS_BETA + 256;  // fp32 [64]: log alpha, then G
-constexpr uint32_t PS_MBAR = PS_G + 256;
+constexpr uint32_t PS_G = PS_BETA + 256;  // fp32 [64]: log alpha, then G, then e^G (after the readout)
+constexpr uint32_t PS_B = PS_G + 256;     // fp32 [64]: b = e^{G_ref - G}
+constexpr uint32_t PS_REF = PS_B + 256;   // fp32 G_ref; int wide
+constexpr uint32_t PS_MBAR = PS_REF + 16;
 constexpr uint32_t PS_TMEMP = PS_MBAR + 8;
 constexpr uint32_t PS_TOTAL = PS_TMEMP + 8;
 static_assert(PS_TOTAL <= 115712, "two CTAs per SM");
@@ -41,6 +46,7 @@ static_assert(PS_R + 32768 <= PS_V, "R tiles below V");
 // after P2: Wr hi, lo and U staged for their bulk copies
 constexpr uint32_t PS_WR = 16384, PS_U = 49152;
 static_assert(PS_U + 32768 <= PS_V, "U below V");
+constexpr float kScalarGMax = 80.f;       // largest |G - G_ref| of the factored form (e^80 < 2^127)
 
 __global__ void __launch_bounds__(kNT, 2)
 prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
@@ -52,6 +58,7 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
     float *sBeta = reinterpret_cast<float *>(smem + PS_BETA);
     float *sG = reinterpret_cast<float *>(smem + PS_G);
+    float *sB = reinterpret_cast<float *>(smem + PS_B);
     const uint32_t mbar = sbase + PS_MBAR;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -137,26 +144,45 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
         a1 += __shfl_sync(0xffffffffu, a0, 31);
         sG[lane] = a0;
         sG[lane + 32] = a1;
+        float mx = fmaxf(a0, a1), mn = fminf(a0, a1);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+        }
+        const float gref = 0.5f * (mx + mn);
+        const bool wide = !(mx - mn <= 2.f * kScalarGMax);
+        sB[lane] = wide ? 0.f : __expf(gref - a0);
+        sB[lane + 32] = wide ? 0.f : __expf(gref - a1);
+        if (lane == 0) {
+            reinterpret_cast<float *>(smem + PS_REF)[0] = gref;
+            reinterpret_cast<int *>(smem + PS_REF)[1] = wide ? 1 : 0;
+        }
     }
     __syncthreads();
     const float g_last = sG[kC - 1];
+    const float gref = reinterpret_cast<const float *>(smem + PS_REF)[0];
+    const bool wide = reinterpret_cast<const int *>(smem + PS_REF)[1] != 0;
     // the record's per-channel decays with m = 0: e^m = 1, e^{G_last}, e^{G_last - m} = 1
     if (tid < kDK) {
         reinterpret_cast<float *>(rec + R_EM)[tid] = 1.f;
         reinterpret_cast<float *>(rec + R_GAM)[tid] = __expf(g_last);
         reinterpret_cast<float *>(rec + R_EL)[tid] = 1.f;
     }
-    // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, staged in the record's order
+    // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, staged in the record's order:
+    // thread (warp w, lane l) takes token 8 w + l % 8 and channel groups l / 8 + 4 r, so a
+    // warp's 16-byte pieces fill 512 contiguous bytes and a thread needs one token's factors
+    const int tq = (lane & 7) + 8 * warp;
+    const float gt = sG[tq];
+    const float fq = scale * __expf(gt), fk = __expf(g_last - gt);
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        const int id = tid + kNT * r, t = (id & 7) | ((id >> 7) << 3), g = (id >> 3) & 15;
-        const uint32_t o = core_off(t, 8 * g, RW_SO, RW_SI);
+        const int g = (lane >> 3) + 4 * r;
+        const uint32_t o = core_off(tq, 8 * g, RW_SO, RW_SI);
         const uint4 qv = *reinterpret_cast<const uint4 *>(smem + PS_Q + o);
         const uint4 kv = *reinterpret_cast<const uint4 *>(smem + PS_K + o);
         const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
         const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv);
-        const float gt = sG[t];
-        const float fq = scale * __expf(gt), fk = __expf(g_last - gt);
         float y[8];
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = fq * __bfloat162float(qb[i]);
@@ -186,29 +212,31 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
         float x[32];
         tmem_ld16(tmem + tlane + TMP_AM + 32 * half, *reinterpret_cast<float (*)[16]>(x));
         tmem_ld16(tmem + tlane + TMP_AM + 32 * half + 16, *reinterpret_cast<float (*)[16]>(x + 16));
+        const int i = lrow & 63;
+        const float gi = sG[i];
+        const float ai = wide ? 0.f : __expf(gi - gref);
+        // e^{G_i - G_j}: a_i b_j, or pair by pair in a wide chunk
+        auto fac = [&](int j) { return wide ? __expf(gi - sG[j]) : ai * sB[j]; };
         if (lrow < 64) {
-            const int i = lrow;
-            const float bi = sBeta[i], gi = sG[i];
+            const float bi = sBeta[i];
 #pragma unroll
             for (int e4 = 0; e4 < 8; ++e4) {
                 float y[4];
 #pragma unroll
                 for (int e = 0; e < 4; ++e) {
                     const int j = 32 * half + 4 * e4 + e;
-                    y[e] = (j < i) ? bi * __expf(gi - sG[j]) * x[4 * e4 + e] : 0.f;
+                    y[e] = (j < i) ? bi * fac(j) * x[4 * e4 + e] : 0.f;
                 }
                 *reinterpret_cast<float4 *>(Am + i * kPitch + 32 * half + 4 * e4) = make_float4(y[0], y[1], y[2], y[3]);
             }
         } else {
-            const int i = lrow - 64;
-            const float gi = sG[i];
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
                 float y[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
                     const int j = 32 * half + 8 * g + e;
-                    y[e] = (j <= i) ? scale * __expf(gi - sG[j]) * x[8 * g + e] : 0.f;
+                    y[e] = (j <= i) ? scale * fac(j) * x[8 * g + e] : 0.f;
                 }
                 const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
                 st_split8(smem, PS_M + o, PS_M + 8192u + o, y);
@@ -224,6 +252,7 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
 
     if (!failed) {
         // ---- T = (I + A)^-1; R = T Diag(beta) and R Diag(e^G), split, as the A of P2
+        if (tid >= kNT - kC) sG[tid - (kNT - kC)] = __expf(sG[tid - (kNT - kC)]);   // G is read no more: e^G
         unit_lower_inverse(Am, Tm, tid);
         if (tid == 0) bulk_wait_read();      // M has left the region R is written to
         __syncthreads();
@@ -232,13 +261,13 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
             const float4 t0v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg);
             const float4 t1v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg + 4);
             const float *bj = sBeta + 8 * jg;
-            const float *gj = sG + 8 * jg;
+            const float *egj = sG + 8 * jg;
             float y[8] = {t0v.x * bj[0], t0v.y * bj[1], t0v.z * bj[2], t0v.w * bj[3],
                           t1v.x * bj[4], t1v.y * bj[5], t1v.z * bj[6], t1v.w * bj[7]};
             const uint32_t o = core_off(i, 8 * jg, H_SO, H_SI);
             st_split8(smem, PS_R + 16384u + o, PS_R + 24576u + o, y);              // R
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] *= __expf(gj[e]);
+            for (int e = 0; e < 8; ++e) y[e] *= egj[e];
             st_split8(smem, PS_R + o, PS_R + 8192u + o, y);                        // R Diag(e^G)
         }
         proxy_fence();
