@@ -845,7 +845,8 @@ def main(argv=None):
             "dtype": "bf16" if tc else "f32", "data": "synthetic",
             "arithmetic": ("tcgen05 bf16 products of hi/lo-split operands (3 terms), fp32 accumulation "
                            "in tensor memory, fp32 CUDA-core solve and scans") if tc else "fp32 CUDA cores",
-            "path": (("two kernels per block of 64 chunks, pipelined: the per-head state chain of block i "
+            "path": (("two kernels per block of up to 64 chunks (first and last 32), pipelined: the per-head "
+                      "state chain of block i "
                       "beside the chunk-local kernel of block i+1 (records in two slots of a %.2f GB caller "
                       "workspace)" if pipelined else
                       "two kernels per call (chunk-local records in a %.2f GB caller workspace, then the "

@@ -1710,11 +1710,14 @@ cudaError_t split_streams(SplitStreams *&out)
     return cudaSuccess;
 }
 
-// Blocks of L chunks: prep(i + 1) fills slot (i + 1) % 2 while chain(i) reads slot i % 2;
-// prep(i + 1) waits for chain(i - 1), the previous reader of its slot.  Only events order
-// the two kernels; neither waits on the other inside a kernel.  (Shorter first and last
-// blocks, to shorten the stretches where only one kernel runs, measured slower: 4.14
-// against 3.85 ms for B1 H32 T65536; blocks of 128 chunks gave 3.87 ms, of 32 4.01 ms.)
+// Blocks of up to L chunks: prep(i + 1) fills slot (i + 1) % 2 while chain(i) reads slot
+// i % 2; prep(i + 1) waits for chain(i - 1), the previous reader of its slot.  Only events
+// order the two kernels; neither waits on the other inside a kernel.  The first and the
+// last block are shorter (kPipeEndChunks), which shortens the stretches where only one of
+// the kernels runs (the first prep, the last chain): B1 H32 T65536 3.74 -> 3.54 ms with
+// end blocks of 32 chunks (16: 3.55, 8: 3.74); uniform blocks of 128 chunks measured
+// slower, of 32 slower still.
+constexpr int kPipeEndChunks = 32;
 
 cudaError_t run_pipelined(const ForwardArgs &a, uint8_t *ws, int L, cudaStream_t stream)
 {
@@ -1722,8 +1725,15 @@ cudaError_t run_pipelined(const ForwardArgs &a, uint8_t *ws, int L, cudaStream_t
     const size_t bh = (size_t)a.B * a.H;
     const size_t slot = bh * (size_t)L * kRec;
     float *carry = reinterpret_cast<float *>(ws + 2 * slot);
-    const int nblk = (nchunks + L - 1) / L;
-    auto block_len = [&](int n0) { return min(L, nchunks - n0); };
+    const int E = min(L, kPipeEndChunks);
+    auto block_len = [&](int n0) {
+        const int rem = nchunks - n0;
+        if (n0 == 0) return min(E, rem);
+        if (rem <= E) return rem;
+        return min(L, rem - E);
+    };
+    int nblk = 0;
+    for (int n0 = 0; n0 < nchunks; n0 += block_len(n0)) ++nblk;
     std::lock_guard<std::mutex> lock(g_split_streams_mu);
     SplitStreams *S = nullptr;
     cudaError_t e = split_streams(S);

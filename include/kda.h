@@ -155,10 +155,11 @@ kda_status kda_forward_ws(const void *q, const void *k, const void *v,
  * carried state).  Both are 0 when the two-kernel path does not apply (dtype, head
  * dimensions, T = 0 or bad sizes).  The records take about 145 KB per chunk of 64
  * tokens per (b, h).  For few heads (2 B H at most the SM count) and sequences of
- * at least 128 chunks, the fastest schedule is pipelined: blocks of 64 chunks whose
- * records alternate between two slots while the chain of one block runs beside the
- * chunk-local kernel of the next, so the size is two blocks' records plus the carried
- * state (0.61 GB for B1 H32 T65536); otherwise it is the whole sequence's records.
+ * at least 128 chunks, the fastest schedule is pipelined: blocks of up to 64 chunks
+ * (the first and the last of 32) whose records alternate between two slots while the
+ * chain of one block runs beside the chunk-local kernel of the next, so the size is
+ * two 64-chunk blocks' records plus the carried state (0.61 GB for B1 H32 T65536);
+ * otherwise it is the whole sequence's records.
  */
 size_t kda_forward_workspace_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
 size_t kda_forward_workspace_min_bytes(int B, int T, int H, int dk, int dv, kda_dtype dtype);
