@@ -587,12 +587,14 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
                         const int j = 32 * half + 8 * g + e;
                         y[e] = (j <= i) ? x[8 * g + e] : 0.f;
                     }
-                    // staged where R goes later (Qr lo, already copied out), then one
-                    // bulk copy to the record
+                    // straight to the record: eight lanes write one core matrix row block,
+                    // 128 contiguous bytes
                     const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
-                    st_split8(smem, PP_R + o, PP_R_LO + o, y);
+                    uint4 hv, lv;
+                    split8(y, hv, lv);
+                    *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
+                    *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
                 }
-                proxy_fence();
             }
         }
     } else {
@@ -632,16 +634,11 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         for (int id = tid; id < 64 * 64; id += kNT) Am[(id >> 6) * kPitch + (id & 63)] = Aw[id];
     }
     __syncthreads();
-    if (!wide_path && !failed && tid == 0) {
-        bulk_s2g(rec + R_M, sbase + PP_R, 16384u);     // M hi and lo, contiguous in both
-        bulk_commit();
-    }
 
     if (!failed) {
         // ---- T = (I + A)^-1 by recursive doubling 16 -> 32 -> 64, fp32; R = T Diag(beta)
         float *Tm = reinterpret_cast<float *>(smem + PP_TMAT);
         unit_lower_inverse(Am, Tm, tid);
-        if (tid == 0) bulk_wait_read();      // M has left the region R is written to
         __syncthreads();
         for (int id = tid; id < 512; id += kNT) {
             const int i = id >> 3, jg = id & 7;

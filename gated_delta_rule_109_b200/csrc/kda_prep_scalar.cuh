@@ -26,8 +26,6 @@
 // shared memory (bytes); tiles in the no-swizzle canonical layout of kda_tc_ptx.cuh
 constexpr uint32_t PS_K = 0;              // K rows: K-major (outer token, inner dk); the B of P1, MN-major B of Wr
 constexpr uint32_t PS_Q = 16384;          // Q rows: rows 64..127 of the [K; Q] A tile of P1
-constexpr uint32_t PS_QR = 32768;         // Qr hi, lo staged in the record's byte order
-constexpr uint32_t PS_KB = 65536;         // Kb hi, lo staged in the record's byte order
 constexpr uint32_t PS_V = 98304;          // V: MN-major B of U
 constexpr uint32_t PS_BETA = 114688;      // fp32 [64]
 constexpr uint32_t PS_G = PS_BETA + 256;  // fp32 [64]: log alpha, then G, then e^G (after the readout)
@@ -37,11 +35,11 @@ constexpr uint32_t PS_MBAR = PS_REF + 16;
 constexpr uint32_t PS_TMEMP = PS_MBAR + 8;
 constexpr uint32_t PS_TOTAL = PS_TMEMP + 8;
 static_assert(PS_TOTAL <= 115712, "two CTAs per SM");
-// after P1 (the [K; Q] tile's Q rows and both staging areas are free): the solve's A and
-// T (fp32, row pitch kPitch), M staged for its bulk copy, then R over M:
-// [R Diag(e^G) hi | lo | R hi | lo], 8 KB each (K-major, outer row, inner token)
+// after P1 (the [K; Q] tile's Q rows are free): the solve's A and T (fp32, row pitch
+// kPitch), then R: [R Diag(e^G) hi | lo | R hi | lo], 8 KB each (K-major, outer row,
+// inner token).  Qr, Kb and M go to the record straight from registers.
 constexpr uint32_t PS_AMAT = 16384, PS_TMAT = PS_AMAT + 64 * kPitch * 4;
-constexpr uint32_t PS_M = PS_TMAT + 64 * kPitch * 4, PS_R = PS_M;
+constexpr uint32_t PS_R = PS_TMAT + 64 * kPitch * 4;
 static_assert(PS_R + 32768 <= PS_V, "R tiles below V");
 // after P2: Wr hi, lo and U staged for their bulk copies
 constexpr uint32_t PS_WR = 16384, PS_U = 49152;
@@ -169,9 +167,10 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
         reinterpret_cast<float *>(rec + R_GAM)[tid] = __expf(g_last);
         reinterpret_cast<float *>(rec + R_EL)[tid] = 1.f;
     }
-    // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, staged in the record's order:
+    // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, straight to the record:
     // thread (warp w, lane l) takes token 8 w + l % 8 and channel groups l / 8 + 4 r, so a
-    // warp's 16-byte pieces fill 512 contiguous bytes and a thread needs one token's factors
+    // warp's 16-byte pieces fill 512 contiguous bytes (of the tiles in shared memory and of
+    // the record) and a thread needs one token's factors
     const int tq = (lane & 7) + 8 * warp;
     const float gt = sG[tq];
     const float fq = scale * __expf(gt), fk = __expf(g_last - gt);
@@ -184,24 +183,20 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
         const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
         const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv);
         float y[8];
+        uint4 hv, lv;
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = fq * __bfloat162float(qb[i]);
-        st_split8(smem, PS_QR + o, PS_QR + 16384u + o, y);
+        split8(y, hv, lv);
+        *reinterpret_cast<uint4 *>(rec + R_WQ + 16384u + o) = hv;
+        *reinterpret_cast<uint4 *>(rec + R_WQ_LO + 16384u + o) = lv;
 #pragma unroll
         for (int i = 0; i < 8; ++i) y[i] = fk * __bfloat162float(kb[i]);
-        st_split8(smem, PS_KB + o, PS_KB + 16384u + o, y);
-    }
-    proxy_fence();
-    __syncthreads();
-    if (tid == 0) {
-        bulk_s2g(rec + R_WQ + 16384u, sbase + PS_QR, 16384u);
-        bulk_s2g(rec + R_WQ_LO + 16384u, sbase + PS_QR + 16384u, 16384u);
-        bulk_s2g(rec + R_KT, sbase + PS_KB, 32768u);
-        bulk_commit();
+        split8(y, hv, lv);
+        *reinterpret_cast<uint4 *>(rec + R_KT + o) = hv;
+        *reinterpret_cast<uint4 *>(rec + R_KT_LO + o) = lv;
     }
     uint32_t phase = 0;
     const bool p1_done = mbar_wait(mbar, phase);
-    if (tid == 0) bulk_wait_read();          // the solve's scratch goes over the staging
     bool failed = __syncthreads_or(!p1_done) != 0;
     phase ^= 1;
 
@@ -239,22 +234,19 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
                     y[e] = (j <= i) ? scale * fac(j) * x[8 * g + e] : 0.f;
                 }
                 const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
-                st_split8(smem, PS_M + o, PS_M + 8192u + o, y);
+                uint4 hv, lv;
+                split8(y, hv, lv);
+                *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
+                *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
             }
-            proxy_fence();
         }
     }
     __syncthreads();
-    if (!failed && tid == 0) {
-        bulk_s2g(rec + R_M, sbase + PS_M, 16384u);        // M hi and lo, contiguous in both
-        bulk_commit();
-    }
 
     if (!failed) {
         // ---- T = (I + A)^-1; R = T Diag(beta) and R Diag(e^G), split, as the A of P2
         if (tid >= kNT - kC) sG[tid - (kNT - kC)] = __expf(sG[tid - (kNT - kC)]);   // G is read no more: e^G
         unit_lower_inverse(Am, Tm, tid);
-        if (tid == 0) bulk_wait_read();      // M has left the region R is written to
         __syncthreads();
         for (int id = tid; id < 512; id += kNT) {
             const int i = id >> 3, jg = id & 7;
