@@ -1090,6 +1090,9 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                        const __grid_constant__ CUtensorMap out_map, int T, int H, int n0, int nb, int mode,
                        const float *__restrict__ s_add)
 {
+    // a chunk-local launch made programmatically dependent on this one may place its CTAs
+    // once every CTA of this grid is resident: they go to the SMs this grid leaves free
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
     volatile uint32_t *sFail = reinterpret_cast<volatile uint32_t *>(smem + TC_FAIL);
@@ -1519,30 +1522,51 @@ bool scalar_records(const ForwardArgs &a) { return a.gate != KDA_GATE_CHANNEL &&
 
 cudaError_t rec_u_tensor_map(uint8_t *ws, size_t nrec, CUtensorMap *m);
 
-cudaError_t run_prep(const ForwardArgs &a, uint8_t *ws, int n0, int nb, cudaStream_t stream)
+// sms_free: the SMs the launch can expect to have (all of them unless a chain runs beside
+// it), which sizes the persistent scalar-gate kernel's grid at two CTAs per SM.
+// pdl: launched programmatically dependent on the kernel before it in the stream (a
+// per-head chain), so that its CTAs are placed once the chain's are resident.
+cudaError_t run_prep(const ForwardArgs &a, uint8_t *ws, int n0, int nb, cudaStream_t stream, int sms_free = 0,
+                     bool pdl = false)
 {
     const size_t bh = (size_t)a.B * a.H;
     CUtensorMap u_map;
     memset(&u_map, 0, sizeof(u_map));
     cudaError_t em = rec_u_tensor_map(ws, bh * (size_t)nb, &u_map);
     if (em != cudaSuccess) return em;
-    // prefetch distance: half the SM count (measured best among an eighth, a quarter,
-    // three eighths, a half, one and two SM counts on the long-context shapes)
     int dev = 0, sms = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e == cudaSuccess) e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    if (scalar_records(a))
-        prefill_prep_scalar_kernel<<<(unsigned)(bh * nb), kNT, PS_TOTAL, stream>>>(
-            static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
-            static_cast<const __nv_bfloat16 *>(a.v), a.gate == KDA_GATE_SCALAR ? a.log_alpha : nullptr, a.beta,
-            ws, a.T, a.H, n0, nb, a.scale, sms / 2, u_map);
-    else
-        prefill_prep_kernel<<<(unsigned)(bh * nb), kNT, PP_TOTAL, stream>>>(
-        static_cast<const __nv_bfloat16 *>(a.q), static_cast<const __nv_bfloat16 *>(a.k),
-        static_cast<const __nv_bfloat16 *>(a.v), a.log_alpha, a.beta, ws, a.T, a.H, n0, nb, a.scale,
-        a.prep_flags, a.gate, sms / 2, u_map);
-    e = cudaGetLastError();
+    // the scalar-gate kernel is persistent, two CTAs per SM that can expect to be free;
+    // the per-channel one takes one CTA per chunk (prefetching for the CTA half the SM
+    // count further on: measured best among an eighth, a quarter, three eighths, a half,
+    // one and two SM counts on the long-context shapes)
+    const size_t nitems = bh * (size_t)nb;
+    const size_t grid = std::min(nitems, (size_t)2 * (size_t)(sms_free > 0 ? std::min(sms_free, sms) : sms));
+    cudaLaunchConfig_t cfg = {};
+    cfg.blockDim = dim3(kNT);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = pdl ? 1 : 0;
+    const __nv_bfloat16 *qb = static_cast<const __nv_bfloat16 *>(a.q), *kb = static_cast<const __nv_bfloat16 *>(a.k),
+                        *vb = static_cast<const __nv_bfloat16 *>(a.v);
+    if (scalar_records(a)) {
+        cfg.gridDim = dim3((unsigned)grid);
+        cfg.dynamicSmemBytes = PS_TOTAL;
+        e = cudaLaunchKernelEx(&cfg, prefill_prep_scalar_kernel, qb, kb, vb,
+                               a.gate == KDA_GATE_SCALAR ? a.log_alpha : (const float *)nullptr, a.beta, ws, a.T, a.H,
+                               n0, nb, (int)nitems, a.scale, u_map);
+    } else {
+        cfg.gridDim = dim3((unsigned)nitems);
+        cfg.dynamicSmemBytes = PP_TOTAL;
+        e = cudaLaunchKernelEx(&cfg, prefill_prep_kernel, qb, kb, vb, a.log_alpha, a.beta, ws, a.T, a.H, n0, nb,
+                               a.scale, a.prep_flags, (int)a.gate, sms / 2, u_map);
+    }
+    if (e == cudaSuccess) e = cudaGetLastError();
     if (e == cudaSuccess) note_launch();
     return e;
 }
@@ -1673,43 +1697,16 @@ affine_compose_kernel(const float *__restrict__ P, const float *__restrict__ F, 
 // workspace after the records.
 namespace {
 
-// Per-device streams and events of the pipelined schedule, created on first use: the
-// chain runs on a stream of the greatest priority, so that its CTAs take SMs as soon as
-// they free up, and the chunk-local kernel on one of the least.
-struct SplitStreams {
-    bool ready = false;
-    cudaStream_t chain = nullptr, prep = nullptr;
-    cudaEvent_t start = nullptr, prep_done[2] = {nullptr, nullptr}, chain_done[2] = {nullptr, nullptr};
-};
-constexpr int kMaxDevices = 64;
-SplitStreams g_split_streams[kMaxDevices];
-std::mutex g_split_streams_mu;
-
-cudaError_t split_streams(SplitStreams *&out)
-{
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-    SplitStreams &S = g_split_streams[dev];
-    if (!S.ready) {
-        int least = 0, greatest = 0;
-        if ((e = cudaDeviceGetStreamPriorityRange(&least, &greatest)) != cudaSuccess) return e;
-        if (!S.chain && (e = cudaStreamCreateWithPriority(&S.chain, cudaStreamNonBlocking, greatest)) != cudaSuccess)
-            return e;
-        if (!S.prep && (e = cudaStreamCreateWithPriority(&S.prep, cudaStreamNonBlocking, least)) != cudaSuccess)
-            return e;
-        for (cudaEvent_t *ev : {&S.start, &S.prep_done[0], &S.prep_done[1], &S.chain_done[0], &S.chain_done[1]})
-            if (!*ev && (e = cudaEventCreateWithFlags(ev, cudaEventDisableTiming)) != cudaSuccess) return e;
-        S.ready = true;
-    }
-    out = &S;
-    return cudaSuccess;
-}
-
-// Blocks of up to L chunks: prep(i + 1) fills slot (i + 1) % 2 while chain(i) reads slot
-// i % 2; prep(i + 1) waits for chain(i - 1), the previous reader of its slot.  Only events
-// order the two kernels; neither waits on the other inside a kernel.  The first and the
+// Blocks of up to L chunks, all on the caller's stream: prep(0), then chain(i) and prep(i + 1)
+// for each block i.  prep(i + 1) is launched programmatically dependent on chain(i): it
+// starts once every chain CTA is resident (the chain releases its dependents first thing),
+// so its CTAs fill the SMs the chain leaves and never hold an SM a chain CTA is waiting
+// for; it fills slot (i + 1) % 2 while chain(i) reads slot i % 2.  chain(i + 1), an
+// ordinary launch, starts after everything before it in the stream has completed, so
+// prep(i + 1) also follows chain(i - 1), the previous reader of its slot.  Neither
+// kernel waits on the other inside a kernel.  (With the two kernels on two streams ordered
+// by events, the chunk-local CTAs, dispatched at the same moment, often took every SM
+// first: the chain of a block then started tens of microseconds late.)  The first and the
 // last block are shorter (kPipeEndChunks), which shortens the stretches where only one of
 // the kernels runs (the first prep, the last chain): B1 H32 T65536 3.74 -> 3.54 ms with
 // end blocks of 32 chunks (16: 3.55, 8: 3.74); uniform blocks of 128 chunks measured
@@ -1731,37 +1728,21 @@ cudaError_t run_pipelined(const ForwardArgs &a, uint8_t *ws, int L, cudaStream_t
     };
     int nblk = 0;
     for (int n0 = 0; n0 < nchunks; n0 += block_len(n0)) ++nblk;
-    std::lock_guard<std::mutex> lock(g_split_streams_mu);
-    SplitStreams *S = nullptr;
-    cudaError_t e = split_streams(S);
-    if (e != cudaSuccess) return e;
-    // fork: both streams start after the work already on the caller's stream
-    if ((e = cudaEventRecord(S->start, stream)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(S->prep, S->start, 0)) != cudaSuccess ||
-        (e = cudaStreamWaitEvent(S->chain, S->start, 0)) != cudaSuccess)
-        return e;
-    e = run_prep(a, ws, 0, block_len(0), S->prep);
-    if (e == cudaSuccess) e = cudaEventRecord(S->prep_done[0], S->prep);
+    const int sms = device_sms();
+    const int sms_beside_chain = sms - (int)std::min<size_t>(bh, (size_t)sms / 2);
+    cudaError_t e = run_prep(a, ws, 0, block_len(0), stream);
     int n0 = 0;
     for (int i = 0; i < nblk && e == cudaSuccess; ++i) {
         const int nb = block_len(n0);
-        e = cudaStreamWaitEvent(S->chain, S->prep_done[i & 1], 0);
-        if (e == cudaSuccess)
-            e = run_chain(a, true, ws + (size_t)(i & 1) * slot, n0, nb, i == 0 ? a.s0 : carry,
-                          i == nblk - 1 ? a.sT : carry, 0, nullptr, S->chain);
-        if (e == cudaSuccess) e = cudaEventRecord(S->chain_done[i & 1], S->chain);
+        e = run_chain(a, true, ws + (size_t)(i & 1) * slot, n0, nb, i == 0 ? a.s0 : carry,
+                      i == nblk - 1 ? a.sT : carry, 0, nullptr, stream);
         if (e == cudaSuccess && i + 1 < nblk) {
             const int n1 = n0 + nb;
-            if (i >= 1) e = cudaStreamWaitEvent(S->prep, S->chain_done[(i - 1) & 1], 0);
-            if (e == cudaSuccess)
-                e = run_prep(a, ws + (size_t)((i + 1) & 1) * slot, n1, block_len(n1), S->prep);
-            if (e == cudaSuccess) e = cudaEventRecord(S->prep_done[(i + 1) & 1], S->prep);
+            e = run_prep(a, ws + (size_t)((i + 1) & 1) * slot, n1, block_len(n1), stream, sms_beside_chain, true);
         }
         n0 += nb;
     }
-    // join: the caller's stream waits for the last chain, which follows every prep
-    const cudaError_t j = cudaStreamWaitEvent(stream, S->chain_done[(nblk - 1) & 1], 0);
-    return e != cudaSuccess ? e : j;
+    return e;
 }
 
 }  // namespace

@@ -41,16 +41,20 @@ static_assert(PS_TOTAL <= 115712, "two CTAs per SM");
 constexpr uint32_t PS_AMAT = 16384, PS_TMAT = PS_AMAT + 64 * kPitch * 4;
 constexpr uint32_t PS_R = PS_TMAT + 64 * kPitch * 4;
 static_assert(PS_R + 32768 <= PS_V, "R tiles below V");
-// after P2: Wr hi, lo and U staged for their bulk copies
-constexpr uint32_t PS_WR = 16384, PS_U = 49152;
+// after P2: U staged for its tensor store (Wr goes to the record from registers)
+constexpr uint32_t PS_U = 49152;
 static_assert(PS_U + 32768 <= PS_V, "U below V");
 constexpr float kScalarGMax = 80.f;       // largest |G - G_ref| of the factored form (e^80 < 2^127)
 
+// Persistent: CTA x takes the chunks x, x + gridDim.x, ... of the launch (chunk index
+// bh * nb + local chunk), and the inputs of its next chunk land while it finishes the
+// current one: the Q rows once the solve has released their space, K, V, the decays and
+// beta once the second product has read them.
 __global__ void __launch_bounds__(kNT, 2)
 prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__restrict__ k,
                            const __nv_bfloat16 *__restrict__ v, const float *__restrict__ log_alpha,
                            const float *__restrict__ beta, uint8_t *__restrict__ ws, int T, int H, int n0, int nb,
-                           float scale, int pf_dist, const __grid_constant__ CUtensorMap u_map)
+                           int nitems, float scale, const __grid_constant__ CUtensorMap u_map)
 {
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(smem);
@@ -60,53 +64,45 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
     const uint32_t mbar = sbase + PS_MBAR;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nloc = blockIdx.x % nb;
-    const int bh = blockIdx.x / nb;
-    const int b = bh / H, h = bh % H;
-    const int t0 = (n0 + nloc) * kC;
-    const int c = min(kC, T - t0);
     const int lrow = 32 * (warp & 3) + lane;          // tensor-memory lane of the readouts
     const int half = warp >> 2;
-    uint8_t *rec = ws + ((size_t)bh * nb + nloc) * kRec;
-    auto row = [&](int t) { return ((size_t)b * T + t0 + t) * H + h; };
-
-    // ---- loads, all at once: k, q, v rows into their operand tiles (rows past the
-    // chunk's end zero-filled), the decays and beta (zero past the end)
+    // (b, h), first token and length of chunk `item`; row(item, t) = its token t's row in [B, T, H]
+    auto chunk_t0 = [&](int item) { return (n0 + item % nb) * kC; };
+    auto chunk_len = [&](int item) { return min(kC, T - chunk_t0(item)); };
+    auto row = [&](int item, int t) {
+        const int bh = item / nb;
+        return ((size_t)(bh / H) * T + chunk_t0(item) + t) * H + bh % H;
+    };
+    // input loads of chunk `item` (rows past the chunk's end zero-filled): eight
+    // consecutive threads take the eight rows of one core matrix, so a warp's 16-byte
+    // pieces fill 512 contiguous bytes of the tile (no bank conflicts)
+    auto load_rows = [&](int item, const __nv_bfloat16 *src, uint32_t dst, int d) {
+        const int c = chunk_len(item);
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        // eight consecutive threads take the eight rows of one core matrix: a warp's
-        // 16-byte pieces then fill 512 contiguous bytes of the tile (no bank conflicts)
-        const int id = tid + kNT * r, t = (id & 7) | ((id >> 7) << 3), g = (id >> 3) & 15;
-        const bool okt = t < c;
-        const size_t o = row(okt ? t : 0);
-        const uint32_t so = core_off(t, 8 * g, RW_SO, RW_SI);
-        cp_async16(sbase + PS_K + so, k + o * kDK + 8 * g, okt ? 16u : 0u);
-        cp_async16(sbase + PS_Q + so, q + o * kDK + 8 * g, okt ? 16u : 0u);
-        cp_async16(sbase + PS_V + so, v + o * kDV + 8 * g, okt ? 16u : 0u);
-    }
-    cp_async_commit();
-    if (tid < kC) {
-        const bool okt = tid < c;
-        sG[tid] = (okt && log_alpha) ? log_alpha[row(tid)] : 0.f;
-        sBeta[tid] = okt ? beta[row(tid)] : 0.f;
-    }
-    // warm L2 with the inputs of the CTA pf_dist places further on
-    if (pf_dist > 0 && blockIdx.x + (unsigned)pf_dist < gridDim.x) {
-        const int xb = (int)blockIdx.x + pf_dist;
-        const int pbh = xb / nb, pb = pbh / H, ph = pbh % H;
-        const int pt0 = (n0 + xb % nb) * kC, pc = min(kC, T - pt0);
-        const int t = tid >> 2, which = tid & 3;
-        if (t < pc) {
-            const size_t r = ((size_t)pb * T + pt0 + t) * H + ph;
-            if (which == 0) l2_prefetch(q + r * kDK, kDK * 2);
-            else if (which == 1) l2_prefetch(k + r * kDK, kDK * 2);
-            else if (which == 2) l2_prefetch(v + r * kDV, kDV * 2);
-            else {
-                asm volatile("prefetch.global.L2 [%0];" :: "l"(beta + r) : "memory");
-                if (log_alpha) asm volatile("prefetch.global.L2 [%0];" :: "l"(log_alpha + r) : "memory");
-            }
+        for (int r = 0; r < 4; ++r) {
+            const int id = tid + kNT * r, t = (id & 7) | ((id >> 7) << 3), g = (id >> 3) & 15;
+            const bool okt = t < c;
+            cp_async16(sbase + dst + core_off(t, 8 * g, RW_SO, RW_SI), src + row(item, okt ? t : 0) * d + 8 * g,
+                       okt ? 16u : 0u);
         }
-    }
+    };
+    auto load_scalars = [&](int item) {
+        if (tid < kC) {
+            const bool okt = tid < chunk_len(item);
+            const size_t r = row(item, okt ? tid : 0);
+            if (log_alpha) cp_async4(sbase + PS_G + 4u * tid, log_alpha + r, okt ? 4u : 0u);
+            else sG[tid] = 0.f;
+            cp_async4(sbase + PS_BETA + 4u * tid, beta + r, okt ? 4u : 0u);
+        }
+    };
+
+    int item = blockIdx.x;
+    if (item >= nitems) return;
+    load_rows(item, q, PS_Q, kDK);
+    load_rows(item, k, PS_K, kDK);
+    load_rows(item, v, PS_V, kDV);
+    load_scalars(item);
+    cp_async_commit();
     if (warp == 0) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
                      :: "r"(sbase + PS_TMEMP), "r"(TMP_COLS) : "memory");
@@ -116,138 +112,155 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
         mbar_init(mbar, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
-    cp_async_wait_all();
-    proxy_fence();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t *>(smem + PS_TMEMP);
     const uint32_t tlane = (uint32_t)(32 * (warp & 3)) << 16;
-
-    // ---- P1: [K; Q] K^T on the exact inputs; rows 0..63 -> A, rows 64..127 -> M
-    if (tid == 0) {
-        mma_split(tmem + TMP_AM, sbase + PS_K, 0u, RW_SI, RW_SO, sbase + PS_K, 0u, RW_SI, RW_SO, kDK / 16,
-                  idesc_bf16(128, 64, 0, 0), false, false, false);
-        umma_commit(mbar);
-    }
-    // ---- in-chunk inclusive sums of the decay (warp 0; padded tokens add 0)
-    if (warp == 0) {
-        float a0 = sG[lane], a1 = sG[lane + 32];
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const float u0 = __shfl_up_sync(0xffffffffu, a0, o);
-            const float u1 = __shfl_up_sync(0xffffffffu, a1, o);
-            if (lane >= o) { a0 += u0; a1 += u1; }
-        }
-        a1 += __shfl_sync(0xffffffffu, a0, 31);
-        sG[lane] = a0;
-        sG[lane + 32] = a1;
-        float mx = fmaxf(a0, a1), mn = fminf(a0, a1);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-            mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
-        }
-        const float gref = 0.5f * (mx + mn);
-        const bool wide = !(mx - mn <= 2.f * kScalarGMax);
-        sB[lane] = wide ? 0.f : __expf(gref - a0);
-        sB[lane + 32] = wide ? 0.f : __expf(gref - a1);
-        if (lane == 0) {
-            reinterpret_cast<float *>(smem + PS_REF)[0] = gref;
-            reinterpret_cast<int *>(smem + PS_REF)[1] = wide ? 1 : 0;
-        }
-    }
-    __syncthreads();
-    const float g_last = sG[kC - 1];
-    const float gref = reinterpret_cast<const float *>(smem + PS_REF)[0];
-    const bool wide = reinterpret_cast<const int *>(smem + PS_REF)[1] != 0;
-    // the record's per-channel decays with m = 0: e^m = 1, e^{G_last}, e^{G_last - m} = 1
-    if (tid < kDK) {
-        reinterpret_cast<float *>(rec + R_EM)[tid] = 1.f;
-        reinterpret_cast<float *>(rec + R_GAM)[tid] = __expf(g_last);
-        reinterpret_cast<float *>(rec + R_EL)[tid] = 1.f;
-    }
-    // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, straight to the record:
-    // thread (warp w, lane l) takes token 8 w + l % 8 and channel groups l / 8 + 4 r, so a
-    // warp's 16-byte pieces fill 512 contiguous bytes (of the tiles in shared memory and of
-    // the record) and a thread needs one token's factors
-    const int tq = (lane & 7) + 8 * warp;
-    const float gt = sG[tq];
-    const float fq = scale * __expf(gt), fk = __expf(g_last - gt);
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int g = (lane >> 3) + 4 * r;
-        const uint32_t o = core_off(tq, 8 * g, RW_SO, RW_SI);
-        const uint4 qv = *reinterpret_cast<const uint4 *>(smem + PS_Q + o);
-        const uint4 kv = *reinterpret_cast<const uint4 *>(smem + PS_K + o);
-        const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
-        const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv);
-        float y[8];
-        uint4 hv, lv;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = fq * __bfloat162float(qb[i]);
-        split8(y, hv, lv);
-        *reinterpret_cast<uint4 *>(rec + R_WQ + 16384u + o) = hv;
-        *reinterpret_cast<uint4 *>(rec + R_WQ_LO + 16384u + o) = lv;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) y[i] = fk * __bfloat162float(kb[i]);
-        split8(y, hv, lv);
-        *reinterpret_cast<uint4 *>(rec + R_KT + o) = hv;
-        *reinterpret_cast<uint4 *>(rec + R_KT_LO + o) = lv;
-    }
-    uint32_t phase = 0;
-    const bool p1_done = mbar_wait(mbar, phase);
-    bool failed = __syncthreads_or(!p1_done) != 0;
-    phase ^= 1;
-
     float *Am = reinterpret_cast<float *>(smem + PS_AMAT);
     float *Tm = reinterpret_cast<float *>(smem + PS_TMAT);
-    if (!failed) {
+    bool failed = false;
+
+    for (; item < nitems; item += gridDim.x) {
+        const int next = item + (int)gridDim.x;
+        uint8_t *rec = ws + (size_t)item * kRec;
+        // ---- this chunk's inputs have landed (and every read of the previous chunk's
+        // tensor memory is done)
+        cp_async_wait_all();
+        proxy_fence();
+        tc_fence_before();
+        __syncthreads();
         tc_fence_after();
-        float x[32];
-        tmem_ld16(tmem + tlane + TMP_AM + 32 * half, *reinterpret_cast<float (*)[16]>(x));
-        tmem_ld16(tmem + tlane + TMP_AM + 32 * half + 16, *reinterpret_cast<float (*)[16]>(x + 16));
-        const int i = lrow & 63;
-        const float gi = sG[i];
-        const float ai = wide ? 0.f : __expf(gi - gref);
-        // e^{G_i - G_j}: a_i b_j, or pair by pair in a wide chunk
-        auto fac = [&](int j) { return wide ? __expf(gi - sG[j]) : ai * sB[j]; };
-        if (lrow < 64) {
-            const float bi = sBeta[i];
+
+        // ---- P1: [K; Q] K^T on the exact inputs; rows 0..63 -> A, rows 64..127 -> M
+        if (tid == 0) {
+            mma_split(tmem + TMP_AM, sbase + PS_K, 0u, RW_SI, RW_SO, sbase + PS_K, 0u, RW_SI, RW_SO, kDK / 16,
+                      idesc_bf16(128, 64, 0, 0), false, false, false);
+            umma_commit(mbar);
+        }
+        // ---- in-chunk inclusive sums of the decay (warp 0; padded tokens add 0)
+        if (warp == 0) {
+            float a0 = sG[lane], a1 = sG[lane + 32];
 #pragma unroll
-            for (int e4 = 0; e4 < 8; ++e4) {
-                float y[4];
-#pragma unroll
-                for (int e = 0; e < 4; ++e) {
-                    const int j = 32 * half + 4 * e4 + e;
-                    y[e] = (j < i) ? bi * fac(j) * x[4 * e4 + e] : 0.f;
-                }
-                *reinterpret_cast<float4 *>(Am + i * kPitch + 32 * half + 4 * e4) = make_float4(y[0], y[1], y[2], y[3]);
+            for (int o = 1; o < 32; o <<= 1) {
+                const float u0 = __shfl_up_sync(0xffffffffu, a0, o);
+                const float u1 = __shfl_up_sync(0xffffffffu, a1, o);
+                if (lane >= o) { a0 += u0; a1 += u1; }
             }
-        } else {
+            a1 += __shfl_sync(0xffffffffu, a0, 31);
+            sG[lane] = a0;
+            sG[lane + 32] = a1;
+            float mx = fmaxf(a0, a1), mn = fminf(a0, a1);
 #pragma unroll
-            for (int g = 0; g < 4; ++g) {
-                float y[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int j = 32 * half + 8 * g + e;
-                    y[e] = (j <= i) ? scale * fac(j) * x[8 * g + e] : 0.f;
-                }
-                const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
-                uint4 hv, lv;
-                split8(y, hv, lv);
-                *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
-                *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
+            for (int o = 16; o > 0; o >>= 1) {
+                mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+                mn = fminf(mn, __shfl_xor_sync(0xffffffffu, mn, o));
+            }
+            const float gref = 0.5f * (mx + mn);
+            const bool wide = !(mx - mn <= 2.f * kScalarGMax);
+            sB[lane] = wide ? 0.f : __expf(gref - a0);
+            sB[lane + 32] = wide ? 0.f : __expf(gref - a1);
+            if (lane == 0) {
+                reinterpret_cast<float *>(smem + PS_REF)[0] = gref;
+                reinterpret_cast<int *>(smem + PS_REF)[1] = wide ? 1 : 0;
             }
         }
-    }
-    __syncthreads();
+        __syncthreads();
+        const float g_last = sG[kC - 1];
+        const float gref = reinterpret_cast<const float *>(smem + PS_REF)[0];
+        const bool wide = reinterpret_cast<const int *>(smem + PS_REF)[1] != 0;
+        // the record's per-channel decays with m = 0: e^m = 1, e^{G_last}, e^{G_last - m} = 1
+        if (tid < kDK) {
+            reinterpret_cast<float *>(rec + R_EM)[tid] = 1.f;
+            reinterpret_cast<float *>(rec + R_GAM)[tid] = __expf(g_last);
+            reinterpret_cast<float *>(rec + R_EL)[tid] = 1.f;
+        }
+        // ---- Qr = scale e^G q and Kb = e^{G_last - G} k, split, straight to the record:
+        // thread (warp w, lane l) takes token 8 w + l % 8 and channel groups l / 8 + 4 r, so
+        // a warp's 16-byte pieces fill 512 contiguous bytes (of the tiles in shared memory
+        // and of the record) and a thread needs one token's factors
+        {
+            const int tq = (lane & 7) + 8 * warp;
+            const float gt = sG[tq];
+            const float fq = scale * __expf(gt), fk = __expf(g_last - gt);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int g = (lane >> 3) + 4 * r;
+                const uint32_t o = core_off(tq, 8 * g, RW_SO, RW_SI);
+                const uint4 qv = *reinterpret_cast<const uint4 *>(smem + PS_Q + o);
+                const uint4 kv = *reinterpret_cast<const uint4 *>(smem + PS_K + o);
+                const __nv_bfloat16 *qb = reinterpret_cast<const __nv_bfloat16 *>(&qv);
+                const __nv_bfloat16 *kb = reinterpret_cast<const __nv_bfloat16 *>(&kv);
+                float y[8];
+                uint4 hv, lv;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = fq * __bfloat162float(qb[i]);
+                split8(y, hv, lv);
+                *reinterpret_cast<uint4 *>(rec + R_WQ + 16384u + o) = hv;
+                *reinterpret_cast<uint4 *>(rec + R_WQ_LO + 16384u + o) = lv;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) y[i] = fk * __bfloat162float(kb[i]);
+                split8(y, hv, lv);
+                *reinterpret_cast<uint4 *>(rec + R_KT + o) = hv;
+                *reinterpret_cast<uint4 *>(rec + R_KT_LO + o) = lv;
+            }
+        }
+        const bool p1_done = mbar_wait(mbar, 0u);
+        if (tid == 0) bulk_wait_read();      // the previous chunk's U store has read its staging
+        if ((failed = __syncthreads_or(!p1_done) != 0)) break;
 
-    if (!failed) {
+        // ---- A = Diag(beta) strictly_lower(...) to shared memory, M to the record
+        {
+            tc_fence_after();
+            float x[32];
+            tmem_ld16(tmem + tlane + TMP_AM + 32 * half, *reinterpret_cast<float (*)[16]>(x));
+            tmem_ld16(tmem + tlane + TMP_AM + 32 * half + 16, *reinterpret_cast<float (*)[16]>(x + 16));
+            const int i = lrow & 63;
+            const float gi = sG[i];
+            const float ai = wide ? 0.f : __expf(gi - gref);
+            // e^{G_i - G_j}: a_i b_j, or pair by pair in a wide chunk
+            auto fac = [&](int j) { return wide ? __expf(gi - sG[j]) : ai * sB[j]; };
+            if (lrow < 64) {
+                const float bi = sBeta[i];
+#pragma unroll
+                for (int e4 = 0; e4 < 8; ++e4) {
+                    float y[4];
+#pragma unroll
+                    for (int e = 0; e < 4; ++e) {
+                        const int j = 32 * half + 4 * e4 + e;
+                        y[e] = (j < i) ? bi * fac(j) * x[4 * e4 + e] : 0.f;
+                    }
+                    *reinterpret_cast<float4 *>(Am + i * kPitch + 32 * half + 4 * e4) =
+                        make_float4(y[0], y[1], y[2], y[3]);
+                }
+            } else {
+#pragma unroll
+                for (int g = 0; g < 4; ++g) {
+                    float y[8];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        const int j = 32 * half + 8 * g + e;
+                        y[e] = (j <= i) ? scale * fac(j) * x[8 * g + e] : 0.f;
+                    }
+                    const uint32_t o = core_off(i, 32 * half + 8 * g, H_SO, H_SI);
+                    uint4 hv, lv;
+                    split8(y, hv, lv);
+                    *reinterpret_cast<uint4 *>(rec + R_M + o) = hv;
+                    *reinterpret_cast<uint4 *>(rec + R_M_LO + o) = lv;
+                }
+            }
+        }
+        __syncthreads();
+
         // ---- T = (I + A)^-1; R = T Diag(beta) and R Diag(e^G), split, as the A of P2
         if (tid >= kNT - kC) sG[tid - (kNT - kC)] = __expf(sG[tid - (kNT - kC)]);   // G is read no more: e^G
         unit_lower_inverse(Am, Tm, tid);
         __syncthreads();
+        // A is free: the next chunk's Q rows land where it was
+        if (next < nitems) {
+            load_rows(next, q, PS_Q, kDK);
+            cp_async_commit();
+        }
         for (int id = tid; id < 512; id += kNT) {
             const int i = id >> 3, jg = id & 7;
             const float4 t0v = *reinterpret_cast<const float4 *>(Tm + i * kPitch + 8 * jg);
@@ -276,10 +289,17 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
                       sbase + PS_V, 0u, RW_SO, RW_SI, kC / 16, idesc_bf16(128, kDV, 0, 1), false, true, false);
             umma_commit(mbar);
         }
-        failed = __syncthreads_or(!mbar_wait(mbar, phase)) != 0;
-        if (!failed) tc_fence_after();
-        if (!failed && lrow < 64) {
-            // Wr: lane = row i, 64 key channels per thread, staged hi then lo
+        if ((failed = __syncthreads_or(!mbar_wait(mbar, 1u)) != 0)) break;
+        tc_fence_after();
+        // K, V, the decays and beta are read: the next chunk's land in their place
+        if (next < nitems) {
+            load_rows(next, k, PS_K, kDK);
+            load_rows(next, v, PS_V, kDV);
+            load_scalars(next);
+            cp_async_commit();
+        }
+        if (lrow < 64) {
+            // Wr: lane = row i, 64 key channels per thread, straight to the record
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 float x[16];
@@ -291,11 +311,13 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
 #pragma unroll
                     for (int e = 0; e < 8; ++e) y[e] = x[8 * g + e];
                     const uint32_t o = core_off(lrow, c0 + 8 * g, RW_SO, RW_SI);
-                    st_split8(smem, PS_WR + o, PS_WR + 16384u + o, y);
+                    uint4 hv, lv;
+                    split8(y, hv, lv);
+                    *reinterpret_cast<uint4 *>(rec + R_WQ + o) = hv;
+                    *reinterpret_cast<uint4 *>(rec + R_WQ_LO + o) = lv;
                 }
             }
-        }
-        if (!failed && lrow >= 64) {
+        } else {
             // U: lane 64 + token, 64 value columns per thread = two slices, staged as the
             // swizzled rows of the tensor store's box
 #pragma unroll
@@ -312,18 +334,19 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
                 }
             }
         }
+        proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+        if (tid == 0) {
+            tma_store_3d(&u_map, sbase + PS_U, 0, 0, item);
+            bulk_commit();
+        }
     }
 
     if (failed && tid == 0) atomicOr(&g_split_device_status, 1u);
-    proxy_fence();
+    cp_async_wait_all();                     // loads in flight land before shared memory goes
     tc_fence_before();
     __syncthreads();
-    if (!failed && tid == 0) {
-        bulk_s2g(rec + R_WQ, sbase + PS_WR, 16384u);
-        bulk_s2g(rec + R_WQ_LO, sbase + PS_WR + 16384u, 16384u);
-        tma_store_3d(&u_map, sbase + PS_U, 0, 0, bh * nb + nloc);
-        bulk_commit();
-    }
     if (warp == 0) {
         tc_fence_after();
         asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"(TMP_COLS) : "memory");

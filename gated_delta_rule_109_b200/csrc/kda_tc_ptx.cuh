@@ -208,6 +208,11 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, uint32
 {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
+// 4-byte global -> shared copy (cp.async.ca); src_bytes = 0 zero-fills
+__device__ __forceinline__ void cp_async4(uint32_t dst, const void *src, uint32_t src_bytes)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" :: "r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
 // L2 prefetch of a global range (16-byte aligned, a multiple of 16 bytes); a hint
 // that nothing waits for
 __device__ __forceinline__ void l2_prefetch(const void *src, uint32_t bytes)

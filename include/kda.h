@@ -123,8 +123,9 @@ kda_status kda_forward(const void *q, const void *k, const void *v,
  *     and room for two blocks of 8 or more chunks: pipelined.  The chain of
  *     block i (one CTA per (b, h)) runs beside the chunk-local kernel of block
  *     i + 1 on the other SMs, their records in alternating halves of the
- *     workspace, on two internal streams (created on first use) ordered by
- *     events; the caller's stream waits for the last kernel.
+ *     workspace.  All launches go to `stream`; the chunk-local launch of block
+ *     i + 1 is programmatically dependent on the chain of block i (it starts
+ *     once the chain's CTAs are resident and does not wait for it to finish).
  *   - otherwise: the chunk-local kernel, then the chain, per block of as many
  *     chunks as fit (the whole sequence with its full record size).
  * Which chain kernel runs depends only on B, T and H, so every workspace size
