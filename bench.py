@@ -74,12 +74,12 @@ MEASURED_TRAFFIC = {
     # the long-context launch by token-heads processed (the kernel streams its inputs once)
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
     ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
-    # two-kernel prefill, one kda_forward_ws call with the pipelined schedule (two blocks
-    # of 64 chunks: prep 169.4 + 247.6 and 169.5 + 244.8 MB, per-head chain 305.3 + 50.9
-    # and 307.3 + 50.6 MB), captured on B1 H32 T8192 and scaled by 8 to T = 65536: every
-    # term (inputs, chunk records, outputs) grows with the token count
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("b4492d60b8c3b70b", 8 * 1545.4e6),
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("b4492d60b8c3b70b", 1545.4e6),
+    # two-kernel prefill, one kda_forward_ws call with the pipelined schedule (blocks of
+    # 32, 64 and 32 chunks: prep 185.0, 424.9, 181.6 MB and per-head chain 169.7, 357.8,
+    # 171.9 MB), captured on B1 H32 T8192 and scaled by 8 to T = 65536: every term
+    # (inputs, chunk records, outputs) grows with the token count
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("88fe9c87fb21f839", 8 * 1490.9e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("88fe9c87fb21f839", 1490.9e6),
 }
 
 
@@ -562,7 +562,8 @@ def _add_gdn(line, args, w, world, device, hbm, use_workspace=True):
         "ms_per_step": ms_total / args.steps, "gpu_launches": pre["launches"],
         "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
                      "traffic": None,
-                     "kernel": ("prefill_prep_kernel + prefill_chain_kernel" if tc and use_workspace
+                     "kernel": ("prefill_prep_scalar_kernel + prefill_chain_t_kernel<kScalar> (pipelined)"
+                                if tc and use_workspace
                                 else "prefill_gdn_tc_kernel" if tc else "prefill_simt_kernel"),
                      "algorithmic_bytes_per_launch": alg_bytes}}
 
