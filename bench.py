@@ -69,7 +69,7 @@ def decode_bytes_per_head(dk, dv, in_bytes):
 # keyed by (kernel source, workload) -> (source digest at capture, bytes).
 # Reported only while the kernel source is unchanged (profiles/ holds the captures).
 MEASURED_TRAFFIC = {
-    ("kda_decode.cu", "decode_bf16_b256_h32_d128_1024steps"): ("ea0a7f230dd3ccec", 1.0301e9),
+    ("kda_decode.cu", "decode_bf16_b256_h32_d128_1024steps"): ("bdf76c3b9b0ab14c", 1.0285e9),
     # captured on B4 H32 T4096 (938.4 MB = 0.979 of its algorithmic bytes) and scaled to
     # the long-context launch by token-heads processed (the kernel streams its inputs once)
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
