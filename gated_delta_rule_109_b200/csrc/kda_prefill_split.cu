@@ -207,8 +207,12 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     const uint32_t mbar = sbase + PP_MBAR;
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int nloc = blockIdx.x % nb;                 // chunk within this block
-    const int bh = blockIdx.x / nb;
+    // CTAs in launch order take the block's chunks from the last to the first, every
+    // (b, h) of a chunk together: the chunks the chain reads first are written last and
+    // are still in L2 when it starts
+    const int nbh = (int)(gridDim.x / (unsigned)nb);
+    const int bh = (int)blockIdx.x % nbh;
+    const int nloc = nb - 1 - (int)blockIdx.x / nbh;  // chunk within this block
     const int b = bh / H, h = bh % H;
     const int t0 = (n0 + nloc) * kC;
     const int c = min(kC, T - t0);
@@ -272,8 +276,8 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
     // this one is still busy: its load phase then reads L2 rather than DRAM
     if (pf_dist > 0 && blockIdx.x + (unsigned)pf_dist < gridDim.x) {
         const int xb = (int)blockIdx.x + pf_dist;
-        const int pbh = xb / nb, pb = pbh / H, ph = pbh % H;
-        const int pt0 = (n0 + xb % nb) * kC, pc = min(kC, T - pt0);
+        const int pbh = xb % nbh, pb = pbh / H, ph = pbh % H;
+        const int pt0 = (n0 + nb - 1 - xb / nbh) * kC, pc = min(kC, T - pt0);
         const int t = tid >> 2, which = tid & 3;
         if (t < pc) {
             const size_t r = ((size_t)pb * T + pt0 + t) * H + ph;

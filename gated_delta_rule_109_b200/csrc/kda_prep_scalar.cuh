@@ -46,8 +46,8 @@ constexpr uint32_t PS_U = 49152;
 static_assert(PS_U + 32768 <= PS_V, "U below V");
 constexpr float kScalarGMax = 80.f;       // largest |G - G_ref| of the factored form (e^80 < 2^127)
 
-// Persistent: CTA x takes the chunks x, x + gridDim.x, ... of the launch (chunk index
-// bh * nb + local chunk), and the inputs of its next chunk land while it finishes the
+// Persistent: CTA x takes the work items x, x + gridDim.x, ... of the launch, and the
+// inputs of its next chunk land while it finishes the
 // current one: the Q rows once the solve has released their space, K, V, the decays and
 // beta once the second product has read them.
 __global__ void __launch_bounds__(kNT, 2)
@@ -66,11 +66,18 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int lrow = 32 * (warp & 3) + lane;          // tensor-memory lane of the readouts
     const int half = warp >> 2;
-    // (b, h), first token and length of chunk `item`; row(item, t) = its token t's row in [B, T, H]
-    auto chunk_t0 = [&](int item) { return (n0 + item % nb) * kC; };
+    // work item -> chunk: items take the block's chunks from the last to the first, every
+    // (b, h) of a chunk together, so the chunks the chain reads first are written last and
+    // are still in L2 when it starts.  Record index bh * nb + local chunk; first token and
+    // length of the chunk; row(item, t) = its token t's row in [B, T, H]
+    const int nbh = nitems / nb;
+    auto item_bh = [&](int item) { return item % nbh; };
+    auto item_loc = [&](int item) { return nb - 1 - item / nbh; };
+    auto rec_index = [&](int item) { return item_bh(item) * nb + item_loc(item); };
+    auto chunk_t0 = [&](int item) { return (n0 + item_loc(item)) * kC; };
     auto chunk_len = [&](int item) { return min(kC, T - chunk_t0(item)); };
     auto row = [&](int item, int t) {
-        const int bh = item / nb;
+        const int bh = item_bh(item);
         return ((size_t)(bh / H) * T + chunk_t0(item) + t) * H + bh % H;
     };
     // input loads of chunk `item` (rows past the chunk's end zero-filled): eight
@@ -123,7 +130,7 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
 
     for (; item < nitems; item += gridDim.x) {
         const int next = item + (int)gridDim.x;
-        uint8_t *rec = ws + (size_t)item * kRec;
+        uint8_t *rec = ws + (size_t)rec_index(item) * kRec;
         // ---- this chunk's inputs have landed (and every read of the previous chunk's
         // tensor memory is done)
         cp_async_wait_all();
@@ -338,7 +345,7 @@ prefill_prep_scalar_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloa
         tc_fence_before();
         __syncthreads();
         if (tid == 0) {
-            tma_store_3d(&u_map, sbase + PS_U, 0, 0, item);
+            tma_store_3d(&u_map, sbase + PS_U, 0, 0, rec_index(item));
             bulk_commit();
         }
     }

@@ -255,13 +255,7 @@ __device__ __forceinline__ void split8(const float (&x)[8], uint4 &hi, uint4 &lo
 {
     uint32_t h[4], l[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        const __nv_bfloat162 hv = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
-        const float2 hf = __bfloat1622float2(hv);
-        const __nv_bfloat162 lv = __floats2bfloat162_rn(x[2 * i] - hf.x, x[2 * i + 1] - hf.y);
-        h[i] = *reinterpret_cast<const uint32_t *>(&hv);
-        l[i] = *reinterpret_cast<const uint32_t *>(&lv);
-    }
+    for (int i = 0; i < 4; ++i) split_pair2(make_float2(x[2 * i], x[2 * i + 1]), h[i], l[i]);
     hi = make_uint4(h[0], h[1], h[2], h[3]);
     lo = make_uint4(l[0], l[1], l[2], l[3]);
 }
