@@ -250,17 +250,11 @@ prefill_prep_kernel(const __nv_bfloat16 *__restrict__ q, const __nv_bfloat16 *__
         for (int j = 0; j < 32; j += 4)
             *reinterpret_cast<float4 *>(Gs + t * kGP + c0 + j) = make_float4(g, g, g, g);
     }
-    if (tid < kC / 4) {
-        const bool okt = 4 * tid < c;
-        // beta is [B, T, H]: the chunk's 64 values are H apart, so they come one by one
-        float4 bv = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (okt) {
-            bv.x = beta[row(4 * tid)];
-            if (4 * tid + 1 < c) bv.y = beta[row(4 * tid + 1)];
-            if (4 * tid + 2 < c) bv.z = beta[row(4 * tid + 2)];
-            if (4 * tid + 3 < c) bv.w = beta[row(4 * tid + 3)];
-        }
-        reinterpret_cast<float4 *>(sBeta)[tid] = bv;
+    if (tid < kC) {
+        // beta is [B, T, H]: the chunk's 64 values are H apart, so they come one by one,
+        // with the log_alpha rows (zero past the chunk's end)
+        const bool okt = tid < c;
+        cp_async4(sbase + PP_BETA + 4u * tid, beta + row(okt ? tid : 0), okt ? 4u : 0u);
     }
     uint4 kv4[4], qv4[4];
 #pragma unroll
@@ -1208,12 +1202,16 @@ prefill_chain_t_kernel(const uint8_t *__restrict__ ws, const float *s_in, float 
                 for (uint32_t o = 0; o < kRec; o += 32768u)
                     l2_prefetch(r + o, (kRec - o) < 32768u ? (kRec - o) : 32768u);
             };
-            for (int kk = 0; kk < 3 && kk < nb; ++kk) prefetch(kk);
-            for (int kk = 0; kk < 2 && kk < nb; ++kk) {
-                load_half(kk, 0);
-                load_half(kk, 1);
-            }
+            // chunk 0's slot and Kb/M/U first (its S'^T split, D1 and Delta wait for
+            // them), then the L2 prefetches and chunk 1's slot
+            load_half(0, 0);
+            load_half(0, 1);
             load_ktm(0);
+            for (int kk = 1; kk < 3 && kk < nb; ++kk) prefetch(kk);
+            if (nb > 1) {
+                load_half(1, 0);
+                load_half(1, 1);
+            }
             for (int kk = 0; kk < nb; ++kk) {
                 if (kk + 3 < nb) prefetch(kk + 3);
                 // D3 done (so D2 and D1 too) and the decays read: the Kb/M slot refills first

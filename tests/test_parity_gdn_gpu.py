@@ -213,6 +213,24 @@ def test_gdn_workspace_path(gate, T, B, H, state):
     _compare("bf16", x, out, sT)
 
 
+def test_gdn_persistent_chunk_local_kernel_many_chunks_per_cta():
+    """More chunks than two per SM, so each CTA of the persistent scalar-gate kernel
+    walks several, loading the next one's inputs while it finishes the current: a
+    ragged last chunk (4 tokens), a wide-range chunk among them, a carried state;
+    blocked workspaces give the same bits."""
+    w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=8, T=4100, seed=9150)
+    assert w.B * w.H * ((w.T + 63) // 64) > 2 * torch.cuda.get_device_properties(0).multi_processor_count
+    x = _inputs(w)
+    x["g"][:, 640:704] = -4.0         # range 256 in that chunk: factors pair by pair
+    ws_full = kda.make_workspace(w.B, w.T, w.H, 128, 128)
+    out_f, s_f = _run(x, workspace=ws_full)
+    _compare("bf16", x, out_f, s_f)
+    bh, rec = w.B * w.H, kda.workspace_bytes(1, 64, 1, 128, 128)
+    ws_b = kda.make_workspace(w.B, w.T, w.H, 128, 128, nbytes=bh * rec * 7 + bh * 128 * 128 * 4)
+    out_b, s_b = _run(x, workspace=ws_b)
+    assert torch.equal(out_f, out_b) and torch.equal(s_f, s_b)
+
+
 def test_gdn_workspace_path_strong_decay_and_blocks():
     w = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=3, T=300, seed=9100)
     x = _inputs(w)
