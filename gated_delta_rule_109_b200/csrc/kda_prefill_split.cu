@@ -1,7 +1,8 @@
 // Two-kernel chunked KDA prefill on the sm_100a tensor cores, bf16 inputs,
 // dk = dv = 128, fp32 state and outputs: the chunk-local work of every chunk
-// runs in parallel (prefill_prep_kernel), and only the short state chain runs
-// in sequence (prefill_chain_kernel).
+// runs in parallel (prefill_prep_kernel; prefill_prep_scalar_kernel for a scalar
+// gate), and only the short state chain runs in sequence (prefill_chain_t_kernel,
+// one CTA per (b, h); prefill_chain_kernel, one per (b, h, 32-column slice)).
 //
 // The token step is the one of "Kimi Delta Attention: The Linear Attention
 // Behind Kimi K2 and Qwen3", §How Kimi Delta Attention works step by step; the
@@ -18,12 +19,13 @@
 //   O     = Qr S' + M Delta
 //   S    <- Diag(e^{G_last}) S + Diag(e^{G_last - m}) Kb^T Delta
 //
-// Nothing above except S', Delta, O and the update depends on S, so
-// prefill_prep_kernel computes it for all chunks at once (one CTA per
-// (b, h, chunk)) and writes one record per chunk to a caller-provided
-// workspace; prefill_chain_kernel then walks the chunks of each (b, h) with two
+// Nothing above except S', Delta, O and the update depends on S, so the
+// chunk-local kernel computes it for all chunks at once and writes one record per
+// chunk to a workspace; a chain kernel then walks the chunks of each (b, h) with two
 // tensor-core round trips per chunk:  D1 = [Wr ; Qr] S'  ->  Delta = U - D1[0:64];
-// D2 = Kb^T Delta, D3 = M Delta  ->  S update and O = D1[64:128] + D3.
+// D2 = Kb^T Delta, D3 = M Delta  ->  S update and O = D1[64:128] + D3.  For few heads
+// and long sequences the two kernels run side by side on alternating blocks of chunks
+// (run_pipelined).
 //
 // m is the midpoint of the chunk's first and last G, so each split factor is at
 // most e^{range/2} for a monotone decay; a chunk where some |G - m| > 40 instead
