@@ -285,6 +285,30 @@ def test_no_device_memory_grows_with_sequence_length():
     assert torch.cuda.mem_get_info()[0] >= free_before + held // 2
 
 
+def test_pooled_workspace_falls_back_to_the_one_kernel_prefill():
+    """A shape whose smallest workspace cannot be had (1.25 M heads of one token: 186
+    GB of records) runs the one-kernel prefill, bit for bit, and leaves the pool and the
+    CUDA error state clean."""
+    w = I.scaled(I.PREFILL_H16_T4K, B=1, H=1_250_000, T=1, seed=21)
+    assert kda.workspace_bytes(w.B, w.T, w.H, 128, 128, minimum=True) > torch.cuda.get_device_properties(0).total_memory
+    x = I.make_inputs(w, "cuda")
+    args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None)
+    held = kda.workspace_pool_bytes()
+    out_p, _ = kda.forward(*args, return_final_state=False)
+    out_1, _ = kda.forward(*args, return_final_state=False, one_kernel=True)
+    torch.cuda.synchronize()
+    kda.check_status()
+    assert torch.equal(out_p, out_1)
+    assert kda.workspace_pool_bytes() <= held + (64 << 20)
+    # and the library still takes the pooled path for an ordinary shape afterwards
+    wb = I.scaled(I.PREFILL_B4_T16K_STATE, B=1, H=2, T=200, seed=22)
+    xb = I.make_inputs(wb, "cuda")
+    ws = kda.make_workspace(wb.B, wb.T, wb.H, 128, 128)
+    o_w, s_w = kda.forward(xb["q"], xb["k"], xb["v"], xb["log_alpha"], xb["beta"], xb["initial_state"], workspace=ws)
+    o_p, s_p = _run_gpu(xb)
+    assert torch.equal(o_p, o_w) and torch.equal(s_p, s_w)
+
+
 def test_pooled_workspace_is_capped_and_shared_by_streams():
     """A shape whose fastest workspace is above 1 GiB runs in blocks within 1 GiB
     (bit-identical to the full workspace); calls on two streams take their own
