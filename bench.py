@@ -75,11 +75,11 @@ MEASURED_TRAFFIC = {
     ("kda_prefill_tc.cu", "prefill_bf16_b1_h32_t65536_d128"): ("411803dd646a1f7c", 0.979 * 3768582144),
     ("kda_prefill_tc.cu", "prefill_bf16_b4_h32_t16384_d128_state_T4096"): ("411803dd646a1f7c", 938.4e6),
     # two-kernel prefill, one kda_forward_ws call with the pipelined schedule (blocks of
-    # 32, 64 and 32 chunks: prep 187.6, 427.9, 183.1 MB and per-head chain 169.8, 358.2,
-    # 171.9 MB), captured on B1 H32 T8192 and scaled by 8 to T = 65536: every term
+    # 32, 64 and 32 chunks: prep 187.6, 427.8, 183.2 MB and per-head chain 169.6, 357.8,
+    # 171.3 MB), captured on B1 H32 T8192 and scaled by 8 to T = 65536: every term
     # (inputs, chunk records, outputs) grows with the token count
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("6076c5c69c33eaeb", 8 * 1498.6e6),
-    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("6076c5c69c33eaeb", 1498.6e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("e1d6d30bca00be24", 8 * 1497.4e6),
+    ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("e1d6d30bca00be24", 1497.4e6),
 }
 
 

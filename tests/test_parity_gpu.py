@@ -286,10 +286,10 @@ def test_no_device_memory_grows_with_sequence_length():
 
 
 def test_pooled_workspace_falls_back_to_the_one_kernel_prefill():
-    """A shape whose smallest workspace cannot be had (1.25 M heads of one token: 186
-    GB of records) runs the one-kernel prefill, bit for bit, and leaves the pool and the
+    """A shape whose smallest workspace cannot be had (1.5 M heads of one token: 223 GB
+    of records) runs the one-kernel prefill, bit for bit, and leaves the pool and the
     CUDA error state clean."""
-    w = I.scaled(I.PREFILL_H16_T4K, B=1, H=1_250_000, T=1, seed=21)
+    w = I.scaled(I.PREFILL_H16_T4K, B=1, H=1_500_000, T=1, seed=21)
     assert kda.workspace_bytes(w.B, w.T, w.H, 128, 128, minimum=True) > torch.cuda.get_device_properties(0).total_memory
     x = I.make_inputs(w, "cuda")
     args = (x["q"], x["k"], x["v"], x["log_alpha"], x["beta"], None)
