@@ -80,15 +80,23 @@ MEASURED_TRAFFIC = {
     # (inputs, chunk records, outputs) grows with the token count
     ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128"): ("e1d6d30bca00be24", 8 * 1497.4e6),
     ("kda_prefill_split.cu", "prefill_bf16_b1_h32_t65536_d128_T8192"): ("e1d6d30bca00be24", 1497.4e6),
+    # Gated DeltaNet two-kernel prefill (kda_gdn_forward_ws, same schedule): chunk-local
+    # kernel 143.2, 344.9, 141.3 MB and the chain's kScalar instance 169.8, 356.4, 171.2 MB
+    # on B1 H32 T8192, scaled by 8; the chunk-local kernel lives in kda_prep_scalar.cuh
+    ("kda_prefill_split.cu", "gdn_prefill_bf16_b1_h32_t65536_d128"):
+        ("e1d6d30bca00be24", 8 * 1326.85e6, {"kda_prep_scalar.cuh": "ad7bde3e303a7b31"}),
 }
 
 
 def measured_traffic(src, workload):
+    """Captured bytes per launch while the kernel source (and any header named with
+    the entry) is the one the capture ran, else None."""
     ent = MEASURED_TRAFFIC.get((src, workload))
     if ent is None:
         return None
-    path = os.path.join(ROOT, "gated_delta_rule_109_b200", "csrc", src)
-    return ent[1] if source_digest(path) == ent[0] else None
+    csrc = os.path.join(ROOT, "gated_delta_rule_109_b200", "csrc")
+    same = {src: ent[0], **(ent[2] if len(ent) > 2 else {})}
+    return ent[1] if all(source_digest(os.path.join(csrc, f)) == d for f, d in same.items()) else None
 
 
 def source_digest(path):
@@ -561,7 +569,8 @@ def _add_gdn(line, args, w, world, device, hbm, use_workspace=True):
         "value": w.B * w.T * args.steps * world / (ms_total / 1e3), "unit": "tokens/s",
         "ms_per_step": ms_total / args.steps, "gpu_launches": pre["launches"],
         "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
-                     "traffic": None,
+                     "traffic": (measured_traffic("kda_prefill_split.cu", "gdn_" + w.name)
+                                 if tc and use_workspace else None),
                      "kernel": ("prefill_prep_scalar_kernel + prefill_chain_t_kernel<kScalar> (pipelined)"
                                 if tc and use_workspace
                                 else "prefill_gdn_tc_kernel" if tc else "prefill_simt_kernel"),
