@@ -12,12 +12,17 @@ pinned here to things outside itself:
 
 A planted mistake in a copy of the backward fails one of them
 (test_oracle_pin_mutations).
+
+The last test runs the other way: the pinned oracle checks the chunkwise gradient
+algebra (tests/chunked_fp64.py) that a chunked backward follows.
 """
 import math
 
 import numpy as np
+import pytest
 
 import oracle
+from tests.chunked_fp64 import chunked_backward
 
 NAMES = ("q", "k", "v", "log_alpha", "beta", "initial_state")
 GRAD = {"q": "dq", "k": "dk", "v": "dv", "log_alpha": "dlog_alpha", "beta": "dbeta",
@@ -122,3 +127,18 @@ def test_backward_without_state_arguments():
     assert g["dinitial_state"].shape == x["initial_state"].shape
     g0 = oracle.backward(*(x[n] for n in NAMES[:5]), np.zeros_like(d_out))
     assert all(np.abs(g0[n]).max() == 0.0 for n in GRAD.values())
+
+
+@pytest.mark.parametrize("C,T,states", [(64, 150, True), (16, 37, True), (8, 21, False), (5, 13, True),
+                                        (1, 6, False)])
+def test_chunked_gradient_algebra_equals_the_oracle(C, T, states):
+    """The chunkwise gradient (tests/chunked_fp64.py: a serial dS chain that is the
+    forward chain transposed, everything else chunk-parallel through the WY
+    factors) equals the pinned gradients of the token recurrence in fp64, over
+    whole chunks and a ragged last chunk."""
+    x, d_out, d_fin = _draw(11 + C, T=T, H=2, dk=8, dv=6)
+    s0, dfin = (x["initial_state"], d_fin) if states else (None, None)
+    ref = oracle.backward(*(x[n] for n in NAMES[:5]), d_out, s0, dfin)
+    got = chunked_backward(*(x[n] for n in NAMES[:5]), d_out, s0, dfin, C=C)
+    for n in GRAD.values():
+        assert oracle.parity_error(got[n], ref[n]) < 1e-12, n
