@@ -63,26 +63,27 @@ def chunked_forward(q, k, v, log_alpha, beta, initial_state=None, scale=None, C=
     return out, S_all
 
 
-def _chunk_terms(kk, qq, vv, bb, la, S, scale):
-    """The chunk's forward quantities (module docstring) for entering state S."""
+def _chunk_terms(kk, qq, vv, bb, la, S, scale, mm=np.matmul):
+    """The chunk's forward quantities (module docstring) for entering state S; every
+    matrix product goes through ``mm``."""
     c = kk.shape[0]
     G = np.cumsum(la, axis=0)
     eG, emG, eL = np.exp(G), np.exp(-G), np.exp(G[-1] - G)
     Kt, Kb, Qt, Kh = kk * eG, kk * emG, scale * qq * eG, kk * eL
-    P = np.tril(Kt @ Kb.T, -1)
+    P = np.tril(mm(Kt, Kb.T), -1)
     A = bb[:, None] * P
-    M = np.tril(Qt @ Kb.T)
+    M = np.tril(mm(Qt, Kb.T))
     Tm = np.linalg.inv(np.eye(c) + A)
-    W = Tm @ (bb[:, None] * Kt)
-    U = Tm @ (bb[:, None] * vv)
-    D = U - W @ S
+    W = mm(Tm, bb[:, None] * Kt)
+    U = mm(Tm, bb[:, None] * vv)
+    D = U - mm(W, S)
     gam = np.exp(G[-1])
     return dict(G=G, eG=eG, emG=emG, eL=eL, Kt=Kt, Kb=Kb, Qt=Qt, Kh=Kh, P=P, M=M, Tm=Tm, W=W, D=D,
-                gam=gam, S_next=gam[:, None] * S + Kh.T @ D)
+                gam=gam, S_next=gam[:, None] * S + mm(Kh.T, D))
 
 
 def chunked_backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_final_state=None,
-                     scale=None, C=64):
+                     scale=None, C=64, mm=np.matmul):
     """Reverse-mode derivative of the chunk algebra above, one chunk at a time.
 
     The loss is L = sum(O * d_out) + sum(S_T * d_final_state).  A forward sweep keeps
@@ -105,7 +106,9 @@ def chunked_backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_fina
       Kh = k e^{G_last - G}, Gam = e^{G_last}) to dk, dq and dG, whose suffix sums
       over the chunk are dlog_alpha (G is an inclusive prefix sum).
 
-    Returns the dict of oracle.backward: dq, dk, dv, dlog_alpha, dbeta, dinitial_state.
+    Every matrix product goes through ``mm`` (a test passes a model of a kernel's
+    product precision).  Returns the dict of oracle.backward: dq, dk, dv, dlog_alpha,
+    dbeta, dinitial_state.
     """
     q, k, v, la, be, g_o = (np.asarray(x, dtype=np.float64) for x in (q, k, v, log_alpha, beta, d_out))
     B, T, H, dk = q.shape
@@ -126,27 +129,27 @@ def chunked_backward(q, k, v, log_alpha, beta, d_out, initial_state=None, d_fina
             S_in, S = [], S0[b, h].copy()
             for s in starts:
                 S_in.append(S)
-                S = _chunk_terms(sl(k, s), sl(q, s), sl(v, s), sl(be, s), sl(la, s), S, scale)["S_next"]
+                S = _chunk_terms(sl(k, s), sl(q, s), sl(v, s), sl(be, s), sl(la, s), S, scale, mm)["S_next"]
             dS = gS[b, h].copy()
             for s, S in zip(reversed(starts), reversed(S_in)):
                 kk, qq, vv, bb, dO = sl(k, s), sl(q, s), sl(v, s), sl(be, s), sl(g_o, s)
-                f = _chunk_terms(kk, qq, vv, bb, sl(la, s), S, scale)
+                f = _chunk_terms(kk, qq, vv, bb, sl(la, s), S, scale, mm)
                 c = kk.shape[0]
-                dD = f["M"].T @ dO + f["Kh"] @ dS
-                dS_in = f["gam"][:, None] * dS + f["Qt"].T @ dO - f["W"].T @ dD
-                dM = np.tril(dO @ f["D"].T)
-                dQt = dO @ S.T + dM @ f["Kb"]
-                dKb = dM.T @ f["Qt"]
-                dKh = f["D"] @ dS.T
+                dD = mm(f["M"].T, dO) + mm(f["Kh"], dS)
+                dS_in = f["gam"][:, None] * dS + mm(f["Qt"].T, dO) - mm(f["W"].T, dD)
+                dM = np.tril(mm(dO, f["D"].T))
+                dQt = mm(dO, S.T) + mm(dM, f["Kb"])
+                dKb = mm(dM.T, f["Qt"])
+                dKh = mm(f["D"], dS.T)
                 dGam = (dS * S).sum(axis=1)
-                dW = -dD @ S.T
+                dW = -mm(dD, S.T)
                 Yv, Yk = bb[:, None] * vv, bb[:, None] * f["Kt"]
-                dTm = dD @ Yv.T + dW @ Yk.T
-                dYv, dYk = f["Tm"].T @ dD, f["Tm"].T @ dW
-                dA = -np.tril(f["Tm"].T @ dTm @ f["Tm"].T, -1)
+                dTm = mm(dD, Yv.T) + mm(dW, Yk.T)
+                dYv, dYk = mm(f["Tm"].T, dD), mm(f["Tm"].T, dW)
+                dA = -np.tril(mm(mm(f["Tm"].T, dTm), f["Tm"].T), -1)
                 dP = bb[:, None] * dA
-                dKt = bb[:, None] * dYk + dP @ f["Kb"]
-                dKb = dKb + dP.T @ f["Kt"]
+                dKt = bb[:, None] * dYk + mm(dP, f["Kb"])
+                dKb = dKb + mm(dP.T, f["Kt"])
                 e = s + c
                 res["dv"][b, s:e, h] = bb[:, None] * dYv
                 res["dbeta"][b, s:e, h] = ((dYv * vv).sum(1) + (dYk * f["Kt"]).sum(1)
