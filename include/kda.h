@@ -354,10 +354,11 @@ kda_status kda_gdn_forward(const void *q, const void *k, const void *v,
  * kda_gdn_forward_ws -- kda_gdn_forward with a caller-provided device workspace,
  * as kda_forward_ws is to kda_forward: bf16 with dk = dv = 128 and a workspace of
  * at least kda_forward_workspace_min_bytes(B, T, H, dk, dv, dtype) bytes (256-byte
- * aligned) take the two-kernel prefill, with each token's scalar decay (or none)
- * staged in every key channel; anything else runs the one-kernel scalar-gate
- * prefill, which needs no device memory beyond its arguments.  Same arguments,
- * statuses and results as kda_gdn_forward.
+ * aligned) take the two-kernel prefill: chunk records from a chunk-local kernel of
+ * the scalar gate's own, in which the per-token decay factors out of every
+ * product, and the per-head chain's scalar-gate form; anything else runs the
+ * one-kernel scalar-gate prefill, which needs no device memory beyond its
+ * arguments.  Same arguments, statuses and results as kda_gdn_forward.
  */
 kda_status kda_gdn_forward_ws(const void *q, const void *k, const void *v,
                               const float *log_alpha, const float *beta,
